@@ -1,0 +1,138 @@
+/*
+ * fir_oracle.c -- plain fp64 CPU oracle for the gated, grouped, depthwise causal FIR.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check in __graft_entry__.py and
+ * the CPU-baseline leg of bench.py may load this library.  It shares no code, header, table
+ * or helper with the CUDA path in gated_causal_fir_b200/, and it never sees a value that the
+ * CUDA path produced.
+ *
+ * Source: the StripedHyena 2 page "04. Hardware-aware convolution kernels"
+ * (imamachi-n.github.io, homemade-llm, stripedhyena2/hardware-algorithms):
+ *   - Sec. 1, causal FIR as a sum: y_t = sum_{k<=t} h_{t-k} x_k, with h_k = 0 outside [0, l_h);
+ *   - Sec. 2, block convolution: yhat_n = sum_k H_{n-k} xhat_k over l_b x l_b sub-blocks of the
+ *     lower-triangular Toeplitz matrix; blocks beyond the filter support are zero;
+ *   - Sec. 3, the worked example (l = 6, l_h = 4, l_b = 3), which fixes the sub-block index rule
+ *     H_m[i][j] = h_{m*l_b + i - j}, and the two-stage form Yhat_n = H0 Xhat_n + H1 Xhat_{n-1}
+ *     with Xhat_{-1} = 0.
+ * The gate y = q * (h_g conv (k * v)), with every d_g consecutive channels sharing filter h_g,
+ * is the operator form of Hyena-SE / Hyena-MR (StripedHyena 2 overview page, Sec. 3 operator
+ * table: SE/MR are gated convolutions with short / medium explicit filters).
+ *
+ * Everything is fp64.  Callers pass the exact fp64 upcast of their (bf16 or fp32) inputs, so
+ * k*v is exact and the only rounding is fp64 summation, in tap order j = 0, 1, ...
+ *
+ * Parity pins (tests/test_oracle_pins.py): worked example (symbolic H0/H1 and integer-exact
+ * two-stage == direct), dense Toeplitz product, numpy.convolve, scipy.signal.lfilter, torch
+ * conv1d, impulse, shift, linearity, causality, closed form of a geometric filter, grouping
+ * and batch independence.  No function below is "parity unpinned".
+ */
+#include <stdint.h>
+#include <stddef.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Return codes shared by every oracle entry point. */
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+
+/*
+ * Direct definition (page 04, Sec. 1 sum, gated as in the Hyena-SE/MR operator):
+ *
+ *   y[b,t,c] = q[b,t,c] * sum_{j=0}^{min(l_h-1, t)} h[c / d_g, j] * (k[b,t-j,c] * v[b,t-j,c])
+ *
+ * q, k, v, y: [B, L, D] row-major (channels contiguous).  h: [D / d_g, l_h] row-major, h[g,0]
+ * multiplies the current token.  Every sequence b starts from zero history.
+ * nthreads <= 0 lets OpenMP choose.
+ */
+int oracle_gated_fir_f64(const double *q, const double *k, const double *v, const double *h,
+                         double *y, int64_t B, int64_t L, int64_t D, int64_t d_g, int64_t l_h,
+                         int nthreads)
+{
+    if (!q || !k || !v || !h || !y) return ORACLE_BAD_ARG;
+    if (B < 0 || L < 0 || D < 1 || d_g < 1 || D % d_g != 0 || l_h < 1) return ORACLE_BAD_ARG;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    const int64_t rows = B * L;
+    #pragma omp parallel for schedule(static)
+    for (int64_t row = 0; row < rows; ++row) {
+        const int64_t b = row / L;
+        const int64_t t = row % L;
+        const int64_t jmax = (l_h - 1 < t) ? l_h - 1 : t;
+        for (int64_t c = 0; c < D; ++c) {
+            const double *hg = h + (c / d_g) * l_h;
+            double s = 0.0;
+            for (int64_t j = 0; j <= jmax; ++j) {
+                const int64_t src = (b * L + (t - j)) * D + c;
+                s += hg[j] * (k[src] * v[src]);
+            }
+            y[row * D + c] = q[row * D + c] * s;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Sub-blocks of the lower-triangular Toeplitz matrix (page 04, Sec. 2 and the Sec. 3 worked
+ * example): H[m][i][j] = h[m*l_b + i - j] when that index lies in [0, l_h), else 0,
+ * for m = 0 .. S-1.  H: [S, l_b, l_b] row-major.
+ */
+int oracle_toeplitz_blocks_f64(const double *h, int64_t l_h, int64_t l_b, int64_t S, double *H)
+{
+    if (!h || !H || l_h < 1 || l_b < 1 || S < 1) return ORACLE_BAD_ARG;
+    for (int64_t m = 0; m < S; ++m)
+        for (int64_t i = 0; i < l_b; ++i)
+            for (int64_t j = 0; j < l_b; ++j) {
+                const int64_t idx = m * l_b + i - j;
+                H[(m * l_b + i) * l_b + j] = (idx >= 0 && idx < l_h) ? h[idx] : 0.0;
+            }
+    return ORACLE_OK;
+}
+
+/*
+ * Block convolution of one channel with S stages (page 04, Sec. 2 block sum, truncated to the
+ * S sub-blocks H_0 .. H_{S-1}; S = 2 is the Sec. 3 two-stage form):
+ *
+ *   Yhat_n = sum_{m=0}^{S-1} H_m Xhat_{n-m},   Xhat_{<0} = 0,
+ *
+ * over the ceil(L / l_b) chunks of x; the tail chunk is zero-padded on read and clipped on
+ * write.  Used by the tests to check the pages' two-stage statements against the direct sum.
+ */
+int oracle_block_conv_f64(const double *h, int64_t l_h, int64_t l_b, int64_t S,
+                          const double *x, int64_t L, double *y)
+{
+    if (!h || !x || !y || l_h < 1 || l_b < 1 || S < 1 || L < 0) return ORACLE_BAD_ARG;
+    const int64_t nchunks = (L + l_b - 1) / l_b;
+    for (int64_t n = 0; n < nchunks; ++n) {
+        for (int64_t i = 0; i < l_b; ++i) {
+            const int64_t t = n * l_b + i;
+            if (t >= L) break;
+            double s = 0.0;
+            for (int64_t m = 0; m < S; ++m) {
+                const int64_t src_chunk = n - m;
+                if (src_chunk < 0) continue;           /* Xhat_{<0} = 0 */
+                for (int64_t jj = 0; jj < l_b; ++jj) {
+                    const int64_t src = src_chunk * l_b + jj;
+                    if (src >= L) continue;             /* zero-padded tail chunk */
+                    const int64_t idx = m * l_b + i - jj;  /* H_m[i][jj] */
+                    if (idx >= 0 && idx < l_h) s += h[idx] * x[src];
+                }
+            }
+            y[t] = s;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Number of threads OpenMP would use (reported as the oracle's core count). */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
