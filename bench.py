@@ -1,0 +1,337 @@
+#!/usr/bin/env python
+"""Throughput of the gated grouped causal FIR forward (Hyena-MR: B=1, L=8192, D=4096, d_g=64,
+l_h=128, l_b=64, bf16) on B200, one process per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mr] [--impl reference]
+
+A step is one pass of the whole forward (one kernel launch) over one batch of synthetic
+inputs already resident in HBM.  Three input sets rotate from step to step (3 x 256 MiB, more
+than the 126 MB L2), so no step reads the previous step's inputs from L2.  The timed region is
+bracketed by a barrier and a device synchronisation, timed with CUDA events on the launching
+stream, and reduced as the max over ranks.  Under torchrun each rank runs an independent
+replica on its own batch (weak scaling, no collective on the data path).
+
+Rank 0 prints one JSON line.  Besides the throughput it reports the roofline of the kernel
+(algorithmic bytes / mean launch time vs the measured HBM copy bandwidth), SM clocks sampled
+through NVML during the timed region, an end-to-end figure through
+``hyena_conv_fwd_from_host`` (pinned host buffers, copies inside the timed region) and the
+fp64 oracle timed on the host cores as a CPU baseline.  ``--impl reference`` times only the
+oracle, one l_b-row chunk of the workload per step.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Hyena-MR fwd tokens/s (D=4096, L=8192, ℓ_h=128); HBM GB/s vs peak"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["hyena_conv.cu", "fir_tc.cuh", "fir_cuda_core.cuh", "ptx.cuh"]
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default="mr")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="target CPU time of the oracle baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "gated_causal_fir_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "%s_%s_traffic.json" % (kernel, workload))
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return rec.get("traffic_bytes_per_launch")
+
+
+class ClockSampler:
+    """Polls SM clock, power and clock-event reasons through NVML in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index, period_s=0.005):
+        self.samples, self.period, self.ok = [], period_s, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report it instead of clocks
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), sm, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"error": "NVML unavailable: " + self.err}
+        win = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples
+        reasons = set()
+        for _, _, rs in win:
+            for bit, name in self.REASONS.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in win) if win else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(win),
+                "source": "NVML, %.0f ms period, during the timed region" % (1e3 * self.period)}
+
+
+def cpu_baseline(wl, q, k, v, h, target_s):
+    """Time the fp64 oracle, as it stands, on this host's cores over whole copies of the
+    workload (repeated until ~target_s of work); returns (record, oracle output of one pass)."""
+    import oracle
+    qh, kh, vh, hh = (x.cpu() for x in (q, k, v, h))
+    reps, t_total, y_ref = 0, 0.0, None
+    while reps < 20 and (reps == 0 or t_total < target_s):
+        t = time.perf_counter()
+        y_ref = oracle.gated_fir(qh, kh, vh, hh, wl.d_g)
+        t_total += time.perf_counter() - t
+        reps += 1
+    rec = {"value": wl.tokens * reps / t_total, "unit": UNIT, "cores": oracle.max_threads(),
+           "kind": "oracle",
+           "sample": "whole %s workload x%d (%.1f s of fp64 direct sums, OpenMP)"
+                     % (wl.name, reps, t_total)}
+    return rec, y_ref
+
+
+def run_reference(args, wl, rank, world):
+    """The oracle arm: one l_b-row chunk of the workload per step, on the host cores."""
+    import oracle
+    import torch
+    from gated_causal_fir_b200.workloads import make_inputs
+    if rank != 0:
+        return
+    q, k, v, h = make_inputs(wl, device="cpu")
+    n_chunks = (wl.L + wl.l_b - 1) // wl.l_b
+
+    def step(i):
+        b = i % wl.B
+        t0 = ((i // wl.B) % n_chunks) * wl.l_b
+        t1 = min(wl.L, t0 + wl.l_b)
+        s = max(0, t0 - (wl.l_h - 1))
+        oracle.gated_fir(q[b, s:t1], k[b, s:t1], v[b, s:t1], h, wl.d_g)
+        return t1 - t0
+
+    for i in range(args.warmup):
+        step(i)
+    t = time.perf_counter()
+    rows = sum(step(args.warmup + i) for i in range(args.steps))
+    dt = time.perf_counter() - t
+    value = rows / dt
+    cores = oracle.max_threads()
+    sample = "one %d-row chunk (all %d channels, with %d history rows) per step" % (
+        wl.l_b, wl.D, wl.l_h - 1)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(wl),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    del torch
+
+
+def workload_config(wl):
+    return {"workload": wl.describe(), "B": wl.B, "L": wl.L, "D": wl.D, "d_g": wl.d_g,
+            "l_h": wl.l_h, "l_b": wl.l_b, "io_dtype": wl.dtype, "filters": wl.filt,
+            "l2": "3 rotating input sets (%.0f MiB) > 126 MB L2"
+                  % (3 * wl.algorithmic_bytes() / 2 ** 20)}
+
+
+def main():
+    args = parse()
+    from gated_causal_fir_b200 import dist as D
+    from gated_causal_fir_b200.workloads import WORKLOADS, make_inputs
+
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        rank, _, world = D.env_world()
+        run_reference(args, wl, rank, world)
+        return
+
+    import torch
+    rank, local_rank, world = D.init("nccl")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+
+    import gated_causal_fir_b200 as g
+    from gated_causal_fir_b200 import _native
+    _native.lib()  # fail loudly here if the library is missing
+
+    # Inputs: three independent sets per rank, resident before the timed region.
+    sets = []
+    for s in range(3):
+        q, k, v, h = make_inputs(wl, device=dev, seed=D.rank_seed(wl.seed + 101 * s, rank),
+                                 l_slice=1 << 16)
+        sets.append((q, k, v, h, torch.empty_like(q)))
+    algo = g.hyena_select_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b,
+                               g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16)
+    fwd = g.hyena_conv_fwd_f32 if wl.dtype == "f32" else g.hyena_conv_fwd
+    stream = torch.cuda.Stream(device=dev)
+
+    def launch(i):
+        q, k, v, h, y = sets[i % 3]
+        fwd(q, k, v, h, wl.d_g, wl.l_b, y=y, stream=stream)
+
+    torch.cuda.synchronize()
+    for i in range(args.warmup):
+        launch(i)
+    torch.cuda.synchronize()
+    assert g.hyena_device_status(clear=True) == 0, "device status raised during warm-up"
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank).start()
+    D.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    start.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        launch(i)
+        ev[i][1].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    D.barrier()
+    clocks.stop()
+    elapsed_ms = start.elapsed_time(stop)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    status = g.hyena_device_status(clear=True)
+    max_ms = D.max_over_ranks(elapsed_ms, device=dev)
+    mean_launch_ms = D.max_over_ranks(sum(launch_ms) / K, device=dev)
+
+    # End to end through the host-buffer entry point, pinned buffers, copies timed.
+    e2e = None
+    if not args.no_e2e and args.e2e_steps > 0:
+        qh, kh, vh, hh = (x.cpu().pin_memory() for x in sets[0][:4])
+        yh = torch.empty_like(qh).pin_memory()
+        g.hyena_conv_fwd_from_host(qh, kh, vh, hh, wl.d_g, wl.l_b, out=yh, device=dev,
+                                   stream=stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        D.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            g.hyena_conv_fwd_from_host(qh, kh, vh, hh, wl.d_g, wl.l_b, out=yh, device=dev,
+                                       stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = D.max_over_ranks(e0.elapsed_time(e1), device=dev)
+        e2e = {"value": world * wl.tokens * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (qh, kh, vh, hh)),
+               "d2h_bytes_per_step": yh.numel() * yh.element_size(),
+               "steps": args.e2e_steps, "api": "hyena_conv_fwd_from_host"}
+
+    cpu, parity = None, None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu, y_ref = cpu_baseline(wl, *sets[0][:4], target_s=args.cpu_seconds)
+        q, k, v, h, y = sets[0]
+        fwd(q, k, v, h, wl.d_g, wl.l_b, y=y, stream=stream)
+        torch.cuda.synchronize()
+        import numpy as np
+        err = np.abs(y.double().cpu().numpy() - y_ref)
+        parity = {"max_err_over_bound": float((err / (1e-2 + 1e-2 * np.abs(y_ref))).max()),
+                  "bound": "|y - y_oracle| <= 1e-2 + 1e-2 |y_oracle|", "checked": "all outputs"}
+
+    D.barrier()
+    if rank == 0:
+        peak, peak_kind = measured_peak_hbm()
+        bytes_per_launch = wl.algorithmic_bytes()
+        achieved = bytes_per_launch / (mean_launch_ms / 1e3) / 1e9
+        kernel = {g.HYENA_ALGO_TENSOR: "fir_tc_kernel", g.HYENA_ALGO_WINDOW: "fir_window_kernel",
+                  g.HYENA_ALGO_DIRECT: "fir_direct_kernel"}[algo]
+        traffic = committed_traffic(kernel, wl.name)
+        line = {
+            "metric": METRIC, "value": world * wl.tokens * K / (max_ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": max_ms / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic", "config": dict(
+                workload_config(wl), parallelism="replicas x%d" % world,
+                mma="f16 x f16 -> f32 (tensor path)" if algo == g.HYENA_ALGO_TENSOR
+                else "fp32 FFMA"),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": "%s (MEASURED_PEAKS hbm_gbs)" % peak_kind
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+                         "algorithmic_bytes_per_launch": bytes_per_launch,
+                         "mean_launch_us": 1e3 * mean_launch_ms, "kernel": kernel},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K,
+            "clocks": clocks.summary(t_wall0, t_wall1),
+            "kernel_algo": g.ALGO_NAMES[algo], "device_status": status, "parity": parity,
+            "wall_s_timed_region": t_wall1 - t_wall0,
+        }
+        print(json.dumps(line), flush=True)
+    D.finalize()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,190 @@
+"""B200-native gated, grouped, depthwise causal FIR: the Hyena-SE / Hyena-MR forward.
+
+    y[b,t,c] = q[b,t,c] * sum_{j<l_h, j<=t} h[c // d_g, j] * k[b,t-j,c] * v[b,t-j,c]
+
+computed by the sm_100a kernels of ``libhyena_conv.so`` through its C ABI
+(``include/hyena_conv.h``).  The functions here carry the C names and only marshal torch CUDA
+tensors into pointers, sizes and the current stream; PyTorch provides device memory and
+streams, nothing else.  There is no CPU path: without a CUDA device or the built library every
+call raises.
+
+Importing the package does not load the library; the first call does.
+"""
+import ctypes
+
+from . import _native
+from ._native import (HYENA_ALGO_AUTO, HYENA_ALGO_DIRECT, HYENA_ALGO_TENSOR, HYENA_ALGO_WINDOW,
+                      HYENA_DEVICE_F16_RANGE, HYENA_DEVICE_TIMEOUT, HYENA_DTYPE_BF16,
+                      HYENA_DTYPE_F32, ALGO_NAMES, HyenaError)
+
+__all__ = [
+    "hyena_conv_fwd", "hyena_conv_fwd_f32", "hyena_conv_fwd_ex", "hyena_select_algo",
+    "hyena_build_toeplitz", "hyena_device_status", "hyena_status_string", "hyena_abi_version",
+    "HyenaError", "HYENA_ALGO_AUTO", "HYENA_ALGO_TENSOR", "HYENA_ALGO_WINDOW",
+    "HYENA_ALGO_DIRECT", "HYENA_DTYPE_BF16", "HYENA_DTYPE_F32", "HYENA_DEVICE_TIMEOUT",
+    "HYENA_DEVICE_F16_RANGE", "ALGO_NAMES", "hyena_conv_fwd_from_host",
+]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return HYENA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return HYENA_DTYPE_F32
+    raise TypeError("q, k, v must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _check(q, k, v, h, d_g, y):
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v), ("h", h)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError("%s must be a CUDA tensor" % name)
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous" % name)
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B, L, D] shape")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    if h.dtype != torch.float32 or h.dim() != 2:
+        raise TypeError("h must be float32 [D // d_g, l_h]")
+    B, L, D = q.shape
+    if d_g < 1 or D % d_g != 0 or h.shape[0] * d_g != D:
+        raise ValueError("h has %d rows; D=%d with d_g=%d needs D // d_g" % (h.shape[0], D, d_g))
+    if y is None:
+        y = torch.empty_like(q)
+    elif (not isinstance(y, torch.Tensor) or y.shape != q.shape or y.dtype != q.dtype
+          or not y.is_cuda or not y.is_contiguous()):
+        raise ValueError("y must be a contiguous CUDA tensor like q")
+    return y
+
+
+def hyena_conv_fwd_ex(q, k, v, h, d_g, l_b, algo=HYENA_ALGO_AUTO, y=None, stream=None):
+    """Forward with the algorithm chosen by the caller (HYENA_ALGO_*); returns y.
+
+    q, k, v: CUDA [B, L, D], all bf16 or all fp32.  h: CUDA fp32 [D // d_g, l_h].
+    l_b: block size of the decomposition (needs l_h <= 2 * l_b; the result does not depend on
+    it).  y: optional preallocated output.  Runs asynchronously on ``stream`` (default: the
+    current torch stream).
+    """
+    y = _check(q, k, v, h, d_g, y)
+    B, L, D = q.shape
+    rc = _native.lib().hyena_conv_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), h.data_ptr(),
+                                         y.data_ptr(), B, L, D, d_g, h.shape[1], l_b,
+                                         _dtype_code(q), algo, _stream(stream))
+    _native.check("hyena_conv_fwd_ex", rc)
+    return y
+
+
+def hyena_conv_fwd(q, k, v, h, d_g, l_b, y=None, stream=None):
+    """bf16 forward, fastest supported algorithm (C: hyena_conv_fwd); returns y."""
+    y = _check(q, k, v, h, d_g, y)
+    if _dtype_code(q) != HYENA_DTYPE_BF16:
+        raise TypeError("hyena_conv_fwd takes bf16 q, k, v; use hyena_conv_fwd_f32 for fp32")
+    B, L, D = q.shape
+    rc = _native.lib().hyena_conv_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), h.data_ptr(),
+                                      y.data_ptr(), B, L, D, d_g, h.shape[1], l_b,
+                                      _stream(stream))
+    _native.check("hyena_conv_fwd", rc)
+    return y
+
+
+def hyena_conv_fwd_f32(q, k, v, h, d_g, l_b, y=None, stream=None):
+    """fp32 forward (C: hyena_conv_fwd_f32); returns y."""
+    y = _check(q, k, v, h, d_g, y)
+    if _dtype_code(q) != HYENA_DTYPE_F32:
+        raise TypeError("hyena_conv_fwd_f32 takes fp32 q, k, v")
+    B, L, D = q.shape
+    rc = _native.lib().hyena_conv_fwd_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                          h.data_ptr(), y.data_ptr(), B, L, D, d_g, h.shape[1],
+                                          l_b, _stream(stream))
+    _native.check("hyena_conv_fwd_f32", rc)
+    return y
+
+
+def hyena_select_algo(B, L, D, d_g, l_h, l_b, dtype=HYENA_DTYPE_BF16, ptrs=(16, 16, 16, 16, 16)):
+    """Host-only: the algorithm AUTO would run (HYENA_ALGO_*), or raises HyenaError.
+
+    ``ptrs`` are the (q, k, v, h, y) addresses to judge alignment by (plain integers); the
+    defaults stand for distinct 16-byte aligned buffers.
+    """
+    n = B * L * D * (4 if dtype == HYENA_DTYPE_F32 else 2)
+    q, k, v, h, y = ptrs
+    if ptrs == (16, 16, 16, 16, 16):  # distinct, non-overlapping, aligned stand-ins
+        q, k, v, h, y = (16 + i * (n + 64) for i in range(5))
+    rc = _native.lib().hyena_select_algo(q, k, v, h, y, B, L, D, d_g, l_h, l_b, dtype)
+    if rc < 0:
+        raise HyenaError("hyena_select_algo", -rc)
+    return rc
+
+
+def hyena_build_toeplitz(h, l_b, stream=None):
+    """H0, H1, H2 (fp32 [G, l_b, l_b] CUDA tensors): H_m[g][i][j] = h[g][m l_b + i - j]."""
+    torch = _torch()
+    if not isinstance(h, torch.Tensor) or not h.is_cuda or h.dtype != torch.float32 \
+            or h.dim() != 2 or not h.is_contiguous():
+        raise TypeError("h must be a contiguous CUDA float32 [G, l_h] tensor")
+    G, l_h = h.shape
+    H = torch.empty((3, G, l_b, l_b), dtype=torch.float32, device=h.device)
+    rc = _native.lib().hyena_build_toeplitz(h.data_ptr(), H[0].data_ptr(), H[1].data_ptr(),
+                                            H[2].data_ptr(), G, l_h, l_b, _stream(stream))
+    _native.check("hyena_build_toeplitz", rc)
+    return H[0], H[1], H[2]
+
+
+def hyena_device_status(clear=True):
+    """The current device's status word (HYENA_DEVICE_* bits); synchronises the device."""
+    out = ctypes.c_uint(0)
+    _native.check("hyena_device_status",
+                  _native.lib().hyena_device_status(ctypes.byref(out), 1 if clear else 0))
+    return out.value
+
+
+def hyena_status_string(status):
+    return _native.status_string(status)
+
+
+def hyena_abi_version():
+    return int(_native.lib().hyena_abi_version())
+
+
+_STAGING = {}
+
+
+def hyena_conv_fwd_from_host(q, k, v, h, d_g, l_b, out=None, device="cuda", stream=None):
+    """End-to-end forward for host tensors: copies q, k, v (bf16 or fp32 [B, L, D]) and h to
+    ``device``, runs the forward there and copies y back into ``out`` (a host tensor; pinned
+    memory makes every copy asynchronous).  Device staging buffers are reused across calls
+    of the same shape.  Queued on ``stream``; synchronise it before reading ``out``.
+    """
+    torch = _torch()
+    key = (tuple(q.shape), q.dtype, tuple(h.shape), str(device))
+    bufs = _STAGING.get(key)
+    if bufs is None:
+        bufs = [torch.empty(q.shape, dtype=q.dtype, device=device) for _ in range(4)]
+        bufs.append(torch.empty(h.shape, dtype=torch.float32, device=device))
+        _STAGING.clear()
+        _STAGING[key] = bufs
+    qd, kd, vd, yd, hd = bufs
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    s = torch.cuda.current_stream() if stream is None else stream
+    with torch.cuda.stream(s):
+        qd.copy_(q, non_blocking=True)
+        kd.copy_(k, non_blocking=True)
+        vd.copy_(v, non_blocking=True)
+        hd.copy_(h, non_blocking=True)
+        hyena_conv_fwd_ex(qd, kd, vd, hd, d_g, l_b, y=yd, stream=s)
+        out.copy_(yd, non_blocking=True)
+    return out

@@ -1,0 +1,436 @@
+// fir_tc.cuh -- tcgen05 tensor-core kernel of the gated grouped causal FIR (bf16 I/O).
+//
+// Method: the block-Toeplitz form of the causal FIR (StripedHyena 2 page "04. Hardware-aware
+// convolution kernels", Sec. 2 block convolution and Sec. 3 two-stage algorithm,
+// Yhat_n = H0 Xhat_n + H1 Xhat_{n-1}, Xhat_{-1} = 0), with the Sec. 4 reuse (the Toeplitz
+// operand of a group is built once on chip and reused for every chunk and every channel of the
+// group, which turns the per-channel products into one GEMM) and the Sec. 6 chunk-direction
+// schedule (each CTA walks consecutive chunks and keeps the previous chunk's input on chip).
+//
+// One tile = 128 output rows x 64 channels (one group of d_g = 64).  The block size of the
+// decomposition is 128 rows, the largest M of one tcgen05.mma: Yhat_n = H0 Xhat_n + H1 Xhat_{n-1}
+// is then exact for l_h <= 129 (two stages suffice iff l_h <= l_b + 1).  As one GEMM per tile:
+//   D[128 x 64] = A[128 x K] * X[K x 64],  K = 128 + halo,  halo = roundup16(l_h - 1),
+// A is the Toeplitz band over input rows [t0 - halo, t0 + 128), X = k*v over those rows.
+//
+// B200 specifics:
+//  * q, k, v tiles arrive by TMA (128-byte swizzle) into a multi-stage ring; y leaves by TMA
+//    store.  The k*v pre-gate is an elementwise pass that writes fp16 X in the same swizzled
+//    layout, which is exactly the MN-major SW128 operand layout of tcgen05: no transpose.
+//  * The Toeplitz band is Hankel once the output rows are reversed (TMEM lane p holds time
+//    t0 + 127 - p): every 8x8 core matrix then depends only on r8 + c8.  A K-major, unswizzled
+//    descriptor with LBO = SBO = 128 bytes aliases those core matrices, so the whole
+//    128 x 256 band lives in 47 core matrices (6 KB) instead of 64 KB.
+//  * Accumulators live in TMEM (2 x 64 columns); the epilogue reads them with tcgen05.ld,
+//    multiplies by q and rounds to bf16 in registers, and writes y over the q tile in place.
+//  * Warp roles: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2-5 pre-gate / operand build,
+//    6-9 epilogue.  Persistent grid: one CTA per SM, each walks a contiguous range of tiles
+//    ordered (group, batch, time), so a halo tile is re-read only where a range starts inside
+//    a sequence.
+//  * Every wait is bounded (ptx.cuh); a timeout raises HYENA_DEVICE_TIMEOUT, all roles leave
+//    their loops, in-flight copies and MMAs are drained and TMEM is freed before exit.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include "ptx.cuh"
+
+namespace hyena {
+
+__device__ unsigned int g_device_status;  // OR of hyena_device_status_bits
+
+namespace tc {
+
+constexpr int kTM = 128;             // output rows per tile (MMA M)
+constexpr int kNC = 64;              // channels per tile = d_g (MMA N)
+constexpr int kMaxHalo = 128;        // supports l_h - 1 <= 128
+constexpr int kNKV = 4;              // k/v stages
+constexpr int kNQ = 2;               // q (and in-place y) stages
+constexpr int kNX = 3;               // fp16 X slots (current, previous, next)
+constexpr int kNAcc = 2;             // TMEM accumulators
+constexpr int kTileBytes = kTM * kNC * 2;                       // 16 KB
+constexpr int kACores = kTM / 8 + (kTM + kMaxHalo) / 8 - 1;     // 47
+constexpr int kABytes = 48 * 128;                               // padded
+constexpr int kTmemCols = kNAcc * kNC;                          // 128
+
+constexpr int kOffKV = 0;
+constexpr int kOffQ = kOffKV + kNKV * 2 * kTileBytes;
+constexpr int kOffX = kOffQ + kNQ * kTileBytes;
+constexpr int kOffA = kOffX + kNX * kTileBytes;
+constexpr int kOffBar = kOffA + 2 * kABytes;
+// barriers
+constexpr int kBarKVFull = 0;
+constexpr int kBarKVEmpty = kBarKVFull + kNKV;
+constexpr int kBarQFull = kBarKVEmpty + kNKV;
+constexpr int kBarQEmpty = kBarQFull + kNQ;
+constexpr int kBarYReady = kBarQEmpty + kNQ;
+constexpr int kBarXFull = kBarYReady + kNQ;
+constexpr int kBarXEmpty = kBarXFull + kNX;
+constexpr int kBarAccFull = kBarXEmpty + kNX;
+constexpr int kBarAccEmpty = kBarAccFull + kNAcc;
+constexpr int kBarAFull = kBarAccEmpty + kNAcc;
+constexpr int kBarAEmpty = kBarAFull + 2;
+constexpr int kBarDone = kBarAEmpty + 2;
+constexpr int kNumBars = kBarDone + 1;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+
+constexpr int kThreads = 320;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGate0 = 2, kWarpEpi0 = 6;
+constexpr int kGroupThreads = 128;
+
+constexpr unsigned kTimeoutBit = 1u;  // HYENA_DEVICE_TIMEOUT
+constexpr unsigned kF16RangeBit = 2u; // HYENA_DEVICE_F16_RANGE
+
+struct Params {
+  const float *h;   // [G, l_h]
+  int B, L, G, l_h;
+  int halo;         // multiple of 16, >= l_h - 1, <= kMaxHalo
+  int nT;           // tiles per sequence = ceil(L / kTM)
+  long long W;      // total tiles = G * B * nT
+};
+
+// One unit of a CTA's walk: a halo tile (input only) or an output tile.
+struct Item {
+  int g, b, i;      // group, sequence, tile index along time
+  int seg;          // running segment number within this CTA (a segment = one sequence run)
+  bool halo;        // input-only tile feeding the first output tile of a segment
+  bool hist;        // the output tile reads the previous tile's X (i > 0)
+  bool last;        // last output tile of its segment
+};
+
+struct WorkIter {
+  long long w, w_begin, w_end;
+  int nT, B, seg;
+  bool entered;
+  __device__ WorkIter(long long b, long long e, int nT_, int B_)
+      : w(b), w_begin(b), w_end(e), nT(nT_), B(B_), seg(-1), entered(false) {}
+  __device__ bool next(Item &it) {
+    if (w >= w_end) return false;
+    const long long seq = w / nT;
+    const int i = static_cast<int>(w - seq * nT);
+    it.g = static_cast<int>(seq / B);
+    it.b = static_cast<int>(seq % B);
+    const bool first = (w == w_begin) || (i == 0);
+    if (first && !entered) {
+      entered = true;
+      ++seg;
+      if (i > 0) {
+        it.i = i - 1;
+        it.seg = seg;
+        it.halo = true;
+        it.hist = false;
+        it.last = false;
+        return true;
+      }
+    }
+    it.i = i;
+    it.seg = seg;
+    it.halo = false;
+    it.hist = i > 0;
+    it.last = (w + 1 == w_end) || (i + 1 == nT);
+    ++w;
+    entered = false;
+    return true;
+  }
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  const bool ok = mbar_wait(bar, parity, abort, &g_device_status, kTimeoutBit);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ bool thread_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  return mbar_wait(bar, parity, abort, &g_device_status, kTimeoutBit);
+}
+
+// Drain wait: bounded by time only (ignores the abort flag), for copies this thread issued.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+  int no_abort = 0;
+  mbar_wait(bar, parity, &no_abort, &g_device_status, kTimeoutBit);
+}
+
+// x = fp16(k * v) for two bf16 lanes packed in a 32-bit word; k*v is exact in fp32.
+__device__ __forceinline__ uint32_t gate_pair(uint32_t kw, uint32_t vw, bool &over) {
+  const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
+  const float v0 = __uint_as_float(vw << 16), v1 = __uint_as_float(vw & 0xFFFF0000u);
+  const float x0 = k0 * v0, x1 = k1 * v1;
+  over |= (fabsf(x0) > 65504.f) | (fabsf(x1) > 65504.f);
+  const __half2 hx = __floats2half2_rn(x0, x1);
+  return *reinterpret_cast<const uint32_t *>(&hx);
+}
+
+// The Toeplitz band as Hankel core matrices: core d, element (i, j) (row i, K column j) holds
+// h[kTM - 1 + halo - 8 d - i - j] (zero outside [0, l_h)), rounded to fp16.
+__device__ __forceinline__ void build_band(uint8_t *a, const float *hg, int l_h, int halo,
+                                           int gt, bool &over) {
+  const int ncores = kTM / 8 + (kTM + halo) / 8 - 1;
+  __half *ah = reinterpret_cast<__half *>(a);
+  for (int e = gt; e < ncores * 64; e += kGroupThreads) {
+    const int d = e >> 6, i = (e >> 3) & 7, j = e & 7;
+    const int idx = kTM - 1 + halo - 8 * d - i - j;
+    const float hv = (idx >= 0 && idx < l_h) ? __ldg(hg + idx) : 0.f;
+    over |= fabsf(hv) > 65504.f;
+    ah[e] = __float2half_rn(hv);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fir_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
+                  const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *kv_st = smem + kOffKV;
+  uint8_t *q_st = smem + kOffQ;
+  uint8_t *x_st = smem + kOffX;
+  uint8_t *a_st = smem + kOffA;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  volatile int *abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long per = p.W / gridDim.x, rem = p.W % gridDim.x;
+  const long long bx = blockIdx.x;
+  const long long w_begin = bx * per + (bx < rem ? bx : rem);
+  const long long w_end = w_begin + per + (bx < rem ? 1 : 0);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNKV; ++i) {
+      mbar_init(&bars[kBarKVFull + i], 1);
+      mbar_init(&bars[kBarKVEmpty + i], kGroupThreads);
+    }
+    for (int i = 0; i < kNQ; ++i) {
+      mbar_init(&bars[kBarQFull + i], 1);
+      mbar_init(&bars[kBarQEmpty + i], 1);
+      mbar_init(&bars[kBarYReady + i], kGroupThreads);
+    }
+    for (int i = 0; i < kNX; ++i) {
+      mbar_init(&bars[kBarXFull + i], kGroupThreads);
+      mbar_init(&bars[kBarXEmpty + i], 1);
+    }
+    for (int i = 0; i < kNAcc; ++i) {
+      mbar_init(&bars[kBarAccFull + i], 1);
+      mbar_init(&bars[kBarAccEmpty + i], kGroupThreads);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[kBarAFull + i], kGroupThreads);
+      mbar_init(&bars[kBarAEmpty + i], 1);
+    }
+    mbar_init(&bars[kBarDone], 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpTma && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_y);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == kWarpTma) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      WorkIter it(w_begin, w_end, p.nT, p.B);
+      Item t;
+      uint32_t kc = 0, qc = 0;
+      while (it.next(t)) {
+        const int ks = kc % kNKV;
+        if (!thread_wait(&bars[kBarKVEmpty + ks], ((kc / kNKV) & 1) ^ 1, abort)) break;
+        mbar_arrive_expect_tx(&bars[kBarKVFull + ks], 2 * kTileBytes);
+        uint8_t *dst = kv_st + ks * 2 * kTileBytes;
+        tma_load_3d(dst, &tm_k, &bars[kBarKVFull + ks], t.g * kNC, t.i * kTM, t.b);
+        tma_load_3d(dst + kTileBytes, &tm_v, &bars[kBarKVFull + ks], t.g * kNC, t.i * kTM, t.b);
+        ++kc;
+        if (!t.halo) {
+          const int qs = qc % kNQ;
+          if (!thread_wait(&bars[kBarQEmpty + qs], ((qc / kNQ) & 1) ^ 1, abort)) break;
+          mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes);
+          tma_load_3d(q_st + qs * kTileBytes, &tm_q, &bars[kBarQFull + qs], t.g * kNC, t.i * kTM,
+                      t.b);
+          ++qc;
+        }
+      }
+      // Every load this thread issued must land before the CTA may exit.
+      for (uint32_t n = kc > kNKV ? kc - kNKV : 0; n < kc; ++n)
+        drain_wait(&bars[kBarKVFull + n % kNKV], (n / kNKV) & 1);
+      for (uint32_t n = qc > kNQ ? qc - kNQ : 0; n < qc; ++n)
+        drain_wait(&bars[kBarQFull + n % kNQ], (n / kNQ) & 1);
+    }
+  } else if (warp == kWarpMma) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      WorkIter it(w_begin, w_end, p.nT, p.B);
+      Item t;
+      uint32_t xc = 0, ac = 0;
+      int cur_seg = -1;
+      const uint32_t idesc = umma_idesc_f16_f32(kTM, kNC, 1);
+      const int ksteps = (kTM + p.halo) / 16, hsteps = p.halo / 16;
+      while (it.next(t)) {
+        const int xs = xc % kNX;
+        if (!thread_wait(&bars[kBarXFull + xs], (xc / kNX) & 1, abort)) break;
+        if (t.halo) {
+          ++xc;
+          continue;
+        }
+        const int pa = t.seg & 1;
+        if (t.seg != cur_seg) {
+          cur_seg = t.seg;
+          if (!thread_wait(&bars[kBarAFull + pa], (t.seg >> 1) & 1, abort)) break;
+        }
+        const int as = ac % kNAcc;
+        if (!thread_wait(&bars[kBarAccEmpty + as], ((ac / kNAcc) & 1) ^ 1, abort)) break;
+        tc_fence_after_sync();
+        const uint32_t a_base = smem_u32(a_st + pa * kABytes);
+        const int xp = (xc + kNX - 1) % kNX;
+        const uint32_t x_cur = smem_u32(x_st + xs * kTileBytes);
+        const uint32_t x_prev = smem_u32(x_st + xp * kTileBytes);
+        const uint32_t d_tmem = tmem_base + as * kNC;
+        uint32_t accumulate = 0;
+        for (int j = 0; j < ksteps; ++j) {
+          uint32_t b_addr;
+          if (j < hsteps) {
+            if (!t.hist) continue;  // zero history before the first tile of a sequence
+            b_addr = x_prev + (kTM - p.halo + 16 * j) * (kNC * 2);
+          } else {
+            b_addr = x_cur + (16 * j - p.halo) * (kNC * 2);
+          }
+          const uint64_t adesc = umma_smem_desc(a_base + j * 256, 128, 128, 0);
+          const uint64_t bdesc = umma_smem_desc(b_addr, kTileBytes, 1024, 2);
+          umma_f16(d_tmem, adesc, bdesc, idesc, accumulate);
+          accumulate = 1;
+        }
+        umma_commit(&bars[kBarAccFull + as]);
+        if (t.hist) umma_commit(&bars[kBarXEmpty + xp]);
+        if (t.last) {
+          umma_commit(&bars[kBarXEmpty + xs]);
+          umma_commit(&bars[kBarAEmpty + pa]);
+        }
+        ++xc;
+        ++ac;
+      }
+      // Every MMA this thread issued must complete before TMEM is freed.
+      umma_commit(&bars[kBarDone]);
+      drain_wait(&bars[kBarDone], 0);
+    }
+  } else if (warp >= kWarpGate0 && warp < kWarpGate0 + 4) {
+    // ---------------------------------------------------------------- pre-gate + band build
+    const int gt = threadIdx.x - kWarpGate0 * 32;
+    WorkIter it(w_begin, w_end, p.nT, p.B);
+    Item t;
+    uint32_t kc = 0, xc = 0;
+    int cur_seg = -1;
+    bool over = false;
+    while (it.next(t)) {
+      if (t.seg != cur_seg) {
+        cur_seg = t.seg;
+        const int pa = t.seg & 1, use = t.seg >> 1;
+        if (use > 0 && !warp_wait(&bars[kBarAEmpty + pa], (use - 1) & 1, abort)) break;
+        build_band(a_st + pa * kABytes, p.h + static_cast<size_t>(t.g) * p.l_h, p.l_h, p.halo,
+                   gt, over);
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[kBarAFull + pa]);
+      }
+      const int ks = kc % kNKV, xs = xc % kNX;
+      if (!warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort)) break;
+      if (!warp_wait(&bars[kBarXEmpty + xs], ((xc / kNX) & 1) ^ 1, abort)) break;
+      const uint4 *ksrc = reinterpret_cast<const uint4 *>(kv_st + ks * 2 * kTileBytes);
+      const uint4 *vsrc = reinterpret_cast<const uint4 *>(kv_st + ks * 2 * kTileBytes + kTileBytes);
+      uint4 *xdst = reinterpret_cast<uint4 *>(x_st + xs * kTileBytes);
+#pragma unroll
+      for (int r = 0; r < kTileBytes / 16 / kGroupThreads; ++r) {
+        const int idx = gt + r * kGroupThreads;
+        const uint4 kk = ksrc[idx], vv = vsrc[idx];
+        uint4 o;
+        o.x = gate_pair(kk.x, vv.x, over);
+        o.y = gate_pair(kk.y, vv.y, over);
+        o.z = gate_pair(kk.z, vv.z, over);
+        o.w = gate_pair(kk.w, vv.w, over);
+        xdst[idx] = o;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[kBarKVEmpty + ks]);
+      mbar_arrive(&bars[kBarXFull + xs]);
+      ++kc;
+      ++xc;
+    }
+    if (over) atomicOr(&g_device_status, kF16RangeBit);
+  } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
+    // ---------------------------------------------------------------- epilogue
+    const int et = threadIdx.x - kWarpEpi0 * 32;
+    const int quad = warp & 3;               // TMEM lanes this warp may read
+    const int row_lane = quad * 32 + lane;   // MMA row = TMEM lane
+    const int r = kTM - 1 - row_lane;        // tile row (time offset) of that lane
+    WorkIter it(w_begin, w_end, p.nT, p.B);
+    Item t;
+    uint32_t ac = 0, qc = 0;
+    while (it.next(t)) {
+      if (t.halo) continue;
+      const int as = ac % kNAcc, qs = qc % kNQ;
+      if (!warp_wait(&bars[kBarAccFull + as], (ac / kNAcc) & 1, abort)) break;
+      tc_fence_after_sync();
+      uint32_t a0[32], a1[32];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + as * kNC;
+      tmem_ld_32x32b_x32(taddr, a0);
+      tmem_ld_32x32b_x32(taddr + 32, a1);
+      tmem_wait_ld();
+      reg_fence(a0);
+      reg_fence(a1);
+      tc_fence_before_sync();
+      mbar_arrive(&bars[kBarAccEmpty + as]);
+      if (!warp_wait(&bars[kBarQFull + qs], (qc / kNQ) & 1, abort)) break;
+      uint8_t *qrow = q_st + qs * kTileBytes + r * (kNC * 2);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 *ptr = reinterpret_cast<uint4 *>(qrow + ((c ^ (r & 7)) << 4));
+        const uint4 qv = *ptr;
+        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+        uint32_t ow[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int ch = 8 * c + 2 * e;
+          const float acc0 = __uint_as_float(ch < 32 ? a0[ch] : a1[ch - 32]);
+          const float acc1 = __uint_as_float(ch + 1 < 32 ? a0[ch + 1] : a1[ch + 1 - 32]);
+          const float q0 = __uint_as_float(qw[e] << 16), q1 = __uint_as_float(qw[e] & 0xFFFF0000u);
+          const __nv_bfloat162 yv = __floats2bfloat162_rn(q0 * acc0, q1 * acc1);
+          ow[e] = *reinterpret_cast<const uint32_t *>(&yv);
+        }
+        *ptr = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[kBarYReady + qs]);
+      bool ok = true;
+      if (et == 0) {
+        ok = thread_wait(&bars[kBarYReady + qs], (qc / kNQ) & 1, abort);
+        if (ok) {
+          tma_store_3d(&tm_y, q_st + qs * kTileBytes, t.g * kNC, t.i * kTM, t.b);
+          bulk_commit_group();
+          bulk_wait_group_read<0>();
+          mbar_arrive(&bars[kBarQEmpty + qs]);
+        }
+      }
+      if (!__all_sync(0xffffffffu, ok)) break;
+      ++ac;
+      ++qc;
+    }
+    if (et == 0) bulk_wait_group<0>();
+  }
+
+  __syncthreads();
+  if (warp == kWarpMma) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace tc
+}  // namespace hyena

@@ -1,0 +1,328 @@
+// hyena_conv.cu -- host side of the C ABI declared in include/hyena_conv.h: argument checks,
+// algorithm selection, TMA descriptor encoding and kernel launches.  Every step of the
+// computation runs in the kernels of fir_tc.cuh and fir_cuda_core.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <limits>
+#include <mutex>
+
+#include "hyena_conv.h"
+#include "fir_cuda_core.cuh"
+#include "fir_tc.cuh"
+
+namespace {
+
+using hyena::cc::WindowParams;
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxWindowTaps = 16;
+constexpr int kWindowRows = 32;
+
+struct DeviceState {
+  std::once_flag once;
+  int sm_count = 0;
+  cudaError_t err = cudaSuccess;
+};
+DeviceState g_devices[kMaxDevices];
+
+// Per-device one-time set-up: SM count and the tensor-core kernel's shared-memory opt-in.
+int current_device(DeviceState *&ds) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYENA_ERR_CUDA;
+  ds = &g_devices[dev];
+  DeviceState *d = ds;
+  std::call_once(d->once, [d, dev]() {
+    cudaError_t e = cudaDeviceGetAttribute(&d->sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(hyena::tc::fir_tc_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               hyena::tc::kSmemBytes);
+    d->err = e;
+  });
+  return d->err == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct Problem {
+  const void *q, *k, *v;
+  const float *h;
+  void *y;
+  int64_t B, L, D;
+  int d_g, l_h, l_b, dtype;
+  int64_t elem() const { return dtype == HYENA_DTYPE_F32 ? 4 : 2; }
+  int64_t numel() const { return B * L * D; }
+  int64_t G() const { return D / d_g; }
+};
+
+constexpr int kEmpty = -1;  // internal: valid problem with nothing to compute
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void *a, const void *b, int64_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + static_cast<uintptr_t>(bytes) && y < x + static_cast<uintptr_t>(bytes);
+}
+
+// Host-side checks shared by every forward entry point (no device access).
+int validate(const Problem &P) {
+  if (P.dtype != HYENA_DTYPE_BF16 && P.dtype != HYENA_DTYPE_F32) return HYENA_ERR_INVALID_ARG;
+  if (P.B < 0 || P.L < 0 || P.D < 1 || P.d_g < 1 || P.l_h < 1 || P.l_b < 1)
+    return HYENA_ERR_INVALID_ARG;
+  if (P.D % P.d_g != 0) return HYENA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(P.l_h) > 2 * static_cast<int64_t>(P.l_b)) return HYENA_ERR_INVALID_ARG;
+  if (P.B == 0 || P.L == 0) return kEmpty;
+  const int64_t lim = std::numeric_limits<int64_t>::max() / 8;
+  if (P.B > lim / P.L || P.B * P.L > lim / P.D) return HYENA_ERR_INVALID_ARG;
+  if (!P.q || !P.k || !P.v || !P.h || !P.y) return HYENA_ERR_INVALID_ARG;
+  const uintptr_t es = static_cast<uintptr_t>(P.elem());
+  if (!aligned(P.q, es) || !aligned(P.k, es) || !aligned(P.v, es) || !aligned(P.y, es) ||
+      !aligned(P.h, 4))
+    return HYENA_ERR_MISALIGNED;
+  const int64_t bytes = P.numel() * P.elem();
+  if (overlaps(P.y, P.q, bytes) || overlaps(P.y, P.k, bytes) || overlaps(P.y, P.v, bytes))
+    return HYENA_ERR_INVALID_ARG;
+  return HYENA_OK;
+}
+
+bool all_aligned16(const Problem &P) {
+  return aligned(P.q, 16) && aligned(P.k, 16) && aligned(P.v, 16) && aligned(P.y, 16);
+}
+
+bool tensor_supported(const Problem &P) {
+  const int64_t i32 = std::numeric_limits<int32_t>::max();
+  return P.dtype == HYENA_DTYPE_BF16 && P.d_g == hyena::tc::kNC &&
+         P.l_h - 1 <= hyena::tc::kMaxHalo && all_aligned16(P) && P.L <= i32 && P.B <= i32 &&
+         P.D <= i32;
+}
+
+bool window_supported(const Problem &P) {
+  const int vec = P.dtype == HYENA_DTYPE_F32 ? 4 : 8;
+  return P.l_h <= kMaxWindowTaps && P.d_g % vec == 0 && all_aligned16(P);
+}
+
+int select_algo(const Problem &P) {
+  if (tensor_supported(P)) return HYENA_ALGO_TENSOR;
+  if (window_supported(P)) return HYENA_ALGO_WINDOW;
+  return HYENA_ALGO_DIRECT;
+}
+
+int launch_tensor(const Problem &P, cudaStream_t s) {
+  DeviceState *ds = nullptr;
+  if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return HYENA_ERR_CUDA;
+  CUtensorMap maps[4];
+  const void *ptrs[4] = {P.q, P.k, P.v, P.y};
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.D), static_cast<cuuint64_t>(P.L),
+                              static_cast<cuuint64_t>(P.B)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.D) * 2,
+                                 static_cast<cuuint64_t>(P.L) * static_cast<cuuint64_t>(P.D) * 2};
+  const cuuint32_t box[3] = {hyena::tc::kNC, hyena::tc::kTM, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  for (int i = 0; i < 4; ++i) {
+    if (enc(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptrs[i]), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return HYENA_ERR_CUDA;
+  }
+  hyena::tc::Params p;
+  p.h = P.h;
+  p.B = static_cast<int>(P.B);
+  p.L = static_cast<int>(P.L);
+  p.G = static_cast<int>(P.G());
+  p.l_h = P.l_h;
+  p.halo = ((P.l_h - 1) + 15) / 16 * 16;
+  p.nT = static_cast<int>((P.L + hyena::tc::kTM - 1) / hyena::tc::kTM);
+  p.W = static_cast<long long>(p.G) * p.B * p.nT;
+  const long long grid = p.W < ds->sm_count ? p.W : ds->sm_count;
+  hyena::tc::fir_tc_kernel<<<static_cast<unsigned>(grid), hyena::tc::kThreads,
+                             hyena::tc::kSmemBytes, s>>>(maps[0], maps[1], maps[2], maps[3], p);
+  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+template <typename T, int LH>
+void launch_window_lh(const Problem &P, const WindowParams &wp, unsigned blocks, cudaStream_t s) {
+  hyena::cc::fir_window_kernel<T, LH><<<blocks, 256, 0, s>>>(
+      static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v), P.h,
+      static_cast<T *>(P.y), wp);
+}
+
+template <typename T, int LH = 1>
+void launch_window_dispatch(const Problem &P, const WindowParams &wp, unsigned blocks,
+                            cudaStream_t s) {
+  if constexpr (LH <= kMaxWindowTaps) {
+    if (P.l_h == LH)
+      launch_window_lh<T, LH>(P, wp, blocks, s);
+    else
+      launch_window_dispatch<T, LH + 1>(P, wp, blocks, s);
+  }
+}
+
+int launch_window(const Problem &P, cudaStream_t s) {
+  const int vec = P.dtype == HYENA_DTYPE_F32 ? 4 : 8;
+  WindowParams wp;
+  wp.B = P.B;
+  wp.L = P.L;
+  wp.D = P.D;
+  wp.d_g = P.d_g;
+  wp.rows = kWindowRows;
+  wp.n_tb = (P.L + kWindowRows - 1) / kWindowRows;
+  wp.cv = P.D / vec;
+  const long long threads = wp.B * wp.n_tb * wp.cv;
+  const long long blocks = (threads + 255) / 256;
+  if (blocks > std::numeric_limits<int32_t>::max()) return HYENA_ERR_UNSUPPORTED;
+  if (P.dtype == HYENA_DTYPE_F32)
+    launch_window_dispatch<float>(P, wp, static_cast<unsigned>(blocks), s);
+  else
+    launch_window_dispatch<__nv_bfloat16>(P, wp, static_cast<unsigned>(blocks), s);
+  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+int launch_direct(const Problem &P, cudaStream_t s) {
+  DeviceState *ds = nullptr;
+  if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
+  const long long n = P.numel();
+  long long blocks = (n + 255) / 256;
+  const long long cap = static_cast<long long>(ds->sm_count) * 16;
+  if (blocks > cap) blocks = cap;
+  if (P.dtype == HYENA_DTYPE_F32)
+    hyena::cc::fir_direct_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        static_cast<const float *>(P.q), static_cast<const float *>(P.k),
+        static_cast<const float *>(P.v), P.h, static_cast<float *>(P.y), P.B, P.L, P.D, P.d_g,
+        P.l_h);
+  else
+    hyena::cc::fir_direct_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16 *>(P.q), static_cast<const __nv_bfloat16 *>(P.k),
+        static_cast<const __nv_bfloat16 *>(P.v), P.h, static_cast<__nv_bfloat16 *>(P.y), P.B,
+        P.L, P.D, P.d_g, P.l_h);
+  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+int run(const Problem &P, int algo, cudaStream_t s) {
+  const int rc = validate(P);
+  if (rc == kEmpty) return HYENA_OK;
+  if (rc != HYENA_OK) return rc;
+  switch (algo) {
+    case HYENA_ALGO_AUTO:
+      algo = select_algo(P);
+      break;
+    case HYENA_ALGO_TENSOR:
+      if (!tensor_supported(P)) return HYENA_ERR_UNSUPPORTED;
+      break;
+    case HYENA_ALGO_WINDOW:
+      if (!window_supported(P)) return HYENA_ERR_UNSUPPORTED;
+      break;
+    case HYENA_ALGO_DIRECT:
+      break;
+    default:
+      return HYENA_ERR_INVALID_ARG;
+  }
+  if (algo == HYENA_ALGO_TENSOR) return launch_tensor(P, s);
+  if (algo == HYENA_ALGO_WINDOW) return launch_window(P, s);
+  return launch_direct(P, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int hyena_conv_fwd(const void *q, const void *k, const void *v, const float *h, void *y,
+                   int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                   cudaStream_t stream) {
+  const Problem P{q, k, v, h, y, B, L, D, d_g, l_h, l_b, HYENA_DTYPE_BF16};
+  return run(P, HYENA_ALGO_AUTO, stream);
+}
+
+int hyena_conv_fwd_f32(const float *q, const float *k, const float *v, const float *h, float *y,
+                       int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                       cudaStream_t stream) {
+  const Problem P{q, k, v, h, y, B, L, D, d_g, l_h, l_b, HYENA_DTYPE_F32};
+  return run(P, HYENA_ALGO_AUTO, stream);
+}
+
+int hyena_conv_fwd_ex(const void *q, const void *k, const void *v, const float *h, void *y,
+                      int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b, int dtype,
+                      int algo, cudaStream_t stream) {
+  const Problem P{q, k, v, h, y, B, L, D, d_g, l_h, l_b, dtype};
+  return run(P, algo, stream);
+}
+
+int hyena_select_algo(const void *q, const void *k, const void *v, const float *h, const void *y,
+                      int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b, int dtype) {
+  const Problem P{q, k, v, h, const_cast<void *>(y), B, L, D, d_g, l_h, l_b, dtype};
+  const int rc = validate(P);
+  if (rc != HYENA_OK && rc != kEmpty) return -rc;
+  return select_algo(P);
+}
+
+int hyena_build_toeplitz(const float *h, float *H0, float *H1, float *H2_or_null, int G,
+                         int l_h, int l_b, cudaStream_t stream) {
+  if (!h || !H0 || !H1 || G < 1 || l_h < 1 || l_b < 1) return HYENA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(l_h) > 2 * static_cast<int64_t>(l_b)) return HYENA_ERR_INVALID_ARG;
+  if (l_h >= l_b + 2 && !H2_or_null) return HYENA_ERR_INVALID_ARG;
+  if (!aligned(h, 4) || !aligned(H0, 4) || !aligned(H1, 4) || !aligned(H2_or_null, 4))
+    return HYENA_ERR_MISALIGNED;
+  DeviceState *ds = nullptr;
+  if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
+  const long long n = static_cast<long long>(G) * l_b * l_b;
+  long long blocks = (n + 255) / 256;
+  const long long cap = static_cast<long long>(ds->sm_count) * 8;
+  if (blocks > cap) blocks = cap;
+  hyena::cc::toeplitz_blocks_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      h, H0, H1, H2_or_null, G, l_h, l_b);
+  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+int hyena_device_status(unsigned int *out, int clear) {
+  if (!out) return HYENA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return HYENA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(out, hyena::g_device_status, sizeof(unsigned int)) != cudaSuccess)
+    return HYENA_ERR_CUDA;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(hyena::g_device_status, &zero, sizeof(unsigned int)) != cudaSuccess)
+      return HYENA_ERR_CUDA;
+  }
+  return HYENA_OK;
+}
+
+const char *hyena_status_string(int status) {
+  switch (status) {
+    case HYENA_OK:
+      return "ok";
+    case HYENA_ERR_INVALID_ARG:
+      return "invalid argument";
+    case HYENA_ERR_UNSUPPORTED:
+      return "unsupported shape or alignment for the requested algorithm";
+    case HYENA_ERR_MISALIGNED:
+      return "pointer not aligned to its element size";
+    case HYENA_ERR_CUDA:
+      return "CUDA runtime error";
+    default:
+      return "unknown status";
+  }
+}
+
+int hyena_abi_version(void) { return 1; }
+
+}  // extern "C"

@@ -1,0 +1,133 @@
+/*
+ * hyena_conv.h -- C ABI of the B200 (sm_100a) gated, grouped, depthwise causal FIR.
+ *
+ * Operation (Hyena-SE / Hyena-MR operators of StripedHyena 2; the convolution is the causal FIR
+ * sum of the page "04. Hardware-aware convolution kernels", Sec. 1, gated by q and by k):
+ *
+ *     y[b,t,c] = q[b,t,c] * sum_{j=0}^{min(l_h-1, t)} h[c / d_g][j] * k[b,t-j,c] * v[b,t-j,c]
+ *
+ * computed with the block-Toeplitz method of the same page (Sec. 2 block convolution, Sec. 3
+ * two-stage form Yhat_n = H0 Xhat_n + H1 Xhat_{n-1}, Xhat_{-1} = 0).
+ *
+ * Conventions shared by every entry point:
+ *   - q, k, v, y are DEVICE pointers to [B, L, D] row-major tensors (channels contiguous).
+ *   - h is a DEVICE pointer to fp32 [D / d_g, l_h], natural tap order: h[g][0] multiplies the
+ *     current token.  Channel c belongs to group c / d_g (contiguous groups).
+ *   - Every sequence b starts from zero history; no state is kept between calls.
+ *   - The caller owns every buffer.  The library allocates no device memory in these calls.
+ *     Each call is asynchronous on `stream` (NULL = the legacy default stream) and returns as
+ *     soon as the work is queued.
+ *   - y must not overlap q, k or v.
+ *   - B == 0 or L == 0 is an empty problem: nothing is launched and HYENA_OK is returned.
+ *   - Return value: HYENA_OK or one of the HYENA_ERR_* codes below.  Argument errors are
+ *     detected on the host before anything is queued.  HYENA_ERR_CUDA reports a launch
+ *     failure (cudaGetLastError).  Errors that happen inside a running kernel (a bounded wait
+ *     that ran out, fp16 operand overflow) are recorded in a per-device status word that
+ *     hyena_device_status() reads.
+ */
+#ifndef HYENA_CONV_H
+#define HYENA_CONV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t (an opaque driver stream handle). */
+typedef struct CUstream_st *cudaStream_t;
+
+enum hyena_status {
+    HYENA_OK = 0,
+    HYENA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, D % d_g != 0, l_h < 1,
+                                    l_b < 1, l_h > 2*l_b, overlapping y, unknown dtype/algo */
+    HYENA_ERR_UNSUPPORTED = 2,   /* a forced algorithm cannot run this shape or alignment */
+    HYENA_ERR_MISALIGNED = 3,    /* a pointer is not aligned to its element size */
+    HYENA_ERR_CUDA = 4           /* the CUDA runtime reported an error for this call */
+};
+
+enum hyena_dtype {
+    HYENA_DTYPE_BF16 = 0,        /* q, k, v, y bf16; fp32 accumulation */
+    HYENA_DTYPE_F32 = 1          /* q, k, v, y fp32; fp32 accumulation */
+};
+
+enum hyena_algo {
+    HYENA_ALGO_AUTO = 0,         /* pick the fastest algorithm that supports the problem */
+    HYENA_ALGO_TENSOR = 1,       /* tcgen05 tensor-core block-Toeplitz GEMM (bf16 only;
+                                    d_g == 64, l_h <= 129, 16-byte aligned tensors) */
+    HYENA_ALGO_WINDOW = 2,       /* CUDA-core register sliding window (l_h <= 16,
+                                    d_g and D multiples of 16 bytes of channels) */
+    HYENA_ALGO_DIRECT = 3        /* CUDA-core direct sum; any supported shape */
+};
+
+/* Bits of the per-device status word (hyena_device_status). */
+enum hyena_device_status_bits {
+    HYENA_DEVICE_TIMEOUT = 1u,      /* a bounded wait inside a kernel gave up; output invalid */
+    HYENA_DEVICE_F16_RANGE = 2u     /* |k*v| or |h| exceeded the fp16 operand range (65504)
+                                       in the tensor-core path; affected outputs are inf/nan */
+};
+
+/*
+ * Gated grouped causal FIR forward, bf16 q/k/v/y (the Hyena-SE / Hyena-MR operator).
+ * l_b is the block size of the block-Toeplitz decomposition.  The result is the same for every
+ * l_b (the decomposition is exact); l_b only bounds the filter length, l_h <= 2*l_b, which is
+ * the domain the two-stage method is stated for.  All tensors 2-byte aligned.
+ */
+int hyena_conv_fwd(const void *q, const void *k, const void *v, const float *h, void *y,
+                   int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                   cudaStream_t stream);
+
+/* The same operation with fp32 q/k/v/y (4-byte aligned). */
+int hyena_conv_fwd_f32(const float *q, const float *k, const float *v, const float *h,
+                       float *y, int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                       cudaStream_t stream);
+
+/*
+ * The same operation with the element type (enum hyena_dtype) and the algorithm
+ * (enum hyena_algo) chosen by the caller.  A forced algorithm that cannot run the problem
+ * returns HYENA_ERR_UNSUPPORTED without queuing anything.
+ */
+int hyena_conv_fwd_ex(const void *q, const void *k, const void *v, const float *h, void *y,
+                      int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                      int dtype, int algo, cudaStream_t stream);
+
+/*
+ * Host-only: the algorithm (enum hyena_algo, > 0) that HYENA_ALGO_AUTO would run for this
+ * problem and these pointers, or minus an error code.  Touches no device.
+ */
+int hyena_select_algo(const void *q, const void *k, const void *v, const float *h,
+                      const void *y, int64_t B, int64_t L, int64_t D, int d_g, int l_h,
+                      int l_b, int dtype);
+
+/*
+ * The l_b x l_b sub-blocks of the lower-triangular Toeplitz matrix of every group
+ * (page 04, Sec. 2; index rule of the Sec. 3 worked example):
+ *     H_m[g][i][j] = h[g][m*l_b + i - j]  if 0 <= m*l_b + i - j < l_h,  else 0,
+ * written for m = 0 (H0), 1 (H1) and 2 (H2) as fp32 [G, l_b, l_b] device arrays.  H2 is the
+ * third diagonal that filters with l_h >= l_b + 2 reach; it may be NULL only when
+ * l_h <= l_b + 1, where it is all zero.  The forward kernels build their own operand tiles
+ * on chip; this entry point exposes the decomposition for inspection and testing.
+ * Errors: HYENA_ERR_INVALID_ARG for null h/H0/H1, G < 1, l_h < 1, l_b < 1, l_h > 2*l_b, or
+ * H2 == NULL when l_h >= l_b + 2.
+ */
+int hyena_build_toeplitz(const float *h, float *H0, float *H1, float *H2_or_null, int G,
+                         int l_h, int l_b, cudaStream_t stream);
+
+/*
+ * Reads (and, if clear != 0, resets) the status word of the current device: an OR of
+ * enum hyena_device_status_bits raised by kernels since the last reset.  Synchronises the
+ * current device.  Returns HYENA_OK or HYENA_ERR_CUDA; *out receives the word.
+ */
+int hyena_device_status(unsigned int *out, int clear);
+
+/* Static description of a status code; never NULL. */
+const char *hyena_status_string(int status);
+
+/* ABI version of this header (incremented on incompatible change). */
+int hyena_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYENA_CONV_H */

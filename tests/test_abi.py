@@ -1,0 +1,110 @@
+"""The C ABI on a host without a GPU: the library builds and loads, exports every function
+include/hyena_conv.h declares, and rejects bad arguments on the host before touching a device.
+No call here reaches a kernel launch."""
+import ctypes
+import shutil
+
+import pytest
+
+import gated_causal_fir_b200 as g
+from gated_causal_fir_b200 import _native, build
+
+pytestmark = pytest.mark.skipif(
+    shutil.which("nvcc") is None and not __import__("os").path.exists(_native.LIB_PATH),
+    reason="needs nvcc or a built library")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _native.lib()
+
+
+def test_exports_every_header_function(lib):
+    declared = _native.header_functions()
+    assert len(declared) >= 8
+    assert set(declared) == set(_native.SIGNATURES), "binding table out of step with the header"
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    assert g.hyena_abi_version() == 1
+    assert g.hyena_status_string(0) == "ok"
+    for code in (1, 2, 3, 4):
+        assert g.hyena_status_string(code) not in ("ok", "unknown status")
+    assert g.hyena_status_string(99) == "unknown status"
+
+
+def test_select_algo_for_the_workloads(lib):
+    from gated_causal_fir_b200.workloads import WORKLOADS
+    want = {"tiny": g.HYENA_ALGO_WINDOW, "se": g.HYENA_ALGO_WINDOW, "mr": g.HYENA_ALGO_TENSOR,
+            "mr_batched": g.HYENA_ALGO_TENSOR, "mr_1m": g.HYENA_ALGO_TENSOR}
+    for name, wl in WORKLOADS.items():
+        dt = g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16
+        assert g.hyena_select_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, dt) == want[name]
+
+
+def test_select_algo_fallbacks(lib):
+    bf, f32 = g.HYENA_DTYPE_BF16, g.HYENA_DTYPE_F32
+    assert g.hyena_select_algo(1, 100, 256, 64, 130, 65, bf) == g.HYENA_ALGO_DIRECT  # l_h > 129
+    assert g.hyena_select_algo(1, 100, 256, 64, 129, 65, bf) == g.HYENA_ALGO_TENSOR
+    assert g.hyena_select_algo(1, 100, 96, 32, 40, 32, bf) == g.HYENA_ALGO_DIRECT   # d_g != 64
+    assert g.hyena_select_algo(1, 100, 96, 32, 16, 32, bf) == g.HYENA_ALGO_WINDOW
+    assert g.hyena_select_algo(1, 100, 96, 4, 3, 2, bf) == g.HYENA_ALGO_DIRECT      # 4 ch < 16 B
+    assert g.hyena_select_algo(1, 100, 96, 4, 3, 2, f32) == g.HYENA_ALGO_WINDOW
+    assert g.hyena_select_algo(1, 64, 128, 64, 128, 64, f32) == g.HYENA_ALGO_DIRECT
+    n = 64 * 128 * 2
+    odd = (16 + 2, 16 + n + 64, 16 + 2 * (n + 64), 16 + 3 * (n + 64), 16 + 4 * (n + 64))
+    assert g.hyena_select_algo(1, 64, 128, 64, 128, 64, bf, ptrs=odd) == g.HYENA_ALGO_DIRECT
+
+
+BASE = dict(B=1, L=64, D=128, d_g=64, l_h=16, l_b=16)
+
+
+def _call(lib, q=0x10000, k=0x20000, v=0x30000, h=0x40000, y=0x50000, dtype=0, algo=0, **kw):
+    a = dict(BASE, **kw)
+    return lib.hyena_conv_fwd_ex(q, k, v, h, y, a["B"], a["L"], a["D"], a["d_g"], a["l_h"],
+                                 a["l_b"], dtype, algo, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(k=None), 1), (dict(v=None), 1), (dict(h=None), 1), (dict(y=None), 1),
+    (dict(B=-1), 1), (dict(L=-5), 1), (dict(D=0), 1), (dict(d_g=0), 1), (dict(d_g=48), 1),
+    (dict(l_h=0), 1), (dict(l_b=0), 1), (dict(l_h=33, l_b=16), 1), (dict(dtype=7), 1),
+    (dict(algo=9), 1), (dict(y=0x10000 + 64), 1), (dict(q=0x10001), 3), (dict(h=0x40002), 3),
+    (dict(algo=1, dtype=1), 2), (dict(algo=1, d_g=32), 2), (dict(algo=2, l_h=17, l_b=16), 2),
+    (dict(algo=1, q=0x10002), 2),
+])
+def test_host_validation(lib, kw, code):
+    assert _call(lib, **kw) == code
+
+
+def test_empty_problem_is_ok_without_launch(lib):
+    assert _call(lib, B=0) == 0
+    assert _call(lib, L=0, q=None, k=None, v=None, y=None) == 0
+
+
+def test_size_overflow_rejected(lib):
+    assert _call(lib, B=1 << 40, L=1 << 20, D=1 << 12) == 1
+
+
+def test_toeplitz_validation(lib):
+    f = lib.hyena_build_toeplitz
+    assert f(None, 0x2000, 0x3000, 0x4000, 4, 4, 3, None) == 1
+    assert f(0x1000, 0x2000, 0x3000, None, 4, 5, 3, None) == 1  # l_h >= l_b + 2 needs H2
+    assert f(0x1000, 0x2000, 0x3000, 0x4000, 4, 9, 4, None) == 1  # l_h > 2 l_b
+    assert f(0x1000, 0x2000, 0x3000, 0x4000, 0, 4, 3, None) == 1
+    assert f(0x1001, 0x2000, 0x3000, 0x4000, 4, 4, 3, None) == 3
+
+
+def test_device_status_needs_out(lib):
+    assert lib.hyena_device_status(None, 0) == 1
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
+    h = torch.zeros(1, 4)
+    with pytest.raises(TypeError):
+        g.hyena_conv_fwd(q, q, q, h, d_g=64, l_b=4)
