@@ -23,8 +23,8 @@
 //    128 x 256 band lives in 47 core matrices (6 KB) instead of 64 KB.
 //  * Accumulators live in TMEM (2 x 64 columns); the epilogue reads them with tcgen05.ld,
 //    multiplies by q and rounds to bf16 in registers, and writes y over the q tile in place.
-//  * Warp roles: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2-5 pre-gate / operand build,
-//    6-9 epilogue.  Persistent grid: one CTA per SM, each walks a contiguous range of tiles
+//  * Warp roles: 0 TMA producer of k and v, 10 TMA producer of q, 1 MMA issuer (+ TMEM
+//    owner), 2-5 pre-gate / operand build, 6-9 epilogue.  Persistent grid: one CTA per SM, each walks a contiguous range of tiles
 //    ordered (group, batch, time), so a halo tile is re-read only where a range starts inside
 //    a sequence.
 //  * Every wait is bounded (ptx.cuh); a timeout raises HYENA_DEVICE_TIMEOUT, all roles leave
@@ -43,14 +43,32 @@ namespace tc {
 constexpr int kTM = 128;             // output rows per tile (MMA M)
 constexpr int kNC = 64;              // channels per tile = d_g (MMA N)
 constexpr int kMaxHalo = 128;        // supports l_h - 1 <= 128
-constexpr int kNKV = 4;              // k/v stages
-constexpr int kNQ = 2;               // q (and in-place y) stages
+#ifndef HYENA_TC_KV_STAGES
+#define HYENA_TC_KV_STAGES 3
+#endif
+#ifndef HYENA_TC_Q_STAGES
+#define HYENA_TC_Q_STAGES 3
+#endif
+constexpr int kNKV = HYENA_TC_KV_STAGES;  // k/v stages
+constexpr int kNQ = HYENA_TC_Q_STAGES;    // q (and in-place y) stages
 constexpr int kNX = 3;               // fp16 X slots (current, previous, next)
-constexpr int kNAcc = 2;             // TMEM accumulators
-constexpr int kTileBytes = kTM * kNC * 2;                       // 16 KB
+constexpr int kNAcc = 2;             // TMEM accumulator sets (tiles in flight)
+#ifndef HYENA_TC_KSPLIT
+#define HYENA_TC_KSPLIT 1
+#endif
+// Independent partial accumulators per tile: k-step n of a tile accumulates into partial
+// n % kKSplit, so consecutive MMAs do not wait on each other's accumulator; the epilogue sums
+// the partials in fp32.
+constexpr int kKSplit = HYENA_TC_KSPLIT;
+constexpr int kRowBytes = kNC * 2;                              // 128 B
+constexpr int kTileBytes = kTM * kRowBytes;                     // 16 KB
+constexpr int kKBlockBytes = kNC * 128;                         // 64 times x 64 channels
 constexpr int kACores = kTM / 8 + (kTM + kMaxHalo) / 8 - 1;     // 47
 constexpr int kABytes = 48 * 128;                               // padded
-constexpr int kTmemCols = kNAcc * kNC;                          // 128
+constexpr int kTmemCols = kNAcc * kKSplit * kNC;                // 512 at kKSplit = 4
+static_assert(kTmemCols == 32 || kTmemCols == 64 || kTmemCols == 128 || kTmemCols == 256 ||
+                  kTmemCols == 512,
+              "TMEM allocation must be a power of two between 32 and 512 columns");
 
 constexpr int kOffKV = 0;
 constexpr int kOffQ = kOffKV + kNKV * 2 * kTileBytes;
@@ -73,9 +91,10 @@ constexpr int kBarDone = kBarAEmpty + 2;
 constexpr int kNumBars = kBarDone + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget of one CTA exceeded");
 
-constexpr int kThreads = 320;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGate0 = 2, kWarpEpi0 = 6;
+constexpr int kThreads = 352;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGate0 = 2, kWarpEpi0 = 6, kWarpTmaQ = 10;
 constexpr int kGroupThreads = 128;
 
 constexpr unsigned kTimeoutBit = 1u;  // HYENA_DEVICE_TIMEOUT
@@ -86,7 +105,11 @@ struct Params {
   int B, L, G, l_h;
   int halo;         // multiple of 16, >= l_h - 1, <= kMaxHalo
   int nT;           // tiles per sequence = ceil(L / kTM)
-  long long W;      // total tiles = G * B * nT
+  long long W;      // tiles of the walk: G * B * nT, or (G / 2) * B * nT when paired
+  int paired;       // CTAs 2p and 2p+1 walk the same (group pair, batch, time) range, one
+                    // group each, so both halves of every 256-byte row are read together
+  int run;          // > 0: strided schedule of runs of `run` tiles (see RunIter)
+  long long units;  // number of runs: B * ceil(nT / run) * G
 };
 
 // One unit of a CTA's walk: a halo tile (input only) or an output tile.
@@ -100,15 +123,18 @@ struct Item {
 
 struct WorkIter {
   long long w, w_begin, w_end;
-  int nT, B, seg;
+  int nT, B, seg, gmul, goff;
   bool entered;
-  __device__ WorkIter(long long b, long long e, int nT_, int B_)
-      : w(b), w_begin(b), w_end(e), nT(nT_), B(B_), seg(-1), entered(false) {}
+  // Tiles [b, e) of the walk ordered (group, batch, time); with gmul = 2 the walk is over
+  // group pairs and this CTA takes group 2 * pair + goff.
+  __device__ WorkIter(long long b, long long e, int nT_, int B_, int gmul_ = 1, int goff_ = 0)
+      : w(b), w_begin(b), w_end(e), nT(nT_), B(B_), seg(-1), gmul(gmul_), goff(goff_),
+        entered(false) {}
   __device__ bool next(Item &it) {
     if (w >= w_end) return false;
     const long long seq = w / nT;
     const int i = static_cast<int>(w - seq * nT);
-    it.g = static_cast<int>(seq / B);
+    it.g = static_cast<int>(seq / B) * gmul + goff;
     it.b = static_cast<int>(seq % B);
     const bool first = (w == w_begin) || (i == 0);
     if (first && !entered) {
@@ -132,6 +158,73 @@ struct WorkIter {
     entered = false;
     return true;
   }
+};
+
+// Strided schedule: the work is cut into runs of `run` consecutive tiles of one (group, batch)
+// sequence, numbered with the group fastest, then the run's time block, then the batch; CTA c
+// takes runs c, c + grid, c + 2 grid, ...  At any moment the CTAs hold neighbouring groups of
+// the same time rows, so together they read whole rows of [B, L, D] (DRAM page locality),
+// and the halo tile a run starts with was usually loaded into L2 moments earlier.
+struct RunIter {
+  long long u, ustep, units;
+  int nT, B, G, run, nblk, seg, i, iend;
+  bool in_run;
+  __device__ RunIter(long long first, long long step, long long n, int nT_, int B_, int G_, int r)
+      : u(first), ustep(step), units(n), nT(nT_), B(B_), G(G_), run(r),
+        nblk((nT_ + r - 1) / r), seg(-1), i(0), iend(0), in_run(false) {}
+  __device__ bool next(Item &it) {
+    if (!in_run) {
+      if (u >= units) return false;
+      const int g = static_cast<int>(u % G);
+      const long long rest = u / G;
+      const int blk = static_cast<int>(rest % nblk);
+      b_ = static_cast<int>(rest / nblk);
+      g_ = g;
+      i = blk * run;
+      iend = min(nT, i + run);
+      ++seg;
+      in_run = true;
+      if (i > 0) {
+        it.g = g_;
+        it.b = b_;
+        it.i = i - 1;
+        it.seg = seg;
+        it.halo = true;
+        it.hist = false;
+        it.last = false;
+        return true;
+      }
+    }
+    it.g = g_;
+    it.b = b_;
+    it.i = i;
+    it.seg = seg;
+    it.halo = false;
+    it.hist = i > 0;
+    it.last = i + 1 == iend;
+    if (++i == iend) {
+      in_run = false;
+      u += ustep;
+    }
+    return true;
+  }
+  int g_ = 0, b_ = 0;
+};
+
+// The walk of this CTA: contiguous tile ranges (kStrided = false) or strided runs.
+template <bool kStrided>
+struct Walk;
+
+template <>
+struct Walk<false> : WorkIter {
+  __device__ Walk(const Params &p, long long w_begin, long long w_end, int gmul, int goff)
+      : WorkIter(w_begin, w_end, p.nT, p.B, gmul, goff) {}
+};
+
+template <>
+struct Walk<true> : RunIter {
+  __device__ Walk(const Params &p, long long, long long, int, int)
+      : RunIter(blockIdx.x, gridDim.x, p.units, p.nT, p.B, p.G, p.run) {}
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
@@ -174,6 +267,7 @@ __device__ __forceinline__ void build_band(uint8_t *a, const float *hg, int l_h,
   }
 }
 
+template <bool kStrided>
 __global__ void __launch_bounds__(kThreads, 1)
     fir_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
@@ -190,8 +284,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long per = p.W / gridDim.x, rem = p.W % gridDim.x;
-  const long long bx = blockIdx.x;
+  const long long nwalk = p.paired ? gridDim.x / 2 : gridDim.x;
+  const long long bx = p.paired ? blockIdx.x / 2 : blockIdx.x;
+  const int gmul = p.paired ? 2 : 1, goff = p.paired ? static_cast<int>(blockIdx.x & 1) : 0;
+  const long long per = p.W / nwalk, rem = p.W % nwalk;
   const long long w_begin = bx * per + (bx < rem ? bx : rem);
   const long long w_end = w_begin + per + (bx < rem ? 1 : 0);
 
@@ -237,11 +333,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == kWarpTma) {
-    // ---------------------------------------------------------------- TMA producer
+    // ---------------------------------------------------------------- TMA producer: k, v
     if (lane == 0) {
-      WorkIter it(w_begin, w_end, p.nT, p.B);
+      Walk<kStrided> it(p, w_begin, w_end, gmul, goff);
       Item t;
-      uint32_t kc = 0, qc = 0;
+      uint32_t kc = 0;
       while (it.next(t)) {
         const int ks = kc % kNKV;
         if (!thread_wait(&bars[kBarKVEmpty + ks], ((kc / kNKV) & 1) ^ 1, abort)) break;
@@ -250,30 +346,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(dst, &tm_k, &bars[kBarKVFull + ks], t.g * kNC, t.i * kTM, t.b);
         tma_load_3d(dst + kTileBytes, &tm_v, &bars[kBarKVFull + ks], t.g * kNC, t.i * kTM, t.b);
         ++kc;
-        if (!t.halo) {
-          const int qs = qc % kNQ;
-          if (!thread_wait(&bars[kBarQEmpty + qs], ((qc / kNQ) & 1) ^ 1, abort)) break;
-          mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes);
-          tma_load_3d(q_st + qs * kTileBytes, &tm_q, &bars[kBarQFull + qs], t.g * kNC, t.i * kTM,
-                      t.b);
-          ++qc;
-        }
       }
       // Every load this thread issued must land before the CTA may exit.
       for (uint32_t n = kc > kNKV ? kc - kNKV : 0; n < kc; ++n)
         drain_wait(&bars[kBarKVFull + n % kNKV], (n / kNKV) & 1);
+    }
+  } else if (warp == kWarpTmaQ) {
+    // ---------------------------------------------------------------- TMA producer: q
+    if (lane == 0) {
+      Walk<kStrided> it(p, w_begin, w_end, gmul, goff);
+      Item t;
+      uint32_t qc = 0;
+      while (it.next(t)) {
+        if (t.halo) continue;
+        const int qs = qc % kNQ;
+        if (!thread_wait(&bars[kBarQEmpty + qs], ((qc / kNQ) & 1) ^ 1, abort)) break;
+        mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes);
+        tma_load_3d(q_st + qs * kTileBytes, &tm_q, &bars[kBarQFull + qs], t.g * kNC, t.i * kTM,
+                    t.b);
+        ++qc;
+      }
       for (uint32_t n = qc > kNQ ? qc - kNQ : 0; n < qc; ++n)
         drain_wait(&bars[kBarQFull + n % kNQ], (n / kNQ) & 1);
     }
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      WorkIter it(w_begin, w_end, p.nT, p.B);
+      Walk<kStrided> it(p, w_begin, w_end, gmul, goff);
       Item t;
       uint32_t xc = 0, ac = 0;
       int cur_seg = -1;
-      const uint32_t idesc = umma_idesc_f16_f32(kTM, kNC, 1);
-      const int ksteps = (kTM + p.halo) / 16, hsteps = p.halo / 16;
+      const uint32_t idesc = umma_idesc_f16_f32(kTM, kNC, 0);  // B K-major
+      const int hsteps = p.halo / 16;
       while (it.next(t)) {
         const int xs = xc % kNX;
         if (!thread_wait(&bars[kBarXFull + xs], (xc / kNX) & 1, abort)) break;
@@ -289,24 +393,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int as = ac % kNAcc;
         if (!thread_wait(&bars[kBarAccEmpty + as], ((ac / kNAcc) & 1) ^ 1, abort)) break;
         tc_fence_after_sync();
-        const uint32_t a_base = smem_u32(a_st + pa * kABytes);
+        // Descriptors advance by plain adds: 16 rows of X = 2048 B = 128 units of 16 B per
+        // k-step, 2 core matrices of the band = 256 B = 16 units (no carry out of the 14-bit
+        // start-address field: every address stays inside shared memory).
         const int xp = (xc + kNX - 1) % kNX;
-        const uint32_t x_cur = smem_u32(x_st + xs * kTileBytes);
-        const uint32_t x_prev = smem_u32(x_st + xp * kTileBytes);
-        const uint32_t d_tmem = tmem_base + as * kNC;
-        uint32_t accumulate = 0;
-        for (int j = 0; j < ksteps; ++j) {
-          uint32_t b_addr;
-          if (j < hsteps) {
-            if (!t.hist) continue;  // zero history before the first tile of a sequence
-            b_addr = x_prev + (kTM - p.halo + 16 * j) * (kNC * 2);
-          } else {
-            b_addr = x_cur + (16 * j - p.halo) * (kNC * 2);
+        const uint32_t d_tmem = tmem_base + as * kKSplit * kNC;
+        uint64_t ad = umma_smem_desc(smem_u32(a_st + pa * kABytes), 128, 128, 0);
+        // B = X^T, K-major with 128-byte swizzle: k-step s of a slot starts at K-block s / 4
+        // (8 KB each) plus 32 bytes per step inside the 128-byte rows.
+        int issued = 0;
+        if (t.hist) {
+          const uint64_t bd0 = umma_smem_desc(smem_u32(x_st + xp * kTileBytes), 16, 1024, 2);
+          const int s0 = (kTM - p.halo) / 16;
+          for (int j = 0; j < hsteps; ++j) {
+            const int st = s0 + j;
+            const uint64_t bd = bd0 + ((st >> 2) * (kKBlockBytes >> 4) + (st & 3) * 2);
+            umma_f16(d_tmem + (issued % kKSplit) * kNC, ad, bd, idesc, issued >= kKSplit);
+            ++issued;
+            ad += 16;
           }
-          const uint64_t adesc = umma_smem_desc(a_base + j * 256, 128, 128, 0);
-          const uint64_t bdesc = umma_smem_desc(b_addr, kTileBytes, 1024, 2);
-          umma_f16(d_tmem, adesc, bdesc, idesc, accumulate);
-          accumulate = 1;
+        } else {
+          ad += 16 * hsteps;  // zero history before the first tile of a sequence
+        }
+        {
+          const uint64_t bd0 = umma_smem_desc(smem_u32(x_st + xs * kTileBytes), 16, 1024, 2);
+#pragma unroll
+          for (int st = 0; st < kTM / 16; ++st) {
+            const uint64_t bd = bd0 + ((st >> 2) * (kKBlockBytes >> 4) + (st & 3) * 2);
+            umma_f16(d_tmem + (issued % kKSplit) * kNC, ad, bd, idesc, issued >= kKSplit);
+            ++issued;
+            ad += 16;
+          }
         }
         umma_commit(&bars[kBarAccFull + as]);
         if (t.hist) umma_commit(&bars[kBarXEmpty + xp]);
@@ -324,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kWarpGate0 && warp < kWarpGate0 + 4) {
     // ---------------------------------------------------------------- pre-gate + band build
     const int gt = threadIdx.x - kWarpGate0 * 32;
-    WorkIter it(w_begin, w_end, p.nT, p.B);
+    Walk<kStrided> it(p, w_begin, w_end, gmul, goff);
     Item t;
     uint32_t kc = 0, xc = 0;
     int cur_seg = -1;
@@ -342,19 +459,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ks = kc % kNKV, xs = xc % kNX;
       if (!warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort)) break;
       if (!warp_wait(&bars[kBarXEmpty + xs], ((xc / kNX) & 1) ^ 1, abort)) break;
-      const uint4 *ksrc = reinterpret_cast<const uint4 *>(kv_st + ks * 2 * kTileBytes);
-      const uint4 *vsrc = reinterpret_cast<const uint4 *>(kv_st + ks * 2 * kTileBytes + kTileBytes);
-      uint4 *xdst = reinterpret_cast<uint4 *>(x_st + xs * kTileBytes);
+      // X^T (channel rows, 64 times per 128-byte row, two 8 KB K-blocks per tile, 128-byte
+      // swizzle) from the time-major k and v tiles: each warp moves 8 x 8 blocks with ldmatrix,
+      // forms k*v in fp32, rounds to fp16 and stores the blocks transposed with stmatrix.
+      const uint32_t kbase = smem_u32(kv_st + ks * 2 * kTileBytes);
+      const uint32_t vbase = kbase + kTileBytes;
+      const uint32_t xbase = smem_u32(x_st + xs * kTileBytes);
+      const int gw = warp - kWarpGate0, mat = lane >> 3, rr = lane & 7;
 #pragma unroll
-      for (int r = 0; r < kTileBytes / 16 / kGroupThreads; ++r) {
-        const int idx = gt + r * kGroupThreads;
-        const uint4 kk = ksrc[idx], vv = vsrc[idx];
-        uint4 o;
-        o.x = gate_pair(kk.x, vv.x, over);
-        o.y = gate_pair(kk.y, vv.y, over);
-        o.z = gate_pair(kk.z, vv.z, over);
-        o.w = gate_pair(kk.w, vv.w, over);
-        xdst[idx] = o;
+      for (int it = 0; it < 8; ++it) {
+        const int bw = it * 4 + mat;
+        const int tg = gw * 4 + (bw >> 3), cg = bw & 7;  // 8-time group, 8-channel group
+        const uint32_t src = (tg * 8 + rr) * kRowBytes + ((cg ^ rr) << 4);
+        uint32_t kf[4], vf[4], xf[4];
+        ldsm_x4(kbase + src, kf);
+        ldsm_x4(vbase + src, vf);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) xf[e] = gate_pair(kf[e], vf[e], over);
+        const int c = cg * 8 + rr;
+        const uint32_t dst = (tg >> 3) * kKBlockBytes + c * kRowBytes + (((tg & 7) ^ rr) << 4);
+        stsm_x4_trans(xbase + dst, xf);
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[kBarKVEmpty + ks]);
@@ -369,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;               // TMEM lanes this warp may read
     const int row_lane = quad * 32 + lane;   // MMA row = TMEM lane
     const int r = kTM - 1 - row_lane;        // tile row (time offset) of that lane
-    WorkIter it(w_begin, w_end, p.nT, p.B);
+    Walk<kStrided> it(p, w_begin, w_end, gmul, goff);
     Item t;
     uint32_t ac = 0, qc = 0;
     while (it.next(t)) {
@@ -378,12 +502,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&bars[kBarAccFull + as], (ac / kNAcc) & 1, abort)) break;
       tc_fence_after_sync();
       uint32_t a0[32], a1[32];
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + as * kNC;
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + as * kKSplit * kNC;
       tmem_ld_32x32b_x32(taddr, a0);
       tmem_ld_32x32b_x32(taddr + 32, a1);
       tmem_wait_ld();
       reg_fence(a0);
       reg_fence(a1);
+#pragma unroll 1
+      for (int part = 1; part < kKSplit; ++part) {
+        uint32_t b0[32], b1[32];
+        tmem_ld_32x32b_x32(taddr + part * kNC, b0);
+        tmem_ld_32x32b_x32(taddr + part * kNC + 32, b1);
+        tmem_wait_ld();
+        reg_fence(b0);
+        reg_fence(b1);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          a0[c] = __float_as_uint(__uint_as_float(a0[c]) + __uint_as_float(b0[c]));
+          a1[c] = __float_as_uint(__uint_as_float(a1[c]) + __uint_as_float(b1[c]));
+        }
+      }
       tc_fence_before_sync();
       mbar_arrive(&bars[kBarAccEmpty + as]);
       if (!warp_wait(&bars[kBarQFull + qs], (qc / kNQ) & 1, abort)) break;
@@ -413,15 +552,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
           tma_store_3d(&tm_y, q_st + qs * kTileBytes, t.g * kNC, t.i * kTM, t.b);
           bulk_commit_group();
-          bulk_wait_group_read<0>();
-          mbar_arrive(&bars[kBarQEmpty + qs]);
+          // One store stays in flight: once the previous tile's store has read its shared
+          // memory, that q/y stage goes back to the producer.
+          bulk_wait_group_read<1>();
+          if (qc > 0) mbar_arrive(&bars[kBarQEmpty + (qc + kNQ - 1) % kNQ]);
         }
       }
       if (!__all_sync(0xffffffffu, ok)) break;
       ++ac;
       ++qc;
     }
-    if (et == 0) bulk_wait_group<0>();
+    if (et == 0) {
+      bulk_wait_group<0>();
+      if (qc > 0) mbar_arrive(&bars[kBarQEmpty + (qc + kNQ - 1) % kNQ]);
+    }
   }
 
   __syncthreads();

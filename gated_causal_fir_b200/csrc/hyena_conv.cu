@@ -16,6 +16,16 @@ namespace {
 
 using hyena::cc::WindowParams;
 
+#ifndef HYENA_TC_L2_PROMOTION
+#define HYENA_TC_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_NONE
+#endif
+#ifndef HYENA_TC_PAIRED
+#define HYENA_TC_PAIRED 1
+#endif
+#ifndef HYENA_TC_RUN
+#define HYENA_TC_RUN 0
+#endif
+
 constexpr int kMaxDevices = 64;
 constexpr int kMaxWindowTaps = 16;
 constexpr int kWindowRows = 32;
@@ -36,7 +46,11 @@ int current_device(DeviceState *&ds) {
   std::call_once(d->once, [d, dev]() {
     cudaError_t e = cudaDeviceGetAttribute(&d->sm_count, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(hyena::tc::fir_tc_kernel,
+      e = cudaFuncSetAttribute(hyena::tc::fir_tc_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               hyena::tc::kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(hyena::tc::fir_tc_kernel<true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                hyena::tc::kSmemBytes);
     d->err = e;
@@ -142,7 +156,7 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
   for (int i = 0; i < 4; ++i) {
     if (enc(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptrs[i]), dims,
             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            HYENA_TC_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return HYENA_ERR_CUDA;
   }
   hyena::tc::Params p;
@@ -153,10 +167,30 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
   p.l_h = P.l_h;
   p.halo = ((P.l_h - 1) + 15) / 16 * 16;
   p.nT = static_cast<int>((P.L + hyena::tc::kTM - 1) / hyena::tc::kTM);
-  p.W = static_cast<long long>(p.G) * p.B * p.nT;
-  const long long grid = p.W < ds->sm_count ? p.W : ds->sm_count;
-  hyena::tc::fir_tc_kernel<<<static_cast<unsigned>(grid), hyena::tc::kThreads,
-                             hyena::tc::kSmemBytes, s>>>(maps[0], maps[1], maps[2], maps[3], p);
+  const long long sms = ds->sm_count;
+  p.run = HYENA_TC_RUN;
+  p.units = 0;
+  p.paired = HYENA_TC_PAIRED && p.G % 2 == 0 && sms >= 2 && p.run == 0;
+  long long grid;
+  if (p.run > 0) {
+    p.units = static_cast<long long>(p.B) * ((p.nT + p.run - 1) / p.run) * p.G;
+    p.W = static_cast<long long>(p.G) * p.B * p.nT;
+    grid = p.units < sms ? p.units : sms;
+  } else if (p.paired) {
+    p.W = static_cast<long long>(p.G / 2) * p.B * p.nT;
+    grid = 2 * (p.W < sms / 2 ? p.W : sms / 2);
+  } else {
+    p.W = static_cast<long long>(p.G) * p.B * p.nT;
+    grid = p.W < sms ? p.W : sms;
+  }
+  if (p.run > 0)
+    hyena::tc::fir_tc_kernel<true><<<static_cast<unsigned>(grid), hyena::tc::kThreads,
+                                     hyena::tc::kSmemBytes, s>>>(maps[0], maps[1], maps[2],
+                                                                 maps[3], p);
+  else
+    hyena::tc::fir_tc_kernel<false><<<static_cast<unsigned>(grid), hyena::tc::kThreads,
+                                      hyena::tc::kSmemBytes, s>>>(maps[0], maps[1], maps[2],
+                                                                  maps[3], p);
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
