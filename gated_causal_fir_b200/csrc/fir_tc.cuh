@@ -63,18 +63,18 @@ constexpr int kKSplit = HYENA_TC_KSPLIT;
 constexpr int kRowBytes = kNC * 2;                              // 128 B
 constexpr int kTileBytes = kTM * kRowBytes;                     // 16 KB
 constexpr int kKBlockBytes = kNC * 128;                         // 64 times x 64 channels
-constexpr int kACores = kTM / 8 + (kTM + kMaxHalo) / 8 - 1;     // 47
-constexpr int kABytes = 48 * 128;                               // padded
-constexpr int kTmemCols = kNAcc * kKSplit * kNC;                // 512 at kKSplit = 4
-static_assert(kTmemCols == 32 || kTmemCols == 64 || kTmemCols == 128 || kTmemCols == 256 ||
-                  kTmemCols == 512,
-              "TMEM allocation must be a power of two between 32 and 512 columns");
+// Tensor memory: accumulators in columns [0, kNAcc * kKSplit * 64); the Toeplitz band (two
+// buffers, one per segment parity) in columns kBandCol0 + 128 * parity: 128 lanes x 128 columns
+// = 128 rows x 256 fp16 K elements each.
+constexpr int kBandCols = (kTM + kMaxHalo) / 2;                  // 128
+constexpr int kBandCol0 = 256;
+constexpr int kTmemCols = 512;
+static_assert(kNAcc * kKSplit * kNC <= kBandCol0, "accumulators overlap the band buffers");
 
 constexpr int kOffKV = 0;
 constexpr int kOffQ = kOffKV + kNKV * 2 * kTileBytes;
 constexpr int kOffX = kOffQ + kNQ * kTileBytes;
-constexpr int kOffA = kOffX + kNX * kTileBytes;
-constexpr int kOffBar = kOffA + 2 * kABytes;
+constexpr int kOffBar = kOffX + kNX * kTileBytes;
 // barriers
 constexpr int kBarKVFull = 0;
 constexpr int kBarKVEmpty = kBarKVFull + kNKV;
@@ -122,22 +122,26 @@ struct Item {
 };
 
 struct WorkIter {
-  long long w, w_begin, w_end;
-  int nT, B, seg, gmul, goff;
-  bool entered;
-  // Tiles [b, e) of the walk ordered (group, batch, time); with gmul = 2 the walk is over
-  // group pairs and this CTA takes group 2 * pair + goff.
-  __device__ WorkIter(long long b, long long e, int nT_, int B_, int gmul_ = 1, int goff_ = 0)
-      : w(b), w_begin(b), w_end(e), nT(nT_), B(B_), seg(-1), gmul(gmul_), goff(goff_),
-        entered(false) {}
+  long long w, w_end;
+  int nT, B, seg, gmul, i, g, b;
+  bool at_begin, entered;
+  // Tiles [w_begin, w_end) of the walk ordered (group, batch, time); with gmul = 2 the walk is
+  // over group pairs and this CTA takes group 2 * pair + goff.  The position is decoded once;
+  // next() only increments (64-bit divisions are software routines on the GPU).
+  __device__ WorkIter(long long w_begin, long long w_end_, int nT_, int B_, int gmul_ = 1,
+                      int goff = 0)
+      : w(w_begin), w_end(w_end_), nT(nT_), B(B_), seg(-1), gmul(gmul_), at_begin(true),
+        entered(false) {
+    const long long seq = w_begin / nT;
+    i = static_cast<int>(w_begin - seq * nT);
+    g = static_cast<int>(seq / B) * gmul + goff;
+    b = static_cast<int>(seq % B);
+  }
   __device__ bool next(Item &it) {
     if (w >= w_end) return false;
-    const long long seq = w / nT;
-    const int i = static_cast<int>(w - seq * nT);
-    it.g = static_cast<int>(seq / B) * gmul + goff;
-    it.b = static_cast<int>(seq % B);
-    const bool first = (w == w_begin) || (i == 0);
-    if (first && !entered) {
+    it.g = g;
+    it.b = b;
+    if ((at_begin || i == 0) && !entered) {
       entered = true;
       ++seg;
       if (i > 0) {
@@ -155,7 +159,15 @@ struct WorkIter {
     it.hist = i > 0;
     it.last = (w + 1 == w_end) || (i + 1 == nT);
     ++w;
+    at_begin = false;
     entered = false;
+    if (++i == nT) {
+      i = 0;
+      if (++b == B) {
+        b = 0;
+        g += gmul;
+      }
+    }
     return true;
   }
 };
@@ -211,18 +223,18 @@ struct RunIter {
   int g_ = 0, b_ = 0;
 };
 
-// The walk of this CTA: contiguous tile ranges (kStrided = false) or strided runs.
-template <bool kStrided>
+// The walk of this CTA: contiguous tile ranges (kSched 0) or strided runs (1).
+template <int kSched>
 struct Walk;
 
 template <>
-struct Walk<false> : WorkIter {
+struct Walk<0> : WorkIter {
   __device__ Walk(const Params &p, long long w_begin, long long w_end, int gmul, int goff)
       : WorkIter(w_begin, w_end, p.nT, p.B, gmul, goff) {}
 };
 
 template <>
-struct Walk<true> : RunIter {
+struct Walk<1> : RunIter {
   __device__ Walk(const Params &p, long long, long long, int, int)
       : RunIter(blockIdx.x, gridDim.x, p.units, p.nT, p.B, p.G, p.run) {}
 };
@@ -252,22 +264,33 @@ __device__ __forceinline__ uint32_t gate_pair(uint32_t kw, uint32_t vw, bool &ov
   return *reinterpret_cast<const uint32_t *>(&hx);
 }
 
-// The Toeplitz band as Hankel core matrices: core d, element (i, j) (row i, K column j) holds
-// h[kTM - 1 + halo - 8 d - i - j] (zero outside [0, l_h)), rounded to fp16.
-__device__ __forceinline__ void build_band(uint8_t *a, const float *hg, int l_h, int halo,
-                                           int gt, bool &over) {
-  const int ncores = kTM / 8 + (kTM + halo) / 8 - 1;
-  __half *ah = reinterpret_cast<__half *>(a);
-  for (int e = gt; e < ncores * 64; e += kGroupThreads) {
-    const int d = e >> 6, i = (e >> 3) & 7, j = e & 7;
-    const int idx = kTM - 1 + halo - 8 * d - i - j;
-    const float hv = (idx >= 0 && idx < l_h) ? __ldg(hg + idx) : 0.f;
-    over |= fabsf(hv) > 65504.f;
-    ah[e] = __float2half_rn(hv);
+// The Toeplitz band of one group in tensor memory.  Output rows are reversed (lane p holds
+// time t0 + 127 - p) and K runs over input rows t0 - halo .. t0 + 127, so
+//     A[p][kk] = h[127 + halo - p - kk]   (zero outside [0, l_h)),  rounded to fp16.
+// Each of the 128 gate threads writes its own lane: 256 K elements = 128 columns.
+__device__ __forceinline__ void build_band_tmem(uint32_t band_col, uint32_t tmem_base,
+                                                const float *hg, int l_h, int halo, int quad,
+                                                int lane, bool &over) {
+  const int row = quad * 32 + lane;
+  const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + band_col;
+#pragma unroll 1
+  for (int c0 = 0; c0 < kBandCols; c0 += 32) {
+    uint32_t r[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const int idx = kTM - 1 + halo - row - 2 * (c0 + c);  // tap of K element 2 (c0 + c)
+      const float v0 = (idx >= 0 && idx < l_h) ? __ldg(hg + idx) : 0.f;
+      const float v1 = (idx - 1 >= 0 && idx - 1 < l_h) ? __ldg(hg + idx - 1) : 0.f;
+      over |= (fabsf(v0) > 65504.f) | (fabsf(v1) > 65504.f);
+      const __half2 hv = __floats2half2_rn(v0, v1);
+      r[c] = *reinterpret_cast<const uint32_t *>(&hv);
+    }
+    tmem_st_32x32b_x32(taddr + c0, r);
   }
+  tmem_wait_st();
 }
 
-template <bool kStrided>
+template <int kSched>
 __global__ void __launch_bounds__(kThreads, 1)
     fir_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
@@ -278,7 +301,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *kv_st = smem + kOffKV;
   uint8_t *q_st = smem + kOffQ;
   uint8_t *x_st = smem + kOffX;
-  uint8_t *a_st = smem + kOffA;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
   volatile int *abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
@@ -317,11 +339,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpTma && lane == 0) {
-    tma_prefetch_desc(&tm_q);
+  // Thread 0 is also the k/v producer: it queues the first k/v stages right away, before the
+  // TMEM allocation and the CTA-wide barrier (no other thread touches those stages yet).
+  Walk<kSched> kv_it(p, w_begin, w_end, gmul, goff);
+  Item kv_t;
+  uint32_t kv_count = 0;
+  bool kv_done = false;
+  if (threadIdx.x == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_y);
+    while (kv_count < kNKV) {
+      if (!kv_it.next(kv_t)) {
+        kv_done = true;
+        break;
+      }
+      mbar_arrive_expect_tx(&bars[kBarKVFull + kv_count], 2 * kTileBytes);
+      uint8_t *dst = kv_st + kv_count * 2 * kTileBytes;
+      tma_load_3d(dst, &tm_k, &bars[kBarKVFull + kv_count], kv_t.g * kNC, kv_t.i * kTM, kv_t.b);
+      tma_load_3d(dst + kTileBytes, &tm_v, &bars[kBarKVFull + kv_count], kv_t.g * kNC,
+                  kv_t.i * kTM, kv_t.b);
+      ++kv_count;
+    }
   }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -335,10 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpTma) {
     // ---------------------------------------------------------------- TMA producer: k, v
     if (lane == 0) {
-      Walk<kStrided> it(p, w_begin, w_end, gmul, goff);
-      Item t;
-      uint32_t kc = 0;
-      while (it.next(t)) {
+      uint32_t kc = kv_count;
+      while (!kv_done && kv_it.next(kv_t)) {
+        const Item &t = kv_t;
         const int ks = kc % kNKV;
         if (!thread_wait(&bars[kBarKVEmpty + ks], ((kc / kNKV) & 1) ^ 1, abort)) break;
         mbar_arrive_expect_tx(&bars[kBarKVFull + ks], 2 * kTileBytes);
@@ -354,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpTmaQ) {
     // ---------------------------------------------------------------- TMA producer: q
     if (lane == 0) {
-      Walk<kStrided> it(p, w_begin, w_end, gmul, goff);
+      Walk<kSched> it(p, w_begin, w_end, gmul, goff);
       Item t;
       uint32_t qc = 0;
       while (it.next(t)) {
@@ -372,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      Walk<kStrided> it(p, w_begin, w_end, gmul, goff);
+      Walk<kSched> it(p, w_begin, w_end, gmul, goff);
       Item t;
       uint32_t xc = 0, ac = 0;
       int cur_seg = -1;
@@ -398,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // start-address field: every address stays inside shared memory).
         const int xp = (xc + kNX - 1) % kNX;
         const uint32_t d_tmem = tmem_base + as * kKSplit * kNC;
-        uint64_t ad = umma_smem_desc(smem_u32(a_st + pa * kABytes), 128, 128, 0);
+        uint32_t ad = tmem_base + kBandCol0 + pa * kBandCols;  // 8 columns = 16 K per step
         // B = X^T, K-major with 128-byte swizzle: k-step s of a slot starts at K-block s / 4
         // (8 KB each) plus 32 bytes per step inside the 128-byte rows.
         int issued = 0;
@@ -408,21 +447,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < hsteps; ++j) {
             const int st = s0 + j;
             const uint64_t bd = bd0 + ((st >> 2) * (kKBlockBytes >> 4) + (st & 3) * 2);
-            umma_f16(d_tmem + (issued % kKSplit) * kNC, ad, bd, idesc, issued >= kKSplit);
+            umma_f16_ts(d_tmem + (issued % kKSplit) * kNC, ad, bd, idesc, issued >= kKSplit);
             ++issued;
-            ad += 16;
+            ad += 8;
           }
         } else {
-          ad += 16 * hsteps;  // zero history before the first tile of a sequence
+          ad += 8 * hsteps;  // zero history before the first tile of a sequence
         }
         {
           const uint64_t bd0 = umma_smem_desc(smem_u32(x_st + xs * kTileBytes), 16, 1024, 2);
 #pragma unroll
           for (int st = 0; st < kTM / 16; ++st) {
             const uint64_t bd = bd0 + ((st >> 2) * (kKBlockBytes >> 4) + (st & 3) * 2);
-            umma_f16(d_tmem + (issued % kKSplit) * kNC, ad, bd, idesc, issued >= kKSplit);
+            umma_f16_ts(d_tmem + (issued % kKSplit) * kNC, ad, bd, idesc, issued >= kKSplit);
             ++issued;
-            ad += 16;
+            ad += 8;
           }
         }
         umma_commit(&bars[kBarAccFull + as]);
@@ -440,8 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kWarpGate0 && warp < kWarpGate0 + 4) {
     // ---------------------------------------------------------------- pre-gate + band build
-    const int gt = threadIdx.x - kWarpGate0 * 32;
-    Walk<kStrided> it(p, w_begin, w_end, gmul, goff);
+    Walk<kSched> it(p, w_begin, w_end, gmul, goff);
     Item t;
     uint32_t kc = 0, xc = 0;
     int cur_seg = -1;
@@ -451,9 +489,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         cur_seg = t.seg;
         const int pa = t.seg & 1, use = t.seg >> 1;
         if (use > 0 && !warp_wait(&bars[kBarAEmpty + pa], (use - 1) & 1, abort)) break;
-        build_band(a_st + pa * kABytes, p.h + static_cast<size_t>(t.g) * p.l_h, p.l_h, p.halo,
-                   gt, over);
-        fence_proxy_async_smem();
+        build_band_tmem(kBandCol0 + pa * kBandCols, tmem_base,
+                        p.h + static_cast<size_t>(t.g) * p.l_h, p.l_h, p.halo, warp & 3, lane,
+                        over);
+        tc_fence_before_sync();
         mbar_arrive(&bars[kBarAFull + pa]);
       }
       const int ks = kc % kNKV, xs = xc % kNX;
@@ -493,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;               // TMEM lanes this warp may read
     const int row_lane = quad * 32 + lane;   // MMA row = TMEM lane
     const int r = kTM - 1 - row_lane;        // tile row (time offset) of that lane
-    Walk<kStrided> it(p, w_begin, w_end, gmul, goff);
+    Walk<kSched> it(p, w_begin, w_end, gmul, goff);
     Item t;
     uint32_t ac = 0, qc = 0;
     while (it.next(t)) {

@@ -26,6 +26,7 @@ using hyena::cc::WindowParams;
 #define HYENA_TC_RUN 0
 #endif
 
+
 constexpr int kMaxDevices = 64;
 constexpr int kMaxWindowTaps = 16;
 constexpr int kWindowRows = 32;
@@ -46,13 +47,14 @@ int current_device(DeviceState *&ds) {
   std::call_once(d->once, [d, dev]() {
     cudaError_t e = cudaDeviceGetAttribute(&d->sm_count, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(hyena::tc::fir_tc_kernel<false>,
+      e = cudaFuncSetAttribute(hyena::tc::fir_tc_kernel<0>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                hyena::tc::kSmemBytes);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(hyena::tc::fir_tc_kernel<true>,
+      e = cudaFuncSetAttribute(hyena::tc::fir_tc_kernel<1>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                hyena::tc::kSmemBytes);
+
     d->err = e;
   });
   return d->err == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
@@ -183,14 +185,12 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
     p.W = static_cast<long long>(p.G) * p.B * p.nT;
     grid = p.W < sms ? p.W : sms;
   }
+  const unsigned g = static_cast<unsigned>(grid);
+  constexpr int T = hyena::tc::kThreads, S = hyena::tc::kSmemBytes;
   if (p.run > 0)
-    hyena::tc::fir_tc_kernel<true><<<static_cast<unsigned>(grid), hyena::tc::kThreads,
-                                     hyena::tc::kSmemBytes, s>>>(maps[0], maps[1], maps[2],
-                                                                 maps[3], p);
+    hyena::tc::fir_tc_kernel<1><<<g, T, S, s>>>(maps[0], maps[1], maps[2], maps[3], p);
   else
-    hyena::tc::fir_tc_kernel<false><<<static_cast<unsigned>(grid), hyena::tc::kThreads,
-                                      hyena::tc::kSmemBytes, s>>>(maps[0], maps[1], maps[2],
-                                                                  maps[3], p);
+    hyena::tc::fir_tc_kernel<0><<<g, T, S, s>>>(maps[0], maps[1], maps[2], maps[3], p);
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
