@@ -79,14 +79,18 @@ struct WindowParams {
 };
 
 // Unroll factor of the time loop: loads of U rows are issued before their arithmetic.
-constexpr int kWindowUnroll = 4;
+#ifndef HYENA_WINDOW_UNROLL
+#define HYENA_WINDOW_UNROLL 8
+#endif
+constexpr int kWindowUnroll = HYENA_WINDOW_UNROLL;
 
 template <typename T, int LH>
 __global__ void __launch_bounds__(256)
     fir_window_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                       const float *__restrict__ h, T *__restrict__ y, const WindowParams p) {
   constexpr int VN = Vec<T>::N;
-  constexpr int U = kWindowUnroll;
+  // Longer windows hold more registers: they unroll less so the loaded rows still fit.
+  constexpr int U = LH <= 8 ? kWindowUnroll : 4;
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (gid >= p.B * p.n_tb * p.cv) return;
   const long long cvi = gid % p.cv;

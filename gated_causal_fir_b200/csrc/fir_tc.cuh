@@ -41,7 +41,7 @@ __device__ unsigned int g_device_status;  // OR of hyena_device_status_bits
 namespace tc {
 
 constexpr int kTM = 128;             // output rows per tile (MMA M)
-constexpr int kNC = 64;              // channels per tile = d_g (MMA N)
+constexpr int kNC = 64;              // channels per tile: 64 / d_g groups of d_g (MMA N = d_g)
 constexpr int kMaxHalo = 128;        // supports l_h - 1 <= 128
 #ifndef HYENA_TC_KV_STAGES
 #define HYENA_TC_KV_STAGES 3
@@ -53,23 +53,15 @@ constexpr int kNKV = HYENA_TC_KV_STAGES;  // k/v stages
 constexpr int kNQ = HYENA_TC_Q_STAGES;    // q (and in-place y) stages
 constexpr int kNX = 3;               // fp16 X slots (current, previous, next)
 constexpr int kNAcc = 2;             // TMEM accumulator sets (tiles in flight)
-#ifndef HYENA_TC_KSPLIT
-#define HYENA_TC_KSPLIT 1
-#endif
-// Independent partial accumulators per tile: k-step n of a tile accumulates into partial
-// n % kKSplit, so consecutive MMAs do not wait on each other's accumulator; the epilogue sums
-// the partials in fp32.
-constexpr int kKSplit = HYENA_TC_KSPLIT;
 constexpr int kRowBytes = kNC * 2;                              // 128 B
 constexpr int kTileBytes = kTM * kRowBytes;                     // 16 KB
 constexpr int kKBlockBytes = kNC * 128;                         // 64 times x 64 channels
-// Tensor memory: accumulators in columns [0, kNAcc * kKSplit * 64); the Toeplitz band (two
-// buffers, one per segment parity) in columns kBandCol0 + 128 * parity: 128 lanes x 128 columns
-// = 128 rows x 256 fp16 K elements each.
-constexpr int kBandCols = (kTM + kMaxHalo) / 2;                  // 128
-constexpr int kBandCol0 = 256;
+// Tensor memory: accumulators in columns [0, kNAcc * 64) (group gg of a tile in columns
+// [gg d_g, (gg+1) d_g) of its set); then `nbuf` sets of Toeplitz bands, one band per group of the
+// tile, each 128 lanes x band_cols columns = 128 rows x 2 band_cols fp16 K elements, with
+// band_cols = (128 + halo) / 2.  The host picks nbuf (2, else 1) so that everything fits.
+constexpr int kBandCol0 = kNAcc * kNC;                           // 128
 constexpr int kTmemCols = 512;
-static_assert(kNAcc * kKSplit * kNC <= kBandCol0, "accumulators overlap the band buffers");
 
 constexpr int kOffKV = 0;
 constexpr int kOffQ = kOffKV + kNKV * 2 * kTileBytes;
@@ -86,7 +78,7 @@ constexpr int kBarXEmpty = kBarXFull + kNX;
 constexpr int kBarAccFull = kBarXEmpty + kNX;
 constexpr int kBarAccEmpty = kBarAccFull + kNAcc;
 constexpr int kBarAFull = kBarAccEmpty + kNAcc;
-constexpr int kBarAEmpty = kBarAFull + 2;
+constexpr int kBarAEmpty = kBarAFull + 2;  // up to two band sets
 constexpr int kBarDone = kBarAEmpty + 2;
 constexpr int kNumBars = kBarDone + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -101,20 +93,23 @@ constexpr unsigned kTimeoutBit = 1u;  // HYENA_DEVICE_TIMEOUT
 constexpr unsigned kF16RangeBit = 2u; // HYENA_DEVICE_F16_RANGE
 
 struct Params {
-  const float *h;   // [G, l_h]
-  int B, L, G, l_h;
+  const float *h;   // [D / d_g, l_h]
+  int B, L, l_h;
+  int CB;           // 64-channel blocks across D (tiles per time row) = D / 64
   int halo;         // multiple of 16, >= l_h - 1, <= kMaxHalo
+  int band_cols;    // TMEM columns of one group's band = (128 + halo) / 2
+  int nbuf;         // band sets in TMEM (1 or 2)
   int nT;           // tiles per sequence = ceil(L / kTM)
-  long long W;      // tiles of the walk: G * B * nT, or (G / 2) * B * nT when paired
-  int paired;       // CTAs 2p and 2p+1 walk the same (group pair, batch, time) range, one
-                    // group each, so both halves of every 256-byte row are read together
+  long long W;      // tiles of the walk: CB * B * nT, or (CB / 2) * B * nT when paired
+  int paired;       // CTAs 2p and 2p+1 walk the same (block pair, batch, time) range, one
+                    // block each, so both halves of every 256-byte row are read together
   int run;          // > 0: strided schedule of runs of `run` tiles (see RunIter)
-  long long units;  // number of runs: B * ceil(nT / run) * G
+  long long units;  // number of runs: B * ceil(nT / run) * CB
 };
 
 // One unit of a CTA's walk: a halo tile (input only) or an output tile.
 struct Item {
-  int g, b, i;      // group, sequence, tile index along time
+  int g, b, i;      // 64-channel block, sequence, tile index along time
   int seg;          // running segment number within this CTA (a segment = one sequence run)
   bool halo;        // input-only tile feeding the first output tile of a segment
   bool hist;        // the output tile reads the previous tile's X (i > 0)
@@ -236,7 +231,7 @@ struct Walk<0> : WorkIter {
 template <>
 struct Walk<1> : RunIter {
   __device__ Walk(const Params &p, long long, long long, int, int)
-      : RunIter(blockIdx.x, gridDim.x, p.units, p.nT, p.B, p.G, p.run) {}
+      : RunIter(blockIdx.x, gridDim.x, p.units, p.nT, p.B, p.CB, p.run) {}
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
@@ -267,30 +262,43 @@ __device__ __forceinline__ uint32_t gate_pair(uint32_t kw, uint32_t vw, bool &ov
 // The Toeplitz band of one group in tensor memory.  Output rows are reversed (lane p holds
 // time t0 + 127 - p) and K runs over input rows t0 - halo .. t0 + 127, so
 //     A[p][kk] = h[127 + halo - p - kk]   (zero outside [0, l_h)),  rounded to fp16.
-// Each of the 128 gate threads writes its own lane: 256 K elements = 128 columns.
-__device__ __forceinline__ void build_band_tmem(uint32_t band_col, uint32_t tmem_base,
-                                                const float *hg, int l_h, int halo, int quad,
-                                                int lane, bool &over) {
+// Each of the 128 gate threads writes its own lane: 128 + halo K elements = band_cols columns.
+// Columns [c0, c0 + N) of one lane's band row: 2 N taps loaded together, then one store.
+template <int N>
+__device__ __forceinline__ void band_chunk(uint32_t taddr, int c0, int row, const float *hg,
+                                           int l_h, int halo, bool &over) {
+  uint32_t r[N];
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    const int idx = kTM - 1 + halo - row - 2 * (c0 + c);  // tap of K element 2 (c0 + c)
+    const float v0 = (idx >= 0 && idx < l_h) ? __ldg(hg + idx) : 0.f;
+    const float v1 = (idx - 1 >= 0 && idx - 1 < l_h) ? __ldg(hg + idx - 1) : 0.f;
+    over |= (fabsf(v0) > 65504.f) | (fabsf(v1) > 65504.f);
+    const __half2 hv = __floats2half2_rn(v0, v1);
+    r[c] = *reinterpret_cast<const uint32_t *>(&hv);
+  }
+  if constexpr (N == 32)
+    tmem_st_32x32b_x32(taddr + c0, r);
+  else
+    tmem_st_32x32b_x8(taddr + c0, r);
+}
+
+__device__ __forceinline__ void build_band_tmem(uint32_t band_col, int band_cols,
+                                                uint32_t tmem_base, const float *hg, int l_h,
+                                                int halo, int quad, int lane, bool &over) {
   const int row = quad * 32 + lane;
   const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + band_col;
+  int c0 = 0;
+  // 32 columns (64 taps in flight) per step, then the 8-column remainder.
 #pragma unroll 1
-  for (int c0 = 0; c0 < kBandCols; c0 += 32) {
-    uint32_t r[32];
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const int idx = kTM - 1 + halo - row - 2 * (c0 + c);  // tap of K element 2 (c0 + c)
-      const float v0 = (idx >= 0 && idx < l_h) ? __ldg(hg + idx) : 0.f;
-      const float v1 = (idx - 1 >= 0 && idx - 1 < l_h) ? __ldg(hg + idx - 1) : 0.f;
-      over |= (fabsf(v0) > 65504.f) | (fabsf(v1) > 65504.f);
-      const __half2 hv = __floats2half2_rn(v0, v1);
-      r[c] = *reinterpret_cast<const uint32_t *>(&hv);
-    }
-    tmem_st_32x32b_x32(taddr + c0, r);
-  }
+  for (; c0 + 32 <= band_cols; c0 += 32) band_chunk<32>(taddr, c0, row, hg, l_h, halo, over);
+#pragma unroll 1
+  for (; c0 < band_cols; c0 += 8) band_chunk<8>(taddr, c0, row, hg, l_h, halo, over);
   tmem_wait_st();
 }
 
-template <int kSched>
+// kNG = 64 / d_g groups per tile (1, 2 or 4); MMA N = d_g.
+template <int kSched, int kNG>
 __global__ void __launch_bounds__(kThreads, 1)
     fir_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
@@ -415,7 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       Item t;
       uint32_t xc = 0, ac = 0;
       int cur_seg = -1;
-      const uint32_t idesc = umma_idesc_f16_f32(kTM, kNC, 0);  // B K-major
+      constexpr int kDG = kNC / kNG;
+      const uint32_t idesc = umma_idesc_f16_f32(kTM, kDG, 0);  // N = d_g, B K-major
       const int hsteps = p.halo / 16;
       while (it.next(t)) {
         const int xs = xc % kNX;
@@ -424,44 +433,55 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++xc;
           continue;
         }
-        const int pa = t.seg & 1;
+        // band set of this segment and how often it was filled before (nbuf is 1 or 2)
+        const int pa = p.nbuf == 2 ? (t.seg & 1) : 0;
         if (t.seg != cur_seg) {
           cur_seg = t.seg;
-          if (!thread_wait(&bars[kBarAFull + pa], (t.seg >> 1) & 1, abort)) break;
+          const int use = p.nbuf == 2 ? (t.seg >> 1) : t.seg;
+          if (!thread_wait(&bars[kBarAFull + pa], use & 1, abort)) break;
         }
         const int as = ac % kNAcc;
         if (!thread_wait(&bars[kBarAccEmpty + as], ((ac / kNAcc) & 1) ^ 1, abort)) break;
         tc_fence_after_sync();
-        // Descriptors advance by plain adds: 16 rows of X = 2048 B = 128 units of 16 B per
-        // k-step, 2 core matrices of the band = 256 B = 16 units (no carry out of the 14-bit
-        // start-address field: every address stays inside shared memory).
         const int xp = (xc + kNX - 1) % kNX;
-        const uint32_t d_tmem = tmem_base + as * kKSplit * kNC;
-        uint32_t ad = tmem_base + kBandCol0 + pa * kBandCols;  // 8 columns = 16 K per step
+        const uint32_t d_tmem = tmem_base + as * kNC;
+        const uint32_t band0 = tmem_base + kBandCol0 + pa * kNG * p.band_cols;
         // B = X^T, K-major with 128-byte swizzle: k-step s of a slot starts at K-block s / 4
-        // (8 KB each) plus 32 bytes per step inside the 128-byte rows.
-        int issued = 0;
+        // (8 KB each) plus 32 bytes per step inside the 128-byte rows; group gg's rows start
+        // gg * d_g channel rows (gg * d_g * 128 bytes) into the block.  A (group gg's band)
+        // advances 8 columns per k-step.
+        uint32_t a_run[kNG];  // next band column of each group
+#pragma unroll
+        for (int gg = 0; gg < kNG; ++gg) a_run[gg] = band0 + gg * p.band_cols;
+        uint32_t acc = 0;     // 0 only for the first MMA of each group's chain
         if (t.hist) {
           const uint64_t bd0 = umma_smem_desc(smem_u32(x_st + xp * kTileBytes), 16, 1024, 2);
           const int s0 = (kTM - p.halo) / 16;
           for (int j = 0; j < hsteps; ++j) {
             const int st = s0 + j;
-            const uint64_t bd = bd0 + ((st >> 2) * (kKBlockBytes >> 4) + (st & 3) * 2);
-            umma_f16_ts(d_tmem + (issued % kKSplit) * kNC, ad, bd, idesc, issued >= kKSplit);
-            ++issued;
-            ad += 8;
+            const uint64_t bdj = bd0 + ((st >> 2) * (kKBlockBytes >> 4) + (st & 3) * 2);
+#pragma unroll
+            for (int gg = 0; gg < kNG; ++gg) {
+              umma_f16_ts(d_tmem + gg * kDG, a_run[gg], bdj + gg * (kDG * 8), idesc, acc);
+              a_run[gg] += 8;
+            }
+            acc = 1;
           }
         } else {
-          ad += 8 * hsteps;  // zero history before the first tile of a sequence
+#pragma unroll
+          for (int gg = 0; gg < kNG; ++gg) a_run[gg] += 8 * hsteps;  // zero history
         }
         {
           const uint64_t bd0 = umma_smem_desc(smem_u32(x_st + xs * kTileBytes), 16, 1024, 2);
 #pragma unroll
           for (int st = 0; st < kTM / 16; ++st) {
-            const uint64_t bd = bd0 + ((st >> 2) * (kKBlockBytes >> 4) + (st & 3) * 2);
-            umma_f16_ts(d_tmem + (issued % kKSplit) * kNC, ad, bd, idesc, issued >= kKSplit);
-            ++issued;
-            ad += 8;
+            const uint64_t bdj = bd0 + ((st >> 2) * (kKBlockBytes >> 4) + (st & 3) * 2);
+#pragma unroll
+            for (int gg = 0; gg < kNG; ++gg) {
+              umma_f16_ts(d_tmem + gg * kDG, a_run[gg], bdj + gg * (kDG * 8), idesc, acc);
+              a_run[gg] += 8;
+            }
+            acc = 1;
           }
         }
         umma_commit(&bars[kBarAccFull + as]);
@@ -487,11 +507,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (it.next(t)) {
       if (t.seg != cur_seg) {
         cur_seg = t.seg;
-        const int pa = t.seg & 1, use = t.seg >> 1;
+        const int pa = p.nbuf == 2 ? (t.seg & 1) : 0, use = p.nbuf == 2 ? (t.seg >> 1) : t.seg;
         if (use > 0 && !warp_wait(&bars[kBarAEmpty + pa], (use - 1) & 1, abort)) break;
-        build_band_tmem(kBandCol0 + pa * kBandCols, tmem_base,
-                        p.h + static_cast<size_t>(t.g) * p.l_h, p.l_h, p.halo, warp & 3, lane,
-                        over);
+#pragma unroll 1
+        for (int gg = 0; gg < kNG; ++gg)
+          build_band_tmem(kBandCol0 + (pa * kNG + gg) * p.band_cols, p.band_cols, tmem_base,
+                          p.h + (static_cast<size_t>(t.g) * kNG + gg) * p.l_h, p.l_h, p.halo,
+                          warp & 3, lane, over);
         tc_fence_before_sync();
         mbar_arrive(&bars[kBarAFull + pa]);
       }
@@ -541,27 +563,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&bars[kBarAccFull + as], (ac / kNAcc) & 1, abort)) break;
       tc_fence_after_sync();
       uint32_t a0[32], a1[32];
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + as * kKSplit * kNC;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + as * kNC;
       tmem_ld_32x32b_x32(taddr, a0);
       tmem_ld_32x32b_x32(taddr + 32, a1);
       tmem_wait_ld();
       reg_fence(a0);
       reg_fence(a1);
-#pragma unroll 1
-      for (int part = 1; part < kKSplit; ++part) {
-        uint32_t b0[32], b1[32];
-        tmem_ld_32x32b_x32(taddr + part * kNC, b0);
-        tmem_ld_32x32b_x32(taddr + part * kNC + 32, b1);
-        tmem_wait_ld();
-        reg_fence(b0);
-        reg_fence(b1);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          a0[c] = __float_as_uint(__uint_as_float(a0[c]) + __uint_as_float(b0[c]));
-          a1[c] = __float_as_uint(__uint_as_float(a1[c]) + __uint_as_float(b1[c]));
-        }
-      }
       tc_fence_before_sync();
       mbar_arrive(&bars[kBarAccEmpty + as]);
       if (!warp_wait(&bars[kBarQFull + qs], (qc / kNQ) & 1, abort)) break;

@@ -29,7 +29,10 @@ using hyena::cc::WindowParams;
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxWindowTaps = 16;
-constexpr int kWindowRows = 32;
+#ifndef HYENA_WINDOW_ROWS
+#define HYENA_WINDOW_ROWS 128
+#endif
+constexpr int kWindowRows = HYENA_WINDOW_ROWS;
 
 struct DeviceState {
   std::once_flag once;
@@ -46,14 +49,17 @@ int current_device(DeviceState *&ds) {
   DeviceState *d = ds;
   std::call_once(d->once, [d, dev]() {
     cudaError_t e = cudaDeviceGetAttribute(&d->sm_count, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(hyena::tc::fir_tc_kernel<0>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               hyena::tc::kSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(hyena::tc::fir_tc_kernel<1>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               hyena::tc::kSmemBytes);
+    const void *kernels[] = {
+        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<0, 1>),
+        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<0, 2>),
+        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<0, 4>),
+        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 1>),
+        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 2>),
+        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 4>)};
+    for (const void *k : kernels)
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 hyena::tc::kSmemBytes);
 
     d->err = e;
   });
@@ -87,7 +93,6 @@ struct Problem {
   int d_g, l_h, l_b, dtype;
   int64_t elem() const { return dtype == HYENA_DTYPE_F32 ? 4 : 2; }
   int64_t numel() const { return B * L * D; }
-  int64_t G() const { return D / d_g; }
 };
 
 constexpr int kEmpty = -1;  // internal: valid problem with nothing to compute
@@ -124,11 +129,28 @@ bool all_aligned16(const Problem &P) {
   return aligned(P.q, 16) && aligned(P.k, 16) && aligned(P.v, 16) && aligned(P.y, 16);
 }
 
+// Tensor-core plan: history rows, one group's band width in TMEM columns and the number of
+// band sets (2 when they fit, else 1; 0 = does not fit).
+struct TcPlan {
+  int halo, band_cols, ng, nbuf;
+};
+
+TcPlan tc_plan(const Problem &P) {
+  TcPlan t{0, 0, 0, 0};
+  if (P.d_g != 16 && P.d_g != 32 && P.d_g != 64) return t;
+  t.halo = ((P.l_h - 1) + 15) / 16 * 16;
+  t.band_cols = (hyena::tc::kTM + t.halo) / 2;
+  t.ng = hyena::tc::kNC / P.d_g;
+  const int room = hyena::tc::kTmemCols - hyena::tc::kBandCol0;
+  t.nbuf = 2 * t.ng * t.band_cols <= room ? 2 : (t.ng * t.band_cols <= room ? 1 : 0);
+  return t;
+}
+
 bool tensor_supported(const Problem &P) {
   const int64_t i32 = std::numeric_limits<int32_t>::max();
-  return P.dtype == HYENA_DTYPE_BF16 && P.d_g == hyena::tc::kNC &&
-         P.l_h - 1 <= hyena::tc::kMaxHalo && all_aligned16(P) && P.L <= i32 && P.B <= i32 &&
-         P.D <= i32;
+  return P.dtype == HYENA_DTYPE_BF16 && P.D % hyena::tc::kNC == 0 &&
+         P.l_h - 1 <= hyena::tc::kMaxHalo && tc_plan(P).nbuf > 0 && all_aligned16(P) &&
+         P.L <= i32 && P.B <= i32 && P.D <= i32;
 }
 
 bool window_supported(const Problem &P) {
@@ -136,9 +158,21 @@ bool window_supported(const Problem &P) {
   return P.l_h <= kMaxWindowTaps && P.d_g % vec == 0 && all_aligned16(P);
 }
 
+// MMAs one 128-row tile issues on the tensor path (groups per tile x k-steps).  Each costs
+// ~55 cycles of issue at any N <= 64; past ~24 per tile the issuing thread, not HBM, sets the
+// pace, and for short filters the CUDA-core window kernel is faster (measured on the SE
+// workload: 36 MMAs per tile, 80 us on tensor cores vs 56 us in the window kernel).
+constexpr int kMaxTileMmas = 24;
+
 int select_algo(const Problem &P) {
-  if (tensor_supported(P)) return HYENA_ALGO_TENSOR;
-  if (window_supported(P)) return HYENA_ALGO_WINDOW;
+  const bool tensor = tensor_supported(P), window = window_supported(P);
+  if (tensor && window) {
+    const TcPlan t = tc_plan(P);
+    return t.ng * ((hyena::tc::kTM + t.halo) / 16) <= kMaxTileMmas ? HYENA_ALGO_TENSOR
+                                                                   : HYENA_ALGO_WINDOW;
+  }
+  if (tensor) return HYENA_ALGO_TENSOR;
+  if (window) return HYENA_ALGO_WINDOW;
   return HYENA_ALGO_DIRECT;
 }
 
@@ -161,36 +195,48 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
             HYENA_TC_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return HYENA_ERR_CUDA;
   }
+  const TcPlan plan = tc_plan(P);
   hyena::tc::Params p;
   p.h = P.h;
   p.B = static_cast<int>(P.B);
   p.L = static_cast<int>(P.L);
-  p.G = static_cast<int>(P.G());
+  p.CB = static_cast<int>(P.D / hyena::tc::kNC);
   p.l_h = P.l_h;
-  p.halo = ((P.l_h - 1) + 15) / 16 * 16;
+  p.halo = plan.halo;
+  p.band_cols = plan.band_cols;
+  p.nbuf = plan.nbuf;
   p.nT = static_cast<int>((P.L + hyena::tc::kTM - 1) / hyena::tc::kTM);
   const long long sms = ds->sm_count;
   p.run = HYENA_TC_RUN;
   p.units = 0;
-  p.paired = HYENA_TC_PAIRED && p.G % 2 == 0 && sms >= 2 && p.run == 0;
+  p.paired = HYENA_TC_PAIRED && p.CB % 2 == 0 && sms >= 2 && p.run == 0;
   long long grid;
   if (p.run > 0) {
-    p.units = static_cast<long long>(p.B) * ((p.nT + p.run - 1) / p.run) * p.G;
-    p.W = static_cast<long long>(p.G) * p.B * p.nT;
+    p.units = static_cast<long long>(p.B) * ((p.nT + p.run - 1) / p.run) * p.CB;
+    p.W = static_cast<long long>(p.CB) * p.B * p.nT;
     grid = p.units < sms ? p.units : sms;
   } else if (p.paired) {
-    p.W = static_cast<long long>(p.G / 2) * p.B * p.nT;
+    p.W = static_cast<long long>(p.CB / 2) * p.B * p.nT;
     grid = 2 * (p.W < sms / 2 ? p.W : sms / 2);
   } else {
-    p.W = static_cast<long long>(p.G) * p.B * p.nT;
+    p.W = static_cast<long long>(p.CB) * p.B * p.nT;
     grid = p.W < sms ? p.W : sms;
   }
   const unsigned g = static_cast<unsigned>(grid);
   constexpr int T = hyena::tc::kThreads, S = hyena::tc::kSmemBytes;
-  if (p.run > 0)
-    hyena::tc::fir_tc_kernel<1><<<g, T, S, s>>>(maps[0], maps[1], maps[2], maps[3], p);
-  else
-    hyena::tc::fir_tc_kernel<0><<<g, T, S, s>>>(maps[0], maps[1], maps[2], maps[3], p);
+#define HYENA_TC_LAUNCH(SCHED, NG) \
+  hyena::tc::fir_tc_kernel<SCHED, NG><<<g, T, S, s>>>(maps[0], maps[1], maps[2], maps[3], p)
+  const int sched = p.run > 0 ? 1 : 0;
+  switch (sched * 8 + plan.ng) {
+    case 1: HYENA_TC_LAUNCH(0, 1); break;
+    case 2: HYENA_TC_LAUNCH(0, 2); break;
+    case 4: HYENA_TC_LAUNCH(0, 4); break;
+    case 9: HYENA_TC_LAUNCH(1, 1); break;
+    case 10: HYENA_TC_LAUNCH(1, 2); break;
+    case 12: HYENA_TC_LAUNCH(1, 4); break;
+    default: return HYENA_ERR_UNSUPPORTED;
+  }
+#undef HYENA_TC_LAUNCH
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 

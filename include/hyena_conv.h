@@ -54,9 +54,11 @@ enum hyena_dtype {
 enum hyena_algo {
     HYENA_ALGO_AUTO = 0,         /* pick the fastest algorithm that supports the problem */
     HYENA_ALGO_TENSOR = 1,       /* tcgen05 tensor-core block-Toeplitz GEMM (bf16 only;
-                                    d_g == 64, l_h <= 129, 16-byte aligned tensors) */
-    HYENA_ALGO_WINDOW = 2,       /* CUDA-core register sliding window (l_h <= 16,
-                                    d_g and D multiples of 16 bytes of channels) */
+                                    D % 64 == 0, d_g in {16, 32, 64}, l_h <= 129, and
+                                    l_h <= 65 when d_g == 16; 16-byte aligned tensors) */
+    HYENA_ALGO_WINDOW = 2,       /* CUDA-core register sliding window (l_h <= 16; d_g a
+                                    multiple of 8 channels for bf16, 4 for fp32; 16-byte
+                                    aligned tensors) */
     HYENA_ALGO_DIRECT = 3        /* CUDA-core direct sum; any supported shape */
 };
 

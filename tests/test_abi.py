@@ -49,8 +49,14 @@ def test_select_algo_fallbacks(lib):
     bf, f32 = g.HYENA_DTYPE_BF16, g.HYENA_DTYPE_F32
     assert g.hyena_select_algo(1, 100, 256, 64, 130, 65, bf) == g.HYENA_ALGO_DIRECT  # l_h > 129
     assert g.hyena_select_algo(1, 100, 256, 64, 129, 65, bf) == g.HYENA_ALGO_TENSOR
-    assert g.hyena_select_algo(1, 100, 96, 32, 40, 32, bf) == g.HYENA_ALGO_DIRECT   # d_g != 64
+    assert g.hyena_select_algo(1, 100, 128, 32, 40, 32, bf) == g.HYENA_ALGO_TENSOR
+    assert g.hyena_select_algo(1, 100, 96, 32, 40, 32, bf) == g.HYENA_ALGO_DIRECT   # D % 64 != 0
     assert g.hyena_select_algo(1, 100, 96, 32, 16, 32, bf) == g.HYENA_ALGO_WINDOW
+    assert g.hyena_select_algo(1, 100, 128, 16, 65, 64, bf) == g.HYENA_ALGO_TENSOR  # 4 bands fit
+    assert g.hyena_select_algo(1, 100, 128, 16, 7, 16, bf) == g.HYENA_ALGO_WINDOW   # 36 MMAs/tile
+    assert g.hyena_select_algo(1, 100, 128, 32, 7, 16, bf) == g.HYENA_ALGO_TENSOR   # 18 MMAs/tile
+    assert g.hyena_select_algo(1, 100, 128, 16, 66, 64, bf) == g.HYENA_ALGO_DIRECT  # they do not
+    assert g.hyena_select_algo(1, 100, 128, 8, 7, 16, bf) == g.HYENA_ALGO_WINDOW    # d_g = 8
     assert g.hyena_select_algo(1, 100, 96, 4, 3, 2, bf) == g.HYENA_ALGO_DIRECT      # 4 ch < 16 B
     assert g.hyena_select_algo(1, 100, 96, 4, 3, 2, f32) == g.HYENA_ALGO_WINDOW
     assert g.hyena_select_algo(1, 64, 128, 64, 128, 64, f32) == g.HYENA_ALGO_DIRECT
@@ -73,7 +79,8 @@ def _call(lib, q=0x10000, k=0x20000, v=0x30000, h=0x40000, y=0x50000, dtype=0, a
     (dict(B=-1), 1), (dict(L=-5), 1), (dict(D=0), 1), (dict(d_g=0), 1), (dict(d_g=48), 1),
     (dict(l_h=0), 1), (dict(l_b=0), 1), (dict(l_h=33, l_b=16), 1), (dict(dtype=7), 1),
     (dict(algo=9), 1), (dict(y=0x10000 + 64), 1), (dict(q=0x10001), 3), (dict(h=0x40002), 3),
-    (dict(algo=1, dtype=1), 2), (dict(algo=1, d_g=32), 2), (dict(algo=2, l_h=17, l_b=16), 2),
+    (dict(algo=1, dtype=1), 2), (dict(algo=1, d_g=8, l_h=8, l_b=8), 2),
+    (dict(algo=2, l_h=17, l_b=16), 2),
     (dict(algo=1, q=0x10002), 2),
 ])
 def test_host_validation(lib, kw, code):

@@ -60,6 +60,9 @@ SHAPES = [
     ("halo_16", 2, 700, 192, 64, 17, 16, "bf16"),
     ("se_like", 2, 777, 512, 16, 7, 16, "bf16"),
     ("dg32", 1, 300, 96, 32, 16, 8, "bf16"),
+    ("dg32_tc", 2, 1100, 256, 32, 40, 32, "bf16"),
+    ("dg16_lh65", 1, 900, 128, 16, 65, 64, "bf16"),
+    ("dg16_multiseg", 3, 2000, 512, 16, 7, 16, "bf16"),
     ("dg4", 1, 200, 60, 4, 5, 3, "bf16"),
     ("dg3_odd", 1, 300, 30, 3, 4, 2, "bf16"),
     ("long_filter", 1, 600, 128, 64, 200, 100, "bf16"),
@@ -69,11 +72,20 @@ SHAPES = [
 ]
 
 
+def _tensor_fits(D, d_g, l_h):
+    """The tensor kernel's plan: 64-channel tiles of 64 / d_g groups, one Toeplitz band of
+    (128 + halo) / 2 TMEM columns per group, next to 128 accumulator columns (512 in all)."""
+    if d_g not in (16, 32, 64) or D % 64 or l_h > 129:
+        return False
+    halo = (l_h - 1 + 15) // 16 * 16
+    return (64 // d_g) * (128 + halo) // 2 <= 384
+
+
 def _supported(algo, B, L, D, d_g, l_h, l_b, dtype):
     if algo == "direct":
         return True
     if algo == "tensor":
-        return dtype == "bf16" and d_g == 64 and l_h <= 129
+        return dtype == "bf16" and _tensor_fits(D, d_g, l_h)
     return l_h <= 16 and d_g % (4 if dtype == "f32" else 8) == 0
 
 
