@@ -159,32 +159,80 @@ def hyena_abi_version():
     return int(_native.lib().hyena_abi_version())
 
 
-_STAGING = {}
+class _Pipeline:
+    """Device slots and streams of hyena_conv_fwd_from_host, reused across calls."""
+
+    def __init__(self, torch, rows, D, dtype, hshape, device, nslots=3):
+        dev = torch.device(device)
+        self.slots = [[torch.empty((1, rows, D), dtype=dtype, device=dev) for _ in range(4)]
+                      for _ in range(nslots)]
+        self.h = torch.empty(hshape, dtype=torch.float32, device=dev)
+        self.h2d, self.comp, self.d2h = (torch.cuda.Stream(device=dev) for _ in range(3))
+        self.free = [torch.cuda.Event() for _ in range(nslots)]
+        self.used = [False] * nslots
 
 
-def hyena_conv_fwd_from_host(q, k, v, h, d_g, l_b, out=None, device="cuda", stream=None):
-    """End-to-end forward for host tensors: copies q, k, v (bf16 or fp32 [B, L, D]) and h to
-    ``device``, runs the forward there and copies y back into ``out`` (a host tensor; pinned
-    memory makes every copy asynchronous).  Device staging buffers are reused across calls
-    of the same shape.  Queued on ``stream``; synchronise it before reading ``out``.
+_PIPES = {}
+
+
+def hyena_conv_fwd_from_host(q, k, v, h, d_g, l_b, out=None, device="cuda", stream=None,
+                             chunk=2048):
+    """End-to-end forward for host tensors: q, k, v (bf16 or fp32 [B, L, D]) and h go to
+    ``device``, the forward runs there, and y comes back into ``out`` (a host tensor).
+
+    The sequence is cut into chunks of ``chunk`` rows.  Chunk c is copied to the device
+    together with the l_h - 1 rows before it (its history), computed as its own sequence, and
+    its rows after the history are copied back: the result is the same as one call on the
+    whole sequence, and the host-to-device copy of one chunk overlaps the kernel and the
+    device-to-host copy of the previous ones (separate streams; PCIe is full duplex).  With
+    pinned host memory every copy is asynchronous.  The call is ordered after the work queued
+    on ``stream`` (default: current stream) and ``stream`` waits for it on return; synchronise
+    ``stream`` before reading ``out``.
     """
     torch = _torch()
-    key = (tuple(q.shape), q.dtype, tuple(h.shape), str(device))
-    bufs = _STAGING.get(key)
-    if bufs is None:
-        bufs = [torch.empty(q.shape, dtype=q.dtype, device=device) for _ in range(4)]
-        bufs.append(torch.empty(h.shape, dtype=torch.float32, device=device))
-        _STAGING.clear()
-        _STAGING[key] = bufs
-    qd, kd, vd, yd, hd = bufs
+    B, L, D = q.shape
+    hist = h.shape[1] - 1
+    rows = min(L, chunk) + hist
+    key = (rows, D, q.dtype, tuple(h.shape), str(device))
+    pipe = _PIPES.get(key)
+    if pipe is None:
+        _PIPES.clear()
+        pipe = _PIPES[key] = _Pipeline(torch, rows, D, q.dtype, h.shape, device)
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-    s = torch.cuda.current_stream() if stream is None else stream
-    with torch.cuda.stream(s):
-        qd.copy_(q, non_blocking=True)
-        kd.copy_(k, non_blocking=True)
-        vd.copy_(v, non_blocking=True)
-        hd.copy_(h, non_blocking=True)
-        hyena_conv_fwd_ex(qd, kd, vd, hd, d_g, l_b, y=yd, stream=s)
-        out.copy_(yd, non_blocking=True)
+    caller = torch.cuda.current_stream(device) if stream is None else stream
+    start = torch.cuda.Event()
+    start.record(caller)
+    pipe.h2d.wait_event(start)
+    with torch.cuda.stream(pipe.h2d):
+        pipe.h.copy_(h, non_blocking=True)
+    n = 0
+    for b in range(B):
+        for t0 in range(0, L, chunk):
+            t1 = min(L, t0 + chunk)
+            s0 = max(0, t0 - hist)           # first row copied (history included)
+            nr = t1 - s0
+            si = n % len(pipe.slots)
+            qd, kd, vd, yd = (x[:, :nr] for x in pipe.slots[si])
+            if pipe.used[si]:                # the slot's previous chunk is back on the host
+                pipe.h2d.wait_event(pipe.free[si])
+            with torch.cuda.stream(pipe.h2d):
+                qd[0].copy_(q[b, s0:t1], non_blocking=True)
+                kd[0].copy_(k[b, s0:t1], non_blocking=True)
+                vd[0].copy_(v[b, s0:t1], non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(pipe.h2d)
+            pipe.comp.wait_event(loaded)
+            hyena_conv_fwd_ex(qd, kd, vd, pipe.h, d_g, l_b, y=yd, stream=pipe.comp)
+            done = torch.cuda.Event()
+            done.record(pipe.comp)
+            pipe.d2h.wait_event(done)
+            with torch.cuda.stream(pipe.d2h):
+                out[b, t0:t1].copy_(yd[0, t0 - s0:], non_blocking=True)
+            pipe.free[si].record(pipe.d2h)
+            pipe.used[si] = True
+            n += 1
+    finish = torch.cuda.Event()
+    finish.record(pipe.d2h)
+    caller.wait_event(finish)
     return out

@@ -84,8 +84,16 @@ struct WindowParams {
 #endif
 constexpr int kWindowUnroll = HYENA_WINDOW_UNROLL;
 
+#ifndef HYENA_WINDOW_BLOCK
+#define HYENA_WINDOW_BLOCK 128
+#endif
+#ifndef HYENA_WINDOW_MIN_BLOCKS
+#define HYENA_WINDOW_MIN_BLOCKS 1
+#endif
+constexpr int kWindowBlock = HYENA_WINDOW_BLOCK;
+
 template <typename T, int LH>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kWindowBlock, HYENA_WINDOW_MIN_BLOCKS)
     fir_window_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                       const float *__restrict__ h, T *__restrict__ y, const WindowParams p) {
   constexpr int VN = Vec<T>::N;

@@ -242,7 +242,7 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
 
 template <typename T, int LH>
 void launch_window_lh(const Problem &P, const WindowParams &wp, unsigned blocks, cudaStream_t s) {
-  hyena::cc::fir_window_kernel<T, LH><<<blocks, 256, 0, s>>>(
+  hyena::cc::fir_window_kernel<T, LH><<<blocks, hyena::cc::kWindowBlock, 0, s>>>(
       static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v), P.h,
       static_cast<T *>(P.y), wp);
 }
@@ -269,7 +269,7 @@ int launch_window(const Problem &P, cudaStream_t s) {
   wp.n_tb = (P.L + kWindowRows - 1) / kWindowRows;
   wp.cv = P.D / vec;
   const long long threads = wp.B * wp.n_tb * wp.cv;
-  const long long blocks = (threads + 255) / 256;
+  const long long blocks = (threads + hyena::cc::kWindowBlock - 1) / hyena::cc::kWindowBlock;
   if (blocks > std::numeric_limits<int32_t>::max()) return HYENA_ERR_UNSUPPORTED;
   if (P.dtype == HYENA_DTYPE_F32)
     launch_window_dispatch<float>(P, wp, static_cast<unsigned>(blocks), s);
