@@ -48,6 +48,8 @@ class OracleLib:
         lib.oracle_toeplitz_blocks_f64.restype = ctypes.c_int
         lib.oracle_block_conv_f64.argtypes = [_dp, i64, i64, i64, _dp, i64, _dp]
         lib.oracle_block_conv_f64.restype = ctypes.c_int
+        lib.oracle_gated_fir_bwd_f64.argtypes = [_dp] * 9 + [i64, i64, i64, i64, i64, ctypes.c_int]
+        lib.oracle_gated_fir_bwd_f64.restype = ctypes.c_int
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
         self.lib = lib
@@ -79,6 +81,26 @@ class OracleLib:
         if rc != 0:
             raise ValueError("oracle_gated_fir_f64 rejected its arguments (rc=%d)" % rc)
         return y[0] if squeeze else y
+
+    def gated_fir_bwd(self, q, k, v, h, dy, d_g: int, nthreads: int = 0):
+        """Gradients (dq, dk, dv, dh) of sum(dy * y) for y = gated_fir(q, k, v, h, d_g)."""
+        q, k, v, h, dy = _f64(q), _f64(k), _f64(v), _f64(h), _f64(dy)
+        squeeze = q.ndim == 2
+        if squeeze:
+            q, k, v, dy = q[None], k[None], v[None], dy[None]
+        B, L, D = q.shape
+        assert k.shape == q.shape and v.shape == q.shape and dy.shape == q.shape
+        assert h.ndim == 2 and h.shape[0] * d_g == D, "h must be [D // d_g, l_h]"
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        dh = np.empty_like(h)
+        rc = self.lib.oracle_gated_fir_bwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(h), _ptr(dy),
+                                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dh), B, L, D,
+                                               d_g, h.shape[1], nthreads)
+        if rc != 0:
+            raise ValueError("oracle_gated_fir_bwd_f64 rejected its arguments (rc=%d)" % rc)
+        if squeeze:
+            dq, dk, dv = dq[0], dk[0], dv[0]
+        return dq, dk, dv, dh
 
     def toeplitz_blocks(self, h, l_b: int, S: int) -> np.ndarray:
         """[S, l_b, l_b]: H[m][i][j] = h[m*l_b + i - j] inside [0, l_h), else 0."""
@@ -121,6 +143,10 @@ def gated_fir(q, k, v, h, d_g: int, nthreads: int = 0) -> np.ndarray:
 
 def toeplitz_blocks(h, l_b: int, S: int) -> np.ndarray:
     return default().toeplitz_blocks(h, l_b, S)
+
+
+def gated_fir_bwd(q, k, v, h, dy, d_g: int, nthreads: int = 0):
+    return default().gated_fir_bwd(q, k, v, h, dy, d_g, nthreads)
 
 
 def block_conv(h, x, l_b: int, S: int) -> np.ndarray:

@@ -136,3 +136,66 @@ int oracle_max_threads(void)
     return 1;
 #endif
 }
+
+/*
+ * Backward of the gated FIR (the gradients the page's Sec. 7 two-pass backward computes):
+ * given dy = dL/dy for y = q * z, z = h_g conv x, x = k * v,
+ *
+ *   dq[b,t,c] = dy[b,t,c] * z[b,t,c]
+ *   dz[b,t,c] = dy[b,t,c] * q[b,t,c]
+ *   dx[b,t,c] = sum_{j=0}^{min(l_h-1, L-1-t)} h[c/d_g, j] * dz[b,t+j,c]   (transposed Toeplitz)
+ *   dk = dx * v,  dv = dx * k
+ *   dh[g, j]  = sum_{b, t >= j, c in g} dz[b,t,c] * x[b,t-j,c]
+ *
+ * written straight from those sums (no blocking).  dh: [D / d_g, l_h].
+ */
+int oracle_gated_fir_bwd_f64(const double *q, const double *k, const double *v, const double *h,
+                             const double *dy, double *dq, double *dk, double *dv, double *dh,
+                             int64_t B, int64_t L, int64_t D, int64_t d_g, int64_t l_h,
+                             int nthreads)
+{
+    if (!q || !k || !v || !h || !dy || !dq || !dk || !dv || !dh) return ORACLE_BAD_ARG;
+    if (B < 0 || L < 0 || D < 1 || d_g < 1 || D % d_g != 0 || l_h < 1) return ORACLE_BAD_ARG;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    const int64_t rows = B * L;
+    #pragma omp parallel for schedule(static)
+    for (int64_t row = 0; row < rows; ++row) {
+        const int64_t b = row / L;
+        const int64_t t = row % L;
+        for (int64_t c = 0; c < D; ++c) {
+            const double *hg = h + (c / d_g) * l_h;
+            double z = 0.0, dx = 0.0;
+            for (int64_t j = 0; j < l_h && j <= t; ++j) {
+                const int64_t src = (b * L + (t - j)) * D + c;
+                z += hg[j] * (k[src] * v[src]);
+            }
+            for (int64_t j = 0; j < l_h && t + j < L; ++j) {
+                const int64_t src = (b * L + (t + j)) * D + c;
+                dx += hg[j] * (dy[src] * q[src]);
+            }
+            const int64_t e = row * D + c;
+            dq[e] = dy[e] * z;
+            dk[e] = dx * v[e];
+            dv[e] = dx * k[e];
+        }
+    }
+    const int64_t G = D / d_g;
+    #pragma omp parallel for schedule(static)
+    for (int64_t gj = 0; gj < G * l_h; ++gj) {
+        const int64_t g = gj / l_h, j = gj % l_h;
+        double s = 0.0;
+        for (int64_t b = 0; b < B; ++b)
+            for (int64_t t = j; t < L; ++t)
+                for (int64_t c = g * d_g; c < (g + 1) * d_g; ++c) {
+                    const int64_t e = (b * L + t) * D + c;
+                    const int64_t src = (b * L + (t - j)) * D + c;
+                    s += (dy[e] * q[e]) * (k[src] * v[src]);
+                }
+        dh[gj] = s;
+    }
+    return ORACLE_OK;
+}

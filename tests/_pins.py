@@ -304,4 +304,60 @@ def pin_index_difference_tile(o):
         assert np.array_equal(tile, o.toeplitz_blocks(h, chunk, 1)[0]), (l_h, chunk)
 
 
+# ---------------------------------------------------------------- backward (Sec. 7)
+
+def _bwd_case(seed, B=2, L=23, D=6, d_g=3, l_h=5):
+    rng = np.random.default_rng(seed)
+    q, k, v, dy = (_rand(rng, B, L, D) for _ in range(4))
+    return q, k, v, _rand(rng, D // d_g, l_h), dy, d_g
+
+
+def pin_bwd_directional_derivatives(o):
+    """y is linear in each of q, k, v and h separately, so for sum(dy * y) the central
+    difference with step 1 along any direction is the directional derivative, exactly: it
+    must equal <gradient, direction> for every one of the four gradients."""
+    q, k, v, h, dy, d_g = _bwd_case(31)
+    dq, dk, dv, dh = o.gated_fir_bwd(q, k, v, h, dy, d_g)
+    rng = np.random.default_rng(32)
+    f = lambda q_, k_, v_, h_: float(np.sum(dy * o.gated_fir(q_, k_, v_, h_, d_g)))
+    for name, grad in (("q", dq), ("k", dk), ("v", dv), ("h", dh)):
+        args = {"q": q, "k": k, "v": v, "h": h}
+        d = rng.standard_normal(args[name].shape)
+        up, dn = dict(args), dict(args)
+        up[name] = args[name] + d
+        dn[name] = args[name] - d
+        num = (f(**{a + "_": up[a] for a in up}) - f(**{a + "_": dn[a] for a in dn})) / 2
+        assert abs(num - float(np.sum(grad * d))) <= 1e-9 * (1 + abs(num)), name
+
+
+def pin_bwd_adjoint_toeplitz(o):
+    """dk = v * T^T (q * dy) with T the dense lower-triangular Toeplitz matrix (scipy)."""
+    q, k, v, h, dy, d_g = _bwd_case(33, B=1, L=19, D=4, d_g=2, l_h=6)
+    dq, dk, dv, dh = o.gated_fir_bwd(q, k, v, h, dy, d_g)
+    L = q.shape[1]
+    for c in range(q.shape[2]):
+        col = np.zeros(L)
+        col[:h.shape[1]] = h[c // d_g]
+        T = scipy.linalg.toeplitz(col, np.zeros(L))
+        dx = T.T @ (q[0, :, c] * dy[0, :, c])
+        _close(dk[0, :, c], dx * v[0, :, c])
+        _close(dv[0, :, c], dx * k[0, :, c])
+        z = T @ (k[0, :, c] * v[0, :, c])
+        _close(dq[0, :, c], dy[0, :, c] * z)
+
+
+def pin_bwd_filter_gradient_correlation(o):
+    """dh[g, j] = sum over sequences and the group's channels of the cross-correlation of
+    dz = q dy with x = k v at lag j (scipy.signal.correlate)."""
+    q, k, v, h, dy, d_g = _bwd_case(34, B=2, L=30, D=6, d_g=3, l_h=7)
+    _, _, _, dh = o.gated_fir_bwd(q, k, v, h, dy, d_g)
+    B, L, D = q.shape
+    ref = np.zeros_like(h)
+    for b in range(B):
+        for c in range(D):
+            cc = scipy.signal.correlate(q[b, :, c] * dy[b, :, c], k[b, :, c] * v[b, :, c], "full")
+            ref[c // d_g] += cc[L - 1:L - 1 + h.shape[1]]
+    _close(dh, ref, rtol=1e-11, atol=1e-11)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
