@@ -19,7 +19,8 @@ from ._native import (HYENA_ALGO_AUTO, HYENA_ALGO_DIRECT, HYENA_ALGO_TENSOR, HYE
 
 __all__ = [
     "hyena_conv_fwd", "hyena_conv_fwd_f32", "hyena_conv_fwd_ex", "hyena_select_algo",
-    "hyena_build_toeplitz", "hyena_device_status", "hyena_status_string", "hyena_abi_version",
+    "hyena_build_toeplitz", "hyena_conv_bwd", "hyena_conv_bwd_workspace_bytes",
+    "hyena_device_status", "hyena_status_string", "hyena_abi_version",
     "HyenaError", "HYENA_ALGO_AUTO", "HYENA_ALGO_TENSOR", "HYENA_ALGO_WINDOW",
     "HYENA_ALGO_DIRECT", "HYENA_DTYPE_BF16", "HYENA_DTYPE_F32", "HYENA_DEVICE_TIMEOUT",
     "HYENA_DEVICE_F16_RANGE", "ALGO_NAMES", "hyena_conv_fwd_from_host",
@@ -127,6 +128,56 @@ def hyena_select_algo(B, L, D, d_g, l_h, l_b, dtype=HYENA_DTYPE_BF16, ptrs=(16, 
     if rc < 0:
         raise HyenaError("hyena_select_algo", -rc)
     return rc
+
+
+def hyena_conv_bwd_workspace_bytes(B, L, D, d_g, l_h):
+    """Host-only: device workspace bytes hyena_conv_bwd needs for this shape."""
+    n = _native.lib().hyena_conv_bwd_workspace_bytes(B, L, D, d_g, l_h)
+    if n < 0:
+        raise HyenaError("hyena_conv_bwd_workspace_bytes", -n)
+    return n
+
+
+def hyena_conv_bwd(q, k, v, h, dy, d_g, l_b, workspace=None, grads=None, stream=None):
+    """Backward of the gated FIR; returns (dq, dk, dv, dh).
+
+    q, k, v, dy: CUDA [B, L, D], one dtype (bf16 or fp32).  h: CUDA fp32 [D // d_g, l_h].
+    dq, dk, dv come back in the dtype of q, dh in fp32 [D // d_g, l_h] (overwritten, not
+    accumulated).  ``workspace``: optional CUDA uint8 tensor of at least
+    hyena_conv_bwd_workspace_bytes() bytes (allocated here from torch when omitted).
+    ``grads``: optional preallocated (dq, dk, dv, dh).
+    """
+    torch = _torch()
+    _check(q, k, v, h, d_g, None)
+    if (not isinstance(dy, torch.Tensor) or not dy.is_cuda or dy.shape != q.shape
+            or dy.dtype != q.dtype or not dy.is_contiguous()):
+        raise ValueError("dy must be a contiguous CUDA tensor like q")
+    B, L, D = q.shape
+    l_h = h.shape[1]
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q),
+                 torch.empty_like(h))
+    dq, dk, dv, dh = grads
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        if (t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda
+                or not t.is_contiguous()):
+            raise ValueError("%s must be a contiguous CUDA tensor like q" % name)
+    if dh.shape != h.shape or dh.dtype != torch.float32 or not dh.is_cuda \
+            or not dh.is_contiguous():
+        raise ValueError("dh must be a contiguous CUDA float32 tensor like h")
+    need = hyena_conv_bwd_workspace_bytes(B, L, D, d_g, l_h)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = _native.lib().hyena_conv_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), h.data_ptr(),
+                                      dy.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                      dv.data_ptr(), dh.data_ptr(), B, L, D, d_g, l_h, l_b,
+                                      _dtype_code(q), workspace.data_ptr(), ws_bytes,
+                                      _stream(stream))
+    _native.check("hyena_conv_bwd", rc)
+    return dq, dk, dv, dh
 
 
 def hyena_build_toeplitz(h, l_b, stream=None):

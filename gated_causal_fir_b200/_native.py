@@ -43,6 +43,9 @@ SIGNATURES = {
                                  _i32, _i32, _vp]),
     "hyena_select_algo": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32,
                                  _i32]),
+    "hyena_conv_bwd_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32, _i32]),
+    "hyena_conv_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                              _i32, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp]),
     "hyena_build_toeplitz": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]),
     "hyena_device_status": (_i32, [ctypes.POINTER(ctypes.c_uint), _i32]),
     "hyena_status_string": (ctypes.c_char_p, [_i32]),

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "hyena_conv.h"
+#include "fir_bwd.cuh"
 #include "fir_cuda_core.cuh"
 #include "fir_tc.cuh"
 
@@ -28,6 +29,9 @@ using hyena::cc::WindowParams;
 
 
 constexpr int kMaxDevices = 64;
+// Shared memory of the dh partial kernel at 64 channels per piece: dz rows + x window.
+constexpr int kDhSmemMax =
+    (2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (64 + 1) * static_cast<int>(sizeof(float));
 constexpr int kMaxWindowTaps = 16;
 #ifndef HYENA_WINDOW_ROWS
 #define HYENA_WINDOW_ROWS 128
@@ -60,6 +64,12 @@ int current_device(DeviceState *&ds) {
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  hyena::tc::kSmemBytes);
+    const void *dh_kernels[] = {
+        reinterpret_cast<const void *>(hyena::bwd::fir_bwd_dh_partial_kernel<float>),
+        reinterpret_cast<const void *>(hyena::bwd::fir_bwd_dh_partial_kernel<__nv_bfloat16>)};
+    for (const void *k : dh_kernels)
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kDhSmemMax);
 
     d->err = e;
   });
@@ -93,6 +103,7 @@ struct Problem {
   int d_g, l_h, l_b, dtype;
   int64_t elem() const { return dtype == HYENA_DTYPE_F32 ? 4 : 2; }
   int64_t numel() const { return B * L * D; }
+  int64_t G() const { return D / d_g; }
 };
 
 constexpr int kEmpty = -1;  // internal: valid problem with nothing to compute
@@ -322,6 +333,96 @@ int run(const Problem &P, int algo, cudaStream_t s) {
   return launch_direct(P, s);
 }
 
+// ------------------------------------------------------------------------------ backward
+struct BwdPlan {
+  int cp, npieces, nchunk;
+  int64_t partial_floats;
+};
+
+BwdPlan bwd_plan(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
+  BwdPlan b;
+  b.cp = hyena::bwd::dh_piece(d_g);
+  b.npieces = static_cast<int>(D / b.cp);
+  b.nchunk = static_cast<int>((L + hyena::bwd::kDhRows - 1) / hyena::bwd::kDhRows);
+  b.partial_floats = B * b.nchunk * static_cast<int64_t>(b.npieces) * l_h;
+  return b;
+}
+
+int64_t bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
+  return (bwd_plan(B, L, D, d_g, l_h).partial_floats * 4 + 255) / 256 * 256;
+}
+
+template <typename T>
+int launch_bwd_cuda_core(const Problem &P, const void *dy, void *dk, void *dv, float *dh,
+                         float *partial, cudaStream_t s) {
+  DeviceState *ds = nullptr;
+  if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
+  const long long n = P.numel();
+  long long blocks = (n + 255) / 256;
+  const long long cap = static_cast<long long>(ds->sm_count) * 16;
+  if (blocks > cap) blocks = cap;
+  hyena::bwd::fir_bwd_dx_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v), P.h,
+      static_cast<const T *>(dy), static_cast<T *>(dk), static_cast<T *>(dv), P.B, P.L, P.D,
+      P.d_g, P.l_h);
+  if (cudaGetLastError() != cudaSuccess) return HYENA_ERR_CUDA;
+  const BwdPlan b = bwd_plan(P.B, P.L, P.D, P.d_g, P.l_h);
+  if (b.nchunk > 2147483647 || P.B > 65535 || b.npieces > 65535) return HYENA_ERR_UNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>(b.nchunk), static_cast<unsigned>(b.npieces),
+                  static_cast<unsigned>(P.B));
+  const int smem = (2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (b.cp + 1) * 4;
+  hyena::bwd::fir_bwd_dh_partial_kernel<T><<<grid, hyena::bwd::kDhTaps, smem, s>>>(
+      static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v),
+      static_cast<const T *>(dy), partial, P.L, P.D, P.l_h, b.cp);
+  if (cudaGetLastError() != cudaSuccess) return HYENA_ERR_CUDA;
+  const long long gn = P.G() * P.l_h;
+  long long rblocks = (gn + 255) / 256;
+  if (rblocks > cap) rblocks = cap;
+  hyena::bwd::fir_bwd_dh_reduce_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
+      partial, dh, static_cast<int>(P.B), b.nchunk, b.npieces, P.d_g / b.cp,
+      static_cast<int>(P.G()), P.l_h);
+  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+int run_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv, float *dh,
+            void *workspace, size_t workspace_bytes, cudaStream_t s) {
+  const int rc = validate(P);  // q, k, v, h and dq (in the place of y)
+  if (rc == kEmpty) {  // no tokens: dh is an empty sum
+    if (!dh || !aligned(dh, 4)) return HYENA_ERR_INVALID_ARG;
+    return cudaMemsetAsync(dh, 0, static_cast<size_t>(P.G() * P.l_h) * 4, s) == cudaSuccess
+               ? HYENA_OK
+               : HYENA_ERR_CUDA;
+  }
+  if (rc != HYENA_OK) return rc;
+  if (!dy || !dk || !dv || !dh) return HYENA_ERR_INVALID_ARG;
+  const uintptr_t es = static_cast<uintptr_t>(P.elem());
+  if (!aligned(dy, es) || !aligned(dk, es) || !aligned(dv, es) || !aligned(dh, 4) ||
+      !aligned(workspace, 16))
+    return HYENA_ERR_MISALIGNED;
+  const int64_t bytes = P.numel() * P.elem();
+  const void *ins[] = {P.q, P.k, P.v, dy};
+  const void *outs[] = {dq, dk, dv};
+  for (int i = 0; i < 3; ++i) {
+    for (const void *in : ins)
+      if (overlaps(outs[i], in, bytes)) return HYENA_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlaps(outs[i], outs[j], bytes)) return HYENA_ERR_INVALID_ARG;
+  }
+  if (!workspace ||
+      static_cast<int64_t>(workspace_bytes) < bwd_workspace_bytes(P.B, P.L, P.D, P.d_g, P.l_h))
+    return HYENA_ERR_INVALID_ARG;
+  // dq = dy * (h conv (k v)): the forward with dy in the place of q.
+  Problem F = P;
+  F.q = dy;
+  F.y = dq;
+  int r = run(F, HYENA_ALGO_AUTO, s);
+  if (r != HYENA_OK) return r;
+  if (P.dtype == HYENA_DTYPE_F32)
+    return launch_bwd_cuda_core<float>(P, dy, dk, dv, dh, static_cast<float *>(workspace), s);
+  return launch_bwd_cuda_core<__nv_bfloat16>(P, dy, dk, dv, dh, static_cast<float *>(workspace),
+                                             s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -353,6 +454,19 @@ int hyena_select_algo(const void *q, const void *k, const void *v, const float *
   const int rc = validate(P);
   if (rc != HYENA_OK && rc != kEmpty) return -rc;
   return select_algo(P);
+}
+
+int64_t hyena_conv_bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
+  if (B < 0 || L < 0 || D < 1 || d_g < 1 || D % d_g != 0 || l_h < 1) return -HYENA_ERR_INVALID_ARG;
+  return bwd_workspace_bytes(B, L, D, d_g, l_h);
+}
+
+int hyena_conv_bwd(const void *q, const void *k, const void *v, const float *h, const void *dy,
+                   void *dq, void *dk, void *dv, float *dh, int64_t B, int64_t L, int64_t D,
+                   int d_g, int l_h, int l_b, int dtype, void *workspace, size_t workspace_bytes,
+                   cudaStream_t stream) {
+  const Problem P{q, k, v, h, dq, B, L, D, d_g, l_h, l_b, dtype};
+  return run_bwd(P, dy, dq, dk, dv, dh, workspace, workspace_bytes, stream);
 }
 
 int hyena_build_toeplitz(const float *h, float *H0, float *H1, float *H2_or_null, int G,

@@ -114,6 +114,32 @@ def make_inputs(wl: Workload, device="cpu", seed=None, l_slice: int = 0):
     return q, k, v, h
 
 
+def make_grad(wl: Workload, device="cpu", seed=None):
+    """Upstream gradient dy [B, L, D] in the workload's dtype, standard normal, seeded apart
+    from the forward inputs (seed + 7919)."""
+    seed = (wl.seed if seed is None else seed) + 7919
+    gen = torch.Generator(device=device).manual_seed(seed)
+    return torch.randn((wl.B, wl.L, wl.D), generator=gen, device=device).to(
+        torch_dtype(wl.dtype))
+
+
+def make_integer_inputs(wl: Workload, device="cpu", seed=None):
+    """q, k, v, dy with integer values in [-2, 2] and h with integers in [-3, 3], seeded.
+
+    Every product and partial sum of the forward and backward is then an integer well inside
+    the fp16/fp32 exact range (for B * L * d_g * 16 < 2**24), so any correct summation order
+    gives the exact result and the GPU path must match the oracle bit for bit.
+    """
+    seed = wl.seed if seed is None else seed
+    gen = torch.Generator(device=device).manual_seed(seed + 104729)
+    shape = (wl.B, wl.L, wl.D)
+    dt = torch_dtype(wl.dtype)
+    q, k, v, dy = (torch.randint(-2, 3, shape, generator=gen, device=device).to(dt)
+                   for _ in range(4))
+    h = torch.randint(-3, 4, (wl.G, wl.l_h), generator=gen, device=device).to(torch.float32)
+    return q, k, v, dy, h
+
+
 def custom(name="custom", B=1, L=256, D=128, d_g=64, l_h=16, l_b=16, dtype="bf16", filt="se",
            seed=7) -> Workload:
     """A workload outside the table (edge cases in the tests)."""

@@ -28,6 +28,7 @@
 #ifndef HYENA_CONV_H
 #define HYENA_CONV_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -100,6 +101,38 @@ int hyena_conv_fwd_ex(const void *q, const void *k, const void *v, const float *
 int hyena_select_algo(const void *q, const void *k, const void *v, const float *h,
                       const void *y, int64_t B, int64_t L, int64_t D, int d_g, int l_h,
                       int l_b, int dtype);
+
+/*
+ * Host-only: the bytes of device workspace hyena_conv_bwd needs for this shape (a multiple of
+ * 256; 4 bytes per partial filter gradient, one partial per sequence, 64-step chunk,
+ * channel piece and tap), or minus HYENA_ERR_INVALID_ARG for a bad shape.  Touches no device.
+ */
+int64_t hyena_conv_bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h);
+
+/*
+ * Backward of the gated FIR (the gradients of the two-pass backward of page 04, Sec. 7).  For
+ * y = q * z, z = h_g conv x, x = k * v and the upstream gradient dy = dLoss/dy:
+ *
+ *     dq[b,t,c] = dy[b,t,c] * z[b,t,c]
+ *     dx[b,t,c] = sum_{j=0}^{min(l_h-1, L-1-t)} h[c / d_g][j] * q[b,t+j,c] * dy[b,t+j,c]
+ *     dk = dx * v,   dv = dx * k
+ *     dh[g][j]  = sum_{b, t >= j, c in group g} q[b,t,c] dy[b,t,c] * k[b,t-j,c] v[b,t-j,c]
+ *
+ * q, k, v, dy, dq, dk, dv: DEVICE [B, L, D] tensors of `dtype`, layout as the forward.
+ * h: DEVICE fp32 [D / d_g, l_h].  dh: DEVICE fp32 [D / d_g, l_h], overwritten (not
+ * accumulated into).  dq is computed by the forward kernels (HYENA_ALGO_AUTO) with dy in the
+ * place of q, so the forward's shape rules (l_h <= 2*l_b) apply; dk, dv and dh by CUDA-core
+ * kernels in fp32.  dh is summed in a fixed order: results are deterministic.
+ * workspace: DEVICE scratch of at least hyena_conv_bwd_workspace_bytes() bytes, 16-byte
+ * aligned, owned by the caller, unused after the queued work ends.  Outputs must not overlap
+ * each other or an input.  B == 0 or L == 0 zeroes dh and launches nothing else.
+ * Errors: as the forward, plus HYENA_ERR_INVALID_ARG for a null dy/dk/dv/dh or a workspace
+ * that is null or too small, and HYENA_ERR_MISALIGNED for a misaligned dy/dk/dv/dh/workspace.
+ */
+int hyena_conv_bwd(const void *q, const void *k, const void *v, const float *h, const void *dy,
+                   void *dq, void *dk, void *dv, float *dh, int64_t B, int64_t L, int64_t D,
+                   int d_g, int l_h, int l_b, int dtype, void *workspace,
+                   size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * The l_b x l_b sub-blocks of the lower-triangular Toeplitz matrix of every group
