@@ -30,6 +30,8 @@ ALGO_NAMES = {HYENA_ALGO_AUTO: "auto", HYENA_ALGO_TENSOR: "tensor", HYENA_ALGO_W
 HYENA_DEVICE_TIMEOUT = 1
 HYENA_DEVICE_F16_RANGE = 2
 
+HYENA_BWD_STATIC_SCRATCH_BYTES = 8 << 20
+
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
 _i32 = ctypes.c_int
@@ -46,6 +48,8 @@ SIGNATURES = {
     "hyena_conv_bwd_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32, _i32]),
     "hyena_conv_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                               _i32, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp]),
+    "hyena_conv_bwd_static_scratch": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
+                                             _i64, _i64, _i32, _i32, _i32, _i32, _vp]),
     "hyena_build_toeplitz": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]),
     "hyena_device_status": (_i32, [ctypes.POINTER(ctypes.c_uint), _i32]),
     "hyena_status_string": (ctypes.c_char_p, [_i32]),

@@ -425,6 +425,37 @@ int run_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv, floa
 
 }  // namespace
 
+// Partials of hyena_conv_bwd_static_scratch: a fixed device array instead of a caller workspace,
+// for callers that cannot allocate device memory (see the header).  Every partial the dh kernel
+// reads is written earlier in the same call, so nothing in it has to start at zero.
+static __device__ __align__(256) float g_bwd_static_scratch[HYENA_BWD_STATIC_SCRATCH_BYTES / 4];
+
+namespace {
+
+struct StaticScratch {
+  std::once_flag once;
+  void *ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+StaticScratch g_static_scratch[kMaxDevices];
+
+// The current device's address of g_bwd_static_scratch, looked up once per device (with that
+// device current) on the first call.
+int static_scratch(void *&ptr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYENA_ERR_CUDA;
+  StaticScratch *sc = &g_static_scratch[dev];
+  std::call_once(sc->once, [sc]() {
+    sc->err = cudaGetSymbolAddress(&sc->ptr, g_bwd_static_scratch);
+    if (sc->err == cudaSuccess && !sc->ptr) sc->err = cudaErrorInvalidSymbol;
+  });
+  if (sc->err != cudaSuccess) return HYENA_ERR_CUDA;
+  ptr = sc->ptr;
+  return HYENA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int hyena_conv_fwd(const void *q, const void *k, const void *v, const float *h, void *y,
@@ -467,6 +498,21 @@ int hyena_conv_bwd(const void *q, const void *k, const void *v, const float *h, 
                    cudaStream_t stream) {
   const Problem P{q, k, v, h, dq, B, L, D, d_g, l_h, l_b, dtype};
   return run_bwd(P, dy, dq, dk, dv, dh, workspace, workspace_bytes, stream);
+}
+
+int hyena_conv_bwd_static_scratch(const void *q, const void *k, const void *v, const float *h,
+                                  const void *dy, void *dq, void *dk, void *dv, float *dh,
+                                  int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                                  int dtype, cudaStream_t stream) {
+  const Problem P{q, k, v, h, dq, B, L, D, d_g, l_h, l_b, dtype};
+  const int rc = validate(P);
+  if (rc != HYENA_OK && rc != kEmpty) return rc;
+  if (rc == HYENA_OK &&
+      bwd_workspace_bytes(B, L, D, d_g, l_h) > static_cast<int64_t>(HYENA_BWD_STATIC_SCRATCH_BYTES))
+    return HYENA_ERR_UNSUPPORTED;
+  void *ws = nullptr;
+  if (static_scratch(ws) != HYENA_OK) return HYENA_ERR_CUDA;
+  return run_bwd(P, dy, dq, dk, dv, dh, ws, HYENA_BWD_STATIC_SCRATCH_BYTES, stream);
 }
 
 int hyena_build_toeplitz(const float *h, float *H0, float *H1, float *H2_or_null, int G,

@@ -134,6 +134,30 @@ int hyena_conv_bwd(const void *q, const void *k, const void *v, const float *h, 
                    int d_g, int l_h, int l_b, int dtype, void *workspace,
                    size_t workspace_bytes, cudaStream_t stream);
 
+/* Size of the fixed device scratch behind hyena_conv_bwd_static_scratch (8 MiB per device). */
+#define HYENA_BWD_STATIC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * hyena_conv_bwd without a workspace argument.  The pages have no counterpart: this is a
+ * convenience of this library.  It is for callers that cannot hand over device memory, such as
+ * a C host program with no device allocator of its own, or a runtime that reserves all device
+ * memory at start-up and allows no allocation afterwards (cudaMalloc also synchronises the
+ * device, which a latency-bound loop cannot afford).  The dh partials go to a fixed array of
+ * HYENA_BWD_STATIC_SCRATCH_BYTES in the library's device memory (one per device); this call
+ * allocates nothing.  Arguments, results and errors are those of hyena_conv_bwd, plus:
+ *   - HYENA_ERR_UNSUPPORTED, with nothing queued, when hyena_conv_bwd_workspace_bytes() of the
+ *     shape exceeds HYENA_BWD_STATIC_SCRATCH_BYTES (e.g. the D = 4096, d_g = 64, l_h = 128
+ *     shape above B * L = 16384 tokens); use hyena_conv_bwd with a workspace there.
+ *   - The first call on each device looks up the array's address (cudaGetSymbolAddress) with
+ *     that device current; make that first call before any stream capture.
+ *   - Calls that overlap in time on one device (different streams, or threads) share the array
+ *     and race: serialise them.  Nothing in the array has to start at zero.
+ */
+int hyena_conv_bwd_static_scratch(const void *q, const void *k, const void *v, const float *h,
+                                  const void *dy, void *dq, void *dk, void *dv, float *dh,
+                                  int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                                  int dtype, cudaStream_t stream);
+
 /*
  * The l_b x l_b sub-blocks of the lower-triangular Toeplitz matrix of every group
  * (page 04, Sec. 2; index rule of the Sec. 3 worked example):

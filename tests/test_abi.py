@@ -115,3 +115,24 @@ def test_python_binding_rejects_cpu_tensors():
     h = torch.zeros(1, 4)
     with pytest.raises(TypeError):
         g.hyena_conv_fwd(q, q, q, h, d_g=64, l_b=4)
+
+
+def test_bwd_workspace_bytes(lib):
+    # D = 4096, d_g = 64 (pieces of 64 channels), l_h = 128, 8192 tokens: 128 chunks x 64 x 128
+    assert lib.hyena_conv_bwd_workspace_bytes(1, 8192, 4096, 64, 128) == 128 * 64 * 128 * 4
+    assert lib.hyena_conv_bwd_workspace_bytes(1, 8192, 4096, 63, 128) == -1
+    assert lib.hyena_conv_bwd_workspace_bytes(0, 8192, 4096, 64, 128) == 0
+    assert lib.hyena_conv_bwd_workspace_bytes(1, 1, 6, 6, 5) == 256  # rounded up
+
+
+def test_bwd_static_scratch_rejects_oversize_on_host(lib):
+    # 16448 tokens of the D = 4096, d_g = 64, l_h = 128 shape need 257 chunks of partials
+    # (8.4 MB > 8 MiB): rejected before any device work.  Distinct aligned stand-in addresses.
+    B, L, D = 1, 16448, 4096
+    n = B * L * D * 2 + 4096
+    p = [4096 + i * n for i in range(9)]
+    assert lib.hyena_conv_bwd_workspace_bytes(B, L, D, 64, 128) > _native.HYENA_BWD_STATIC_SCRATCH_BYTES
+    rc = lib.hyena_conv_bwd_static_scratch(*p, B, L, D, 64, 128, 64, 0, None)
+    assert rc == _native.HYENA_ERR_UNSUPPORTED
+    rc = lib.hyena_conv_bwd_static_scratch(*p, B, L, D, 63, 128, 64, 0, None)
+    assert rc == _native.HYENA_ERR_INVALID_ARG
