@@ -49,6 +49,8 @@ def parse():
                    help="target CPU time of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--bwd-steps", type=int, default=200,
+                   help="timed steps of the backward (hyena_conv_bwd); 0 skips it")
     return p.parse_args()
 
 
@@ -197,6 +199,67 @@ def run_reference(args, wl, rank, world):
     del torch
 
 
+def time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind):
+    """The backward (hyena_conv_bwd: dq, dk, dv, dh) over the same rotating input sets, timed
+    like the forward: CUDA events on the launching stream, max over ranks.
+
+    Algorithmic bytes per step: read q, k, v, dy, write dq, dk, dv (7 tensors of B L D
+    elements), plus h read and dh written (G l_h fp32 each); the workspace of partials is
+    overhead, not counted."""
+    import torch
+    from gated_causal_fir_b200.workloads import make_grad
+    code = g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    ws_bytes = g.hyena_conv_bwd_workspace_bytes(wl.B, wl.L, wl.D, wl.d_g, wl.l_h)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    bufs = []
+    for n, (q, k, v, h, _) in enumerate(sets):
+        dy = make_grad(wl, device=dev, seed=wl.seed + 977 * n)
+        dq, dk, dv, dh = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q),
+                          torch.empty_like(h))
+        g.hyena_conv_bwd(q, k, v, h, dy, wl.d_g, wl.l_b, workspace=ws,
+                         grads=(dq, dk, dv, dh), stream=stream)  # binding checks, once
+        bufs.append((q, k, v, h, dy, dq, dk, dv, dh))
+    cfn = _native.lib().hyena_conv_bwd
+    algo = g.hyena_select_bwd_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, code)
+    kernels = (["fir_tc_bwd_kernel", "fir_bwd_tc_reduce_kernel"] if algo == g.HYENA_ALGO_TENSOR
+               else ["forward kernel (dq)", "fir_bwd_dx_kernel", "fir_bwd_dh_partial_kernel",
+                     "fir_bwd_dh_reduce_kernel"])
+    cargs = [tuple(t.data_ptr() for t in b) + (wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, code,
+                                                ws.data_ptr(), ws.numel(), sh) for b in bufs]
+
+    def launch(i):
+        rc = cfn(*cargs[i % 3])
+        if rc != 0:
+            raise _native.HyenaError("hyena_conv_bwd", rc)
+
+    for i in range(max(3, args.warmup)):
+        launch(i)
+    torch.cuda.synchronize()
+    K = args.bwd_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(K):
+        launch(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = D.max_over_ranks(e0.elapsed_time(e1), device=dev) / K
+    world = D.env_world()[2]
+    elem = 4 if wl.dtype == "f32" else 2
+    nbytes = 7 * wl.B * wl.L * wl.D * elem + 2 * wl.G * wl.l_h * 4
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {"metric": "Hyena-MR bwd tokens/s (dq, dk, dv, dh)",
+            "value": world * wl.tokens / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+            "steps": K, "gpu_launches": len(kernels) * K, "kernels": kernels,
+            "algo": g.ALGO_NAMES[algo],
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "algorithmic_bytes_per_step": nbytes,
+                         "peak_source": peak_kind,
+                         "note": "whole backward (all its kernels) per step"}}
+
+
 def workload_config(wl):
     return {"workload": wl.describe(), "B": wl.B, "L": wl.L, "D": wl.D, "d_g": wl.d_g,
             "l_h": wl.l_h, "l_b": wl.l_b, "io_dtype": wl.dtype, "filters": wl.filt,
@@ -300,6 +363,11 @@ def main():
                "d2h_bytes_per_step": yh.numel() * yh.element_size(),
                "steps": args.e2e_steps, "api": "hyena_conv_fwd_from_host"}
 
+    bwd = None
+    if args.bwd_steps > 0:
+        peak, peak_kind = measured_peak_hbm()
+        bwd = time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind)
+
     cpu, parity = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu, y_ref = cpu_baseline(wl, *sets[0][:4], target_s=args.cpu_seconds)
@@ -335,7 +403,7 @@ def main():
                          "mean_launch_us": 1e3 * mean_launch_ms, "kernel": kernel},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K,
             "clocks": clocks.summary(t_wall0, t_wall1),
-            "kernel_algo": g.ALGO_NAMES[algo], "device_status": status, "parity": parity,
+            "backward": bwd, "kernel_algo": g.ALGO_NAMES[algo], "device_status": status, "parity": parity,
             "wall_s_timed_region": t_wall1 - t_wall0,
         }
         print(json.dumps(line), flush=True)

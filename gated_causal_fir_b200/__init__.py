@@ -19,7 +19,8 @@ from ._native import (HYENA_ALGO_AUTO, HYENA_ALGO_DIRECT, HYENA_ALGO_TENSOR, HYE
 
 __all__ = [
     "hyena_conv_fwd", "hyena_conv_fwd_f32", "hyena_conv_fwd_ex", "hyena_select_algo",
-    "hyena_build_toeplitz", "hyena_conv_bwd", "hyena_conv_bwd_workspace_bytes",
+    "hyena_build_toeplitz", "hyena_conv_bwd", "hyena_conv_bwd_ex", "hyena_select_bwd_algo",
+    "hyena_conv_bwd_workspace_bytes",
     "hyena_device_status", "hyena_status_string", "hyena_abi_version",
     "HyenaError", "HYENA_ALGO_AUTO", "HYENA_ALGO_TENSOR", "HYENA_ALGO_WINDOW",
     "HYENA_ALGO_DIRECT", "HYENA_DTYPE_BF16", "HYENA_DTYPE_F32", "HYENA_DEVICE_TIMEOUT",
@@ -139,7 +140,25 @@ def hyena_conv_bwd_workspace_bytes(B, L, D, d_g, l_h):
 
 
 def hyena_conv_bwd(q, k, v, h, dy, d_g, l_b, workspace=None, grads=None, stream=None):
-    """Backward of the gated FIR; returns (dq, dk, dv, dh).
+    """Backward, fastest supported algorithm (C: hyena_conv_bwd); see hyena_conv_bwd_ex."""
+    return hyena_conv_bwd_ex(q, k, v, h, dy, d_g, l_b, HYENA_ALGO_AUTO, workspace, grads,
+                             stream)
+
+
+def hyena_select_bwd_algo(B, L, D, d_g, l_h, l_b, dtype=HYENA_DTYPE_BF16):
+    """Host-only: the backward algorithm AUTO would run for distinct 16-byte aligned buffers."""
+    n = B * L * D * (4 if dtype == HYENA_DTYPE_F32 else 2)
+    p = [16 + i * (n + 64) for i in range(8)]
+    rc = _native.lib().hyena_select_bwd_algo(*p, B, L, D, d_g, l_h, l_b, dtype)
+    if rc < 0:
+        raise HyenaError("hyena_select_bwd_algo", -rc)
+    return rc
+
+
+def hyena_conv_bwd_ex(q, k, v, h, dy, d_g, l_b, algo=HYENA_ALGO_AUTO, workspace=None,
+                      grads=None, stream=None):
+    """Backward of the gated FIR with the algorithm chosen by the caller; returns
+    (dq, dk, dv, dh).
 
     q, k, v, dy: CUDA [B, L, D], one dtype (bf16 or fp32).  h: CUDA fp32 [D // d_g, l_h].
     dq, dk, dv come back in the dtype of q, dh in fp32 [D // d_g, l_h] (overwritten, not
@@ -171,12 +190,12 @@ def hyena_conv_bwd(q, k, v, h, dy, d_g, l_b, workspace=None, grads=None, stream=
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
-    rc = _native.lib().hyena_conv_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), h.data_ptr(),
-                                      dy.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                                      dv.data_ptr(), dh.data_ptr(), B, L, D, d_g, l_h, l_b,
-                                      _dtype_code(q), workspace.data_ptr(), ws_bytes,
-                                      _stream(stream))
-    _native.check("hyena_conv_bwd", rc)
+    rc = _native.lib().hyena_conv_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                         h.data_ptr(), dy.data_ptr(), dq.data_ptr(),
+                                         dk.data_ptr(), dv.data_ptr(), dh.data_ptr(), B, L, D,
+                                         d_g, l_h, l_b, _dtype_code(q), algo,
+                                         workspace.data_ptr(), ws_bytes, _stream(stream))
+    _native.check("hyena_conv_bwd_ex", rc)
     return dq, dk, dv, dh
 
 

@@ -48,6 +48,10 @@ SIGNATURES = {
     "hyena_conv_bwd_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32, _i32]),
     "hyena_conv_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                               _i32, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp]),
+    "hyena_conv_bwd_ex": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                 _i32, _i32, _i32, _i32, _i32, _vp, ctypes.c_size_t, _vp]),
+    "hyena_select_bwd_algo": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                     _i32, _i32, _i32, _i32]),
     "hyena_conv_bwd_static_scratch": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                              _i64, _i64, _i32, _i32, _i32, _i32, _vp]),
     "hyena_build_toeplitz": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]),

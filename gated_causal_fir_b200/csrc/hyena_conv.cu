@@ -12,6 +12,7 @@
 #include "fir_bwd.cuh"
 #include "fir_cuda_core.cuh"
 #include "fir_tc.cuh"
+#include "fir_tc_bwd.cuh"
 
 namespace {
 
@@ -70,6 +71,10 @@ int current_device(DeviceState *&ds) {
     for (const void *k : dh_kernels)
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kDhSmemMax);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(reinterpret_cast<const void *>(hyena::tcb::fir_tc_bwd_kernel),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               hyena::tcb::kSmemBytes);
 
     d->err = e;
   });
@@ -348,8 +353,36 @@ BwdPlan bwd_plan(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
   return b;
 }
 
+int64_t round256(int64_t n) { return (n + 255) / 256 * 256; }
+
+// Workspace of the tensor-core backward: one dh partial (l_h floats) and one group id per
+// (CTA, segment) slot, then one segment count per CTA.
+constexpr int64_t kTcBwdMaxGrid = 1024;
+struct TcBwdLayout {
+  int64_t off_group, off_count, bytes;
+};
+TcBwdLayout tc_bwd_layout(int64_t slots, int64_t grid, int l_h) {
+  TcBwdLayout o;
+  o.off_group = round256(slots * l_h * 4);
+  o.off_count = o.off_group + round256(slots * 4);
+  o.bytes = o.off_count + round256(grid * 4);
+  return o;
+}
+
+// Upper bound over every grid size: a CTA of a walk of W tiles split over `grid` CTAs touches
+// at most per / nT + 2 sequences, so slots <= B G + 2 grid.
+int64_t tc_bwd_bytes_bound(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
+  if (d_g != hyena::tc::kNC || D % hyena::tc::kNC != 0) return 0;
+  const int64_t nT = (L + hyena::tc::kTM - 1) / hyena::tc::kTM, G = D / hyena::tc::kNC;
+  const int64_t W = G * B * nT;
+  const int64_t grid = W < kTcBwdMaxGrid ? W : kTcBwdMaxGrid;
+  return tc_bwd_layout(B * G + 2 * grid, grid, l_h).bytes;
+}
+
 int64_t bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
-  return (bwd_plan(B, L, D, d_g, l_h).partial_floats * 4 + 255) / 256 * 256;
+  const int64_t cc = round256(bwd_plan(B, L, D, d_g, l_h).partial_floats * 4);
+  const int64_t tc = tc_bwd_bytes_bound(B, L, D, d_g, l_h);
+  return cc > tc ? cc : tc;
 }
 
 template <typename T>
@@ -384,15 +417,96 @@ int launch_bwd_cuda_core(const Problem &P, const void *dy, void *dk, void *dv, f
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
-int run_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv, float *dh,
-            void *workspace, size_t workspace_bytes, cudaStream_t s) {
-  const int rc = validate(P);  // q, k, v, h and dq (in the place of y)
-  if (rc == kEmpty) {  // no tokens: dh is an empty sum
-    if (!dh || !aligned(dh, 4)) return HYENA_ERR_INVALID_ARG;
-    return cudaMemsetAsync(dh, 0, static_cast<size_t>(P.G() * P.l_h) * 4, s) == cudaSuccess
-               ? HYENA_OK
-               : HYENA_ERR_CUDA;
+// dq through the forward kernels (dy in the place of q), then the CUDA-core dx/dk/dv and dh
+// kernels.
+int run_bwd_cuda_core(const Problem &P, const void *dy, void *dq, void *dk, void *dv, float *dh,
+                      void *workspace, cudaStream_t s) {
+  Problem F = P;
+  F.q = dy;
+  F.y = dq;
+  const int r = run(F, HYENA_ALGO_AUTO, s);
+  if (r != HYENA_OK) return r;
+  if (P.dtype == HYENA_DTYPE_F32)
+    return launch_bwd_cuda_core<float>(P, dy, dk, dv, dh, static_cast<float *>(workspace), s);
+  return launch_bwd_cuda_core<__nv_bfloat16>(P, dy, dk, dv, dh, static_cast<float *>(workspace),
+                                             s);
+}
+
+bool tc_bwd_supported(const Problem &P, const void *dy, const void *dq, const void *dk,
+                      const void *dv) {
+  return P.dtype == HYENA_DTYPE_BF16 && P.d_g == hyena::tc::kNC && P.D % hyena::tc::kNC == 0 &&
+         P.l_h <= hyena::tc::kMaxHalo + 1 && P.L <= (int64_t{1} << 30) &&
+         P.B <= (int64_t{1} << 30) && aligned(P.q, 16) && aligned(P.k, 16) &&
+         aligned(P.v, 16) && aligned(dy, 16) && aligned(dq, 16) && aligned(dk, 16) &&
+         aligned(dv, 16);
+}
+
+int launch_tensor_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv, float *dh,
+                      void *workspace, size_t workspace_bytes, cudaStream_t s) {
+  namespace tb = hyena::tcb;
+  DeviceState *ds = nullptr;
+  if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return HYENA_ERR_CUDA;
+  CUtensorMap maps[4];
+  const void *ptrs[4] = {P.q, P.k, P.v, dy};
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.D), static_cast<cuuint64_t>(P.L),
+                              static_cast<cuuint64_t>(P.B)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.D) * 2,
+                                 static_cast<cuuint64_t>(P.L) * static_cast<cuuint64_t>(P.D) * 2};
+  const cuuint32_t box[3] = {hyena::tc::kNC, hyena::tc::kTM, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  for (int i = 0; i < 4; ++i) {
+    if (enc(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptrs[i]), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            HYENA_TC_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return HYENA_ERR_CUDA;
   }
+  tb::Params p;
+  p.h = P.h;
+  p.B = static_cast<int>(P.B);
+  p.L = static_cast<int>(P.L);
+  p.l_h = P.l_h;
+  p.G = static_cast<int>(P.D / hyena::tc::kNC);
+  p.halo = (P.l_h - 1 + 15) / 16 * 16;
+  p.band_cols = (hyena::tc::kTM + p.halo) / 2;
+  p.nT = static_cast<int>((P.L + hyena::tc::kTM - 1) / hyena::tc::kTM);
+  p.W = static_cast<long long>(p.G) * P.B * p.nT;
+  int64_t grid = ds->sm_count;
+  if (grid > p.W) grid = p.W;
+  if (grid > kTcBwdMaxGrid) grid = kTcBwdMaxGrid;
+  const int64_t per = p.W / grid;
+  p.max_segs = static_cast<int>(per / p.nT + 2);
+  const TcBwdLayout lay = tc_bwd_layout(grid * p.max_segs, grid, P.l_h);
+  if (lay.bytes > static_cast<int64_t>(workspace_bytes)) return HYENA_ERR_INVALID_ARG;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  p.partial = reinterpret_cast<float *>(ws);
+  p.seg_group = reinterpret_cast<int *>(ws + lay.off_group);
+  p.seg_count = reinterpret_cast<int *>(ws + lay.off_count);
+  p.D = P.D;
+  p.k = static_cast<const __nv_bfloat16 *>(P.k);
+  p.v = static_cast<const __nv_bfloat16 *>(P.v);
+  p.dy = static_cast<const __nv_bfloat16 *>(dy);
+  p.dq = static_cast<__nv_bfloat16 *>(dq);
+  p.dk = static_cast<__nv_bfloat16 *>(dk);
+  p.dv = static_cast<__nv_bfloat16 *>(dv);
+  tb::fir_tc_bwd_kernel<<<static_cast<unsigned>(grid), tb::kThreads, tb::kSmemBytes, s>>>(
+      maps[0], maps[1], maps[2], maps[3], p);
+  if (cudaGetLastError() != cudaSuccess) return HYENA_ERR_CUDA;
+  const long long gn = static_cast<long long>(p.G) * P.l_h;
+  long long rblocks = (gn + 255) / 256;
+  if (rblocks > ds->sm_count) rblocks = ds->sm_count;
+  tb::fir_bwd_tc_reduce_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
+      p.partial, p.seg_group, p.seg_count, p.max_segs, dh, p.G, P.l_h, per, p.W % grid,
+      static_cast<long long>(P.B) * p.nT);
+  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+// Host checks of a backward call; HYENA_OK, kEmpty or an error code.
+int validate_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv, float *dh,
+                 void *workspace, size_t workspace_bytes) {
+  const int rc = validate(P);  // q, k, v, h and dq (in the place of y)
+  if (rc == kEmpty) return (!dh || !aligned(dh, 4)) ? HYENA_ERR_INVALID_ARG : kEmpty;
   if (rc != HYENA_OK) return rc;
   if (!dy || !dk || !dv || !dh) return HYENA_ERR_INVALID_ARG;
   const uintptr_t es = static_cast<uintptr_t>(P.elem());
@@ -411,17 +525,38 @@ int run_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv, floa
   if (!workspace ||
       static_cast<int64_t>(workspace_bytes) < bwd_workspace_bytes(P.B, P.L, P.D, P.d_g, P.l_h))
     return HYENA_ERR_INVALID_ARG;
-  // dq = dy * (h conv (k v)): the forward with dy in the place of q.
-  Problem F = P;
-  F.q = dy;
-  F.y = dq;
-  int r = run(F, HYENA_ALGO_AUTO, s);
-  if (r != HYENA_OK) return r;
-  if (P.dtype == HYENA_DTYPE_F32)
-    return launch_bwd_cuda_core<float>(P, dy, dk, dv, dh, static_cast<float *>(workspace), s);
-  return launch_bwd_cuda_core<__nv_bfloat16>(P, dy, dk, dv, dh, static_cast<float *>(workspace),
-                                             s);
+  return HYENA_OK;
 }
+
+// The backward algorithm: HYENA_ALGO_TENSOR (fused tcgen05 kernel) or HYENA_ALGO_DIRECT
+// (CUDA-core kernels, dq through the forward), or minus HYENA_ERR_UNSUPPORTED.
+int select_bwd(const Problem &P, const void *dy, const void *dq, const void *dk, const void *dv,
+               int algo) {
+  const bool tc = tc_bwd_supported(P, dy, dq, dk, dv);
+  switch (algo) {
+    case HYENA_ALGO_AUTO: return tc ? HYENA_ALGO_TENSOR : HYENA_ALGO_DIRECT;
+    case HYENA_ALGO_TENSOR: return tc ? HYENA_ALGO_TENSOR : -HYENA_ERR_UNSUPPORTED;
+    case HYENA_ALGO_DIRECT: return HYENA_ALGO_DIRECT;
+    case HYENA_ALGO_WINDOW: return -HYENA_ERR_UNSUPPORTED;
+    default: return -HYENA_ERR_INVALID_ARG;
+  }
+}
+
+int run_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv, float *dh,
+            void *workspace, size_t workspace_bytes, cudaStream_t s, int algo) {
+  const int rc = validate_bwd(P, dy, dq, dk, dv, dh, workspace, workspace_bytes);
+  if (rc == kEmpty)  // no tokens: dh is an empty sum
+    return cudaMemsetAsync(dh, 0, static_cast<size_t>(P.G() * P.l_h) * 4, s) == cudaSuccess
+               ? HYENA_OK
+               : HYENA_ERR_CUDA;
+  if (rc != HYENA_OK) return rc;
+  const int a = select_bwd(P, dy, dq, dk, dv, algo);
+  if (a < 0) return -a;
+  if (a == HYENA_ALGO_TENSOR)
+    return launch_tensor_bwd(P, dy, dq, dk, dv, dh, workspace, workspace_bytes, s);
+  return run_bwd_cuda_core(P, dy, dq, dk, dv, dh, workspace, s);
+}
+
 
 }  // namespace
 
@@ -497,7 +632,25 @@ int hyena_conv_bwd(const void *q, const void *k, const void *v, const float *h, 
                    int d_g, int l_h, int l_b, int dtype, void *workspace, size_t workspace_bytes,
                    cudaStream_t stream) {
   const Problem P{q, k, v, h, dq, B, L, D, d_g, l_h, l_b, dtype};
-  return run_bwd(P, dy, dq, dk, dv, dh, workspace, workspace_bytes, stream);
+  return run_bwd(P, dy, dq, dk, dv, dh, workspace, workspace_bytes, stream, HYENA_ALGO_AUTO);
+}
+
+int hyena_conv_bwd_ex(const void *q, const void *k, const void *v, const float *h,
+                      const void *dy, void *dq, void *dk, void *dv, float *dh, int64_t B,
+                      int64_t L, int64_t D, int d_g, int l_h, int l_b, int dtype, int algo,
+                      void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const Problem P{q, k, v, h, dq, B, L, D, d_g, l_h, l_b, dtype};
+  return run_bwd(P, dy, dq, dk, dv, dh, workspace, workspace_bytes, stream, algo);
+}
+
+int hyena_select_bwd_algo(const void *q, const void *k, const void *v, const float *h,
+                          const void *dy, const void *dq, const void *dk, const void *dv,
+                          int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                          int dtype) {
+  const Problem P{q, k, v, h, const_cast<void *>(dq), B, L, D, d_g, l_h, l_b, dtype};
+  const int rc = validate(P);
+  if (rc != HYENA_OK && rc != kEmpty) return -rc;
+  return select_bwd(P, dy, dq, dk, dv, HYENA_ALGO_AUTO);
 }
 
 int hyena_conv_bwd_static_scratch(const void *q, const void *k, const void *v, const float *h,
@@ -512,7 +665,8 @@ int hyena_conv_bwd_static_scratch(const void *q, const void *k, const void *v, c
     return HYENA_ERR_UNSUPPORTED;
   void *ws = nullptr;
   if (static_scratch(ws) != HYENA_OK) return HYENA_ERR_CUDA;
-  return run_bwd(P, dy, dq, dk, dv, dh, ws, HYENA_BWD_STATIC_SCRATCH_BYTES, stream);
+  return run_bwd(P, dy, dq, dk, dv, dh, ws, HYENA_BWD_STATIC_SCRATCH_BYTES, stream,
+                 HYENA_ALGO_AUTO);
 }
 
 int hyena_build_toeplitz(const float *h, float *H0, float *H1, float *H2_or_null, int G,

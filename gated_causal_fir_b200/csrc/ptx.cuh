@@ -36,6 +36,13 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
                : "memory");
 }
 
+// Arrival that counts as `count` arrivals (one thread releasing for a whole group).
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(count)
+               : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
                    smem_u32(bar)),
@@ -92,6 +99,14 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
 }
 
 // 3-D tiled store from shared memory; rows outside the tensor are clipped by the hardware.
+// Fetch a tile into L2 ahead of its load (no shared memory, no completion signal).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int c0,
                                              int c1, int c2) {
   asm volatile(
@@ -215,6 +230,17 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
 }
 
 // Each thread of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -278,6 +304,13 @@ __host__ __device__ constexpr uint32_t umma_idesc_f16_f32(int M, int N, int b_mn
          | (static_cast<uint32_t>(b_mn_major) << 16)   // B major-ness
          | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);      // M / 16
+}
+
+// Same with both operands' major-ness chosen (1 = MN-major), e.g. A^T B products of tiles
+// stored with the M/N index contiguous.
+__host__ __device__ constexpr uint32_t umma_idesc_f16_f32_mn(int M, int N, int a_mn_major,
+                                                            int b_mn_major) {
+  return umma_idesc_f16_f32(M, N, b_mn_major) | (static_cast<uint32_t>(a_mn_major) << 15);
 }
 
 }  // namespace hyena

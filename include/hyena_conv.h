@@ -103,9 +103,11 @@ int hyena_select_algo(const void *q, const void *k, const void *v, const float *
                       int l_b, int dtype);
 
 /*
- * Host-only: the bytes of device workspace hyena_conv_bwd needs for this shape (a multiple of
- * 256; 4 bytes per partial filter gradient, one partial per sequence, 64-step chunk,
- * channel piece and tap), or minus HYENA_ERR_INVALID_ARG for a bad shape.  Touches no device.
+ * Host-only: the bytes of device workspace the backward entry points need for this shape, on
+ * any algorithm and any device (a multiple of 256), or minus HYENA_ERR_INVALID_ARG for a bad
+ * shape.  The workspace holds fp32 partial filter gradients: on the CUDA-core path one per
+ * sequence, 64-step chunk, channel piece and tap; on the tensor path one per (CTA, sequence
+ * run) and tap, with the run's group and a run count per CTA.  Touches no device.
  */
 int64_t hyena_conv_bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h);
 
@@ -120,9 +122,12 @@ int64_t hyena_conv_bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g,
  *
  * q, k, v, dy, dq, dk, dv: DEVICE [B, L, D] tensors of `dtype`, layout as the forward.
  * h: DEVICE fp32 [D / d_g, l_h].  dh: DEVICE fp32 [D / d_g, l_h], overwritten (not
- * accumulated into).  dq is computed by the forward kernels (HYENA_ALGO_AUTO) with dy in the
- * place of q, so the forward's shape rules (l_h <= 2*l_b) apply; dk, dv and dh by CUDA-core
- * kernels in fp32.  dh is summed in a fixed order: results are deterministic.
+ * accumulated into).  The forward's shape rules (l_h <= 2*l_b) apply.  Algorithm (AUTO): where
+ * the tensor path applies (bf16, d_g == 64, D % 64 == 0, l_h <= 129, all seven tensors
+ * 16-byte aligned) one fused tcgen05 kernel reads q, k, v, dy once and writes dq, dk, dv once,
+ * with fp16 operands (x = k v, dz = q dy, h rounded to fp16) and fp32 accumulation; otherwise
+ * dq comes from the forward kernels and dk, dv, dh from CUDA-core kernels in fp32.  dh is
+ * summed in a fixed order on either path: results are deterministic on a given device.
  * workspace: DEVICE scratch of at least hyena_conv_bwd_workspace_bytes() bytes, 16-byte
  * aligned, owned by the caller, unused after the queued work ends.  Outputs must not overlap
  * each other or an input.  B == 0 or L == 0 zeroes dh and launches nothing else.
@@ -133,6 +138,26 @@ int hyena_conv_bwd(const void *q, const void *k, const void *v, const float *h, 
                    void *dq, void *dk, void *dv, float *dh, int64_t B, int64_t L, int64_t D,
                    int d_g, int l_h, int l_b, int dtype, void *workspace,
                    size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * hyena_conv_bwd with the algorithm chosen by the caller: HYENA_ALGO_AUTO, HYENA_ALGO_TENSOR
+ * (the fused tcgen05 kernel; HYENA_ERR_UNSUPPORTED where it does not apply) or
+ * HYENA_ALGO_DIRECT (the CUDA-core kernels; any shape).  HYENA_ALGO_WINDOW has no backward
+ * and returns HYENA_ERR_UNSUPPORTED.  Nothing is queued when an error is returned.
+ */
+int hyena_conv_bwd_ex(const void *q, const void *k, const void *v, const float *h,
+                      const void *dy, void *dq, void *dk, void *dv, float *dh, int64_t B,
+                      int64_t L, int64_t D, int d_g, int l_h, int l_b, int dtype, int algo,
+                      void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Host-only: the algorithm (HYENA_ALGO_TENSOR or HYENA_ALGO_DIRECT) HYENA_ALGO_AUTO would run
+ * for this backward problem and these pointers, or minus an error code.  Touches no device.
+ */
+int hyena_select_bwd_algo(const void *q, const void *k, const void *v, const float *h,
+                          const void *dy, const void *dq, const void *dk, const void *dv,
+                          int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                          int dtype);
 
 /* Size of the fixed device scratch behind hyena_conv_bwd_static_scratch (8 MiB per device). */
 #define HYENA_BWD_STATIC_SCRATCH_BYTES (8u << 20)

@@ -136,3 +136,14 @@ def test_bwd_static_scratch_rejects_oversize_on_host(lib):
     assert rc == _native.HYENA_ERR_UNSUPPORTED
     rc = lib.hyena_conv_bwd_static_scratch(*p, B, L, D, 63, 128, 64, 0, None)
     assert rc == _native.HYENA_ERR_INVALID_ARG
+
+
+def test_select_bwd_algo(lib):
+    T, Dd = g.HYENA_ALGO_TENSOR, g.HYENA_ALGO_DIRECT
+    assert g.hyena_select_bwd_algo(1, 8192, 4096, 64, 128, 64) == T   # MR: fused tensor kernel
+    assert g.hyena_select_bwd_algo(1, 8192, 4096, 16, 7, 16) == Dd    # d_g 16: CUDA cores
+    assert g.hyena_select_bwd_algo(1, 8192, 4096, 64, 128, 64, g.HYENA_DTYPE_F32) == Dd
+    assert g.hyena_select_bwd_algo(1, 300, 4096, 64, 130, 65) == Dd   # l_h > 129
+    assert g.hyena_select_bwd_algo(1, 300, 96, 32, 16, 16) == Dd
+    with pytest.raises(g.HyenaError):
+        g.hyena_select_bwd_algo(1, 300, 96, 32, 100, 16)                # l_h > 2 l_b

@@ -3,12 +3,18 @@
 Tolerances:
   * dq, dk, dv: those of the forward (bf16: 1e-2 + 1e-2 |ref| elementwise; fp32 normwise 1e-5);
     each is one fp32 sum of at most l_h exact products, rounded once to the output type.
-  * dh (fp32 output): normwise max|dh - ref| <= 1e-4 max|ref|.  Each dh[g][j] is a sum of
-    N = B * L * d_g terms of rms ~1 for these inputs, so |ref| ~ sqrt(N).  The kernels add
-    them as fp32 partials of 64 rows x (up to) 64 channels, then a fixed-order sum of the
-    partials; rounding errors of random sign give about u * 64 * sqrt(4096) * sqrt(N / 4096)
-    ~ 2e-6 sqrt(N), i.e. ~2e-6 normwise, so 1e-4 keeps a 50x margin while a single dropped
-    or doubled term (~1 / sqrt(N) normwise, 1.4e-3 at the MR size) still fails.
+  * dh (fp32 output), CUDA-core path: normwise max|dh - ref| <= 1e-4 max|ref|.  Each
+    dh[g][j] is a sum of N = B * L * d_g terms of rms ~1 for these inputs, so |ref| ~ sqrt(N).
+    The kernels add them as fp32 partials of 64 rows x (up to) 64 channels, then a fixed-order
+    sum of the partials; rounding errors of random sign give about
+    u * 64 * sqrt(4096) * sqrt(N / 4096) ~ 2e-6 sqrt(N), i.e. ~2e-6 normwise, so 1e-4 keeps a
+    50x margin while a single dropped or doubled term (~1 / sqrt(N) normwise, 1.4e-3 at the MR
+    size) still fails.
+  * dh, tensor path: normwise 2e-3.  Its products take x = k v and dz = q dy rounded to fp16
+    (relative error <= 2^-11 each, ~4e-4 rms per product); the sum of N such errors of random
+    sign is ~4e-4 sqrt(N), i.e. ~4e-4 / 3.5 ~ 1.2e-4 of max|ref| on average and ~5e-4 at the
+    worst of the G * l_h outputs.  2e-3 keeps a 4x margin; a wrong lag, tile or group moves
+    dh by O(max|ref|).  The integer cases pin this path exactly.
   * Integer-valued inputs (test_integer_exact): every product and partial sum is an exact
     integer, so all four gradients must equal the oracle's bit for bit.
 """
@@ -24,7 +30,12 @@ import oracle
 
 pytestmark = pytest.mark.gpu
 
-DH_NORMWISE = 1e-4
+DH_NORMWISE = {g.HYENA_ALGO_DIRECT: 1e-4, g.HYENA_ALGO_TENSOR: 2e-3}
+ALGOS = {"direct": g.HYENA_ALGO_DIRECT, "tensor": g.HYENA_ALGO_TENSOR}
+
+
+def _tensor_fits(B, L, D, d_g, l_h, dt):
+    return dt == "bf16" and d_g == 64 and D % 64 == 0 and l_h <= 129
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -38,13 +49,13 @@ def _device():
     assert g.hyena_device_status(clear=True) == 0, "a kernel raised its device status word"
 
 
-def _bwd(q, k, v, h, dy, wl):
-    out = g.hyena_conv_bwd(q, k, v, h, dy, wl.d_g, wl.l_b)
+def _bwd(q, k, v, h, dy, wl, algo=g.HYENA_ALGO_AUTO):
+    out = g.hyena_conv_bwd_ex(q, k, v, h, dy, wl.d_g, wl.l_b, algo=algo)
     torch.cuda.synchronize()
     return out
 
 
-def _check_all(out, ref, dtype):
+def _check_all(out, ref, dtype, algo):
     dq, dk, dv, dh = out
     rq, rk, rv, rh = ref
     U.assert_parity(dq, rq, dtype)
@@ -53,17 +64,23 @@ def _check_all(out, ref, dtype):
     got = dh.detach().cpu().double().numpy()
     assert np.all(np.isfinite(got)), "non-finite dh"
     r = U.f32_normwise(got, rh)
-    assert r <= DH_NORMWISE, "dh normwise error %.3e > %.1e" % (r, DH_NORMWISE)
+    tol = DH_NORMWISE[algo]
+    assert r <= tol, "dh normwise error %.3e > %.1e" % (r, tol)
 
 
 @pytest.mark.parametrize("name", ["tiny", "se", "mr"])
 def test_bwd_workload(name):
+    """The default entry point on the workloads; MR runs the fused tensor kernel."""
     wl = WORKLOADS[name]
     q, k, v, h = make_inputs(wl, device="cuda")
     dy = make_grad(wl, device="cuda")
-    out = _bwd(q, k, v, h, dy, wl)
+    algo = g.hyena_select_bwd_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b,
+                                   g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16)
+    assert algo == (g.HYENA_ALGO_TENSOR if name == "mr" else g.HYENA_ALGO_DIRECT)
+    out = g.hyena_conv_bwd(q, k, v, h, dy, wl.d_g, wl.l_b)
+    torch.cuda.synchronize()
     ref = oracle.gated_fir_bwd(q, k, v, h, dy, wl.d_g)
-    _check_all(out, ref, q.dtype)
+    _check_all(out, ref, q.dtype, algo)
 
 
 SHAPES = [
@@ -78,35 +95,52 @@ SHAPES = [
     ("long_filter", 1, 600, 64, 64, 200, 100, "bf16"),
     ("f32_dg6", 2, 301, 12, 6, 5, 4, "f32"),
     ("f32_mr", 1, 900, 128, 64, 128, 64, "f32"),
+    ("runs_across_seqs", 3, 3000, 512, 64, 100, 64, "bf16"),
+    ("long_seq_one_group", 1, 40000, 64, 64, 128, 64, "bf16"),
+    ("batched_halo16", 4, 2048, 128, 64, 17, 16, "bf16"),
 ]
+CASES = [(s, a) for s in SHAPES for a in ALGOS if a == "direct" or _tensor_fits(*s[1:6], s[7])]
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=[s[0] for s in SHAPES])
-def test_bwd_shapes(shape):
+@pytest.mark.parametrize("shape,algo", CASES, ids=["%s-%s" % (s[0], a) for s, a in CASES])
+def test_bwd_shapes(shape, algo):
     name, B, L, D, d_g, l_h, l_b, dt = shape
     wl = custom(name, B, L, D, d_g, l_h, l_b, dt, filt="mr" if l_h > 16 else "se", seed=11)
     q, k, v, h = make_inputs(wl, device="cuda")
     dy = make_grad(wl, device="cuda")
-    out = _bwd(q, k, v, h, dy, wl)
+    out = _bwd(q, k, v, h, dy, wl, ALGOS[algo])
     ref = oracle.gated_fir_bwd(q, k, v, h, dy, wl.d_g)
-    _check_all(out, ref, q.dtype)
+    _check_all(out, ref, q.dtype, ALGOS[algo])
+
+
+def test_bwd_tensor_unsupported_is_rejected():
+    wl = custom("dg32", 1, 300, 128, 32, 16, 16, "bf16")
+    q, k, v, h = make_inputs(wl, device="cuda")
+    dy = make_grad(wl, device="cuda")
+    with pytest.raises(g.HyenaError) as e:
+        _bwd(q, k, v, h, dy, wl, g.HYENA_ALGO_TENSOR)
+    assert e.value.status == 2
 
 
 INT_SHAPES = [
     ("mr", 2, 1500, 256, 64, 128, 64, "bf16"),
+    ("mr_halo_129", 1, 3000, 128, 64, 129, 65, "bf16"),
     ("se", 1, 2000, 512, 16, 7, 16, "bf16"),
     ("dg32", 1, 1000, 128, 32, 65, 64, "bf16"),
     ("f32", 2, 700, 64, 8, 12, 8, "f32"),
 ]
+INT_CASES = [(s, a) for s in INT_SHAPES for a in ALGOS
+             if a == "direct" or _tensor_fits(*s[1:6], s[7])]
 
 
-@pytest.mark.parametrize("shape", INT_SHAPES, ids=[s[0] for s in INT_SHAPES])
-def test_integer_exact(shape):
+@pytest.mark.parametrize("shape,algo", INT_CASES,
+                         ids=["%s-%s" % (s[0], a) for s, a in INT_CASES])
+def test_integer_exact(shape, algo):
     name, B, L, D, d_g, l_h, l_b, dt = shape
     assert B * L * d_g * 16 < 2 ** 24
     wl = custom("int_" + name, B, L, D, d_g, l_h, l_b, dt, seed=5)
     q, k, v, dy, h = make_integer_inputs(wl, device="cuda")
-    dq, dk, dv, dh = _bwd(q, k, v, h, dy, wl)
+    dq, dk, dv, dh = _bwd(q, k, v, h, dy, wl, ALGOS[algo])
     rq, rk, rv, rh = oracle.gated_fir_bwd(q, k, v, h, dy, wl.d_g)
     tdt = q.dtype
     for got, ref, nm in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
@@ -115,12 +149,13 @@ def test_integer_exact(shape):
     assert np.array_equal(dh.cpu().double().numpy(), rh), "dh differs from the exact sum"
 
 
-def test_bwd_deterministic():
+@pytest.mark.parametrize("algo", list(ALGOS))
+def test_bwd_deterministic(algo):
     wl = custom("det", 2, 1000, 256, 64, 128, 64, "bf16", filt="mr", seed=3)
     q, k, v, h = make_inputs(wl, device="cuda")
     dy = make_grad(wl, device="cuda")
-    a = [t.clone() for t in _bwd(q, k, v, h, dy, wl)]
-    b = _bwd(q, k, v, h, dy, wl)
+    a = [t.clone() for t in _bwd(q, k, v, h, dy, wl, ALGOS[algo])]
+    b = _bwd(q, k, v, h, dy, wl, ALGOS[algo])
     for x, y in zip(a, b):
         assert torch.equal(x, y)
 
