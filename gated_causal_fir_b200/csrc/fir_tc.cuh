@@ -346,18 +346,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[kBarDone], 1);
     *abort = 0;
     fence_mbar_init();
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_y);
   }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  // Everything above touches no global memory, so under a programmatic dependent launch it
+  // overlaps the end of the previous kernel.  From here on the inputs may be read.
+  griddep_wait();
+  griddep_launch_dependents();
   // Thread 0 is also the k/v producer: it queues the first k/v stages right away, before the
-  // TMEM allocation and the CTA-wide barrier (no other thread touches those stages yet).
+  // CTA-wide barrier (no other thread touches those stages yet).
   Walk<kSched> kv_it(p, w_begin, w_end, gmul, goff);
   Item kv_t;
   uint32_t kv_count = 0;
   bool kv_done = false;
   if (threadIdx.x == 0) {
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_y);
     while (kv_count < kNKV) {
       if (!kv_it.next(kv_t)) {
         kv_done = true;
@@ -370,10 +378,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                   kv_t.i * kTM, kv_t.b);
       ++kv_count;
     }
-  }
-  if (warp == kWarpMma) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -609,7 +613,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++qc;
     }
     if (et == 0) {
-      bulk_wait_group<0>();
+      // The stores must have read their shared memory before the CTA exits; their global
+      // writes complete with the grid.
+      bulk_wait_group_read<0>();
       if (qc > 0) mbar_arrive(&bars[kBarQEmpty + (qc + kNQ - 1) % kNQ]);
     }
   }

@@ -27,6 +27,9 @@ using hyena::cc::WindowParams;
 #ifndef HYENA_TC_RUN
 #define HYENA_TC_RUN 0
 #endif
+#ifndef HYENA_PDL
+#define HYENA_PDL 1
+#endif
 
 
 constexpr int kMaxDevices = 64;
@@ -240,8 +243,22 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
   }
   const unsigned g = static_cast<unsigned>(grid);
   constexpr int T = hyena::tc::kThreads, S = hyena::tc::kSmemBytes;
-#define HYENA_TC_LAUNCH(SCHED, NG) \
-  hyena::tc::fir_tc_kernel<SCHED, NG><<<g, T, S, s>>>(maps[0], maps[1], maps[2], maps[3], p)
+  // Programmatic dependent launch: the kernel's set-up (barriers, tensor memory) overlaps the
+  // tail of the previous kernel in the stream; it reads nothing before that kernel is done.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = HYENA_PDL;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(g);
+  cfg.blockDim = dim3(T);
+  cfg.dynamicSmemBytes = S;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t le = cudaSuccess;
+#define HYENA_TC_LAUNCH(SCHED, NG)                                                          \
+  le = cudaLaunchKernelEx(&cfg, hyena::tc::fir_tc_kernel<SCHED, NG>, maps[0], maps[1], maps[2], \
+                          maps[3], p)
   const int sched = p.run > 0 ? 1 : 0;
   switch (sched * 8 + plan.ng) {
     case 1: HYENA_TC_LAUNCH(0, 1); break;
@@ -253,7 +270,7 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
     default: return HYENA_ERR_UNSUPPORTED;
   }
 #undef HYENA_TC_LAUNCH
-  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+  return le == cudaSuccess && cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
 template <typename T, int LH>

@@ -83,6 +83,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   }
 }
 
+// ------------------------------------------------------------------------------ launch order
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialisation may
+// start while the previous kernel of its stream is still running; griddep_wait() blocks the
+// calling thread until that kernel has completed and its memory writes are visible, so every
+// thread calls it before its first global-memory access.  griddep_launch_dependents() lets the
+// next such kernel of the stream be scheduled (its CTAs still wait in griddep_wait()).
+// Without the launch attribute both are no-ops.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
