@@ -25,6 +25,7 @@ __all__ = [
     "HyenaError", "HYENA_ALGO_AUTO", "HYENA_ALGO_TENSOR", "HYENA_ALGO_WINDOW",
     "HYENA_ALGO_DIRECT", "HYENA_DTYPE_BF16", "HYENA_DTYPE_F32", "HYENA_DEVICE_TIMEOUT",
     "HYENA_DEVICE_F16_RANGE", "ALGO_NAMES", "hyena_conv_fwd_from_host",
+    "hyena_toeplitz_stages", "hyena_build_toeplitz_blocks",
 ]
 
 
@@ -76,8 +77,8 @@ def hyena_conv_fwd_ex(q, k, v, h, d_g, l_b, algo=HYENA_ALGO_AUTO, y=None, stream
     """Forward with the algorithm chosen by the caller (HYENA_ALGO_*); returns y.
 
     q, k, v: CUDA [B, L, D], all bf16 or all fp32.  h: CUDA fp32 [D // d_g, l_h].
-    l_b: block size of the decomposition (needs l_h <= 2 * l_b; the result does not depend on
-    it).  y: optional preallocated output.  Runs asynchronously on ``stream`` (default: the
+    l_b: block size of the decomposition (any l_h >= 1 is accepted; the result does not depend
+    on l_b).  y: optional preallocated output.  Runs asynchronously on ``stream`` (default: the
     current torch stream).
     """
     y = _check(q, k, v, h, d_g, y)
@@ -211,6 +212,31 @@ def hyena_build_toeplitz(h, l_b, stream=None):
                                             H[2].data_ptr(), G, l_h, l_b, _stream(stream))
     _native.check("hyena_build_toeplitz", rc)
     return H[0], H[1], H[2]
+
+
+def hyena_toeplitz_stages(l_h, l_b):
+    """Sub-block diagonals S = 1 + ceil((l_h - 1) / l_b) of the block-Toeplitz decomposition."""
+    rc = int(_native.lib().hyena_toeplitz_stages(l_h, l_b))
+    if rc < 0:
+        _native.check("hyena_toeplitz_stages", -rc)
+    return rc
+
+
+def hyena_build_toeplitz_blocks(h, l_b, S=None, stream=None):
+    """fp32 CUDA tensor [S, G, l_b, l_b] with Hm[m][g][i][j] = h[g][m l_b + i - j] (zero outside
+    [0, l_h)); S defaults to the number of non-zero sub-block diagonals."""
+    torch = _torch()
+    if not isinstance(h, torch.Tensor) or not h.is_cuda or h.dtype != torch.float32 \
+            or h.dim() != 2 or not h.is_contiguous():
+        raise TypeError("h must be a contiguous CUDA float32 [G, l_h] tensor")
+    G, l_h = h.shape
+    if S is None:
+        S = hyena_toeplitz_stages(l_h, l_b)
+    H = torch.empty((S, G, l_b, l_b), dtype=torch.float32, device=h.device)
+    rc = _native.lib().hyena_build_toeplitz_blocks(h.data_ptr(), H.data_ptr(), S, G, l_h, l_b,
+                                                   _stream(stream))
+    _native.check("hyena_build_toeplitz_blocks", rc)
+    return H
 
 
 def hyena_device_status(clear=True):

@@ -55,6 +55,8 @@ SIGNATURES = {
     "hyena_conv_bwd_static_scratch": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                              _i64, _i64, _i32, _i32, _i32, _i32, _vp]),
     "hyena_build_toeplitz": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]),
+    "hyena_toeplitz_stages": (_i32, [_i32, _i32]),
+    "hyena_build_toeplitz_blocks": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp]),
     "hyena_device_status": (_i32, [ctypes.POINTER(ctypes.c_uint), _i32]),
     "hyena_status_string": (ctypes.c_char_p, [_i32]),
     "hyena_abi_version": (_i32, []),

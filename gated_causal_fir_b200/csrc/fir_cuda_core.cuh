@@ -221,5 +221,24 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// All S sub-block diagonals: Hm[m][g][i][j] = h[g][m l_b + i - j] inside [0, l_h), else 0, for
+// m < S (the general block form of the same page, any filter length).
+__global__ void __launch_bounds__(256)
+    toeplitz_stack_kernel(const float *__restrict__ h, float *__restrict__ Hm, int S, int G,
+                          int l_h, int l_b) {
+  const long long blk = static_cast<long long>(l_b) * l_b;
+  const long long n = static_cast<long long>(S) * G * blk;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long mg = e / blk;
+    const int m = static_cast<int>(mg / G);
+    const long long g = mg % G;
+    const int i = static_cast<int>((e / l_b) % l_b);
+    const int j = static_cast<int>(e % l_b);
+    const long long idx = static_cast<long long>(m) * l_b + i - j;
+    Hm[e] = (idx >= 0 && idx < l_h) ? __ldg(h + g * l_h + idx) : 0.f;
+  }
+}
+
 }  // namespace cc
 }  // namespace hyena

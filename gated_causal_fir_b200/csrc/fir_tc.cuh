@@ -42,16 +42,12 @@ namespace tc {
 
 constexpr int kTM = 128;             // output rows per tile (MMA M)
 constexpr int kNC = 64;              // channels per tile: 64 / d_g groups of d_g (MMA N = d_g)
-constexpr int kMaxHalo = 128;        // supports l_h - 1 <= 128
+constexpr int kMaxHist = 4;          // history tiles a tile may read: l_h - 1 <= 4 * 128
+constexpr int kMaxHalo = kMaxHist * kTM;
 #ifndef HYENA_TC_KV_STAGES
 #define HYENA_TC_KV_STAGES 3
 #endif
-#ifndef HYENA_TC_Q_STAGES
-#define HYENA_TC_Q_STAGES 3
-#endif
 constexpr int kNKV = HYENA_TC_KV_STAGES;  // k/v stages
-constexpr int kNQ = HYENA_TC_Q_STAGES;    // q (and in-place y) stages
-constexpr int kNX = 3;               // fp16 X slots (current, previous, next)
 constexpr int kNAcc = 2;             // TMEM accumulator sets (tiles in flight)
 constexpr int kRowBytes = kNC * 2;                              // 128 B
 constexpr int kTileBytes = kTM * kRowBytes;                     // 16 KB
@@ -63,27 +59,35 @@ constexpr int kKBlockBytes = kNC * 128;                         // 64 times x 64
 constexpr int kBandCol0 = kNAcc * kNC;                           // 128
 constexpr int kTmemCols = 512;
 
-constexpr int kOffKV = 0;
-constexpr int kOffQ = kOffKV + kNKV * 2 * kTileBytes;
-constexpr int kOffX = kOffQ + kNQ * kTileBytes;
-constexpr int kOffBar = kOffX + kNX * kTileBytes;
-// barriers
-constexpr int kBarKVFull = 0;
-constexpr int kBarKVEmpty = kBarKVFull + kNKV;
-constexpr int kBarQFull = kBarKVEmpty + kNKV;
-constexpr int kBarQEmpty = kBarQFull + kNQ;
-constexpr int kBarYReady = kBarQEmpty + kNQ;
-constexpr int kBarXFull = kBarYReady + kNQ;
-constexpr int kBarXEmpty = kBarXFull + kNX;
-constexpr int kBarAccFull = kBarXEmpty + kNX;
-constexpr int kBarAccEmpty = kBarAccFull + kNAcc;
-constexpr int kBarAFull = kBarAccEmpty + kNAcc;
-constexpr int kBarAEmpty = kBarAFull + 2;  // up to two band sets
-constexpr int kBarDone = kBarAEmpty + 2;
-constexpr int kNumBars = kBarDone + 1;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget of one CTA exceeded");
+// Shared-memory layout for a kernel whose tiles read kNH earlier tiles (halo <= 128 kNH rows):
+// k/v stages, q stages (reused in place for y), and kNH + 2 fp16 X slots (the kNH tiles of
+// history, the current tile and the next one being gated).
+template <int kNH>
+struct Layout {
+  static constexpr int kNQ = kNH >= 4 ? 2 : 3;   // q (and in-place y) stages
+  static constexpr int kNX = kNH + 2;            // fp16 X slots
+  static constexpr int kOffKV = 0;
+  static constexpr int kOffQ = kOffKV + kNKV * 2 * kTileBytes;
+  static constexpr int kOffX = kOffQ + kNQ * kTileBytes;
+  static constexpr int kOffBar = kOffX + kNX * kTileBytes;
+  // barriers
+  static constexpr int kBarKVFull = 0;
+  static constexpr int kBarKVEmpty = kBarKVFull + kNKV;
+  static constexpr int kBarQFull = kBarKVEmpty + kNKV;
+  static constexpr int kBarQEmpty = kBarQFull + kNQ;
+  static constexpr int kBarYReady = kBarQEmpty + kNQ;
+  static constexpr int kBarXFull = kBarYReady + kNQ;
+  static constexpr int kBarXEmpty = kBarXFull + kNX;
+  static constexpr int kBarAccFull = kBarXEmpty + kNX;
+  static constexpr int kBarAccEmpty = kBarAccFull + kNAcc;
+  static constexpr int kBarAFull = kBarAccEmpty + kNAcc;
+  static constexpr int kBarAEmpty = kBarAFull + 2;  // up to two band sets
+  static constexpr int kBarDone = kBarAEmpty + 2;
+  static constexpr int kNumBars = kBarDone + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget of one CTA exceeded");
+};
 
 constexpr int kThreads = 352;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGate0 = 2, kWarpEpi0 = 6, kWarpTmaQ = 10;
@@ -96,37 +100,36 @@ struct Params {
   const float *h;   // [D / d_g, l_h]
   int B, L, l_h;
   int CB;           // 64-channel blocks across D (tiles per time row) = D / 64
-  int halo;         // multiple of 16, >= l_h - 1, <= kMaxHalo
+  int halo;         // multiple of 16, >= l_h - 1, <= 128 * (history tiles of the kernel)
   int band_cols;    // TMEM columns of one group's band = (128 + halo) / 2
   int nbuf;         // band sets in TMEM (1 or 2)
   int nT;           // tiles per sequence = ceil(L / kTM)
   long long W;      // tiles of the walk: CB * B * nT, or (CB / 2) * B * nT when paired
   int paired;       // CTAs 2p and 2p+1 walk the same (block pair, batch, time) range, one
                     // block each, so both halves of every 256-byte row are read together
-  int run;          // > 0: strided schedule of runs of `run` tiles (see RunIter)
-  long long units;  // number of runs: B * ceil(nT / run) * CB
 };
 
 // One unit of a CTA's walk: a halo tile (input only) or an output tile.
 struct Item {
   int g, b, i;      // 64-channel block, sequence, tile index along time
   int seg;          // running segment number within this CTA (a segment = one sequence run)
-  bool halo;        // input-only tile feeding the first output tile of a segment
-  bool hist;        // the output tile reads the previous tile's X (i > 0)
+  bool halo;        // input-only tile feeding the first output tiles of a segment
   bool last;        // last output tile of its segment
 };
 
+// The walk of one CTA: tiles [w_begin, w_end) of the order (group, batch, time); with gmul = 2
+// the walk is over group pairs and this CTA takes group 2 * pair + goff.  A segment that starts
+// at tile i > 0 of a sequence is preceded by its min(i, nh) history tiles as halo items (input
+// only).  The position is decoded once; next() only increments (64-bit divisions are software
+// routines on the GPU).
 struct WorkIter {
   long long w, w_end;
-  int nT, B, seg, gmul, i, g, b;
+  int nT, B, seg, gmul, nh, hpend, i, g, b;
   bool at_begin, entered;
-  // Tiles [w_begin, w_end) of the walk ordered (group, batch, time); with gmul = 2 the walk is
-  // over group pairs and this CTA takes group 2 * pair + goff.  The position is decoded once;
-  // next() only increments (64-bit divisions are software routines on the GPU).
-  __device__ WorkIter(long long w_begin, long long w_end_, int nT_, int B_, int gmul_ = 1,
-                      int goff = 0)
-      : w(w_begin), w_end(w_end_), nT(nT_), B(B_), seg(-1), gmul(gmul_), at_begin(true),
-        entered(false) {
+  __device__ WorkIter(long long w_begin, long long w_end_, int nT_, int B_, int gmul_, int goff,
+                      int nh_)
+      : w(w_begin), w_end(w_end_), nT(nT_), B(B_), seg(-1), gmul(gmul_), nh(nh_), hpend(0),
+        at_begin(true), entered(false) {
     const long long seq = w_begin / nT;
     i = static_cast<int>(w_begin - seq * nT);
     g = static_cast<int>(seq / B) * gmul + goff;
@@ -139,19 +142,18 @@ struct WorkIter {
     if ((at_begin || i == 0) && !entered) {
       entered = true;
       ++seg;
-      if (i > 0) {
-        it.i = i - 1;
-        it.seg = seg;
-        it.halo = true;
-        it.hist = false;
-        it.last = false;
-        return true;
-      }
+      hpend = min(i, nh);
+    }
+    it.seg = seg;
+    if (hpend > 0) {
+      it.i = i - hpend;
+      it.halo = true;
+      it.last = false;
+      --hpend;
+      return true;
     }
     it.i = i;
-    it.seg = seg;
     it.halo = false;
-    it.hist = i > 0;
     it.last = (w + 1 == w_end) || (i + 1 == nT);
     ++w;
     at_begin = false;
@@ -165,73 +167,6 @@ struct WorkIter {
     }
     return true;
   }
-};
-
-// Strided schedule: the work is cut into runs of `run` consecutive tiles of one (group, batch)
-// sequence, numbered with the group fastest, then the run's time block, then the batch; CTA c
-// takes runs c, c + grid, c + 2 grid, ...  At any moment the CTAs hold neighbouring groups of
-// the same time rows, so together they read whole rows of [B, L, D] (DRAM page locality),
-// and the halo tile a run starts with was usually loaded into L2 moments earlier.
-struct RunIter {
-  long long u, ustep, units;
-  int nT, B, G, run, nblk, seg, i, iend;
-  bool in_run;
-  __device__ RunIter(long long first, long long step, long long n, int nT_, int B_, int G_, int r)
-      : u(first), ustep(step), units(n), nT(nT_), B(B_), G(G_), run(r),
-        nblk((nT_ + r - 1) / r), seg(-1), i(0), iend(0), in_run(false) {}
-  __device__ bool next(Item &it) {
-    if (!in_run) {
-      if (u >= units) return false;
-      const int g = static_cast<int>(u % G);
-      const long long rest = u / G;
-      const int blk = static_cast<int>(rest % nblk);
-      b_ = static_cast<int>(rest / nblk);
-      g_ = g;
-      i = blk * run;
-      iend = min(nT, i + run);
-      ++seg;
-      in_run = true;
-      if (i > 0) {
-        it.g = g_;
-        it.b = b_;
-        it.i = i - 1;
-        it.seg = seg;
-        it.halo = true;
-        it.hist = false;
-        it.last = false;
-        return true;
-      }
-    }
-    it.g = g_;
-    it.b = b_;
-    it.i = i;
-    it.seg = seg;
-    it.halo = false;
-    it.hist = i > 0;
-    it.last = i + 1 == iend;
-    if (++i == iend) {
-      in_run = false;
-      u += ustep;
-    }
-    return true;
-  }
-  int g_ = 0, b_ = 0;
-};
-
-// The walk of this CTA: contiguous tile ranges (kSched 0) or strided runs (1).
-template <int kSched>
-struct Walk;
-
-template <>
-struct Walk<0> : WorkIter {
-  __device__ Walk(const Params &p, long long w_begin, long long w_end, int gmul, int goff)
-      : WorkIter(w_begin, w_end, p.nT, p.B, gmul, goff) {}
-};
-
-template <>
-struct Walk<1> : RunIter {
-  __device__ Walk(const Params &p, long long, long long, int, int)
-      : RunIter(blockIdx.x, gridDim.x, p.units, p.nT, p.B, p.CB, p.run) {}
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
@@ -297,12 +232,23 @@ __device__ __forceinline__ void build_band_tmem(uint32_t band_col, int band_cols
   tmem_wait_st();
 }
 
-// kNG = 64 / d_g groups per tile (1, 2 or 4); MMA N = d_g.
-template <int kSched, int kNG>
+// kNG = 64 / d_g groups per tile (1, 2 or 4); MMA N = d_g.  kNH = ceil(halo / 128) earlier
+// tiles feed each tile's product (1 for l_h <= 129, up to 4 for l_h <= 513).
+template <int kNG, int kNH>
 __global__ void __launch_bounds__(kThreads, 1)
     fir_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
                   const Params p) {
+  using Ly = Layout<kNH>;
+  constexpr int kNQ = Ly::kNQ, kNX = Ly::kNX;
+  constexpr int kOffKV = Ly::kOffKV, kOffQ = Ly::kOffQ, kOffX = Ly::kOffX, kOffBar = Ly::kOffBar,
+                kOffMisc = Ly::kOffMisc;
+  constexpr int kBarKVFull = Ly::kBarKVFull, kBarKVEmpty = Ly::kBarKVEmpty,
+                kBarQFull = Ly::kBarQFull, kBarQEmpty = Ly::kBarQEmpty,
+                kBarYReady = Ly::kBarYReady, kBarXFull = Ly::kBarXFull,
+                kBarXEmpty = Ly::kBarXEmpty, kBarAccFull = Ly::kBarAccFull,
+                kBarAccEmpty = Ly::kBarAccEmpty, kBarAFull = Ly::kBarAFull,
+                kBarAEmpty = Ly::kBarAEmpty, kBarDone = Ly::kBarDone;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -361,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_launch_dependents();
   // Thread 0 is also the k/v producer: it queues the first k/v stages right away, before the
   // CTA-wide barrier (no other thread touches those stages yet).
-  Walk<kSched> kv_it(p, w_begin, w_end, gmul, goff);
+  WorkIter kv_it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH);
   Item kv_t;
   uint32_t kv_count = 0;
   bool kv_done = false;
@@ -405,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpTmaQ) {
     // ---------------------------------------------------------------- TMA producer: q
     if (lane == 0) {
-      Walk<kSched> it(p, w_begin, w_end, gmul, goff);
+      WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH);
       Item t;
       uint32_t qc = 0;
       while (it.next(t)) {
@@ -423,15 +369,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      Walk<kSched> it(p, w_begin, w_end, gmul, goff);
+      WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH);
       Item t;
-      uint32_t xc = 0, ac = 0;
-      int cur_seg = -1;
+      uint32_t xc = 0, ac = 0, seg_x0 = 0;
+      int cur_seg = -1, x_seg = -1;
       constexpr int kDG = kNC / kNG;
       const uint32_t idesc = umma_idesc_f16_f32(kTM, kDG, 0);  // N = d_g, B K-major
       const int hsteps = p.halo / 16;
+      // B = X^T, K-major with 128-byte swizzle: k-step s of a slot starts at K-block s / 4
+      // (8 KB each) plus 32 bytes per step inside the 128-byte rows; group gg's rows start
+      // gg * d_g channel rows (gg * d_g * 128 bytes) into the block.  Slot n starts n * 16 KB
+      // after slot 0 (descriptor address field in 16-byte units).
+      const uint64_t bd_x0 = umma_smem_desc(smem_u32(x_st), 16, 1024, 2);
+      // History k-step j covers input rows t0 - halo + 16 j ..; counted from the start of the
+      // oldest history tile (kNH tiles back) that is row hrow0 + 16 j.
+      const int hrow0 = kNH * kTM - p.halo;
       while (it.next(t)) {
         const int xs = xc % kNX;
+        if (t.seg != x_seg) {  // first item (halo or output) of a segment
+          x_seg = t.seg;
+          seg_x0 = xc;
+        }
         if (!thread_wait(&bars[kBarXFull + xs], (xc / kNX) & 1, abort)) break;
         if (t.halo) {
           ++xc;
@@ -447,36 +405,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int as = ac % kNAcc;
         if (!thread_wait(&bars[kBarAccEmpty + as], ((ac / kNAcc) & 1) ^ 1, abort)) break;
         tc_fence_after_sync();
-        const int xp = (xc + kNX - 1) % kNX;
         const uint32_t d_tmem = tmem_base + as * kNC;
         const uint32_t band0 = tmem_base + kBandCol0 + pa * kNG * p.band_cols;
-        // B = X^T, K-major with 128-byte swizzle: k-step s of a slot starts at K-block s / 4
-        // (8 KB each) plus 32 bytes per step inside the 128-byte rows; group gg's rows start
-        // gg * d_g channel rows (gg * d_g * 128 bytes) into the block.  A (group gg's band)
-        // advances 8 columns per k-step.
+        // A (group gg's band) advances 8 columns (16 K elements) per k-step.  History steps
+        // whose rows lie before the start of the sequence are zero and skipped.
+        const int jstart = max(0, (p.halo - t.i * kTM) / 16);
         uint32_t a_run[kNG];  // next band column of each group
 #pragma unroll
-        for (int gg = 0; gg < kNG; ++gg) a_run[gg] = band0 + gg * p.band_cols;
+        for (int gg = 0; gg < kNG; ++gg) a_run[gg] = band0 + gg * p.band_cols + 8 * jstart;
         uint32_t acc = 0;     // 0 only for the first MMA of each group's chain
-        if (t.hist) {
-          const uint64_t bd0 = umma_smem_desc(smem_u32(x_st + xp * kTileBytes), 16, 1024, 2);
-          const int s0 = (kTM - p.halo) / 16;
-          for (int j = 0; j < hsteps; ++j) {
-            const int st = s0 + j;
-            const uint64_t bdj = bd0 + ((st >> 2) * (kKBlockBytes >> 4) + (st & 3) * 2);
+        for (int j = jstart; j < hsteps; ++j) {
+          const int u = hrow0 + 16 * j;
+          // with one history tile (u < 128) the slot is the same for every step
+          const uint32_t slot = (xc + kNX - kNH + (kNH == 1 ? 0 : (u >> 7))) % kNX;
+          const int st = (u & (kTM - 1)) >> 4;
+          const uint64_t bdj = bd_x0 + (slot * (kTileBytes >> 4) + (st >> 2) * (kKBlockBytes >> 4) +
+                                        (st & 3) * 2);
 #pragma unroll
-            for (int gg = 0; gg < kNG; ++gg) {
-              umma_f16_ts(d_tmem + gg * kDG, a_run[gg], bdj + gg * (kDG * 8), idesc, acc);
-              a_run[gg] += 8;
-            }
-            acc = 1;
+          for (int gg = 0; gg < kNG; ++gg) {
+            umma_f16_ts(d_tmem + gg * kDG, a_run[gg], bdj + gg * (kDG * 8), idesc, acc);
+            a_run[gg] += 8;
           }
-        } else {
-#pragma unroll
-          for (int gg = 0; gg < kNG; ++gg) a_run[gg] += 8 * hsteps;  // zero history
+          acc = 1;
         }
         {
-          const uint64_t bd0 = umma_smem_desc(smem_u32(x_st + xs * kTileBytes), 16, 1024, 2);
+          const uint64_t bd0 = bd_x0 + xs * (kTileBytes >> 4);
 #pragma unroll
           for (int st = 0; st < kTM / 16; ++st) {
             const uint64_t bdj = bd0 + ((st >> 2) * (kKBlockBytes >> 4) + (st & 3) * 2);
@@ -489,9 +442,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         umma_commit(&bars[kBarAccFull + as]);
-        if (t.hist) umma_commit(&bars[kBarXEmpty + xp]);
+        // X slots go back to the gate warps after their last reader: the slot kNH items back
+        // is read by no later tile; at the end of a segment every slot still held is free.
+        if (xc >= seg_x0 + kNH) umma_commit(&bars[kBarXEmpty + (xc - kNH) % kNX]);
         if (t.last) {
-          umma_commit(&bars[kBarXEmpty + xs]);
+          for (uint32_t n = xc + 1 > seg_x0 + kNH ? xc + 1 - kNH : seg_x0; n <= xc; ++n)
+            umma_commit(&bars[kBarXEmpty + n % kNX]);
           umma_commit(&bars[kBarAEmpty + pa]);
         }
         ++xc;
@@ -503,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kWarpGate0 && warp < kWarpGate0 + 4) {
     // ---------------------------------------------------------------- pre-gate + band build
-    Walk<kSched> it(p, w_begin, w_end, gmul, goff);
+    WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH);
     Item t;
     uint32_t kc = 0, xc = 0;
     int cur_seg = -1;
@@ -558,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;               // TMEM lanes this warp may read
     const int row_lane = quad * 32 + lane;   // MMA row = TMEM lane
     const int r = kTM - 1 - row_lane;        // tile row (time offset) of that lane
-    Walk<kSched> it(p, w_begin, w_end, gmul, goff);
+    WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH);
     Item t;
     uint32_t ac = 0, qc = 0;
     while (it.next(t)) {

@@ -49,6 +49,7 @@ using tc::kRowBytes;
 using tc::kGroupThreads;
 using tc::kTimeoutBit;
 using tc::kF16RangeBit;
+constexpr int kMaxHalo = 128;  // one tile of history: l_h - 1 <= 128
 
 constexpr int kNKV = 2;   // k/v stages (32 KB each)
 constexpr int kNQ = 3;    // q stages; each becomes the tile's fp16 dz (channel-major, reversed)

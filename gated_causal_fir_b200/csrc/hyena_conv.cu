@@ -24,9 +24,6 @@ using hyena::cc::WindowParams;
 #ifndef HYENA_TC_PAIRED
 #define HYENA_TC_PAIRED 1
 #endif
-#ifndef HYENA_TC_RUN
-#define HYENA_TC_RUN 0
-#endif
 #ifndef HYENA_PDL
 #define HYENA_PDL 1
 #endif
@@ -57,17 +54,21 @@ int current_device(DeviceState *&ds) {
   DeviceState *d = ds;
   std::call_once(d->once, [d, dev]() {
     cudaError_t e = cudaDeviceGetAttribute(&d->sm_count, cudaDevAttrMultiProcessorCount, dev);
-    const void *kernels[] = {
-        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<0, 1>),
-        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<0, 2>),
-        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<0, 4>),
-        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 1>),
-        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 2>),
-        reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 4>)};
-    for (const void *k : kernels)
+    // Every (groups per tile, history tiles) instantiation with its shared-memory size.
+    const struct {
+      const void *fn;
+      int smem;
+    } kernels[] = {
+        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 1>), hyena::tc::Layout<1>::kSmemBytes},
+        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 2>), hyena::tc::Layout<2>::kSmemBytes},
+        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 3>), hyena::tc::Layout<3>::kSmemBytes},
+        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 4>), hyena::tc::Layout<4>::kSmemBytes},
+        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<2, 1>), hyena::tc::Layout<1>::kSmemBytes},
+        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<2, 2>), hyena::tc::Layout<2>::kSmemBytes},
+        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<4, 1>), hyena::tc::Layout<1>::kSmemBytes}};
+    for (const auto &k : kernels)
       if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 hyena::tc::kSmemBytes);
+        e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
     const void *dh_kernels[] = {
         reinterpret_cast<const void *>(hyena::bwd::fir_bwd_dh_partial_kernel<float>),
         reinterpret_cast<const void *>(hyena::bwd::fir_bwd_dh_partial_kernel<__nv_bfloat16>)};
@@ -129,7 +130,6 @@ int validate(const Problem &P) {
   if (P.B < 0 || P.L < 0 || P.D < 1 || P.d_g < 1 || P.l_h < 1 || P.l_b < 1)
     return HYENA_ERR_INVALID_ARG;
   if (P.D % P.d_g != 0) return HYENA_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(P.l_h) > 2 * static_cast<int64_t>(P.l_b)) return HYENA_ERR_INVALID_ARG;
   if (P.B == 0 || P.L == 0) return kEmpty;
   const int64_t lim = std::numeric_limits<int64_t>::max() / 8;
   if (P.B > lim / P.L || P.B * P.L > lim / P.D) return HYENA_ERR_INVALID_ARG;
@@ -148,16 +148,18 @@ bool all_aligned16(const Problem &P) {
   return aligned(P.q, 16) && aligned(P.k, 16) && aligned(P.v, 16) && aligned(P.y, 16);
 }
 
-// Tensor-core plan: history rows, one group's band width in TMEM columns and the number of
-// band sets (2 when they fit, else 1; 0 = does not fit).
+// Tensor-core plan: history rows, history tiles, one group's band width in TMEM columns and the
+// number of band sets (2 when they fit, else 1; 0 = does not fit).
 struct TcPlan {
-  int halo, band_cols, ng, nbuf;
+  int halo, nh, band_cols, ng, nbuf;
 };
 
 TcPlan tc_plan(const Problem &P) {
-  TcPlan t{0, 0, 0, 0};
+  TcPlan t{0, 0, 0, 0, 0};
   if (P.d_g != 16 && P.d_g != 32 && P.d_g != 64) return t;
+  if (P.l_h - 1 > hyena::tc::kMaxHalo) return t;
   t.halo = ((P.l_h - 1) + 15) / 16 * 16;
+  t.nh = t.halo <= hyena::tc::kTM ? 1 : (t.halo + hyena::tc::kTM - 1) / hyena::tc::kTM;
   t.band_cols = (hyena::tc::kTM + t.halo) / 2;
   t.ng = hyena::tc::kNC / P.d_g;
   const int room = hyena::tc::kTmemCols - hyena::tc::kBandCol0;
@@ -167,9 +169,8 @@ TcPlan tc_plan(const Problem &P) {
 
 bool tensor_supported(const Problem &P) {
   const int64_t i32 = std::numeric_limits<int32_t>::max();
-  return P.dtype == HYENA_DTYPE_BF16 && P.D % hyena::tc::kNC == 0 &&
-         P.l_h - 1 <= hyena::tc::kMaxHalo && tc_plan(P).nbuf > 0 && all_aligned16(P) &&
-         P.L <= i32 && P.B <= i32 && P.D <= i32;
+  return P.dtype == HYENA_DTYPE_BF16 && P.D % hyena::tc::kNC == 0 && tc_plan(P).nbuf > 0 &&
+         all_aligned16(P) && P.L <= i32 && P.B <= i32 && P.D <= i32;
 }
 
 bool window_supported(const Problem &P) {
@@ -226,15 +227,9 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
   p.nbuf = plan.nbuf;
   p.nT = static_cast<int>((P.L + hyena::tc::kTM - 1) / hyena::tc::kTM);
   const long long sms = ds->sm_count;
-  p.run = HYENA_TC_RUN;
-  p.units = 0;
-  p.paired = HYENA_TC_PAIRED && p.CB % 2 == 0 && sms >= 2 && p.run == 0;
+  p.paired = HYENA_TC_PAIRED && p.CB % 2 == 0 && sms >= 2;
   long long grid;
-  if (p.run > 0) {
-    p.units = static_cast<long long>(p.B) * ((p.nT + p.run - 1) / p.run) * p.CB;
-    p.W = static_cast<long long>(p.CB) * p.B * p.nT;
-    grid = p.units < sms ? p.units : sms;
-  } else if (p.paired) {
+  if (p.paired) {
     p.W = static_cast<long long>(p.CB / 2) * p.B * p.nT;
     grid = 2 * (p.W < sms / 2 ? p.W : sms / 2);
   } else {
@@ -242,7 +237,7 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
     grid = p.W < sms ? p.W : sms;
   }
   const unsigned g = static_cast<unsigned>(grid);
-  constexpr int T = hyena::tc::kThreads, S = hyena::tc::kSmemBytes;
+  constexpr int T = hyena::tc::kThreads;
   // Programmatic dependent launch: the kernel's set-up (barriers, tensor memory) overlaps the
   // tail of the previous kernel in the stream; it reads nothing before that kernel is done.
   cudaLaunchAttribute attr[1];
@@ -251,22 +246,23 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(g);
   cfg.blockDim = dim3(T);
-  cfg.dynamicSmemBytes = S;
+  cfg.dynamicSmemBytes = 0;  // set per instantiation below
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t le = cudaSuccess;
-#define HYENA_TC_LAUNCH(SCHED, NG)                                                          \
-  le = cudaLaunchKernelEx(&cfg, hyena::tc::fir_tc_kernel<SCHED, NG>, maps[0], maps[1], maps[2], \
+#define HYENA_TC_LAUNCH(NG, NH)                                                            \
+  cfg.dynamicSmemBytes = hyena::tc::Layout<NH>::kSmemBytes;                                  \
+  le = cudaLaunchKernelEx(&cfg, hyena::tc::fir_tc_kernel<NG, NH>, maps[0], maps[1], maps[2], \
                           maps[3], p)
-  const int sched = p.run > 0 ? 1 : 0;
-  switch (sched * 8 + plan.ng) {
-    case 1: HYENA_TC_LAUNCH(0, 1); break;
-    case 2: HYENA_TC_LAUNCH(0, 2); break;
-    case 4: HYENA_TC_LAUNCH(0, 4); break;
+  switch (plan.ng * 8 + plan.nh) {
     case 9: HYENA_TC_LAUNCH(1, 1); break;
     case 10: HYENA_TC_LAUNCH(1, 2); break;
+    case 11: HYENA_TC_LAUNCH(1, 3); break;
     case 12: HYENA_TC_LAUNCH(1, 4); break;
+    case 17: HYENA_TC_LAUNCH(2, 1); break;
+    case 18: HYENA_TC_LAUNCH(2, 2); break;
+    case 33: HYENA_TC_LAUNCH(4, 1); break;
     default: return HYENA_ERR_UNSUPPORTED;
   }
 #undef HYENA_TC_LAUNCH
@@ -452,7 +448,7 @@ int run_bwd_cuda_core(const Problem &P, const void *dy, void *dq, void *dk, void
 bool tc_bwd_supported(const Problem &P, const void *dy, const void *dq, const void *dk,
                       const void *dv) {
   return P.dtype == HYENA_DTYPE_BF16 && P.d_g == hyena::tc::kNC && P.D % hyena::tc::kNC == 0 &&
-         P.l_h <= hyena::tc::kMaxHalo + 1 && P.L <= (int64_t{1} << 30) &&
+         P.l_h <= hyena::tcb::kMaxHalo + 1 && P.L <= (int64_t{1} << 30) &&
          P.B <= (int64_t{1} << 30) && aligned(P.q, 16) && aligned(P.k, 16) &&
          aligned(P.v, 16) && aligned(dy, 16) && aligned(dq, 16) && aligned(dk, 16) &&
          aligned(dv, 16);
@@ -701,6 +697,28 @@ int hyena_build_toeplitz(const float *h, float *H0, float *H1, float *H2_or_null
   if (blocks > cap) blocks = cap;
   hyena::cc::toeplitz_blocks_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
       h, H0, H1, H2_or_null, G, l_h, l_b);
+  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+int hyena_toeplitz_stages(int l_h, int l_b) {
+  if (l_h < 1 || l_b < 1) return -HYENA_ERR_INVALID_ARG;
+  return 1 + static_cast<int>((static_cast<int64_t>(l_h) - 1 + l_b - 1) / l_b);
+}
+
+int hyena_build_toeplitz_blocks(const float *h, float *Hm, int S, int G, int l_h, int l_b,
+                                cudaStream_t stream) {
+  if (!h || !Hm || S < 1 || G < 1 || l_h < 1 || l_b < 1) return HYENA_ERR_INVALID_ARG;
+  const int64_t sg = static_cast<int64_t>(S) * G, blk = static_cast<int64_t>(l_b) * l_b;
+  if (blk > std::numeric_limits<int64_t>::max() / 8 / sg) return HYENA_ERR_INVALID_ARG;
+  const int64_t n = sg * blk;
+  if (!aligned(h, 4) || !aligned(Hm, 4)) return HYENA_ERR_MISALIGNED;
+  DeviceState *ds = nullptr;
+  if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
+  long long blocks = (n + 255) / 256;
+  const long long cap = static_cast<long long>(ds->sm_count) * 8;
+  if (blocks > cap) blocks = cap;
+  hyena::cc::toeplitz_stack_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      h, Hm, S, G, l_h, l_b);
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 

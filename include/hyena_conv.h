@@ -41,7 +41,7 @@ typedef struct CUstream_st *cudaStream_t;
 enum hyena_status {
     HYENA_OK = 0,
     HYENA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, D % d_g != 0, l_h < 1,
-                                    l_b < 1, l_h > 2*l_b, overlapping y, unknown dtype/algo */
+                                    l_b < 1, overlapping y, unknown dtype/algo */
     HYENA_ERR_UNSUPPORTED = 2,   /* a forced algorithm cannot run this shape or alignment */
     HYENA_ERR_MISALIGNED = 3,    /* a pointer is not aligned to its element size */
     HYENA_ERR_CUDA = 4           /* the CUDA runtime reported an error for this call */
@@ -55,8 +55,9 @@ enum hyena_dtype {
 enum hyena_algo {
     HYENA_ALGO_AUTO = 0,         /* pick the fastest algorithm that supports the problem */
     HYENA_ALGO_TENSOR = 1,       /* tcgen05 tensor-core block-Toeplitz GEMM (bf16 only;
-                                    D % 64 == 0, d_g in {16, 32, 64}, l_h <= 129, and
-                                    l_h <= 65 when d_g == 16; 16-byte aligned tensors) */
+                                    D % 64 == 0, d_g in {16, 32, 64}; l_h <= 513 for
+                                    d_g == 64, <= 257 for d_g == 32, <= 65 for d_g == 16;
+                                    16-byte aligned tensors) */
     HYENA_ALGO_WINDOW = 2,       /* CUDA-core register sliding window (l_h <= 16; d_g a
                                     multiple of 8 channels for bf16, 4 for fp32; 16-byte
                                     aligned tensors) */
@@ -72,9 +73,12 @@ enum hyena_device_status_bits {
 
 /*
  * Gated grouped causal FIR forward, bf16 q/k/v/y (the Hyena-SE / Hyena-MR operator).
- * l_b is the block size of the block-Toeplitz decomposition.  The result is the same for every
- * l_b (the decomposition is exact); l_b only bounds the filter length, l_h <= 2*l_b, which is
- * the domain the two-stage method is stated for.  All tensors 2-byte aligned.
+ * l_b is the block size of the block-Toeplitz decomposition (page 04, Sec. 2).  Any l_h >= 1 is
+ * accepted: the block form with S = 1 + ceil((l_h - 1) / l_b) sub-block diagonals is exact for
+ * every filter length (the two-stage form of Sec. 3 is the case S = 2, l_h <= l_b + 1), so the
+ * result does not depend on l_b.  The kernels pick their own internal block size.  Filters
+ * longer than the tensor path's limit (HYENA_ALGO_TENSOR above) run on the CUDA-core direct
+ * kernel.  All tensors 2-byte aligned.
  */
 int hyena_conv_fwd(const void *q, const void *k, const void *v, const float *h, void *y,
                    int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
@@ -122,7 +126,7 @@ int64_t hyena_conv_bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g,
  *
  * q, k, v, dy, dq, dk, dv: DEVICE [B, L, D] tensors of `dtype`, layout as the forward.
  * h: DEVICE fp32 [D / d_g, l_h].  dh: DEVICE fp32 [D / d_g, l_h], overwritten (not
- * accumulated into).  The forward's shape rules (l_h <= 2*l_b) apply.  Algorithm (AUTO): where
+ * accumulated into).  The forward's shape rules apply (any l_h >= 1).  Algorithm (AUTO): where
  * the tensor path applies (bf16, d_g == 64, D % 64 == 0, l_h <= 129, all seven tensors
  * 16-byte aligned) one fused tcgen05 kernel reads q, k, v, dy once and writes dq, dk, dv once,
  * with fp16 operands (x = k v, dz = q dy, h rounded to fp16) and fp32 accumulation; otherwise
@@ -196,6 +200,27 @@ int hyena_conv_bwd_static_scratch(const void *q, const void *k, const void *v, c
  */
 int hyena_build_toeplitz(const float *h, float *H0, float *H1, float *H2_or_null, int G,
                          int l_h, int l_b, cudaStream_t stream);
+
+/*
+ * Host-only: the number S = 1 + ceil((l_h - 1) / l_b) of sub-block diagonals of the
+ * lower-triangular Toeplitz matrix that hold a filter tap (page 04, Sec. 2 block convolution:
+ * H_m is zero for m >= S).  Returns minus HYENA_ERR_INVALID_ARG for l_h < 1 or l_b < 1.
+ */
+int hyena_toeplitz_stages(int l_h, int l_b);
+
+/*
+ * All S sub-block diagonals of the block-Toeplitz decomposition (page 04, Sec. 2, with the
+ * index rule of the Sec. 3 worked example), for any filter length:
+ *     Hm[m][g][i][j] = h[g][m*l_b + i - j]  if 0 <= m*l_b + i - j < l_h,  else 0,
+ * for m = 0 .. S-1, written to Hm, a DEVICE fp32 [S, G, l_b, l_b] array owned by the caller.
+ * h: DEVICE fp32 [G, l_h].  The decomposition y_n = sum_m H_m x_{n-m} is exact when
+ * S >= hyena_toeplitz_stages(l_h, l_b); a smaller S gives the leading diagonals only.
+ * Asynchronous on `stream`.  Errors: HYENA_ERR_INVALID_ARG for null h/Hm, S < 1, G < 1,
+ * l_h < 1, l_b < 1 or an output too large to index; HYENA_ERR_MISALIGNED for pointers that
+ * are not 4-byte aligned; HYENA_ERR_CUDA for a launch failure.
+ */
+int hyena_build_toeplitz_blocks(const float *h, float *Hm, int S, int G, int l_h, int l_b,
+                                cudaStream_t stream);
 
 /*
  * Reads (and, if clear != 0, resets) the status word of the current device: an OR of

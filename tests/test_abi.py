@@ -47,7 +47,8 @@ def test_select_algo_for_the_workloads(lib):
 
 def test_select_algo_fallbacks(lib):
     bf, f32 = g.HYENA_DTYPE_BF16, g.HYENA_DTYPE_F32
-    assert g.hyena_select_algo(1, 100, 256, 64, 130, 65, bf) == g.HYENA_ALGO_DIRECT  # l_h > 129
+    assert g.hyena_select_algo(1, 100, 256, 64, 514, 65, bf) == g.HYENA_ALGO_DIRECT  # l_h > 513
+    assert g.hyena_select_algo(1, 100, 256, 64, 130, 65, bf) == g.HYENA_ALGO_TENSOR  # 2 tiles back
     assert g.hyena_select_algo(1, 100, 256, 64, 129, 65, bf) == g.HYENA_ALGO_TENSOR
     assert g.hyena_select_algo(1, 100, 128, 32, 40, 32, bf) == g.HYENA_ALGO_TENSOR
     assert g.hyena_select_algo(1, 100, 96, 32, 40, 32, bf) == g.HYENA_ALGO_DIRECT   # D % 64 != 0
@@ -77,11 +78,13 @@ def _call(lib, q=0x10000, k=0x20000, v=0x30000, h=0x40000, y=0x50000, dtype=0, a
 @pytest.mark.parametrize("kw,code", [
     (dict(q=None), 1), (dict(k=None), 1), (dict(v=None), 1), (dict(h=None), 1), (dict(y=None), 1),
     (dict(B=-1), 1), (dict(L=-5), 1), (dict(D=0), 1), (dict(d_g=0), 1), (dict(d_g=48), 1),
-    (dict(l_h=0), 1), (dict(l_b=0), 1), (dict(l_h=33, l_b=16), 1), (dict(dtype=7), 1),
+    (dict(l_h=0), 1), (dict(l_b=0), 1), (dict(dtype=7), 1),
     (dict(algo=9), 1), (dict(y=0x10000 + 64), 1), (dict(q=0x10001), 3), (dict(h=0x40002), 3),
     (dict(algo=1, dtype=1), 2), (dict(algo=1, d_g=8, l_h=8, l_b=8), 2),
     (dict(algo=2, l_h=17, l_b=16), 2),
     (dict(algo=1, q=0x10002), 2),
+    (dict(algo=1, l_h=514, l_b=16), 2),                  # past the tensor path's 513 taps
+    (dict(algo=1, d_g=32, l_h=258, l_b=16), 2),          # d_g 32: bands fit up to 257 taps
 ])
 def test_host_validation(lib, kw, code):
     assert _call(lib, **kw) == code
@@ -103,6 +106,44 @@ def test_toeplitz_validation(lib):
     assert f(0x1000, 0x2000, 0x3000, 0x4000, 4, 9, 4, None) == 1  # l_h > 2 l_b
     assert f(0x1000, 0x2000, 0x3000, 0x4000, 0, 4, 3, None) == 1
     assert f(0x1001, 0x2000, 0x3000, 0x4000, 4, 4, 3, None) == 3
+
+
+def test_toeplitz_blocks_validation(lib):
+    f = lib.hyena_build_toeplitz_blocks
+    assert f(None, 0x2000, 3, 4, 9, 4, None) == 1
+    assert f(0x1000, None, 3, 4, 9, 4, None) == 1
+    assert f(0x1000, 0x2000, 0, 4, 9, 4, None) == 1
+    assert f(0x1000, 0x2000, 3, 0, 9, 4, None) == 1
+    assert f(0x1000, 0x2000, 3, 4, 0, 4, None) == 1
+    assert f(0x1000, 0x2000, 3, 4, 9, 0, None) == 1
+    assert f(0x1000, 0x2000, 1 << 30, 1 << 30, 9, 1 << 20, None) == 1  # too large to index
+    assert f(0x1002, 0x2000, 3, 4, 9, 4, None) == 3
+    assert f(0x1000, 0x2001, 3, 4, 9, 4, None) == 3
+
+
+@pytest.mark.parametrize("l_h,l_b,S", [(1, 1, 1), (2, 1, 2), (4, 3, 2), (5, 3, 3), (7, 16, 2),
+                                       (17, 16, 2), (18, 16, 3), (128, 64, 3), (129, 64, 3),
+                                       (130, 64, 4), (300, 64, 6), (1000, 7, 144)])
+def test_toeplitz_stages(lib, l_h, l_b, S):
+    import oracle
+    assert lib.hyena_toeplitz_stages(l_h, l_b) == S == oracle.stages_needed(l_h, l_b)
+
+
+def test_toeplitz_stages_validation(lib):
+    assert lib.hyena_toeplitz_stages(0, 4) == -1
+    assert lib.hyena_toeplitz_stages(4, 0) == -1
+
+
+def test_long_filters_select_an_algorithm():
+    bf = g.HYENA_DTYPE_BF16
+    assert g.hyena_select_algo(1, 8192, 4096, 64, 130, 64, bf) == g.HYENA_ALGO_TENSOR
+    assert g.hyena_select_algo(1, 8192, 4096, 64, 513, 64, bf) == g.HYENA_ALGO_TENSOR
+    assert g.hyena_select_algo(1, 8192, 4096, 64, 514, 64, bf) == g.HYENA_ALGO_DIRECT
+    assert g.hyena_select_algo(1, 8192, 4096, 32, 257, 64, bf) == g.HYENA_ALGO_TENSOR
+    assert g.hyena_select_algo(1, 8192, 4096, 32, 258, 64, bf) == g.HYENA_ALGO_DIRECT
+    assert g.hyena_select_algo(1, 8192, 4096, 16, 66, 16, bf) == g.HYENA_ALGO_DIRECT
+    assert g.hyena_select_algo(1, 8192, 4096, 64, 300, 64, g.HYENA_DTYPE_F32) == \
+        g.HYENA_ALGO_DIRECT
 
 
 def test_device_status_needs_out(lib):
@@ -145,5 +186,4 @@ def test_select_bwd_algo(lib):
     assert g.hyena_select_bwd_algo(1, 8192, 4096, 64, 128, 64, g.HYENA_DTYPE_F32) == Dd
     assert g.hyena_select_bwd_algo(1, 300, 4096, 64, 130, 65) == Dd   # l_h > 129
     assert g.hyena_select_bwd_algo(1, 300, 96, 32, 16, 16) == Dd
-    with pytest.raises(g.HyenaError):
-        g.hyena_select_bwd_algo(1, 300, 96, 32, 100, 16)                # l_h > 2 l_b
+    assert g.hyena_select_bwd_algo(1, 300, 4096, 64, 300, 16) == Dd   # l_h > 2 l_b: block form

@@ -66,6 +66,17 @@ SHAPES = [
     ("dg4", 1, 200, 60, 4, 5, 3, "bf16"),
     ("dg3_odd", 1, 300, 30, 3, 4, 2, "bf16"),
     ("long_filter", 1, 600, 128, 64, 200, 100, "bf16"),
+    # filters past 2 l_b (the general block form; 2 to 4 earlier tiles feed each output tile)
+    ("lh256_lb64", 2, 1500, 256, 64, 256, 64, "bf16"),
+    ("lh385_ragged", 1, 2000, 128, 64, 385, 64, "bf16"),
+    ("lh513_ragged", 2, 1700, 128, 64, 513, 32, "bf16"),
+    ("lh300_multiseg", 3, 1100, 512, 64, 300, 64, "bf16"),
+    ("lh513_short_runs", 1, 19200, 128, 64, 513, 64, "bf16"),
+    ("lh400_L77", 1, 77, 128, 64, 400, 64, "bf16"),
+    ("dg32_lh257", 1, 900, 128, 32, 257, 64, "bf16"),
+    ("dg32_lh200_multiseg", 2, 3000, 256, 32, 200, 16, "bf16"),
+    ("lh600_direct", 1, 400, 64, 64, 600, 64, "bf16"),
+    ("f32_long", 1, 500, 64, 16, 300, 8, "f32"),
     ("f32_tiny_like", 2, 1000, 64, 16, 7, 16, "f32"),
     ("f32_mr_like", 1, 500, 128, 64, 128, 64, "f32"),
     ("f32_dg2", 1, 300, 10, 2, 3, 2, "f32"),
@@ -74,8 +85,9 @@ SHAPES = [
 
 def _tensor_fits(D, d_g, l_h):
     """The tensor kernel's plan: 64-channel tiles of 64 / d_g groups, one Toeplitz band of
-    (128 + halo) / 2 TMEM columns per group, next to 128 accumulator columns (512 in all)."""
-    if d_g not in (16, 32, 64) or D % 64 or l_h > 129:
+    (128 + halo) / 2 TMEM columns per group, next to 128 accumulator columns (512 in all);
+    at most 4 earlier 128-row tiles of history (halo <= 512)."""
+    if d_g not in (16, 32, 64) or D % 64 or l_h > 513:
         return False
     halo = (l_h - 1 + 15) // 16 * 16
     return (64 // d_g) * (128 + halo) // 2 <= 384
@@ -167,6 +179,42 @@ def test_toeplitz_builder(l_h, l_b):
         ref = oracle.toeplitz_blocks(h[gi].cpu(), l_b, 3)
         for m, Hm in enumerate((H0, H1, H2)):
             assert np.array_equal(Hm[gi].cpu().double().numpy(), ref[m]), (gi, m)
+
+
+@pytest.mark.parametrize("l_h,l_b,S", [(4, 3, None), (128, 64, None), (300, 64, None),
+                                       (513, 32, None), (9, 4, 5), (200, 100, 1)])
+def test_toeplitz_blocks_builder(l_h, l_b, S):
+    """All sub-block diagonals of any filter length, against the oracle's decomposition."""
+    G = 3
+    h = torch.randn(G, l_h, generator=torch.Generator().manual_seed(l_h + 1)).cuda()
+    Hm = g.hyena_build_toeplitz_blocks(h, l_b, S)
+    torch.cuda.synchronize()
+    S = oracle.stages_needed(l_h, l_b) if S is None else S
+    assert Hm.shape == (S, G, l_b, l_b)
+    for gi in range(G):
+        ref = oracle.toeplitz_blocks(h[gi].cpu(), l_b, S)
+        assert np.array_equal(Hm[:, gi].cpu().double().numpy(), ref), gi
+
+
+@pytest.mark.parametrize("shape", [
+    # name, B, L, D, d_g, l_h
+    ("int_lh200", 2, 1300, 256, 64, 200),
+    ("int_lh385", 1, 2100, 128, 64, 385),
+    ("int_lh513", 3, 900, 128, 64, 513),
+    ("int_lh513_runs", 1, 19200, 128, 64, 513),
+    ("int_dg32_lh250", 2, 1000, 128, 32, 250),
+], ids=lambda s: s[0])
+def test_long_filter_integer_exact(shape):
+    """Integer inputs make every fp16 operand, product and fp32 partial sum exact, so the tensor
+    path must give the oracle's result rounded once to bf16, bit for bit: any tap applied to
+    the wrong row (a history tile or slot off by one) changes an output."""
+    from gated_causal_fir_b200.workloads import make_integer_inputs
+    name, B, L, D, d_g, l_h = shape
+    wl = custom(name, B, L, D, d_g, l_h, 64, "bf16", "mr", seed=l_h)
+    q, k, v, _, h = make_integer_inputs(wl, device="cuda")
+    y = _run(q, k, v, h, wl, g.HYENA_ALGO_TENSOR)
+    ref = torch.from_numpy(U.oracle_full(q, k, v, h, d_g)).to(torch.bfloat16)
+    assert torch.equal(y.cpu(), ref)
 
 
 def test_f16_operand_range_is_reported():
