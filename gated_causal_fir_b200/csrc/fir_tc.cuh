@@ -7,26 +7,29 @@
 // group, which turns the per-channel products into one GEMM) and the Sec. 6 chunk-direction
 // schedule (each CTA walks consecutive chunks and keeps the previous chunk's input on chip).
 //
-// One tile = 128 output rows x 64 channels (one group of d_g = 64).  The block size of the
-// decomposition is 128 rows, the largest M of one tcgen05.mma: Yhat_n = H0 Xhat_n + H1 Xhat_{n-1}
-// is then exact for l_h <= 129 (two stages suffice iff l_h <= l_b + 1).  As one GEMM per tile:
-//   D[128 x 64] = A[128 x K] * X[K x 64],  K = 128 + halo,  halo = roundup16(l_h - 1),
+// One tile = 128 output rows x 64 channels (64 / d_g groups).  The block size of the
+// decomposition is 128 rows, the largest M of one tcgen05.mma.  A tile reads its own 128 input
+// rows and halo = roundup16(l_h - 1) rows before them, which lie in the kNH = ceil(halo / 128)
+// earlier tiles (one for l_h <= 129, where this is the two-stage form of Sec. 3; up to four for
+// l_h <= 513, the general block form of Sec. 2).  As one GEMM per tile and group:
+//   D[128 x d_g] = A[128 x K] * X[K x d_g],  K = 128 + halo,
 // A is the Toeplitz band over input rows [t0 - halo, t0 + 128), X = k*v over those rows.
 //
 // B200 specifics:
 //  * q, k, v tiles arrive by TMA (128-byte swizzle) into a multi-stage ring; y leaves by TMA
-//    store.  The k*v pre-gate is an elementwise pass that writes fp16 X in the same swizzled
-//    layout, which is exactly the MN-major SW128 operand layout of tcgen05: no transpose.
-//  * The Toeplitz band is Hankel once the output rows are reversed (TMEM lane p holds time
-//    t0 + 127 - p): every 8x8 core matrix then depends only on r8 + c8.  A K-major, unswizzled
-//    descriptor with LBO = SBO = 128 bytes aliases those core matrices, so the whole
-//    128 x 256 band lives in 47 core matrices (6 KB) instead of 64 KB.
+//    store.  The gate warps turn each time-major k, v tile into fp16 X^T (channels as rows,
+//    K-major, 128-byte swizzle) with ldmatrix / stmatrix.trans: the B operand of tcgen05.
+//  * The band lives in tensor memory (A operand of tcgen05.mma read from TMEM), written once
+//    per sequence run by the gate warps with tcgen05.st: output rows are reversed (TMEM lane p
+//    holds time t0 + 127 - p), so lane p's row is A[p][kk] = h[127 + halo - p - kk].
 //  * Accumulators live in TMEM (2 x 64 columns); the epilogue reads them with tcgen05.ld,
 //    multiplies by q and rounds to bf16 in registers, and writes y over the q tile in place.
 //  * Warp roles: 0 TMA producer of k and v, 10 TMA producer of q, 1 MMA issuer (+ TMEM
-//    owner), 2-5 pre-gate / operand build, 6-9 epilogue.  Persistent grid: one CTA per SM, each walks a contiguous range of tiles
-//    ordered (group, batch, time), so a halo tile is re-read only where a range starts inside
-//    a sequence.
+//    owner), 2-5 pre-gate / operand build, 6-9 epilogue.  Persistent grid: one CTA per SM, each
+//    walks a contiguous range of tiles ordered (group, batch, time), so halo tiles are re-read
+//    only where a range starts inside a sequence.
+//  * Launched with programmatic stream serialisation: barrier set-up and the TMEM allocation
+//    overlap the previous kernel; nothing global is read before griddepcontrol.wait.
 //  * Every wait is bounded (ptx.cuh); a timeout raises HYENA_DEVICE_TIMEOUT, all roles leave
 //    their loops, in-flight copies and MMAs are drained and TMEM is freed before exit.
 #pragma once
