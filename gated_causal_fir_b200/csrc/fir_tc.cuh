@@ -62,6 +62,10 @@ constexpr int kKBlockBytes = kNC * 128;                         // 64 times x 64
 constexpr int kBandCol0 = kNAcc * kNC;                           // 128
 constexpr int kTmemCols = 512;
 
+constexpr int kThreads = 352;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGate0 = 2, kWarpEpi0 = 6, kWarpTmaQ = 10;
+constexpr int kGroupThreads = 128;
+
 // Shared-memory layout for a kernel whose tiles read kNH earlier tiles (halo <= 128 kNH rows):
 // k/v stages, q stages (reused in place for y), and kNH + 2 fp16 X slots (the kNH tiles of
 // history, the current tile and the next one being gated).
@@ -72,7 +76,12 @@ struct Layout {
   static constexpr int kOffKV = 0;
   static constexpr int kOffQ = kOffKV + kNKV * 2 * kTileBytes;
   static constexpr int kOffX = kOffQ + kNQ * kTileBytes;
-  static constexpr int kOffBar = kOffX + kNX * kTileBytes;
+  // fp16 filter taps of the tile's groups, zero-padded: 258 + halo per group (see stage_taps);
+  // kPer of them per gate thread
+  static constexpr int kHzBytes = kNH == 1 ? 2688 : (kNH == 2 ? 2064 : 1552);
+  static constexpr int kPer = (kHzBytes / 2 + kGroupThreads - 1) / kGroupThreads;
+  static constexpr int kOffHz = kOffX + kNX * kTileBytes;
+  static constexpr int kOffBar = kOffHz + kHzBytes;
   // barriers
   static constexpr int kBarKVFull = 0;
   static constexpr int kBarKVEmpty = kBarKVFull + kNKV;
@@ -85,16 +94,14 @@ struct Layout {
   static constexpr int kBarAccEmpty = kBarAccFull + kNAcc;
   static constexpr int kBarAFull = kBarAccEmpty + kNAcc;
   static constexpr int kBarAEmpty = kBarAFull + 2;  // up to two band sets
-  static constexpr int kBarDone = kBarAEmpty + 2;
+  static constexpr int kBarGate = kBarAEmpty + 2;   // the 128 gate threads among themselves
+  static constexpr int kBarDone = kBarGate + 1;
   static constexpr int kNumBars = kBarDone + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget of one CTA exceeded");
 };
 
-constexpr int kThreads = 352;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGate0 = 2, kWarpEpi0 = 6, kWarpTmaQ = 10;
-constexpr int kGroupThreads = 128;
 
 constexpr unsigned kTimeoutBit = 1u;  // HYENA_DEVICE_TIMEOUT
 constexpr unsigned kF16RangeBit = 2u; // HYENA_DEVICE_F16_RANGE
@@ -197,24 +204,55 @@ __device__ __forceinline__ uint32_t gate_pair(uint32_t kw, uint32_t vw, bool &ov
   return *reinterpret_cast<const uint32_t *>(&hx);
 }
 
+// Filter taps of the tile's kNG groups, staged once per sequence run by the 128 gate threads:
+// group gg's taps start at hz + gg (258 + halo) + 2, and hz_g[i] = fp16(h[g kNG + gg][i - 127])
+// for 0 <= i - 127 < l_h, else 0, for -2 <= i < 256 + halo.  One coalesced pass over the
+// filters instead of each band lane fetching its own taps.  The loads (tap_load) are issued
+// into registers and written to shared memory later (tap_store), so their latency can overlap
+// other work.
+template <int kPer>
+__device__ __forceinline__ void tap_load(float (&v)[kPer], const float *hblk, int l_h, int halo,
+                                         int ng, int tid) {
+  const int stride = 258 + halo;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int e = tid + k * kGroupThreads;
+    const int gg = e / stride, idx = e - gg * stride - 2 - 127;
+    v[k] = (gg < ng && idx >= 0 && idx < l_h) ? __ldg(hblk + gg * l_h + idx) : 0.f;
+  }
+}
+
+template <int kPer>
+__device__ __forceinline__ void tap_store(uint16_t *hz, const float (&v)[kPer], int halo, int ng,
+                                          int tid, bool &over) {
+  const int n = ng * (258 + halo);
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int e = tid + k * kGroupThreads;
+    if (e < n) {
+      over |= fabsf(v[k]) > 65504.f;
+      const __half hv = __float2half_rn(v[k]);
+      hz[e] = *reinterpret_cast<const uint16_t *>(&hv);
+    }
+  }
+}
+
 // The Toeplitz band of one group in tensor memory.  Output rows are reversed (lane p holds
 // time t0 + 127 - p) and K runs over input rows t0 - halo .. t0 + 127, so
-//     A[p][kk] = h[127 + halo - p - kk]   (zero outside [0, l_h)),  rounded to fp16.
-// Each of the 128 gate threads writes its own lane: 128 + halo K elements = band_cols columns.
-// Columns [c0, c0 + N) of one lane's band row: 2 N taps loaded together, then one store.
+//     A[p][kk] = h[127 + halo - p - kk]   (zero outside [0, l_h))  = hz_g[254 + halo - p - kk].
+// Each of the 128 gate threads writes its own lane, 128 + halo K elements = band_cols columns
+// (two fp16 K elements per 32-bit column, the lower K index in the low half), 32 (then 8)
+// columns per tcgen05.st.  Column c needs hz_g[i0 - 2c] and hz_g[i0 - 2c - 1], i0 = 254 + halo
+// - p: with i0 odd both lie in 32-bit word (i0 - 1) / 2 - c (halves swapped); with i0 even they
+// are the low half of word i0 / 2 - c and the high half of the word below it.
 template <int N>
-__device__ __forceinline__ void band_chunk(uint32_t taddr, int c0, int row, const float *hg,
-                                           int l_h, int halo, bool &over) {
-  uint32_t r[N];
+__device__ __forceinline__ void band_chunk(uint32_t taddr, int c0, const uint32_t *hw, int m0,
+                                           uint32_t sel) {
+  uint32_t w[N + 1], r[N];
 #pragma unroll
-  for (int c = 0; c < N; ++c) {
-    const int idx = kTM - 1 + halo - row - 2 * (c0 + c);  // tap of K element 2 (c0 + c)
-    const float v0 = (idx >= 0 && idx < l_h) ? __ldg(hg + idx) : 0.f;
-    const float v1 = (idx - 1 >= 0 && idx - 1 < l_h) ? __ldg(hg + idx - 1) : 0.f;
-    over |= (fabsf(v0) > 65504.f) | (fabsf(v1) > 65504.f);
-    const __half2 hv = __floats2half2_rn(v0, v1);
-    r[c] = *reinterpret_cast<const uint32_t *>(&hv);
-  }
+  for (int c = 0; c <= N; ++c) w[c] = hw[m0 - c0 - c];
+#pragma unroll
+  for (int c = 0; c < N; ++c) r[c] = __byte_perm(w[c], w[c + 1], sel);
   if constexpr (N == 32)
     tmem_st_32x32b_x32(taddr + c0, r);
   else
@@ -222,16 +260,19 @@ __device__ __forceinline__ void band_chunk(uint32_t taddr, int c0, int row, cons
 }
 
 __device__ __forceinline__ void build_band_tmem(uint32_t band_col, int band_cols,
-                                                uint32_t tmem_base, const float *hg, int l_h,
-                                                int halo, int quad, int lane, bool &over) {
+                                                uint32_t tmem_base, const uint16_t *hzg, int halo,
+                                                int quad, int lane) {
   const int row = quad * 32 + lane;
   const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + band_col;
+  const int i0 = 254 + halo - row;
+  const uint32_t sel = (i0 & 1) ? 0x1032u : 0x7610u;
+  const uint32_t *hw = reinterpret_cast<const uint32_t *>(hzg);  // hzg is 4-byte aligned
+  const int m0 = i0 >> 1;  // the lowest word read is m0 - band_cols >= -1 (the zero pad)
   int c0 = 0;
-  // 32 columns (64 taps in flight) per step, then the 8-column remainder.
 #pragma unroll 1
-  for (; c0 + 32 <= band_cols; c0 += 32) band_chunk<32>(taddr, c0, row, hg, l_h, halo, over);
+  for (; c0 + 32 <= band_cols; c0 += 32) band_chunk<32>(taddr, c0, hw, m0, sel);
 #pragma unroll 1
-  for (; c0 < band_cols; c0 += 8) band_chunk<8>(taddr, c0, row, hg, l_h, halo, over);
+  for (; c0 < band_cols; c0 += 8) band_chunk<8>(taddr, c0, hw, m0, sel);
   tmem_wait_st();
 }
 
@@ -251,13 +292,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 kBarYReady = Ly::kBarYReady, kBarXFull = Ly::kBarXFull,
                 kBarXEmpty = Ly::kBarXEmpty, kBarAccFull = Ly::kBarAccFull,
                 kBarAccEmpty = Ly::kBarAccEmpty, kBarAFull = Ly::kBarAFull,
-                kBarAEmpty = Ly::kBarAEmpty, kBarDone = Ly::kBarDone;
+                kBarAEmpty = Ly::kBarAEmpty, kBarGate = Ly::kBarGate, kBarDone = Ly::kBarDone;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *kv_st = smem + kOffKV;
   uint8_t *q_st = smem + kOffQ;
   uint8_t *x_st = smem + kOffX;
+  uint16_t *hz = reinterpret_cast<uint16_t *>(smem + Ly::kOffHz);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
   volatile int *abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
@@ -292,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[kBarAFull + i], kGroupThreads);
       mbar_init(&bars[kBarAEmpty + i], 1);
     }
+    mbar_init(&bars[kBarGate], kGroupThreads);
     mbar_init(&bars[kBarDone], 1);
     *abort = 0;
     fence_mbar_init();
@@ -327,6 +370,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                   kv_t.i * kTM, kv_t.b);
       ++kv_count;
     }
+  }
+  // The gate threads issue the loads of the first run's filter taps now; they land while the
+  // CTA-wide barrier below completes and are written to shared memory after it.
+  bool over = false;
+  float taps[Ly::kPer];
+  const bool gate_role = warp >= kWarpGate0 && warp < kWarpGate0 + 4;
+  if (gate_role && w_begin < w_end) {
+    const int g0 = static_cast<int>((w_begin / p.nT) / p.B) * gmul + goff;
+    tap_load(taps, p.h + static_cast<size_t>(g0) * kNG * p.l_h, p.l_h, p.halo, kNG,
+             threadIdx.x - kWarpGate0 * 32);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -466,17 +519,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     Item t;
     uint32_t kc = 0, xc = 0;
     int cur_seg = -1;
-    bool over = false;
+    const int gtid = threadIdx.x - kWarpGate0 * 32;
+    uint32_t gphase = 0;  // phases of the gate threads' own barrier
     while (it.next(t)) {
       if (t.seg != cur_seg) {
         cur_seg = t.seg;
+        if (t.seg > 0) {
+          // every gate thread has finished reading the previous taps ...
+          tap_load(taps, p.h + static_cast<size_t>(t.g) * kNG * p.l_h, p.l_h, p.halo, kNG, gtid);
+          mbar_arrive(&bars[kBarGate]);
+          if (!warp_wait(&bars[kBarGate], gphase++ & 1, abort)) break;
+        }
+        tap_store(hz, taps, p.halo, kNG, gtid, over);
+        // ... and has written its share of the new ones
+        mbar_arrive(&bars[kBarGate]);
+        if (!warp_wait(&bars[kBarGate], gphase++ & 1, abort)) break;
         const int pa = p.nbuf == 2 ? (t.seg & 1) : 0, use = p.nbuf == 2 ? (t.seg >> 1) : t.seg;
         if (use > 0 && !warp_wait(&bars[kBarAEmpty + pa], (use - 1) & 1, abort)) break;
 #pragma unroll 1
         for (int gg = 0; gg < kNG; ++gg)
           build_band_tmem(kBandCol0 + (pa * kNG + gg) * p.band_cols, p.band_cols, tmem_base,
-                          p.h + (static_cast<size_t>(t.g) * kNG + gg) * p.l_h, p.l_h, p.halo,
-                          warp & 3, lane, over);
+                          hz + gg * (258 + p.halo) + 2, p.halo, warp & 3, lane);
         tc_fence_before_sync();
         mbar_arrive(&bars[kBarAFull + pa]);
       }

@@ -51,6 +51,46 @@ using tc::kTimeoutBit;
 using tc::kF16RangeBit;
 constexpr int kMaxHalo = 128;  // one tile of history: l_h - 1 <= 128
 
+// The Toeplitz band of one group in tensor memory, each lane fetching its own taps from
+// global memory.  Output rows are reversed (lane p holds
+// time t0 + 127 - p) and K runs over input rows t0 - halo .. t0 + 127, so
+//     A[p][kk] = h[127 + halo - p - kk]   (zero outside [0, l_h)),  rounded to fp16.
+// Each of the 128 gate threads writes its own lane: 128 + halo K elements = band_cols columns.
+// Columns [c0, c0 + N) of one lane's band row: 2 N taps loaded together, then one store.
+template <int N>
+__device__ __forceinline__ void band_chunk_gmem(uint32_t taddr, int c0, int row, const float *hg,
+                                           int l_h, int halo, bool &over) {
+  uint32_t r[N];
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    const int idx = kTM - 1 + halo - row - 2 * (c0 + c);  // tap of K element 2 (c0 + c)
+    const float v0 = (idx >= 0 && idx < l_h) ? __ldg(hg + idx) : 0.f;
+    const float v1 = (idx - 1 >= 0 && idx - 1 < l_h) ? __ldg(hg + idx - 1) : 0.f;
+    over |= (fabsf(v0) > 65504.f) | (fabsf(v1) > 65504.f);
+    const __half2 hv = __floats2half2_rn(v0, v1);
+    r[c] = *reinterpret_cast<const uint32_t *>(&hv);
+  }
+  if constexpr (N == 32)
+    tmem_st_32x32b_x32(taddr + c0, r);
+  else
+    tmem_st_32x32b_x8(taddr + c0, r);
+}
+
+__device__ __forceinline__ void build_band_gmem(uint32_t band_col, int band_cols,
+                                                uint32_t tmem_base, const float *hg, int l_h,
+                                                int halo, int quad, int lane, bool &over) {
+  const int row = quad * 32 + lane;
+  const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + band_col;
+  int c0 = 0;
+  // 32 columns (64 taps in flight) per step, then the 8-column remainder.
+#pragma unroll 1
+  for (; c0 + 32 <= band_cols; c0 += 32) band_chunk_gmem<32>(taddr, c0, row, hg, l_h, halo, over);
+#pragma unroll 1
+  for (; c0 < band_cols; c0 += 8) band_chunk_gmem<8>(taddr, c0, row, hg, l_h, halo, over);
+  tmem_wait_st();
+}
+
+
 constexpr int kNKV = 2;   // k/v stages (32 KB each)
 constexpr int kNQ = 3;    // q stages; each becomes the tile's fp16 dz (channel-major, reversed)
 constexpr int kNDY = 3;   // dy stages
@@ -537,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (it.next(t)) {
       if (t.seg_first) {
         if (t.seg > 0 && !tc::warp_wait(&bars[kBarAEmpty], (t.seg - 1) & 1, abort)) break;
-        tc::build_band_tmem(kColBand, p.band_cols, tmem_base, p.h + static_cast<size_t>(t.g) * p.l_h,
+        build_band_gmem(kColBand, p.band_cols, tmem_base, p.h + static_cast<size_t>(t.g) * p.l_h,
                             p.l_h, p.halo, warp & 3, lane, over);
         tc_fence_before_sync();
         mbar_arrive(&bars[kBarAFull]);
