@@ -25,7 +25,7 @@ __all__ = [
     "HyenaError", "HYENA_ALGO_AUTO", "HYENA_ALGO_TENSOR", "HYENA_ALGO_WINDOW",
     "HYENA_ALGO_DIRECT", "HYENA_DTYPE_BF16", "HYENA_DTYPE_F32", "HYENA_DEVICE_TIMEOUT",
     "HYENA_DEVICE_F16_RANGE", "ALGO_NAMES", "hyena_conv_fwd_from_host",
-    "hyena_toeplitz_stages", "hyena_build_toeplitz_blocks",
+    "hyena_toeplitz_stages", "hyena_build_toeplitz_blocks", "hyena_conv_fwd_hist",
 ]
 
 
@@ -87,6 +87,35 @@ def hyena_conv_fwd_ex(q, k, v, h, d_g, l_b, algo=HYENA_ALGO_AUTO, y=None, stream
                                          y.data_ptr(), B, L, D, d_g, h.shape[1], l_b,
                                          _dtype_code(q), algo, _stream(stream))
     _native.check("hyena_conv_fwd_ex", rc)
+    return y
+
+
+def hyena_conv_fwd_hist(q, k, v, h, d_g, l_b, k_hist, v_hist, algo=HYENA_ALGO_AUTO, y=None,
+                        stream=None):
+    """Forward of one shard of longer sequences: k_hist, v_hist [B, L_hist, D] are the rows that
+    precede row 0 of every sequence (their last l_h - 1 rows are read); returns y [B, L, D].
+    L_hist = 0 (or k_hist None) is zero history."""
+    torch = _torch()
+    y = _check(q, k, v, h, d_g, y)
+    B, L, D = q.shape
+    if k_hist is None or k_hist.shape[1] == 0:
+        kp = vp = None
+        L_hist = 0
+    else:
+        for t in (k_hist, v_hist):
+            if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != q.dtype \
+                    or t.dim() != 3 or not t.is_contiguous() or t.device != q.device:
+                raise TypeError("k_hist, v_hist must be contiguous CUDA [B, L_hist, D] tensors of "
+                                "q's dtype on q's device")
+        if k_hist.shape != v_hist.shape or k_hist.shape[0] != B or k_hist.shape[2] != D:
+            raise ValueError("k_hist, v_hist must both be [B, L_hist, D] with q's B and D")
+        kp, vp = k_hist.data_ptr(), v_hist.data_ptr()
+        L_hist = k_hist.shape[1]
+    rc = _native.lib().hyena_conv_fwd_hist(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           h.data_ptr(), y.data_ptr(), kp, vp, L_hist, B, L, D,
+                                           d_g, h.shape[1], l_b, _dtype_code(q), algo,
+                                           _stream(stream))
+    _native.check("hyena_conv_fwd_hist", rc)
     return y
 
 

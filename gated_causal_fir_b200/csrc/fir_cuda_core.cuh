@@ -76,6 +76,8 @@ struct WindowParams {
   int rows;        // time steps per thread
   long long n_tb;  // time blocks per sequence = ceil(L / rows)
   long long cv;    // channel vectors per row = D / VEC
+  const void *kh, *vh;  // [B, Lh, D]: the rows before row 0 of every sequence (Lh = 0: zeros)
+  long long Lh;
 };
 
 // Unroll factor of the time loop: loads of U rows are issued before their arithmetic.
@@ -122,7 +124,7 @@ __global__ void __launch_bounds__(kWindowBlock, HYENA_WINDOW_MIN_BLOCKS)
   const long long t_end = min(t0 + p.rows, p.L);
   const long long seq = b * p.L * p.D + c0;
 
-  // Halo: the l_h - 1 rows before t0 (zero before the start of the sequence).
+  // Halo: the l_h - 1 rows before t0 (before row 0: the history rows, then zeros).
 #pragma unroll
   for (int s = LH - 1; s >= 1; --s) {
 #pragma unroll
@@ -130,10 +132,14 @@ __global__ void __launch_bounds__(kWindowBlock, HYENA_WINDOW_MIN_BLOCKS)
 #pragma unroll
       for (int e = 0; e < VN; ++e) xw[j][e] = xw[j - 1][e];
     const long long t = t0 - s;
-    if (t >= 0) {
+    if (t >= -p.Lh) {
+      const T *kp = t >= 0 ? k + seq + t * p.D
+                           : static_cast<const T *>(p.kh) + (b * p.Lh + p.Lh + t) * p.D + c0;
+      const T *vp = t >= 0 ? v + seq + t * p.D
+                           : static_cast<const T *>(p.vh) + (b * p.Lh + p.Lh + t) * p.D + c0;
       float kk[VN], vv[VN];
-      Vec<T>::unpack(Vec<T>::load(k + seq + t * p.D), kk);
-      Vec<T>::unpack(Vec<T>::load(v + seq + t * p.D), vv);
+      Vec<T>::unpack(Vec<T>::load(kp), kk);
+      Vec<T>::unpack(Vec<T>::load(vp), vv);
 #pragma unroll
       for (int e = 0; e < VN; ++e) xw[0][e] = kk[e] * vv[e];
     } else {
@@ -184,7 +190,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
     fir_direct_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                       const float *__restrict__ h, T *__restrict__ y, long long B, long long L,
-                      long long D, int d_g, int l_h) {
+                      long long D, int d_g, int l_h, const T *__restrict__ kh,
+                      const T *__restrict__ vh, long long Lh) {
   const long long n = B * L * D;
   for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -196,6 +203,15 @@ __global__ void __launch_bounds__(256)
     for (long long j = 0; j <= jmax; ++j) {
       const long long src = e - j * D;
       acc = fmaf(__ldg(hg + j), to_f32(k[src]) * to_f32(v[src]), acc);
+    }
+    // taps that reach before row 0: the history rows [B, Lh, D] (row Lh - 1 precedes row 0)
+    const long long jh = min(static_cast<long long>(l_h - 1), t + Lh);
+    if (jh > t) {
+      const long long hrow = (e / (L * D)) * Lh + Lh + t;  // history row of tap j: hrow - j
+      for (long long j = t + 1; j <= jh; ++j) {
+        const long long src = (hrow - j) * D + c;
+        acc = fmaf(__ldg(hg + j), to_f32(kh[src]) * to_f32(vh[src]), acc);
+      }
     }
     from_f32(to_f32(q[e]) * acc, y + e);
   }

@@ -117,11 +117,14 @@ struct Params {
   long long W;      // tiles of the walk: CB * B * nT, or (CB / 2) * B * nT when paired
   int paired;       // CTAs 2p and 2p+1 walk the same (block pair, batch, time) range, one
                     // block each, so both halves of every 256-byte row are read together
+  int hist_tiles;   // 0: zero history before row 0; kNH: the rows before row 0 come from the
+                    // history tensors (tile i < 0 = their rows Lh + 128 i .. Lh + 128 i + 127)
+  int Lh;           // rows of the history tensors
 };
 
 // One unit of a CTA's walk: a halo tile (input only) or an output tile.
 struct Item {
-  int g, b, i;      // 64-channel block, sequence, tile index along time
+  int g, b, i;      // 64-channel block, sequence, tile index along time (< 0: history tile)
   int seg;          // running segment number within this CTA (a segment = one sequence run)
   bool halo;        // input-only tile feeding the first output tiles of a segment
   bool last;        // last output tile of its segment
@@ -129,17 +132,17 @@ struct Item {
 
 // The walk of one CTA: tiles [w_begin, w_end) of the order (group, batch, time); with gmul = 2
 // the walk is over group pairs and this CTA takes group 2 * pair + goff.  A segment that starts
-// at tile i > 0 of a sequence is preceded by its min(i, nh) history tiles as halo items (input
-// only).  The position is decoded once; next() only increments (64-bit divisions are software
+// at tile i of a sequence is preceded by its min(i + hist_tiles, nh) history tiles as halo
+// items (input only; tiles with i < 0 come from the history tensors).  The position is decoded once; next() only increments (64-bit divisions are software
 // routines on the GPU).
 struct WorkIter {
   long long w, w_end;
-  int nT, B, seg, gmul, nh, hpend, i, g, b;
+  int nT, B, seg, gmul, nh, hist, hpend, i, g, b;
   bool at_begin, entered;
   __device__ WorkIter(long long w_begin, long long w_end_, int nT_, int B_, int gmul_, int goff,
-                      int nh_)
-      : w(w_begin), w_end(w_end_), nT(nT_), B(B_), seg(-1), gmul(gmul_), nh(nh_), hpend(0),
-        at_begin(true), entered(false) {
+                      int nh_, int hist_tiles)
+      : w(w_begin), w_end(w_end_), nT(nT_), B(B_), seg(-1), gmul(gmul_), nh(nh_),
+        hist(hist_tiles), hpend(0), at_begin(true), entered(false) {
     const long long seq = w_begin / nT;
     i = static_cast<int>(w_begin - seq * nT);
     g = static_cast<int>(seq / B) * gmul + goff;
@@ -152,7 +155,7 @@ struct WorkIter {
     if ((at_begin || i == 0) && !entered) {
       entered = true;
       ++seg;
-      hpend = min(i, nh);
+      hpend = min(i + hist, nh);
     }
     it.seg = seg;
     if (hpend > 0) {
@@ -282,7 +285,8 @@ template <int kNG, int kNH>
 __global__ void __launch_bounds__(kThreads, 1)
     fir_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
-                  const Params p) {
+                  const __grid_constant__ CUtensorMap tm_kh,
+                  const __grid_constant__ CUtensorMap tm_vh, const Params p) {
   using Ly = Layout<kNH>;
   constexpr int kNQ = Ly::kNQ, kNX = Ly::kNX;
   constexpr int kOffKV = Ly::kOffKV, kOffQ = Ly::kOffQ, kOffX = Ly::kOffX, kOffBar = Ly::kOffBar,
@@ -342,6 +346,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_y);
+    if (p.hist_tiles) {
+      tma_prefetch_desc(&tm_kh);
+      tma_prefetch_desc(&tm_vh);
+    }
   }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -353,7 +361,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_launch_dependents();
   // Thread 0 is also the k/v producer: it queues the first k/v stages right away, before the
   // CTA-wide barrier (no other thread touches those stages yet).
-  WorkIter kv_it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH);
+  WorkIter kv_it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH, p.hist_tiles);
+  // k and v of one item into stage `slot`: tiles i < 0 from the history tensors.
+  auto load_kv = [&](uint32_t slot, const Item &t) {
+    uint8_t *dst = kv_st + slot * 2 * kTileBytes;
+    const bool h = t.i < 0;
+    const int row = h ? p.Lh + t.i * kTM : t.i * kTM;
+    tma_load_3d(dst, h ? &tm_kh : &tm_k, &bars[kBarKVFull + slot], t.g * kNC, row, t.b);
+    tma_load_3d(dst + kTileBytes, h ? &tm_vh : &tm_v, &bars[kBarKVFull + slot], t.g * kNC, row,
+                t.b);
+  };
   Item kv_t;
   uint32_t kv_count = 0;
   bool kv_done = false;
@@ -364,10 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       mbar_arrive_expect_tx(&bars[kBarKVFull + kv_count], 2 * kTileBytes);
-      uint8_t *dst = kv_st + kv_count * 2 * kTileBytes;
-      tma_load_3d(dst, &tm_k, &bars[kBarKVFull + kv_count], kv_t.g * kNC, kv_t.i * kTM, kv_t.b);
-      tma_load_3d(dst + kTileBytes, &tm_v, &bars[kBarKVFull + kv_count], kv_t.g * kNC,
-                  kv_t.i * kTM, kv_t.b);
+      load_kv(kv_count, kv_t);
       ++kv_count;
     }
   }
@@ -395,9 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ks = kc % kNKV;
         if (!thread_wait(&bars[kBarKVEmpty + ks], ((kc / kNKV) & 1) ^ 1, abort)) break;
         mbar_arrive_expect_tx(&bars[kBarKVFull + ks], 2 * kTileBytes);
-        uint8_t *dst = kv_st + ks * 2 * kTileBytes;
-        tma_load_3d(dst, &tm_k, &bars[kBarKVFull + ks], t.g * kNC, t.i * kTM, t.b);
-        tma_load_3d(dst + kTileBytes, &tm_v, &bars[kBarKVFull + ks], t.g * kNC, t.i * kTM, t.b);
+        load_kv(ks, t);
         ++kc;
       }
       // Every load this thread issued must land before the CTA may exit.
@@ -407,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpTmaQ) {
     // ---------------------------------------------------------------- TMA producer: q
     if (lane == 0) {
-      WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH);
+      WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH, p.hist_tiles);
       Item t;
       uint32_t qc = 0;
       while (it.next(t)) {
@@ -425,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH);
+      WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH, p.hist_tiles);
       Item t;
       uint32_t xc = 0, ac = 0, seg_x0 = 0;
       int cur_seg = -1, x_seg = -1;
@@ -464,8 +476,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem_base + as * kNC;
         const uint32_t band0 = tmem_base + kBandCol0 + pa * kNG * p.band_cols;
         // A (group gg's band) advances 8 columns (16 K elements) per k-step.  History steps
-        // whose rows lie before the start of the sequence are zero and skipped.
-        const int jstart = max(0, (p.halo - t.i * kTM) / 16);
+        // whose rows lie before the start of the sequence (and its history) are zero and skipped.
+        const int jstart = max(0, (p.halo - (t.i + p.hist_tiles) * kTM) / 16);
         uint32_t a_run[kNG];  // next band column of each group
 #pragma unroll
         for (int gg = 0; gg < kNG; ++gg) a_run[gg] = band0 + gg * p.band_cols + 8 * jstart;
@@ -515,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kWarpGate0 && warp < kWarpGate0 + 4) {
     // ---------------------------------------------------------------- pre-gate + band build
-    WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH);
+    WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH, p.hist_tiles);
     Item t;
     uint32_t kc = 0, xc = 0;
     int cur_seg = -1;
@@ -580,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;               // TMEM lanes this warp may read
     const int row_lane = quad * 32 + lane;   // MMA row = TMEM lane
     const int r = kTM - 1 - row_lane;        // tile row (time offset) of that lane
-    WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH);
+    WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH, p.hist_tiles);
     Item t;
     uint32_t ac = 0, qc = 0;
     while (it.next(t)) {

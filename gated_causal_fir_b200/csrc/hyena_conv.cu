@@ -110,6 +110,8 @@ struct Problem {
   void *y;
   int64_t B, L, D;
   int d_g, l_h, l_b, dtype;
+  const void *kh = nullptr, *vh = nullptr;  // [B, Lh, D] rows before row 0 (Lh = 0: zeros)
+  int64_t Lh = 0;
   int64_t elem() const { return dtype == HYENA_DTYPE_F32 ? 4 : 2; }
   int64_t numel() const { return B * L * D; }
   int64_t G() const { return D / d_g; }
@@ -141,11 +143,24 @@ int validate(const Problem &P) {
   const int64_t bytes = P.numel() * P.elem();
   if (overlaps(P.y, P.q, bytes) || overlaps(P.y, P.k, bytes) || overlaps(P.y, P.v, bytes))
     return HYENA_ERR_INVALID_ARG;
+  if (P.Lh > 0) {
+    if (!P.kh || !P.vh || P.Lh > lim / P.B / P.D) return HYENA_ERR_INVALID_ARG;
+    if (!aligned(P.kh, es) || !aligned(P.vh, es)) return HYENA_ERR_MISALIGNED;
+    const int64_t hb = P.B * P.Lh * P.D * P.elem();
+    // y must not overlap the history either (the intervals differ in length)
+    const uintptr_t y0 = reinterpret_cast<uintptr_t>(P.y);
+    for (const void *hp : {P.kh, P.vh}) {
+      const uintptr_t h0 = reinterpret_cast<uintptr_t>(hp);
+      if (y0 < h0 + static_cast<uintptr_t>(hb) && h0 < y0 + static_cast<uintptr_t>(bytes))
+        return HYENA_ERR_INVALID_ARG;
+    }
+  }
   return HYENA_OK;
 }
 
 bool all_aligned16(const Problem &P) {
-  return aligned(P.q, 16) && aligned(P.k, 16) && aligned(P.v, 16) && aligned(P.y, 16);
+  return aligned(P.q, 16) && aligned(P.k, 16) && aligned(P.v, 16) && aligned(P.y, 16) &&
+         (P.Lh == 0 || (aligned(P.kh, 16) && aligned(P.vh, 16)));
 }
 
 // Tensor-core plan: history rows, history tiles, one group's band width in TMEM columns and the
@@ -170,7 +185,7 @@ TcPlan tc_plan(const Problem &P) {
 bool tensor_supported(const Problem &P) {
   const int64_t i32 = std::numeric_limits<int32_t>::max();
   return P.dtype == HYENA_DTYPE_BF16 && P.D % hyena::tc::kNC == 0 && tc_plan(P).nbuf > 0 &&
-         all_aligned16(P) && P.L <= i32 && P.B <= i32 && P.D <= i32;
+         all_aligned16(P) && P.L <= i32 && P.B <= i32 && P.D <= i32 && P.Lh <= i32;
 }
 
 bool window_supported(const Problem &P) {
@@ -201,15 +216,18 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
   if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
   EncodeTiledFn enc = encode_tiled();
   if (!enc) return HYENA_ERR_CUDA;
-  CUtensorMap maps[4];
-  const void *ptrs[4] = {P.q, P.k, P.v, P.y};
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.D), static_cast<cuuint64_t>(P.L),
-                              static_cast<cuuint64_t>(P.B)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.D) * 2,
-                                 static_cast<cuuint64_t>(P.L) * static_cast<cuuint64_t>(P.D) * 2};
+  // q, k, v, y over [B, L, D]; then k, v history over [B, Lh, D] (without history the k, v
+  // maps stand in: the kernel never reads them then).
+  CUtensorMap maps[6];
+  const bool hist = P.Lh > 0;
+  const void *ptrs[6] = {P.q, P.k, P.v, P.y, hist ? P.kh : P.k, hist ? P.vh : P.v};
   const cuuint32_t box[3] = {hyena::tc::kNC, hyena::tc::kTM, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 6; ++i) {
+    const cuuint64_t rows = static_cast<cuuint64_t>(i >= 4 && hist ? P.Lh : P.L);
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.D), rows, static_cast<cuuint64_t>(P.B)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.D) * 2,
+                                   rows * static_cast<cuuint64_t>(P.D) * 2};
     if (enc(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptrs[i]), dims,
             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             HYENA_TC_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -226,6 +244,8 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
   p.band_cols = plan.band_cols;
   p.nbuf = plan.nbuf;
   p.nT = static_cast<int>((P.L + hyena::tc::kTM - 1) / hyena::tc::kTM);
+  p.hist_tiles = hist ? plan.nh : 0;
+  p.Lh = static_cast<int>(P.Lh);
   const long long sms = ds->sm_count;
   p.paired = HYENA_TC_PAIRED && p.CB % 2 == 0 && sms >= 2;
   long long grid;
@@ -254,7 +274,7 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
 #define HYENA_TC_LAUNCH(NG, NH)                                                            \
   cfg.dynamicSmemBytes = hyena::tc::Layout<NH>::kSmemBytes;                                  \
   le = cudaLaunchKernelEx(&cfg, hyena::tc::fir_tc_kernel<NG, NH>, maps[0], maps[1], maps[2], \
-                          maps[3], p)
+                          maps[3], maps[4], maps[5], p)
   switch (plan.ng * 8 + plan.nh) {
     case 9: HYENA_TC_LAUNCH(1, 1); break;
     case 10: HYENA_TC_LAUNCH(1, 2); break;
@@ -297,6 +317,9 @@ int launch_window(const Problem &P, cudaStream_t s) {
   wp.rows = kWindowRows;
   wp.n_tb = (P.L + kWindowRows - 1) / kWindowRows;
   wp.cv = P.D / vec;
+  wp.kh = P.kh;
+  wp.vh = P.vh;
+  wp.Lh = P.Lh;
   const long long threads = wp.B * wp.n_tb * wp.cv;
   const long long blocks = (threads + hyena::cc::kWindowBlock - 1) / hyena::cc::kWindowBlock;
   if (blocks > std::numeric_limits<int32_t>::max()) return HYENA_ERR_UNSUPPORTED;
@@ -318,12 +341,13 @@ int launch_direct(const Problem &P, cudaStream_t s) {
     hyena::cc::fir_direct_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
         static_cast<const float *>(P.q), static_cast<const float *>(P.k),
         static_cast<const float *>(P.v), P.h, static_cast<float *>(P.y), P.B, P.L, P.D, P.d_g,
-        P.l_h);
+        P.l_h, static_cast<const float *>(P.kh), static_cast<const float *>(P.vh), P.Lh);
   else
     hyena::cc::fir_direct_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
         static_cast<const __nv_bfloat16 *>(P.q), static_cast<const __nv_bfloat16 *>(P.k),
         static_cast<const __nv_bfloat16 *>(P.v), P.h, static_cast<__nv_bfloat16 *>(P.y), P.B,
-        P.L, P.D, P.d_g, P.l_h);
+        P.L, P.D, P.d_g, P.l_h, static_cast<const __nv_bfloat16 *>(P.kh),
+        static_cast<const __nv_bfloat16 *>(P.vh), P.Lh);
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
@@ -624,6 +648,18 @@ int hyena_conv_fwd_ex(const void *q, const void *k, const void *v, const float *
                       int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b, int dtype,
                       int algo, cudaStream_t stream) {
   const Problem P{q, k, v, h, y, B, L, D, d_g, l_h, l_b, dtype};
+  return run(P, algo, stream);
+}
+
+int hyena_conv_fwd_hist(const void *q, const void *k, const void *v, const float *h, void *y,
+                        const void *k_hist, const void *v_hist, int64_t L_hist, int64_t B,
+                        int64_t L, int64_t D, int d_g, int l_h, int l_b, int dtype, int algo,
+                        cudaStream_t stream) {
+  if (L_hist < 0) return HYENA_ERR_INVALID_ARG;
+  Problem P{q, k, v, h, y, B, L, D, d_g, l_h, l_b, dtype};
+  P.kh = k_hist;
+  P.vh = v_hist;
+  P.Lh = L_hist;
   return run(P, algo, stream);
 }
 

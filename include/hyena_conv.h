@@ -99,6 +99,29 @@ int hyena_conv_fwd_ex(const void *q, const void *k, const void *v, const float *
                       int dtype, int algo, cudaStream_t stream);
 
 /*
+ * One shard of longer sequences: the same operation as hyena_conv_fwd_ex over rows 0 .. L-1
+ * of every sequence, where the L_hist rows that precede row 0 are given instead of zero
+ * history (page 04, Sec. 3: output chunk n needs input chunk n-1; page 01, Sec. 5 names
+ * point-to-point context parallelism, which cuts a sequence across devices):
+ *
+ *     y[b,t,c] = q[b,t,c] * sum_{j=0}^{min(l_h-1, t+L_hist)} h[c/d_g][j] * x(b, t-j, c),
+ *     x(b, s, c) = k[b,s,c] v[b,s,c] for s >= 0,
+ *                  k_hist[b, L_hist+s, c] v_hist[b, L_hist+s, c] for s < 0.
+ *
+ * k_hist, v_hist: DEVICE [B, L_hist, D] tensors of `dtype` (row L_hist-1 immediately precedes
+ * row 0); only their last min(L_hist, l_h-1) rows are read.  L_hist == 0 is zero history
+ * (k_hist, v_hist may then be NULL) and gives exactly hyena_conv_fwd_ex.  The history must not
+ * overlap y.  Every algorithm takes history; HYENA_ALGO_TENSOR and HYENA_ALGO_WINDOW also need
+ * k_hist and v_hist 16-byte aligned.  Errors: as hyena_conv_fwd_ex, plus HYENA_ERR_INVALID_ARG
+ * for L_hist < 0, NULL history with L_hist > 0 or history that overlaps y, and
+ * HYENA_ERR_MISALIGNED for history not aligned to its element size.
+ */
+int hyena_conv_fwd_hist(const void *q, const void *k, const void *v, const float *h, void *y,
+                        const void *k_hist, const void *v_hist, int64_t L_hist, int64_t B,
+                        int64_t L, int64_t D, int d_g, int l_h, int l_b, int dtype, int algo,
+                        cudaStream_t stream);
+
+/*
  * Host-only: the algorithm (enum hyena_algo, > 0) that HYENA_ALGO_AUTO would run for this
  * problem and these pointers, or minus an error code.  Touches no device.
  */

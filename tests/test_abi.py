@@ -146,6 +146,20 @@ def test_long_filters_select_an_algorithm():
         g.HYENA_ALGO_DIRECT
 
 
+def test_history_validation(lib):
+    f = lib.hyena_conv_fwd_hist
+    q, k, v, h, y = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+    kh, vh = 0x60000, 0x70000
+    a = (1, 64, 128, 64, 16, 16, 0, 0, None)  # B, L, D, d_g, l_h, l_b, dtype, algo, stream
+    assert f(q, k, v, h, y, kh, vh, -1, *a) == 1                    # negative L_hist
+    assert f(q, k, v, h, y, None, vh, 8, *a) == 1                   # missing history
+    assert f(q, k, v, h, y, kh, None, 8, *a) == 1
+    assert f(q, k, v, h, y, kh + 1, vh, 8, *a) == 3                 # misaligned history
+    assert f(q, k, v, h, y, y + 64, vh, 8, *a) == 1                 # history overlaps y
+    assert f(q, k, v, h, y, y - 1024, vh, 8, *a) == 1               # history runs into y
+    assert f(q, k, v, h, y, kh, vh, 8, 0, 64, 128, 64, 16, 16, 0, 0, None) == 0  # empty: no launch
+
+
 def test_device_status_needs_out(lib):
     assert lib.hyena_device_status(None, 0) == 1
 
