@@ -1,40 +1,41 @@
-// fir_tc_bwd.cuh -- fused tcgen05 backward of the gated grouped causal FIR (bf16, d_g = 64).
+// fir_tc_bwd.cuh -- tcgen05 kernel of the backward of the gated grouped causal FIR (bf16,
+// d_g = 64): the anti-causal product and the filter gradient.
 //
 // For y = q * z, z = h_g conv x, x = k * v and the upstream gradient dy (page "04.
 // Hardware-aware convolution kernels", Sec. 7 backward; Sec. 2-3 block-Toeplitz form):
-//   dq = dy * z                      z  = T x           (causal Toeplitz product)
+//   dq = dy * z                      -- the forward kernel with dy in the place of q (host)
 //   dk = dx * v,  dv = dx * k        dx = T^T (q * dy)  (anti-causal: the transposed product)
 //   dh[g][j] = sum_{t, c in g} dz[t, c] x[t - j, c],  dz = q * dy
-// One kernel reads q, k, v, dy once and writes dq, dk, dv once; dh leaves as one fp32 partial
-// per (CTA, segment), summed in a fixed order by fir_bwd_tc_reduce_kernel.
+// This kernel reads q, k, v, dy once and writes dk, dv once; dh leaves as one fp32 partial per
+// (CTA, segment), summed in a fixed order by fir_bwd_tc_reduce_kernel (the two passes of Sec. 7).
+// Computing dq here as well (recomputing z = T x on chip) saves three tensor streams but puts
+// 40 MMAs on every 128 x 64 tile; with 24 this kernel and the forward each run near the HBM
+// bound, which measured faster than the fused form.
 //
 // Tiles are 128 time rows x 64 channels (one group).  Each CTA walks contiguous tile ranges
 // like the forward kernel, but every sequence run ("segment", tiles lo..hi) in DECREASING time,
-// so the anti-causal product of a tile finds the next tile's dz already on chip.  The causal
-// product of tile i+1 is issued once tile i's x exists (one tile of lag), which costs one extra
-// dy stage instead of keeping k and v longer.
+// so the anti-causal product of a tile finds the next tile's dz already on chip.
 //
 // B200 specifics:
-//  * One Toeplitz band in tensor memory serves both products.  The forward's band
-//    A[p][kk] = h[127 + halo - p - kk] multiplies x rows t0 - halo + kk into output lane
-//    p = time t0 + 127 - p.  Fed with dz in REVERSED time (operand row kk = time
-//    t0 + 127 + halo - kk), the same band yields lane p = dx[t0 + p]: so dz tiles are stored
-//    time-reversed, and the anti-causal chain is the causal chain's code with the next tile in
-//    the place of the previous one.
+//  * The forward's Toeplitz band in tensor memory, A[p][kk] = h[127 + halo - p - kk], computes
+//    z = T x with output lane p = time t0 + 127 - p.  Fed with dz in REVERSED time (operand row
+//    kk = time t0 + 127 + halo - kk), the same band yields lane p = dx[t0 + p]: dz tiles are
+//    stored time-reversed, and the anti-causal chain is the causal chain with the next tile in
+//    the place of the previous one.  The band is built from the filter taps staged in shared
+//    memory, as in the forward.
 //  * dh as a GEMM: C[m][n] = sum_c x[t0 + m, c] dz[tau(n), c] over the 256 dz times of tiles
 //    i and i+1 (two M128 N128 K64 MMAs with both operands MN-major, read straight from the
-//    channel-major fp16 tiles the Toeplitz chains use).  C accumulates in tensor memory over a
-//    whole segment; the lag j = tau(n) - t0 - m is constant along anti-diagonals, which the
-//    epilogue sums once per segment.
-//  * Tensor memory (512 columns): z accumulator [0, 64), dx accumulator [64, 128), band
-//    [128, 128 + band_cols), C [256, 512).
+//    channel-major fp16 tiles).  C accumulates in tensor memory over a whole segment; the lag
+//    j = tau(n) - t0 - m is constant along anti-diagonals, which the epilogue sums once per
+//    segment.
+//  * Tensor memory (512 columns): two dx accumulators [0, 128) (the MMA issuer fills one while
+//    the epilogue drains the other), band [128, 256), C [256, 512).
 //  * Warp roles as the forward: 0 TMA k/v, 10 TMA q/dy (both fetch their tiles into L2 a few
 //    items ahead, then into shared memory), 1 MMA issuer + TMEM owner, 2-5 operand build
-//    (x = k v; dz = q dy written over the q tile; the band), 6-9 epilogue.  The epilogue reads
-//    its k, v, dy rows from global memory (L2-resident: just loaded) and stores dq, dk, dv rows
-//    directly, so every input stage is released as soon as its operand is built; it also sums
-//    the dh anti-diagonals.  Every wait is bounded; a timeout raises HYENA_DEVICE_TIMEOUT and
-//    all roles drain and leave.
+//    (x = k v; dz = q dy written over the q tile; the band), 6-9 epilogue.  The epilogue copies
+//    its k, v rows from the stage into registers, releases it, and stores dk, dv rows directly;
+//    it also sums the dh anti-diagonals.  Every wait is bounded; a timeout raises
+//    HYENA_DEVICE_TIMEOUT and all roles drain and leave.
 #pragma once
 #include "fir_tc.cuh"
 
@@ -51,57 +52,19 @@ using tc::kTimeoutBit;
 using tc::kF16RangeBit;
 constexpr int kMaxHalo = 128;  // one tile of history: l_h - 1 <= 128
 
-// The Toeplitz band of one group in tensor memory, each lane fetching its own taps from
-// global memory.  Output rows are reversed (lane p holds
-// time t0 + 127 - p) and K runs over input rows t0 - halo .. t0 + 127, so
-//     A[p][kk] = h[127 + halo - p - kk]   (zero outside [0, l_h)),  rounded to fp16.
-// Each of the 128 gate threads writes its own lane: 128 + halo K elements = band_cols columns.
-// Columns [c0, c0 + N) of one lane's band row: 2 N taps loaded together, then one store.
-template <int N>
-__device__ __forceinline__ void band_chunk_gmem(uint32_t taddr, int c0, int row, const float *hg,
-                                           int l_h, int halo, bool &over) {
-  uint32_t r[N];
-#pragma unroll
-  for (int c = 0; c < N; ++c) {
-    const int idx = kTM - 1 + halo - row - 2 * (c0 + c);  // tap of K element 2 (c0 + c)
-    const float v0 = (idx >= 0 && idx < l_h) ? __ldg(hg + idx) : 0.f;
-    const float v1 = (idx - 1 >= 0 && idx - 1 < l_h) ? __ldg(hg + idx - 1) : 0.f;
-    over |= (fabsf(v0) > 65504.f) | (fabsf(v1) > 65504.f);
-    const __half2 hv = __floats2half2_rn(v0, v1);
-    r[c] = *reinterpret_cast<const uint32_t *>(&hv);
-  }
-  if constexpr (N == 32)
-    tmem_st_32x32b_x32(taddr + c0, r);
-  else
-    tmem_st_32x32b_x8(taddr + c0, r);
-}
-
-__device__ __forceinline__ void build_band_gmem(uint32_t band_col, int band_cols,
-                                                uint32_t tmem_base, const float *hg, int l_h,
-                                                int halo, int quad, int lane, bool &over) {
-  const int row = quad * 32 + lane;
-  const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + band_col;
-  int c0 = 0;
-  // 32 columns (64 taps in flight) per step, then the 8-column remainder.
-#pragma unroll 1
-  for (; c0 + 32 <= band_cols; c0 += 32) band_chunk_gmem<32>(taddr, c0, row, hg, l_h, halo, over);
-#pragma unroll 1
-  for (; c0 < band_cols; c0 += 8) band_chunk_gmem<8>(taddr, c0, row, hg, l_h, halo, over);
-  tmem_wait_st();
-}
-
-
-constexpr int kNKV = 2;   // k/v stages (32 KB each)
+constexpr int kNKV = 3;   // k/v stages (32 KB each)
 constexpr int kNQ = 3;    // q stages; each becomes the tile's fp16 dz (channel-major, reversed)
-constexpr int kNDY = 3;   // dy stages
-constexpr int kNX = 3;    // fp16 x tiles, channel-major
+constexpr int kNDY = 2;   // dy stages (free once dz is built)
+constexpr int kNX = 2;    // fp16 x tiles, channel-major (free once the tile's dh product ran)
 constexpr int kPrefetch = 3;  // items a producer fetches into L2 ahead of its loads
 
-constexpr uint32_t kColZ = 0, kColDX = 64, kColBand = 128, kColC = 256;
+constexpr uint32_t kColDX = 0, kColBand = 128, kColC = 256;
 constexpr int kTmemCols = 512;
 
 constexpr int kRedLd = 17;                       // 32 x 16 scratch per epilogue warp, padded
 constexpr int kPartLen = 132;                    // dh taps per epilogue warp (l_h <= 129)
+constexpr int kHzStride = 258 + kMaxHalo;        // staged fp16 taps of one group (see tc::tap_load)
+constexpr int kTapPer = (kHzStride + kGroupThreads - 1) / kGroupThreads;
 
 constexpr int kOffKV = 0;
 constexpr int kOffQ = kOffKV + kNKV * 2 * kTileBytes;
@@ -109,7 +72,8 @@ constexpr int kOffDY = kOffQ + kNQ * kTileBytes;
 constexpr int kOffX = kOffDY + kNDY * kTileBytes;
 constexpr int kOffRed = kOffX + kNX * kTileBytes;
 constexpr int kOffPart = kOffRed + 4 * 32 * kRedLd * 4;
-constexpr int kOffBar = kOffPart + 4 * kPartLen * 4;
+constexpr int kOffHz = kOffPart + 4 * kPartLen * 4;
+constexpr int kOffBar = (kOffHz + kHzStride * 2 + 15) / 16 * 16;
 
 constexpr int kBarKVFull = 0;
 constexpr int kBarKVEmpty = kBarKVFull + kNKV;
@@ -121,11 +85,10 @@ constexpr int kBarXFull = kBarDYEmpty + kNDY;
 constexpr int kBarXEmpty = kBarXFull + kNX;
 constexpr int kBarDZFull = kBarXEmpty + kNX;   // dz built over q stage s
 constexpr int kBarGateRead = kBarDZFull + kNQ; // every gate thread has read its q, dy fragments
-constexpr int kBarZFull = kBarGateRead + 1;
-constexpr int kBarZEmpty = kBarZFull + 1;
-constexpr int kBarDXFull = kBarZEmpty + 1;
-constexpr int kBarDXEmpty = kBarDXFull + 1;
-constexpr int kBarCFull = kBarDXEmpty + 1;
+constexpr int kBarGate = kBarGateRead + 1;     // the gate threads among themselves (tap staging)
+constexpr int kBarDXFull = kBarGate + 1;       // two of each: one per accumulator set
+constexpr int kBarDXEmpty = kBarDXFull + 2;
+constexpr int kBarCFull = kBarDXEmpty + 2;
 constexpr int kBarCEmpty = kBarCFull + 1;
 constexpr int kBarAFull = kBarCEmpty + 1;
 constexpr int kBarAEmpty = kBarAFull + 1;
@@ -152,18 +115,16 @@ struct Params {
   long long W;        // tiles of the walk: G * B * nT
   int max_segs;       // partial slots per CTA
   long long D;        // channels (row length of every [B, L, D] tensor)
-  const __nv_bfloat16 *k, *v, *dy;  // inputs the epilogue reads by rows
-  __nv_bfloat16 *dq, *dk, *dv;      // outputs, written by rows
+  __nv_bfloat16 *dk, *dv;  // outputs, written by rows
 };
 
-enum ItemKind { kNextHalo = 0, kMain = 1, kTail = 2 };
+enum ItemKind { kNextHalo = 0, kMain = 1 };
 
 // One unit of a CTA's walk.  A segment (tiles lo..hi of one (group, batch) sequence) is walked
-//   [next-halo: tile hi + 1's q, dy -> dz only]  main hi, main hi-1, ..., main lo,
-//   tail: tile lo - 1's k, v -> x only (when lo > 0), then z of tile lo.
+//   [next-halo: tile hi + 1's q, dy -> dz only]  main hi, main hi-1, ..., main lo.
 struct BItem {
   int kind;
-  int g, b, i;        // group, sequence, tile (main: the tile; halos: the halo tile)
+  int g, b, i;        // group, sequence, tile (next-halo: tile hi + 1)
   int lo, hi, seg;
   bool seg_first;     // first item of its segment
 };
@@ -201,17 +162,13 @@ struct BwdWalk {
       it.kind = kNextHalo;
       it.i = hi + 1;
       state = 2;
-    } else if (state == 2) {
+    } else {
       it.kind = kMain;
       it.i = i;
       if (i == lo)
-        state = 3;
+        state = 0;
       else
         --i;
-    } else {
-      it.kind = kTail;
-      it.i = lo - 1;
-      state = 0;
     }
     return true;
   }
@@ -322,6 +279,27 @@ __device__ __forceinline__ uint4 *row_chunk(uint8_t *tile, int r, int c) {
   return reinterpret_cast<uint4 *>(tile + r * kRowBytes + ((c ^ (r & 7)) << 4));
 }
 
+// One 16-byte shared-memory load that the compiler may neither repeat nor move: a stage's
+// rows must be read before the stage is handed back to its producer, and a plain load could be
+// re-issued after that point (rematerialised instead of spilled) and see the next tile.
+// An instruction that reads every loaded register, so the warp waits until the loads have
+// returned their data (an empty asm would emit nothing and wait for nothing).
+__device__ __forceinline__ void consume_rows(const uint4 (&r)[8]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    asm volatile("{\n\t.reg .b32 t;\n\txor.b32 t, %0, %1;\n\txor.b32 t, t, %2;\n\t"
+                 "xor.b32 t, t, %3;\n\t}" ::"r"(r[c].x), "r"(r[c].y), "r"(r[c].z), "r"(r[c].w));
+}
+
+__device__ __forceinline__ uint4 lds_v4(const void *p) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(smem_u32(p))
+               : "memory");
+  return r;
+}
+
 __device__ __forceinline__ void unpack_bf16x8(const uint4 &u, float (&o)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -356,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *x_st = smem + kOffX;
   float *red = reinterpret_cast<float *>(smem + kOffRed);
   float *part = reinterpret_cast<float *>(smem + kOffPart);
+  uint16_t *hz = reinterpret_cast<uint16_t *>(smem + kOffHz);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
   volatile int *abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
@@ -367,8 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long w_end = w_begin + per + (bx < rem ? 1 : 0);
 
   if (threadIdx.x == 0) {
-    // k/v and dy stages are released by both readers: the operand builders and the epilogue
-    // (the builders arrive twice for halo tiles, which the epilogue never reads)
+    // k/v stages are released by both readers: the operand builders and the epilogue
     for (int i = 0; i < kNKV; ++i) {
       mbar_init(&bars[kBarKVFull + i], 1);
       mbar_init(&bars[kBarKVEmpty + i], 2 * kGroupThreads);
@@ -380,17 +358,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kNDY; ++i) {
       mbar_init(&bars[kBarDYFull + i], 1);
-      mbar_init(&bars[kBarDYEmpty + i], 2 * kGroupThreads);
+      mbar_init(&bars[kBarDYEmpty + i], kGroupThreads);
     }
     for (int i = 0; i < kNX; ++i) {
       mbar_init(&bars[kBarXFull + i], kGroupThreads);
       mbar_init(&bars[kBarXEmpty + i], 1);
     }
     mbar_init(&bars[kBarGateRead], kGroupThreads);
-    mbar_init(&bars[kBarZFull], 1);
-    mbar_init(&bars[kBarZEmpty], kGroupThreads);
-    mbar_init(&bars[kBarDXFull], 1);
-    mbar_init(&bars[kBarDXEmpty], kGroupThreads);
+    mbar_init(&bars[kBarGate], kGroupThreads);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[kBarDXFull + i], 1);
+      mbar_init(&bars[kBarDXEmpty + i], kGroupThreads);
+    }
     mbar_init(&bars[kBarCFull], 1);
     mbar_init(&bars[kBarCEmpty], kGroupThreads);
     mbar_init(&bars[kBarAFull], kGroupThreads);
@@ -404,6 +383,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  // Nothing above touches global memory: under a programmatic dependent launch it overlaps the
+  // previous kernel (the dq forward).  From here on the inputs may be read.
+  griddep_wait();
+  griddep_launch_dependents();
+  // The gate threads issue the loads of the first segment's filter taps before the barrier.
+  bool over = false;
+  float taps[kTapPer];
+  if (warp >= kWarpGate0 && warp < kWarpGate0 + 4 && w_begin < w_end) {
+    const int g0 = static_cast<int>((w_begin / p.nT) / p.B);
+    tc::tap_load(taps, p.h + static_cast<size_t>(g0) * p.l_h, p.l_h, p.halo, 1,
+                 threadIdx.x - kWarpGate0 * 32);
+  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -416,11 +407,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_v);
       BwdWalk it(w_begin, w_end, p.nT, p.B), pf(w_begin, w_end, p.nT, p.B);
       BItem t, u;
-      auto kv_item = [](const BItem &x) { return x.kind == kMain || (x.kind == kTail && x.lo > 0); };
       // L2 prefetch runs kPrefetch loads ahead: the loads then find their tiles in L2.
       auto prefetch_next = [&]() {
         while (pf.next(u)) {
-          if (!kv_item(u)) continue;
+          if (u.kind != kMain) continue;
           tma_prefetch_l2_3d(&tm_k, u.g * kNC, u.i * kTM, u.b);
           tma_prefetch_l2_3d(&tm_v, u.g * kNC, u.i * kTM, u.b);
           return;
@@ -429,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = 0; n < kPrefetch; ++n) prefetch_next();
       uint32_t kc = 0;
       while (it.next(t)) {
-        if (!kv_item(t)) continue;
+        if (t.kind != kMain) continue;
         prefetch_next();
         const int ks = kc % kNKV;
         if (!tc::thread_wait(&bars[kBarKVEmpty + ks], ((kc / kNKV) & 1) ^ 1, abort)) break;
@@ -450,17 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       BwdWalk it(w_begin, w_end, p.nT, p.B), pf(w_begin, w_end, p.nT, p.B);
       BItem t, u;
       auto prefetch_next = [&]() {
-        while (pf.next(u)) {
-          if (u.kind == kTail) continue;
+        if (pf.next(u)) {
           tma_prefetch_l2_3d(&tm_q, u.g * kNC, u.i * kTM, u.b);
           tma_prefetch_l2_3d(&tm_dy, u.g * kNC, u.i * kTM, u.b);
-          return;
         }
       };
       for (int n = 0; n < kPrefetch; ++n) prefetch_next();
       uint32_t qc = 0, dc = 0;
       while (it.next(t)) {
-        if (t.kind == kTail) continue;
         prefetch_next();
         const int qs = qc % kNQ, ds = dc % kNDY;
         if (!tc::thread_wait(&bars[kBarQEmpty + qs], ((qc / kNQ) & 1) ^ 1, abort)) break;
@@ -484,84 +471,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       BwdWalk it(w_begin, w_end, p.nT, p.B);
       BItem t;
-      uint32_t xc = 0, dzc = 0, zc = 0, dxc = 0, cc = 0;
+      uint32_t xc = 0, dzc = 0, dxc = 0, cc = 0;
       const uint32_t id_t = umma_idesc_f16_f32(kTM, kNC, 0);        // Toeplitz chains
       const uint32_t id_c = umma_idesc_f16_f32_mn(kTM, 128, 1, 1);  // dh products
       const uint32_t band0 = tmem_base + kColBand;
       const uint32_t xs_base = smem_u32(x_st), dz_base = smem_u32(q_st);  // dz over q
       bool lo_init = false, hi_init = false;
-      bool ok = true;
-      while (ok && it.next(t)) {
+      while (it.next(t)) {
         if (t.kind == kNextHalo) {
-          ok = tc::thread_wait(&bars[kBarDZFull + dzc % kNQ], (dzc / kNQ) & 1, abort);
+          if (!tc::thread_wait(&bars[kBarDZFull + dzc % kNQ], (dzc / kNQ) & 1, abort)) break;
           ++dzc;
           continue;
         }
-        if (t.kind == kMain) {
-          if (t.i == t.hi) {  // first main tile: this segment's band
-            if (!tc::thread_wait(&bars[kBarAFull], t.seg & 1, abort)) break;
-          }
-          const int xs = xc % kNX, ds = dzc % kNQ;
-          if (!tc::thread_wait(&bars[kBarXFull + xs], (xc / kNX) & 1, abort)) break;
-          if (!tc::thread_wait(&bars[kBarDZFull + ds], (dzc / kNQ) & 1, abort)) break;
-          const bool has_next = t.i + 1 < p.nT;
-          const int dn = (dzc + kNQ - 1) % kNQ;  // dz of tile i + 1 (previous acquisition)
-          // dx(i): the band against dz of tiles i+1 (halo rows) and i
-          if (!tc::thread_wait(&bars[kBarDXEmpty], (dxc & 1) ^ 1, abort)) break;
-          tc_fence_after_sync();
-          toeplitz_chain(tmem_base + kColDX, band0, dz_base, has_next ? dn : -1, ds, p.halo,
-                         id_t);
-          umma_commit(&bars[kBarDXFull]);
-          ++dxc;
-          // C += x(i) dz(i), x(i) dz(i+1)
-          if (t.i == t.hi) {
-            if (!tc::thread_wait(&bars[kBarCEmpty], (cc & 1) ^ 1, abort)) break;
-            tc_fence_after_sync();
-            lo_init = hi_init = false;
-          }
-          c_chain(tmem_base + kColC, xs_base + xs * kTileBytes, dz_base + ds * kTileBytes, id_c,
-                  lo_init);
-          lo_init = true;
-          if (has_next) {
-            c_chain(tmem_base + kColC + 128, xs_base + xs * kTileBytes,
-                    dz_base + dn * kTileBytes, id_c, hi_init);
-            hi_init = true;
-            umma_commit(&bars[kBarQEmpty + dn]);
-          }
-          // z(i+1): the band against x of tiles i (halo rows) and i+1
-          if (t.i < t.hi) {
-            const int xn = (xc + kNX - 1) % kNX;
-            if (!tc::thread_wait(&bars[kBarZEmpty], (zc & 1) ^ 1, abort)) break;
-            tc_fence_after_sync();
-            toeplitz_chain(tmem_base + kColZ, band0, xs_base, xs, xn, p.halo, id_t);
-            umma_commit(&bars[kBarZFull]);
-            ++zc;
-            umma_commit(&bars[kBarXEmpty + xn]);
-          }
-          if (t.i == t.lo) {
-            umma_commit(&bars[kBarCFull]);
-            ++cc;
-          }
-          ++xc;
-          ++dzc;
-          continue;
+        if (t.i == t.hi) {  // first main tile: this segment's band
+          if (!tc::thread_wait(&bars[kBarAFull], t.seg & 1, abort)) break;
         }
-        // tail: z(lo) against x of tile lo - 1 (when it exists) and lo
-        const bool has_prev = t.lo > 0;
-        const int xl = (xc + kNX - 1) % kNX, xp = xc % kNX;
-        if (has_prev && !tc::thread_wait(&bars[kBarXFull + xp], (xc / kNX) & 1, abort)) break;
-        if (!tc::thread_wait(&bars[kBarZEmpty], (zc & 1) ^ 1, abort)) break;
+        const int xs = xc % kNX, ds = dzc % kNQ;
+        if (!tc::thread_wait(&bars[kBarXFull + xs], (xc / kNX) & 1, abort)) break;
+        if (!tc::thread_wait(&bars[kBarDZFull + ds], (dzc / kNQ) & 1, abort)) break;
+        const bool has_next = t.i + 1 < p.nT;
+        const int dn = (dzc + kNQ - 1) % kNQ;  // dz of tile i + 1 (previous acquisition)
+        // dx(i): the band against dz of tiles i+1 (halo rows) and i
+        const int xb = dxc & 1;
+        if (!tc::thread_wait(&bars[kBarDXEmpty + xb], ((dxc >> 1) & 1) ^ 1, abort)) break;
         tc_fence_after_sync();
-        toeplitz_chain(tmem_base + kColZ, band0, xs_base, has_prev ? xp : -1, xl, p.halo, id_t);
-        umma_commit(&bars[kBarZFull]);
-        ++zc;
-        umma_commit(&bars[kBarXEmpty + xl]);
-        if (has_prev) {
-          umma_commit(&bars[kBarXEmpty + xp]);
-          ++xc;
+        toeplitz_chain(tmem_base + kColDX + 64 * xb, band0, dz_base, has_next ? dn : -1, ds,
+                       p.halo, id_t);
+        umma_commit(&bars[kBarDXFull + xb]);
+        ++dxc;
+        // C += x(i) dz(i), x(i) dz(i+1)
+        if (t.i == t.hi) {
+          if (!tc::thread_wait(&bars[kBarCEmpty], (cc & 1) ^ 1, abort)) break;
+          tc_fence_after_sync();
+          lo_init = hi_init = false;
         }
-        umma_commit(&bars[kBarQEmpty + (dzc + kNQ - 1) % kNQ]);
-        umma_commit(&bars[kBarAEmpty]);
+        c_chain(tmem_base + kColC, xs_base + xs * kTileBytes, dz_base + ds * kTileBytes, id_c,
+                lo_init);
+        lo_init = true;
+        if (has_next) {
+          c_chain(tmem_base + kColC + 128, xs_base + xs * kTileBytes, dz_base + dn * kTileBytes,
+                  id_c, hi_init);
+          hi_init = true;
+          umma_commit(&bars[kBarQEmpty + dn]);  // dz(i+1) is used up
+        }
+        umma_commit(&bars[kBarXEmpty + xs]);    // x(i) is used up
+        if (t.i == t.lo) {
+          umma_commit(&bars[kBarQEmpty + ds]);  // dz(lo) is used up
+          umma_commit(&bars[kBarCFull]);
+          umma_commit(&bars[kBarAEmpty]);
+          ++cc;
+        }
+        ++xc;
+        ++dzc;
       }
       // Every MMA this thread issued must complete before TMEM is freed.
       umma_commit(&bars[kBarDone]);
@@ -571,19 +532,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ operand build
     BwdWalk it(w_begin, w_end, p.nT, p.B);
     BItem t;
-    uint32_t kc = 0, qc = 0, dc = 0, xc = 0, rc = 0;
-    const int gw = warp - kWarpGate0;
-    bool over = false;
+    uint32_t kc = 0, qc = 0, dc = 0, xc = 0, rc = 0, gphase = 0;
+    const int gw = warp - kWarpGate0, gtid = threadIdx.x - kWarpGate0 * 32;
     while (it.next(t)) {
       if (t.seg_first) {
-        if (t.seg > 0 && !tc::warp_wait(&bars[kBarAEmpty], (t.seg - 1) & 1, abort)) break;
-        build_band_gmem(kColBand, p.band_cols, tmem_base, p.h + static_cast<size_t>(t.g) * p.l_h,
-                            p.l_h, p.halo, warp & 3, lane, over);
+        if (t.seg > 0) {
+          if (!tc::warp_wait(&bars[kBarAEmpty], (t.seg - 1) & 1, abort)) break;
+          tc::tap_load(taps, p.h + static_cast<size_t>(t.g) * p.l_h, p.l_h, p.halo, 1, gtid);
+          // every gate thread has finished reading the previous taps ...
+          mbar_arrive(&bars[kBarGate]);
+          if (!tc::warp_wait(&bars[kBarGate], gphase++ & 1, abort)) break;
+        }
+        tc::tap_store(hz, taps, p.halo, 1, gtid, over);
+        // ... and has written its share of the new ones
+        mbar_arrive(&bars[kBarGate]);
+        if (!tc::warp_wait(&bars[kBarGate], gphase++ & 1, abort)) break;
+        tc::build_band_tmem(kColBand, p.band_cols, tmem_base, hz + 2, p.halo, warp & 3, lane);
         tc_fence_before_sync();
         mbar_arrive(&bars[kBarAFull]);
       }
-      if (t.kind == kTail && t.lo == 0) continue;
-      const bool need_x = t.kind != kNextHalo, need_dz = t.kind != kTail;
+      const bool need_x = t.kind == kMain;
       const int ks = kc % kNKV, qs = qc % kNQ, ds = dc % kNDY, xs = xc % kNX;
       if (need_x) {
         if (!tc::warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort)) break;
@@ -591,35 +559,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t kb = smem_u32(kv_st + ks * 2 * kTileBytes);
         gate_tile<false>(kb, kb + kTileBytes, smem_u32(x_st + xs * kTileBytes), gw, lane, over);
       }
-      if (need_dz) {
-        if (!tc::warp_wait(&bars[kBarQFull + qs], (qc / kNQ) & 1, abort)) break;
-        if (!tc::warp_wait(&bars[kBarDYFull + ds], (dc / kNDY) & 1, abort)) break;
-        if (!gate_dz_inplace(smem_u32(q_st + qs * kTileBytes), smem_u32(dy_st + ds * kTileBytes),
-                             gw, lane, over, &bars[kBarGateRead], rc & 1, abort))
-          break;
-        ++rc;
-      }
+      if (!tc::warp_wait(&bars[kBarQFull + qs], (qc / kNQ) & 1, abort)) break;
+      if (!tc::warp_wait(&bars[kBarDYFull + ds], (dc / kNDY) & 1, abort)) break;
+      if (!gate_dz_inplace(smem_u32(q_st + qs * kTileBytes), smem_u32(dy_st + ds * kTileBytes),
+                           gw, lane, over, &bars[kBarGateRead], rc & 1, abort))
+        break;
+      ++rc;
       fence_proxy_async_smem();
-      // this group is done with k, v (and dy); halo tiles have no second reader
       if (need_x) {
         mbar_arrive(&bars[kBarXFull + xs]);
-        mbar_arrive_cnt(&bars[kBarKVEmpty + ks], t.kind == kTail ? 2 : 1);
+        mbar_arrive(&bars[kBarKVEmpty + ks]);  // the epilogue is the stage's other reader
         ++kc;
         ++xc;
       }
-      if (need_dz) {
-        mbar_arrive(&bars[kBarDZFull + qs]);
-        mbar_arrive_cnt(&bars[kBarDYEmpty + ds], t.kind == kNextHalo ? 2 : 1);
-        ++qc;
-        ++dc;
-      }
+      mbar_arrive(&bars[kBarDZFull + qs]);
+      mbar_arrive(&bars[kBarDYEmpty + ds]);
+      ++qc;
+      ++dc;
     }
     if (over) atomicOr(&g_device_status, kF16RangeBit);
   } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
     // ------------------------------------------------------------ epilogue
-    // Thread = one tile row.  It copies its k, v (and later dy) rows from the input stages into
-    // registers and releases the stage at once; dq, dk, dv rows go straight out with streaming
-    // stores, so no stage waits for an output to drain.
+    // Thread = one tile row.  It copies its k, v rows from the input stage into registers and
+    // releases the stage at once; dk, dv rows go straight out with streaming stores.
     const int et = threadIdx.x - kWarpEpi0 * 32;
     const int quad = warp & 3;              // TMEM lanes this warp may read
     const int row_lane = quad * 32 + lane;  // MMA row = TMEM lane
@@ -628,112 +590,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *pw = part + quad * kPartLen;
     BwdWalk it(w_begin, w_end, p.nT, p.B);
     BItem t;
-    uint32_t zc = 0, dxc = 0, cc = 0, kc = 0, dc = 0;
-    int prev_ds = 0;        // dy stage of the previous main tile (its dq comes one step later)
-    uint32_t prev_dc = 0;   // and that stage's use count
+    uint32_t dxc = 0, cc = 0, kc = 0;
     int nseg = 0;
-    // Element offset of row `tt` of sequence b, group g (channel 64 g), or -1 past the end.
-    auto row_off = [&](int b, long long tt, int g) -> long long {
-      return tt < p.L ? (static_cast<long long>(b) * p.L + tt) * p.D + static_cast<long long>(g) * kNC
-                      : -1;
-    };
-    auto smem_row = [&](uint8_t *tile, int r, uint4 (&o)[8]) {
+    while (it.next(t)) {
+      if (t.kind != kMain) continue;
+      // dk = dx * v and dv = dx * k (dx lane p = time 128 i + p)
+      const int ks = kc % kNKV;
+      const uint32_t kcount = kc++;
+      const long long tt = static_cast<long long>(t.i) * kTM + row_lane;
+      if (!tc::warp_wait(&bars[kBarKVFull + ks], (kcount / kNKV) & 1, abort)) break;
+      uint4 kr[8], vr[8];
+      uint8_t *ktile = kv_st + ks * 2 * kTileBytes;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) o[c] = *row_chunk(tile, r, c);
-    };
-    // dq = dy * z for tile i (z lane p = time 128 i + 127 - p); dy from stage ds.
-    auto dq_tile = [&](int g, int i, int b, int ds, uint32_t dcount) -> bool {
-      const int r = kTM - 1 - row_lane;
-      const long long off = row_off(b, static_cast<long long>(i) * kTM + r, g);
-      if (!tc::warp_wait(&bars[kBarDYFull + ds], (dcount / kNDY) & 1, abort)) return false;
-      uint4 dr[8];
-      smem_row(dy_st + ds * kTileBytes, r, dr);
-      mbar_arrive(&bars[kBarDYEmpty + ds]);
-      if (!tc::warp_wait(&bars[kBarZFull], zc & 1, abort)) return false;
+      for (int c = 0; c < 8; ++c) {
+        kr[c] = lds_v4(row_chunk(ktile, row_lane, c));
+        vr[c] = lds_v4(row_chunk(ktile + kTileBytes, row_lane, c));
+      }
+      const int xb = dxc & 1;
+      if (!tc::warp_wait(&bars[kBarDXFull + xb], (dxc >> 1) & 1, abort)) break;
       tc_fence_after_sync();
       uint32_t a0[32], a1[32];
-      tmem_ld_32x32b_x32(tl + kColZ, a0);
-      tmem_ld_32x32b_x32(tl + kColZ + 32, a1);
+      tmem_ld_32x32b_x32(tl + kColDX + 64 * xb, a0);
+      tmem_ld_32x32b_x32(tl + kColDX + 64 * xb + 32, a1);
       tmem_wait_ld();
       reg_fence(a0);
       reg_fence(a1);
       tc_fence_before_sync();
-      mbar_arrive(&bars[kBarZEmpty]);
-      ++zc;
-      if (off >= 0) {
-        uint4 *dst = reinterpret_cast<uint4 *>(p.dq + off);
+      mbar_arrive(&bars[kBarDXEmpty + xb]);
+      ++dxc;
+      if (tt < p.L) {
+        const long long off = (static_cast<long long>(t.b) * p.L + tt) * p.D +
+                              static_cast<long long>(t.g) * kNC;
+        uint4 *dk = reinterpret_cast<uint4 *>(p.dk + off);
+        uint4 *dv = reinterpret_cast<uint4 *>(p.dv + off);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          float d[8], o[8];
-          unpack_bf16x8(dr[c], d);
+          float kf[8], vf[8], ok8[8], ov8[8];
+          unpack_bf16x8(kr[c], kf);
+          unpack_bf16x8(vr[c], vf);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int ch = 8 * c + e;
-            o[e] = d[e] * __uint_as_float(ch < 32 ? a0[ch] : a1[ch - 32]);
+            const float dx = __uint_as_float(ch < 32 ? a0[ch] : a1[ch - 32]);
+            ok8[e] = dx * vf[e];
+            ov8[e] = dx * kf[e];
           }
-          __stcs(dst + c, pack_bf16x8(o));
+          __stcs(dk + c, pack_bf16x8(ok8));
+          __stcs(dv + c, pack_bf16x8(ov8));
         }
       }
-      return true;
-    };
-    bool ok = true;
-    while (ok && it.next(t)) {
-      if (t.kind == kNextHalo) {
-        ++dc;
-        continue;
-      }
-      if (t.kind == kMain) {
-        // dk = dx * v and dv = dx * k (dx lane p = time 128 i + p)
-        const int ks = kc % kNKV, ds = dc % kNDY;
-        const uint32_t kcount = kc, dcount = dc;
-        ++kc;
-        ++dc;
-        const long long off = row_off(t.b, static_cast<long long>(t.i) * kTM + row_lane, t.g);
-        if (!tc::warp_wait(&bars[kBarKVFull + ks], (kcount / kNKV) & 1, abort)) break;
-        uint4 kr[8], vr[8];
-        uint8_t *ktile = kv_st + ks * 2 * kTileBytes;
-        smem_row(ktile, row_lane, kr);
-        smem_row(ktile + kTileBytes, row_lane, vr);
-        mbar_arrive(&bars[kBarKVEmpty + ks]);
-        if (!tc::warp_wait(&bars[kBarDXFull], dxc & 1, abort)) break;
-        tc_fence_after_sync();
-        uint32_t a0[32], a1[32];
-        tmem_ld_32x32b_x32(tl + kColDX, a0);
-        tmem_ld_32x32b_x32(tl + kColDX + 32, a1);
-        tmem_wait_ld();
-        reg_fence(a0);
-        reg_fence(a1);
-        tc_fence_before_sync();
-        mbar_arrive(&bars[kBarDXEmpty]);
-        ++dxc;
-        if (off >= 0) {
-          uint4 *dk = reinterpret_cast<uint4 *>(p.dk + off);
-          uint4 *dv = reinterpret_cast<uint4 *>(p.dv + off);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            float kf[8], vf[8], ok8[8], ov8[8];
-            unpack_bf16x8(kr[c], kf);
-            unpack_bf16x8(vr[c], vf);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int ch = 8 * c + e;
-              const float dx = __uint_as_float(ch < 32 ? a0[ch] : a1[ch - 32]);
-              ok8[e] = dx * vf[e];
-              ov8[e] = dx * kf[e];
-            }
-            __stcs(dk + c, pack_bf16x8(ok8));
-            __stcs(dv + c, pack_bf16x8(ov8));
-          }
-        }
-        // dq of tile i + 1 (its z was issued with this tile)
-        if (t.i < t.hi && !dq_tile(t.g, t.i + 1, t.b, prev_ds, prev_dc)) break;
-        prev_ds = ds;
-        prev_dc = dcount;
-        continue;
-      }
-      // tail: dq of tile lo, then the dh sums of the segment
-      if (t.lo > 0) ++kc;
-      if (!dq_tile(t.g, t.lo, t.b, prev_ds, prev_dc)) break;
+      // The stage goes back to the producer (whose next TMA write to it is an async-proxy
+      // access) only once every row load has returned its data and is ordered before the
+      // arrive: an arrive issued right after the loads let the next tile's TMA write land under
+      // them (seen as sporadic wrong rows in one warp's quarter of a tile).
+      consume_rows(kr);
+      consume_rows(vr);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[kBarKVEmpty + ks]);
+      if (t.i != t.lo) continue;
+      // end of the segment: the dh sums
       if (!tc::warp_wait(&bars[kBarCFull], cc & 1, abort)) break;
       tc_fence_after_sync();
       for (int j = lane; j < kPartLen; j += 32) pw[j] = 0.f;

@@ -478,6 +478,8 @@ bool tc_bwd_supported(const Problem &P, const void *dy, const void *dq, const vo
          aligned(dv, 16);
 }
 
+// dq = dy * (h conv x) is the forward with dy in the place of q (the tuned forward kernel);
+// then fir_tc_bwd_kernel (dx, dk, dv and the dh partials) and the fixed-order dh reduction.
 int launch_tensor_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv, float *dh,
                       void *workspace, size_t workspace_bytes, cudaStream_t s) {
   namespace tb = hyena::tcb;
@@ -521,15 +523,28 @@ int launch_tensor_bwd(const Problem &P, const void *dy, void *dq, void *dk, void
   p.seg_group = reinterpret_cast<int *>(ws + lay.off_group);
   p.seg_count = reinterpret_cast<int *>(ws + lay.off_count);
   p.D = P.D;
-  p.k = static_cast<const __nv_bfloat16 *>(P.k);
-  p.v = static_cast<const __nv_bfloat16 *>(P.v);
-  p.dy = static_cast<const __nv_bfloat16 *>(dy);
-  p.dq = static_cast<__nv_bfloat16 *>(dq);
   p.dk = static_cast<__nv_bfloat16 *>(dk);
   p.dv = static_cast<__nv_bfloat16 *>(dv);
-  tb::fir_tc_bwd_kernel<<<static_cast<unsigned>(grid), tb::kThreads, tb::kSmemBytes, s>>>(
-      maps[0], maps[1], maps[2], maps[3], p);
-  if (cudaGetLastError() != cudaSuccess) return HYENA_ERR_CUDA;
+  Problem F = P;  // dq through the forward kernels
+  F.q = dy;
+  F.y = dq;
+  const int rf = run(F, HYENA_ALGO_AUTO, s);
+  if (rf != HYENA_OK) return rf;
+  // Programmatic dependent launch: the set-up overlaps the end of the dq forward.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = HYENA_PDL;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(tb::kThreads);
+  cfg.dynamicSmemBytes = tb::kSmemBytes;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, tb::fir_tc_bwd_kernel, maps[0], maps[1], maps[2], maps[3], p) !=
+          cudaSuccess ||
+      cudaGetLastError() != cudaSuccess)
+    return HYENA_ERR_CUDA;
   const long long gn = static_cast<long long>(p.G) * P.l_h;
   long long rblocks = (gn + 255) / 256;
   if (rblocks > ds->sm_count) rblocks = ds->sm_count;
