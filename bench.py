@@ -222,7 +222,8 @@ def time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind):
         bufs.append((q, k, v, h, dy, dq, dk, dv, dh))
     cfn = _native.lib().hyena_conv_bwd
     algo = g.hyena_select_bwd_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, code)
-    kernels = (["fir_tc_bwd_kernel", "fir_bwd_tc_reduce_kernel"] if algo == g.HYENA_ALGO_TENSOR
+    kernels = (["fir_tc_kernel (dq)", "fir_tc_bwd_kernel", "fir_bwd_tc_reduce_kernel"]
+               if algo == g.HYENA_ALGO_TENSOR
                else ["forward kernel (dq)", "fir_bwd_dx_kernel", "fir_bwd_dh_partial_kernel",
                      "fir_bwd_dh_reduce_kernel"])
     cargs = [tuple(t.data_ptr() for t in b) + (wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, code,

@@ -26,6 +26,7 @@ __all__ = [
     "HYENA_ALGO_DIRECT", "HYENA_DTYPE_BF16", "HYENA_DTYPE_F32", "HYENA_DEVICE_TIMEOUT",
     "HYENA_DEVICE_F16_RANGE", "ALGO_NAMES", "hyena_conv_fwd_from_host",
     "hyena_toeplitz_stages", "hyena_build_toeplitz_blocks", "hyena_conv_fwd_hist",
+    "hyena_conv_fwd_fft", "hyena_conv_fwd_fft_workspace_bytes",
 ]
 
 
@@ -116,6 +117,33 @@ def hyena_conv_fwd_hist(q, k, v, h, d_g, l_b, k_hist, v_hist, algo=HYENA_ALGO_AU
                                            d_g, h.shape[1], l_b, _dtype_code(q), algo,
                                            _stream(stream))
     _native.check("hyena_conv_fwd_hist", rc)
+    return y
+
+
+def hyena_conv_fwd_fft_workspace_bytes(B, L, D, d_g, l_h):
+    """Bytes of workspace hyena_conv_fwd_fft needs (raises where the FFT path does not apply)."""
+    n = int(_native.lib().hyena_conv_fwd_fft_workspace_bytes(B, L, D, d_g, l_h))
+    if n < 0:
+        _native.check("hyena_conv_fwd_fft_workspace_bytes", -n)
+    return n
+
+
+def hyena_conv_fwd_fft(q, k, v, h, d_g, l_b, workspace=None, y=None, stream=None):
+    """Forward by FFT convolution (long filters): same operation and arguments as
+    hyena_conv_fwd_ex; ``workspace`` is a CUDA uint8 tensor of at least
+    hyena_conv_fwd_fft_workspace_bytes() bytes (allocated here when None)."""
+    torch = _torch()
+    y = _check(q, k, v, h, d_g, y)
+    B, L, D = q.shape
+    need = hyena_conv_fwd_fft_workspace_bytes(B, L, D, d_g, h.shape[1])
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    rc = _native.lib().hyena_conv_fwd_fft(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                          h.data_ptr(), y.data_ptr(), B, L, D, d_g, h.shape[1],
+                                          l_b, _dtype_code(q), workspace.data_ptr(),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream(stream))
+    _native.check("hyena_conv_fwd_fft", rc)
     return y
 
 

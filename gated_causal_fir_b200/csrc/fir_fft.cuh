@@ -1,0 +1,214 @@
+// fir_fft.cuh -- FFT kernels of the gated grouped causal convolution for long filters (the
+// Hyena-LI class of the StripedHyena 2 overview, Sec. 3 operator table: long implicit filters,
+// evaluated by FFT convolution, O(L log L) per channel instead of O(L l_h)).
+//
+// The convolution y = q * (h_g conv x), x = k * v, is evaluated as a cyclic convolution of
+// length N = N1 N2 >= L + l_h - 1 (a power of two): zero padding makes the cyclic sum equal
+// the causal one for every t < L.  The length-N DFT uses the four-step factorisation
+//     X[k1 + N1 k2] = sum_{n2} W_N2^{n2 k2} W_N^{n2 k1} sum_{n1} x[N2 n1 + n2] W_N1^{n1 k1},
+// W_M = exp(-2 pi i / M), and its inverse in the mirrored order.  Three kernels:
+//   pass 1 (per n2): x = k v over the rows t = N2 n1 + n2, length-N1 FFT, times W_N^{n2 k1};
+//   pass 2 (per k1): length-N2 FFT, times the filter spectrum H[k1 + N1 k2], inverse FFT;
+//   pass 3 (per n2): times W_N^{-n2 k1}, inverse length-N1 FFT, / N, times q, store t < L.
+// The filter spectrum comes from passes 1 and 2 run on h ("spectrum" mode).
+//
+// Two channels of one group travel as one complex signal x_c + i x_{c+1}: their filter (and
+// so its spectrum) is the same and both signals are real, so the inverse transform of
+// H (X_c + i X_{c+1}) is y_c + i y_{c+1} exactly -- no separation step.
+//
+// Every FFT runs in shared memory: P signals (channel pairs) side by side, radix-2 Stockham
+// stages (self-sorting: natural order in, natural order out), twiddles from sincospif.  The
+// intermediate spectra live in a caller-owned fp32 workspace laid out [b][k1][n2][pair], so
+// every pass reads and writes P contiguous complex values (128 bytes) per index.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "fir_cuda_core.cuh"
+
+namespace hyena {
+namespace fft {
+
+constexpr int kP = 16;          // signals (channel pairs) per CTA
+constexpr int kThreads = 256;
+constexpr int kMaxLen = 256;    // N1, N2 <= 256: N <= 65536
+
+struct FftParams {
+  long long B, L, D;
+  int d_g, l_h;
+  int N1, N2, log1, log2;
+  long long PT;      // signals per sequence: D / 2 (data) or G (spectrum)
+  int G;
+};
+
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+  return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
+}
+
+// exp(-2 pi i num / den) (den a power of two, |num| < den), accurate to a few ulp.
+__device__ __forceinline__ float2 twiddle(long long num, long long den) {
+  float s, c;
+  sincospif(-2.0f * static_cast<float>(num) / static_cast<float>(den), &s, &c);
+  return make_float2(c, s);
+}
+
+// Radix-2 Stockham FFT of n = 2^logn points for kP signals laid out a[point * kP + signal];
+// b is scratch of the same size; tw[k] = W_n^k for k < n / 2.  Forward (W) or inverse (W^-1,
+// unscaled).  Returns the buffer holding the result.  All threads of the CTA take part.
+template <bool kInverse>
+__device__ float2 *fft_smem(float2 *a, float2 *b, int n, int logn, const float2 *tw) {
+  const int half = n >> 1;
+  for (int s = 0; s < logn; ++s) {
+    const int ns = 1 << s;
+    for (int e = threadIdx.x; e < half * kP; e += blockDim.x) {
+      const int j = e / kP, sig = e % kP;
+      const int k = j & (ns - 1);
+      float2 w = tw[k << (logn - 1 - s)];  // W_{2 ns}^k
+      if (kInverse) w.y = -w.y;
+      const float2 u = a[j * kP + sig];
+      const float2 t = cmul(a[(j + half) * kP + sig], w);
+      const int d = ((j - k) << 1) + k;
+      b[d * kP + sig] = make_float2(u.x + t.x, u.y + t.y);
+      b[(d + ns) * kP + sig] = make_float2(u.x - t.x, u.y - t.y);
+    }
+    __syncthreads();
+    float2 *x = a;
+    a = b;
+    b = x;
+  }
+  return a;
+}
+
+__device__ __forceinline__ void fill_twiddles(float2 *tw, int n) {
+  for (int k = threadIdx.x; k < (n >> 1); k += blockDim.x) tw[k] = twiddle(k, n);
+}
+
+// Pass 1.  Block (n2, signal block, b).  Data mode: signal s of sequence b is
+// k v at channels 2s, 2s+1 (real, imaginary); spectrum mode: signal s is filter s (real).
+// Writes A[b][k1][n2][s] = W_N^{n2 k1} * sum_{n1} z[N2 n1 + n2] W_N1^{n1 k1}.
+template <typename T, bool kSpectrum>
+__global__ void __launch_bounds__(kThreads)
+    fft_pass1_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ h,
+                     float2 *__restrict__ A, const FftParams p) {
+  extern __shared__ float2 fsm[];
+  const int n1len = p.N1;
+  float2 *b0 = fsm, *b1 = fsm + n1len * kP, *tw = fsm + 2 * n1len * kP;
+  const int n2 = blockIdx.x;
+  const long long s0 = static_cast<long long>(blockIdx.y) * kP;
+  const long long b = blockIdx.z;
+  const long long N = static_cast<long long>(p.N1) * p.N2;
+  fill_twiddles(tw, n1len);
+  for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
+    const int n1 = e / kP, sig = e % kP;
+    const long long t = static_cast<long long>(p.N2) * n1 + n2;
+    const long long s = s0 + sig;
+    float2 z = make_float2(0.f, 0.f);
+    if (s < p.PT) {
+      if (kSpectrum) {
+        if (t < p.l_h) z.x = __ldg(h + s * p.l_h + t);
+      } else if (t < p.L) {
+        const long long off = (b * p.L + t) * p.D + 2 * s;
+        z.x = cc::to_f32(k[off]) * cc::to_f32(v[off]);
+        z.y = cc::to_f32(k[off + 1]) * cc::to_f32(v[off + 1]);
+      }
+    }
+    b0[e] = z;
+  }
+  __syncthreads();
+  const float2 *r = fft_smem<false>(b0, b1, n1len, p.log1, tw);
+  for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
+    const int k1 = e / kP, sig = e % kP;
+    const long long s = s0 + sig;
+    if (s < p.PT)
+      A[((b * p.N1 + k1) * p.N2 + n2) * p.PT + s] =
+          cmul(r[e], twiddle((static_cast<long long>(n2) * k1) % N, N));
+  }
+}
+
+// Pass 2.  Block (k1, signal block, b): length-N2 FFT over n2 of A[b][k1][.][s].  Spectrum
+// mode writes the spectrum H[k1][k2][g] (signal = group); data mode multiplies by the group's
+// H, inverse-transforms over k2 and writes the result back in place.
+template <bool kSpectrum>
+__global__ void __launch_bounds__(kThreads)
+    fft_pass2_kernel(float2 *__restrict__ A, float2 *__restrict__ H, const FftParams p) {
+  extern __shared__ float2 fsm[];
+  const int n2len = p.N2;
+  float2 *b0 = fsm, *b1 = fsm + n2len * kP, *tw = fsm + 2 * n2len * kP;
+  const int k1 = blockIdx.x;
+  const long long s0 = static_cast<long long>(blockIdx.y) * kP;
+  const long long b = blockIdx.z;
+  fill_twiddles(tw, n2len);
+  float2 *row = A + (b * p.N1 + k1) * p.N2 * p.PT;
+  for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
+    const int n2 = e / kP, sig = e % kP;
+    const long long s = s0 + sig;
+    b0[e] = s < p.PT ? row[n2 * p.PT + s] : make_float2(0.f, 0.f);
+  }
+  __syncthreads();
+  float2 *r = fft_smem<false>(b0, b1, n2len, p.log2, tw);
+  float2 *o = r == b0 ? b1 : b0;
+  if constexpr (kSpectrum) {
+    for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
+      const int k2 = e / kP, sig = e % kP;
+      const long long s = s0 + sig;
+      if (s < p.PT) H[(static_cast<long long>(k1) * p.N2 + k2) * p.G + s] = r[e];
+    }
+  } else {
+    for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
+      const int k2 = e / kP, sig = e % kP;
+      const long long s = s0 + sig;
+      const long long g = s < p.PT ? (2 * s) / p.d_g : 0;
+      r[e] = cmul(r[e], H[(static_cast<long long>(k1) * p.N2 + k2) * p.G + g]);
+    }
+    __syncthreads();
+    const float2 *y = fft_smem<true>(r, o, n2len, p.log2, tw);
+    for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
+      const int n2 = e / kP, sig = e % kP;
+      const long long s = s0 + sig;
+      if (s < p.PT) row[n2 * p.PT + s] = y[e];
+    }
+  }
+}
+
+// Pass 3.  Block (n2, signal block, b): W_N^{-n2 k1} times A[b][.][n2][s], inverse length-N1
+// FFT over k1, scaled by 1/N: the convolution at t = N2 n1 + n2; y = q * conv for t < L.
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+    fft_pass3_kernel(const float2 *__restrict__ A, const T *__restrict__ q, T *__restrict__ y,
+                     const FftParams p) {
+  extern __shared__ float2 fsm[];
+  const int n1len = p.N1;
+  float2 *b0 = fsm, *b1 = fsm + n1len * kP, *tw = fsm + 2 * n1len * kP;
+  const int n2 = blockIdx.x;
+  const long long s0 = static_cast<long long>(blockIdx.y) * kP;
+  const long long b = blockIdx.z;
+  const long long N = static_cast<long long>(p.N1) * p.N2;
+  fill_twiddles(tw, n1len);
+  for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
+    const int k1 = e / kP, sig = e % kP;
+    const long long s = s0 + sig;
+    float2 z = make_float2(0.f, 0.f);
+    if (s < p.PT) {
+      float2 w = twiddle((static_cast<long long>(n2) * k1) % N, N);
+      w.y = -w.y;
+      z = cmul(A[((b * p.N1 + k1) * p.N2 + n2) * p.PT + s], w);
+    }
+    b0[e] = z;
+  }
+  __syncthreads();
+  const float2 *r = fft_smem<true>(b0, b1, n1len, p.log1, tw);
+  const float inv = 1.0f / static_cast<float>(N);
+  for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
+    const int n1 = e / kP, sig = e % kP;
+    const long long t = static_cast<long long>(p.N2) * n1 + n2;
+    const long long s = s0 + sig;
+    if (s < p.PT && t < p.L) {
+      const long long off = (b * p.L + t) * p.D + 2 * s;
+      cc::from_f32(cc::to_f32(q[off]) * (r[e].x * inv), y + off);
+      cc::from_f32(cc::to_f32(q[off + 1]) * (r[e].y * inv), y + off + 1);
+    }
+  }
+}
+
+}  // namespace fft
+}  // namespace hyena

@@ -11,6 +11,7 @@
 #include "hyena_conv.h"
 #include "fir_bwd.cuh"
 #include "fir_cuda_core.cuh"
+#include "fir_fft.cuh"
 #include "fir_tc.cuh"
 #include "fir_tc_bwd.cuh"
 
@@ -34,6 +35,11 @@ constexpr int kMaxDevices = 64;
 constexpr int kDhSmemMax =
     (2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (64 + 1) * static_cast<int>(sizeof(float));
 constexpr int kMaxWindowTaps = 16;
+// Shared memory of an FFT pass over n points: two buffers of n x kP complex and n / 2 twiddles.
+constexpr int fft_smem_bytes(int n) {
+  return (2 * n * hyena::fft::kP + n / 2) * static_cast<int>(sizeof(float2));
+}
+constexpr int kFftSmemMax = fft_smem_bytes(hyena::fft::kMaxLen);
 #ifndef HYENA_WINDOW_ROWS
 #define HYENA_WINDOW_ROWS 128
 #endif
@@ -75,6 +81,17 @@ int current_device(DeviceState *&ds) {
     for (const void *k : dh_kernels)
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kDhSmemMax);
+    const void *fft_kernels[] = {
+        reinterpret_cast<const void *>(hyena::fft::fft_pass1_kernel<float, true>),
+        reinterpret_cast<const void *>(hyena::fft::fft_pass1_kernel<float, false>),
+        reinterpret_cast<const void *>(hyena::fft::fft_pass1_kernel<__nv_bfloat16, false>),
+        reinterpret_cast<const void *>(hyena::fft::fft_pass2_kernel<true>),
+        reinterpret_cast<const void *>(hyena::fft::fft_pass2_kernel<false>),
+        reinterpret_cast<const void *>(hyena::fft::fft_pass3_kernel<float>),
+        reinterpret_cast<const void *>(hyena::fft::fft_pass3_kernel<__nv_bfloat16>)};
+    for (const void *k : fft_kernels)
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kFftSmemMax);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(reinterpret_cast<const void *>(hyena::tcb::fir_tc_bwd_kernel),
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -554,6 +571,91 @@ int launch_tensor_bwd(const Problem &P, const void *dy, void *dq, void *dk, void
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
+// FFT path: N = N1 N2 >= L + l_h - 1 (power of two, >= 64), N1 >= N2, both <= 256.
+struct FftPlan {
+  int N1, N2, log1, log2;
+  int64_t N;
+  bool ok;
+};
+
+FftPlan fft_plan(int64_t L, int l_h) {
+  FftPlan f{0, 0, 0, 0, 0, false};
+  const int64_t need = L + l_h - 1;
+  int m = 6;
+  while ((int64_t{1} << m) < need && m < 40) ++m;
+  f.log1 = (m + 1) / 2;
+  f.log2 = m / 2;
+  f.N1 = 1 << f.log1;
+  f.N2 = 1 << f.log2;
+  f.N = int64_t{1} << m;
+  f.ok = f.N1 <= hyena::fft::kMaxLen;
+  return f;
+}
+
+struct FftLayout {
+  int64_t off_hspec, off_h, bytes;
+};
+
+// Workspace: the data spectra [B][N1][N2][D/2] complex, the filters' pass-1 output and their
+// spectrum [N1 N2][G] complex.
+FftLayout fft_layout(int64_t B, int64_t D, int64_t G, int64_t N) {
+  FftLayout o;
+  o.off_hspec = round256(B * N * (D / 2) * 8);
+  o.off_h = o.off_hspec + round256(N * G * 8);
+  o.bytes = o.off_h + round256(N * G * 8);
+  return o;
+}
+
+// 0 when the FFT path takes the shape, else the error it returns.
+int fft_supported(const Problem &P, FftPlan &f) {
+  if (P.D % 2 != 0 || P.d_g % 2 != 0) return HYENA_ERR_UNSUPPORTED;
+  f = fft_plan(P.L, P.l_h);
+  if (!f.ok || P.B > 65535 || (P.D / 2 + hyena::fft::kP - 1) / hyena::fft::kP > 65535 ||
+      (P.G() + hyena::fft::kP - 1) / hyena::fft::kP > 65535)
+    return HYENA_ERR_UNSUPPORTED;
+  return HYENA_OK;
+}
+
+template <typename T>
+int launch_fft(const Problem &P, const FftPlan &f, uint8_t *ws, cudaStream_t s) {
+  namespace hf = hyena::fft;
+  const FftLayout lay = fft_layout(P.B, P.D, P.G(), f.N);
+  float2 *A = reinterpret_cast<float2 *>(ws);
+  float2 *Hs = reinterpret_cast<float2 *>(ws + lay.off_hspec);
+  float2 *Hh = reinterpret_cast<float2 *>(ws + lay.off_h);
+  hf::FftParams p;
+  p.B = P.B;
+  p.L = P.L;
+  p.D = P.D;
+  p.d_g = P.d_g;
+  p.l_h = P.l_h;
+  p.N1 = f.N1;
+  p.N2 = f.N2;
+  p.log1 = f.log1;
+  p.log2 = f.log2;
+  p.G = static_cast<int>(P.G());
+  // the filters' spectrum H[k1][k2][g]
+  hf::FftParams ph = p;
+  ph.PT = P.G();
+  ph.B = 1;
+  const unsigned gb = static_cast<unsigned>((ph.PT + hf::kP - 1) / hf::kP);
+  hf::fft_pass1_kernel<float, true><<<dim3(f.N2, gb, 1), hf::kThreads, fft_smem_bytes(f.N1), s>>>(
+      nullptr, nullptr, P.h, Hh, ph);
+  hf::fft_pass2_kernel<true><<<dim3(f.N1, gb, 1), hf::kThreads, fft_smem_bytes(f.N2), s>>>(
+      Hh, Hs, ph);
+  // the data: pass 1, pass 2 (times H, inverse), pass 3 (inverse, q gate)
+  p.PT = P.D / 2;
+  const unsigned db = static_cast<unsigned>((p.PT + hf::kP - 1) / hf::kP);
+  const unsigned nb = static_cast<unsigned>(P.B);
+  hf::fft_pass1_kernel<T, false><<<dim3(f.N2, db, nb), hf::kThreads, fft_smem_bytes(f.N1), s>>>(
+      static_cast<const T *>(P.k), static_cast<const T *>(P.v), nullptr, A, p);
+  hf::fft_pass2_kernel<false><<<dim3(f.N1, db, nb), hf::kThreads, fft_smem_bytes(f.N2), s>>>(
+      A, Hs, p);
+  hf::fft_pass3_kernel<T><<<dim3(f.N2, db, nb), hf::kThreads, fft_smem_bytes(f.N1), s>>>(
+      A, static_cast<const T *>(P.q), static_cast<T *>(P.y), p);
+  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
 // Host checks of a backward call; HYENA_OK, kEmpty or an error code.
 int validate_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv, float *dh,
                  void *workspace, size_t workspace_bytes) {
@@ -676,6 +778,37 @@ int hyena_conv_fwd_hist(const void *q, const void *k, const void *v, const float
   P.vh = v_hist;
   P.Lh = L_hist;
   return run(P, algo, stream);
+}
+
+int64_t hyena_conv_fwd_fft_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
+  if (B < 0 || L < 0 || D < 1 || d_g < 1 || D % d_g != 0 || l_h < 1) return -HYENA_ERR_INVALID_ARG;
+  const Problem P{nullptr, nullptr, nullptr, nullptr, nullptr, B, L, D, d_g, l_h, 1,
+                  HYENA_DTYPE_BF16};
+  if (B == 0 || L == 0) return 0;
+  FftPlan f{};
+  if (fft_supported(P, f) != HYENA_OK) return -HYENA_ERR_UNSUPPORTED;
+  return fft_layout(B, D, P.G(), f.N).bytes;
+}
+
+int hyena_conv_fwd_fft(const void *q, const void *k, const void *v, const float *h, void *y,
+                       int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b, int dtype,
+                       void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const Problem P{q, k, v, h, y, B, L, D, d_g, l_h, l_b, dtype};
+  const int rc = validate(P);
+  if (rc == kEmpty) return HYENA_OK;
+  if (rc != HYENA_OK) return rc;
+  FftPlan f{};
+  const int fs = fft_supported(P, f);
+  if (fs != HYENA_OK) return fs;
+  if (!workspace) return HYENA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16)) return HYENA_ERR_MISALIGNED;
+  if (static_cast<int64_t>(workspace_bytes) < fft_layout(B, D, P.G(), f.N).bytes)
+    return HYENA_ERR_INVALID_ARG;
+  DeviceState *ds = nullptr;
+  if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  if (dtype == HYENA_DTYPE_F32) return launch_fft<float>(P, f, ws, stream);
+  return launch_fft<__nv_bfloat16>(P, f, ws, stream);
 }
 
 int hyena_select_algo(const void *q, const void *k, const void *v, const float *h, const void *y,

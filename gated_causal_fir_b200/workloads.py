@@ -69,6 +69,8 @@ WORKLOADS = {
     "mr": Workload("mr", 1, 8192, 4096, 64, 128, 64, "bf16", "mr", 2),
     "mr_batched": Workload("mr_batched", 8, 32768, 4096, 64, 128, 64, "bf16", "mr", 3),
     "mr_1m": Workload("mr_1m", 1, 1 << 20, 4096, 64, 128, 64, "bf16", "mr", 4),
+    # long filters (the Hyena-LI class): filter as long as the sequence, decayed like MR's
+    "li": Workload("li", 1, 8192, 4096, 64, 8192, 64, "bf16", "mr", 5),
 }
 
 

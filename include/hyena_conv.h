@@ -122,6 +122,34 @@ int hyena_conv_fwd_hist(const void *q, const void *k, const void *v, const float
                         cudaStream_t stream);
 
 /*
+ * Host-only: bytes of device workspace hyena_conv_fwd_fft needs for this shape (a multiple of
+ * 256), minus HYENA_ERR_INVALID_ARG for a bad shape, or minus HYENA_ERR_UNSUPPORTED where the
+ * FFT path does not apply (odd D or d_g, or L + l_h - 1 > 65536).  Touches no device.  The
+ * workspace holds the fp32 spectra: 4 B L_fft D bytes for the data plus 16 L_fft D / d_g for
+ * the filters, L_fft the power of two >= max(64, L + l_h - 1) (256 MiB of data spectra at
+ * B = 1, L = l_h = 8192, D = 4096).
+ */
+int64_t hyena_conv_fwd_fft_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h);
+
+/*
+ * The same operation as hyena_conv_fwd_ex, evaluated by FFT: the convolution of every channel
+ * with its group's filter as a cyclic convolution of length L_fft (zero-padded, so exact for
+ * t < L), computed with a four-step FFT in three passes over the workspace.  For long filters
+ * (the Hyena-LI operator of StripedHyena 2, overview page, Sec. 3 operator table: long
+ * implicit filters, FFT convolution; the direct and block-Toeplitz forms cost O(L l_h) per
+ * channel, this one O(L log L)).  Any l_h >= 1; needs D and d_g even (two channels of a group
+ * share one complex transform) and L + l_h - 1 <= 65536.  dtype bf16 or fp32 (q, k, v, y);
+ * the transforms run in fp32.
+ * workspace: DEVICE scratch of at least hyena_conv_fwd_fft_workspace_bytes() bytes, 16-byte
+ * aligned, owned by the caller, unused after the queued work ends.
+ * Errors: as hyena_conv_fwd_ex, plus HYENA_ERR_UNSUPPORTED as above, HYENA_ERR_INVALID_ARG for
+ * a NULL or too small workspace, HYENA_ERR_MISALIGNED for a misaligned one.
+ */
+int hyena_conv_fwd_fft(const void *q, const void *k, const void *v, const float *h, void *y,
+                       int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b, int dtype,
+                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Host-only: the algorithm (enum hyena_algo, > 0) that HYENA_ALGO_AUTO would run for this
  * problem and these pointers, or minus an error code.  Touches no device.
  */

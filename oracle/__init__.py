@@ -9,6 +9,7 @@ marshals numpy arrays.  What each function computes, with its source on the Stri
 page "04. Hardware-aware convolution kernels":
 
 * :func:`gated_fir` -- the direct sum of Sec. 1, gated: y = q * sum_j h_g[j] (k v)[t-j].
+* :func:`gated_fir_rows` -- the same direct sum for selected output rows only.
 * :func:`toeplitz_blocks` -- the l_b x l_b sub-blocks H_m[i][j] = h[m l_b + i - j] of the
   lower-triangular Toeplitz matrix (Sec. 2; index rule fixed by the Sec. 3 worked example).
 * :func:`block_conv` -- the S-stage block form Yhat_n = sum_{m<S} H_m Xhat_{n-m} (Sec. 2/3;
@@ -44,6 +45,10 @@ class OracleLib:
         lib.oracle_gated_fir_f64.argtypes = [_dp, _dp, _dp, _dp, _dp, i64, i64, i64, i64, i64,
                                              ctypes.c_int]
         lib.oracle_gated_fir_f64.restype = ctypes.c_int
+        lib.oracle_gated_fir_rows_f64.argtypes = [_dp, _dp, _dp, _dp,
+                                                  ctypes.POINTER(ctypes.c_int64), i64, _dp, i64,
+                                                  i64, i64, i64, i64, ctypes.c_int]
+        lib.oracle_gated_fir_rows_f64.restype = ctypes.c_int
         lib.oracle_toeplitz_blocks_f64.argtypes = [_dp, i64, i64, i64, _dp]
         lib.oracle_toeplitz_blocks_f64.restype = ctypes.c_int
         lib.oracle_block_conv_f64.argtypes = [_dp, i64, i64, i64, _dp, i64, _dp]
@@ -81,6 +86,24 @@ class OracleLib:
         if rc != 0:
             raise ValueError("oracle_gated_fir_f64 rejected its arguments (rc=%d)" % rc)
         return y[0] if squeeze else y
+
+    def gated_fir_rows(self, q, k, v, h, d_g: int, rows, nthreads: int = 0) -> np.ndarray:
+        """y[b, t, :] of :meth:`gated_fir` for each (b, t) in ``rows`` only: [len(rows), D]."""
+        q, k, v, h = _f64(q), _f64(k), _f64(v), _f64(h)
+        if q.ndim == 2:
+            q, k, v = q[None], k[None], v[None]
+        B, L, D = q.shape
+        assert k.shape == q.shape and v.shape == q.shape, "q, k, v shapes differ"
+        assert h.ndim == 2 and h.shape[0] * d_g == D, "h must be [D // d_g, l_h]"
+        flat = np.ascontiguousarray([b * L + t for b, t in rows], dtype=np.int64)
+        out = np.empty((len(flat), D), dtype=np.float64)
+        rc = self.lib.oracle_gated_fir_rows_f64(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(h),
+            flat.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), len(flat), _ptr(out), B, L, D,
+            d_g, h.shape[1], nthreads)
+        if rc != 0:
+            raise ValueError("oracle_gated_fir_rows_f64 rejected its arguments (rc=%d)" % rc)
+        return out
 
     def gated_fir_bwd(self, q, k, v, h, dy, d_g: int, nthreads: int = 0):
         """Gradients (dq, dk, dv, dh) of sum(dy * y) for y = gated_fir(q, k, v, h, d_g)."""
@@ -139,6 +162,10 @@ def max_threads() -> int:
 
 def gated_fir(q, k, v, h, d_g: int, nthreads: int = 0) -> np.ndarray:
     return default().gated_fir(q, k, v, h, d_g, nthreads)
+
+
+def gated_fir_rows(q, k, v, h, d_g: int, rows, nthreads: int = 0) -> np.ndarray:
+    return default().gated_fir_rows(q, k, v, h, d_g, rows, nthreads)
 
 
 def toeplitz_blocks(h, l_b: int, S: int) -> np.ndarray:

@@ -76,6 +76,45 @@ int oracle_gated_fir_f64(const double *q, const double *k, const double *v, cons
 }
 
 /*
+ * The same direct definition for a list of output rows only: for i < n_rows with
+ * rows[i] = b * L + t,  y_rows[i * D + c] = y[b, t, c]  of oracle_gated_fir_f64, computed with
+ * the same products in the same tap order.  Lets a test check sampled rows of sequences whose
+ * full oracle (O(L l_h D)) would take too long, e.g. filters as long as the sequence.
+ */
+int oracle_gated_fir_rows_f64(const double *q, const double *k, const double *v, const double *h,
+                              const int64_t *rows, int64_t n_rows, double *y_rows, int64_t B,
+                              int64_t L, int64_t D, int64_t d_g, int64_t l_h, int nthreads)
+{
+    if (!q || !k || !v || !h || (!rows && n_rows > 0) || (!y_rows && n_rows > 0))
+        return ORACLE_BAD_ARG;
+    if (B < 0 || L < 0 || D < 1 || d_g < 1 || D % d_g != 0 || l_h < 1 || n_rows < 0)
+        return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < n_rows; ++i)
+        if (rows[i] < 0 || rows[i] >= B * L) return ORACLE_BAD_ARG;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    #pragma omp parallel for schedule(static)
+    for (int64_t ic = 0; ic < n_rows * D; ++ic) {
+        const int64_t i = ic / D, c = ic % D;
+        const int64_t row = rows[i];
+        const int64_t b = row / L;
+        const int64_t t = row % L;
+        const int64_t last = (l_h - 1 < t) ? l_h - 1 : t;
+        const double *hg = h + (c / d_g) * l_h;
+        double acc = 0.0;
+        for (int64_t tap = 0; tap <= last; ++tap) {
+            const int64_t at = (b * L + (t - tap)) * D + c;
+            acc += hg[tap] * (k[at] * v[at]);
+        }
+        y_rows[ic] = q[row * D + c] * acc;
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Sub-blocks of the lower-triangular Toeplitz matrix (page 04, Sec. 2 and the Sec. 3 worked
  * example): H[m][i][j] = h[m*l_b + i - j] when that index lies in [0, l_h), else 0,
  * for m = 0 .. S-1.  H: [S, l_b, l_b] row-major.

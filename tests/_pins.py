@@ -142,6 +142,24 @@ def pin_torch_conv1d(o):
 
 # ---------------------------------------------------------------- invariants
 
+def pin_rows_match_the_full_sum(o):
+    """Selected rows of the direct sum equal the same rows of the full direct sum (incl. the
+    first row, a row inside the filter's reach of t = 0 and the last), and numpy.convolve for
+    one channel."""
+    rng = np.random.default_rng(41)
+    B, L, D, d_g, l_h = 2, 57, 6, 3, 20
+    q, k, v = (rng.standard_normal((B, L, D)) for _ in range(3))
+    h = rng.standard_normal((D // d_g, l_h))
+    full = o.gated_fir(q, k, v, h, d_g)
+    rows = [(0, 0), (0, 5), (1, 19), (1, 20), (0, 56), (1, 56)]
+    got = o.gated_fir_rows(q, k, v, h, d_g, rows)
+    for i, (b, t) in enumerate(rows):
+        assert np.array_equal(got[i], full[b, t]), (b, t)
+    x = k[1, :, 4] * v[1, :, 4]
+    ref = np.convolve(x, h[4 // d_g])[:L]
+    assert np.allclose(got[3, 4], q[1, 20, 4] * ref[20], rtol=1e-12, atol=1e-12)
+
+
 def pin_impulse(o):
     """x = delta_0, q = 1: the output is the filter itself, then zeros."""
     L, l_h = 20, 7

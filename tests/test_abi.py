@@ -39,7 +39,8 @@ def test_status_strings_and_version(lib):
 def test_select_algo_for_the_workloads(lib):
     from gated_causal_fir_b200.workloads import WORKLOADS
     want = {"tiny": g.HYENA_ALGO_WINDOW, "se": g.HYENA_ALGO_WINDOW, "mr": g.HYENA_ALGO_TENSOR,
-            "mr_batched": g.HYENA_ALGO_TENSOR, "mr_1m": g.HYENA_ALGO_TENSOR}
+            "mr_batched": g.HYENA_ALGO_TENSOR, "mr_1m": g.HYENA_ALGO_TENSOR,
+            "li": g.HYENA_ALGO_DIRECT}  # long filters: the FFT entry point (workspace) is separate
     for name, wl in WORKLOADS.items():
         dt = g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16
         assert g.hyena_select_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, dt) == want[name]
@@ -158,6 +159,31 @@ def test_history_validation(lib):
     assert f(q, k, v, h, y, y + 64, vh, 8, *a) == 1                 # history overlaps y
     assert f(q, k, v, h, y, y - 1024, vh, 8, *a) == 1               # history runs into y
     assert f(q, k, v, h, y, kh, vh, 8, 0, 64, 128, 64, 16, 16, 0, 0, None) == 0  # empty: no launch
+
+
+def test_fft_workspace_bytes(lib):
+    f = lib.hyena_conv_fwd_fft_workspace_bytes
+    # L = l_h = 8192, D = 4096, d_g = 64: N = 16384; 4 B N D of data spectra + 2 x 8 N G
+    assert f(1, 8192, 4096, 64, 8192) == 4 * 16384 * 4096 + 2 * 8 * 16384 * 64
+    assert f(2, 8, 4, 2, 3) == 2 * 64 * 2 * 8 + 2 * 64 * 2 * 8   # N = 64, the smallest
+    assert f(1, 8192, 4096, 63, 8192) == -1                  # D % d_g
+    assert f(1, 8192, 4095, 4095, 10) == -2                  # odd D: channel pairs
+    assert f(1, 100, 96, 3, 10) == -2                        # odd d_g
+    assert f(1, 40000, 64, 64, 30000) == -2                  # L + l_h - 1 > 65536
+    assert f(0, 100, 64, 2, 10) == 0
+
+
+def test_fft_validation(lib):
+    f = lib.hyena_conv_fwd_fft
+    q, k, v, h, y = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+    a = (1, 64, 128, 64, 16, 16, 0)   # B, L, D, d_g, l_h, l_b, dtype
+    need = lib.hyena_conv_fwd_fft_workspace_bytes(1, 64, 128, 64, 16)
+    assert f(q, k, v, h, y, *a, None, need, None) == 1               # no workspace
+    assert f(q, k, v, h, y, *a, 0x600000, need - 1, None) == 1       # too small
+    assert f(q, k, v, h, y, *a, 0x600008, need, None) == 3           # misaligned
+    assert f(q, k, v, h, y, 1, 64, 128, 3, 16, 16, 0, 0x600000, need, None) == 1  # D % d_g
+    assert f(q, k, v, h, y, 1, 64, 126, 63, 16, 16, 0, 0x600000, need, None) == 2  # odd d_g
+    assert f(q, k, v, h, y, 0, 64, 128, 64, 16, 16, 0, None, 0, None) == 0  # empty: no launch
 
 
 def test_device_status_needs_out(lib):

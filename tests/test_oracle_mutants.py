@@ -35,6 +35,8 @@ MUTANTS = [
     ("bwd_dk_wrong_factor", "dk[e] = dx * v[e];", "dk[e] = dx * k[e];"),
     ("bwd_dq_wrong_factor", "dq[e] = dy[e] * z;", "dq[e] = q[e] * z;"),
     ("bwd_dh_no_lag", "s += (dy[e] * q[e]) * (k[src] * v[src]);", "s += (dy[e] * q[e]) * (k[e] * v[e]);"),
+    ("rows_reversed_taps", "acc += hg[tap] * (k[at] * v[at]);", "acc += hg[l_h - 1 - tap] * (k[at] * v[at]);"),
+    ("rows_drops_last_tap", "for (int64_t tap = 0; tap <= last; ++tap) {", "for (int64_t tap = 0; tap < last; ++tap) {"),
     ("bwd_dx_drops_tap0", "for (int64_t j = 0; j < l_h && t + j < L; ++j) {", "for (int64_t j = 1; j < l_h && t + j < L; ++j) {"),
 ]
 
