@@ -16,8 +16,9 @@
 // so its spectrum) is the same and both signals are real, so the inverse transform of
 // H (X_c + i X_{c+1}) is y_c + i y_{c+1} exactly -- no separation step.
 //
-// Every FFT runs in shared memory: P signals (channel pairs) side by side, radix-2 Stockham
-// stages (self-sorting: natural order in, natural order out), twiddles from sincospif.  The
+// Every FFT runs in shared memory: P signals (channel pairs) side by side, radix-4 (and one
+// radix-2) Stockham stages (self-sorting: natural order in, natural order out), twiddles from
+// sincospif tabled once per CTA.  The
 // intermediate spectra live in a caller-owned fp32 workspace laid out [b][k1][n2][pair], so
 // every pass reads and writes P contiguous complex values (128 bytes) per index.
 #pragma once
@@ -36,9 +37,10 @@ constexpr int kMaxLen = 256;    // N1, N2 <= 256: N <= 65536
 struct FftParams {
   long long B, L, D;
   int d_g, l_h;
-  int N1, N2, log1, log2;
+  int N1, N2;
   long long PT;      // signals per sequence: D / 2 (data) or G (spectrum)
   int G;
+  int vec;           // q, k, v, y 16-byte aligned and D a multiple of one 16-byte vector
 };
 
 __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
@@ -52,35 +54,94 @@ __device__ __forceinline__ float2 twiddle(long long num, long long den) {
   return make_float2(c, s);
 }
 
-// Radix-2 Stockham FFT of n = 2^logn points for kP signals laid out a[point * kP + signal];
-// b is scratch of the same size; tw[k] = W_n^k for k < n / 2.  Forward (W) or inverse (W^-1,
-// unscaled).  Returns the buffer holding the result.  All threads of the CTA take part.
+__device__ __forceinline__ float2 times_i(float2 a, bool neg) {  // +i a, or -i a when neg
+  return neg ? make_float2(a.y, -a.x) : make_float2(-a.y, a.x);
+}
+
+// Stockham FFT (self-sorting) of n = 2^k points for kP signals laid out a[point * kP + signal]:
+// radix-4 stages while four or more points per sub-transform remain, then one radix-2 stage
+// when log2 n is odd.  b is scratch of the same size; tw[k] = W_n^k for k < n.  Forward (W)
+// or inverse (W^-1, unscaled).  Returns the buffer holding the result.  All threads take part.
 template <bool kInverse>
-__device__ float2 *fft_smem(float2 *a, float2 *b, int n, int logn, const float2 *tw) {
-  const int half = n >> 1;
-  for (int s = 0; s < logn; ++s) {
-    const int ns = 1 << s;
-    for (int e = threadIdx.x; e < half * kP; e += blockDim.x) {
+__device__ float2 *fft_smem(float2 *a, float2 *b, int n, const float2 *tw) {
+  for (int ns = 1; ns < n;) {
+    const bool r4 = n / ns >= 4;
+    const int R = r4 ? 4 : 2;
+    const int m = n / R;
+    const int step = n / (R * ns);
+    for (int e = threadIdx.x; e < m * kP; e += blockDim.x) {
       const int j = e / kP, sig = e % kP;
       const int k = j & (ns - 1);
-      float2 w = tw[k << (logn - 1 - s)];  // W_{2 ns}^k
-      if (kInverse) w.y = -w.y;
-      const float2 u = a[j * kP + sig];
-      const float2 t = cmul(a[(j + half) * kP + sig], w);
-      const int d = ((j - k) << 1) + k;
-      b[d * kP + sig] = make_float2(u.x + t.x, u.y + t.y);
-      b[(d + ns) * kP + sig] = make_float2(u.x - t.x, u.y - t.y);
+      const int d = (j - k) * R + k;
+      if (r4) {
+        float2 w1 = tw[k * step], w2 = tw[2 * k * step], w3 = tw[3 * k * step];
+        if (kInverse) {
+          w1.y = -w1.y;
+          w2.y = -w2.y;
+          w3.y = -w3.y;
+        }
+        const float2 v0 = a[j * kP + sig];
+        const float2 v1 = cmul(a[(j + m) * kP + sig], w1);
+        const float2 v2 = cmul(a[(j + 2 * m) * kP + sig], w2);
+        const float2 v3 = cmul(a[(j + 3 * m) * kP + sig], w3);
+        const float2 a0 = make_float2(v0.x + v2.x, v0.y + v2.y);
+        const float2 a1 = make_float2(v0.x - v2.x, v0.y - v2.y);
+        const float2 b0 = make_float2(v1.x + v3.x, v1.y + v3.y);
+        const float2 b1 = times_i(make_float2(v1.x - v3.x, v1.y - v3.y), !kInverse);
+        b[d * kP + sig] = make_float2(a0.x + b0.x, a0.y + b0.y);
+        b[(d + ns) * kP + sig] = make_float2(a1.x + b1.x, a1.y + b1.y);
+        b[(d + 2 * ns) * kP + sig] = make_float2(a0.x - b0.x, a0.y - b0.y);
+        b[(d + 3 * ns) * kP + sig] = make_float2(a1.x - b1.x, a1.y - b1.y);
+      } else {
+        float2 w = tw[k * step];
+        if (kInverse) w.y = -w.y;
+        const float2 u = a[j * kP + sig];
+        const float2 t = cmul(a[(j + m) * kP + sig], w);
+        b[d * kP + sig] = make_float2(u.x + t.x, u.y + t.y);
+        b[(d + ns) * kP + sig] = make_float2(u.x - t.x, u.y - t.y);
+      }
     }
     __syncthreads();
     float2 *x = a;
     a = b;
     b = x;
+    ns *= R;
   }
   return a;
 }
 
-__device__ __forceinline__ void fill_twiddles(float2 *tw, int n) {
-  for (int k = threadIdx.x; k < (n >> 1); k += blockDim.x) tw[k] = twiddle(k, n);
+// tw[k] = W_n^k for k < n; with n2 >= 0 also tw2[k1] = W_N^{n2 k1} for k1 < n (the twiddles
+// between the two factors of the four-step transform, for this CTA's n2).
+__device__ __forceinline__ void fill_twiddles(float2 *tw, int n, float2 *tw2 = nullptr,
+                                              long long n2 = 0, long long N = 1) {
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    tw[k] = twiddle(k, n);
+    if (tw2) tw2[k] = twiddle((n2 * k) % N, N);
+  }
+}
+
+// 16-byte vectors of T: 8 / sizeof(T) channel pairs.
+template <typename T>
+struct PairVec {
+  static constexpr int VP = 8 / static_cast<int>(sizeof(T));
+  __device__ static void load(const T *p, float (&o)[2 * VP]);
+  __device__ static void store(T *p, const float (&o)[2 * VP]);
+};
+template <>
+__device__ inline void PairVec<__nv_bfloat16>::load(const __nv_bfloat16 *p, float (&o)[8]) {
+  cc::Vec<__nv_bfloat16>::unpack(cc::Vec<__nv_bfloat16>::load(p), o);
+}
+template <>
+__device__ inline void PairVec<__nv_bfloat16>::store(__nv_bfloat16 *p, const float (&o)[8]) {
+  cc::Vec<__nv_bfloat16>::store(p, o);
+}
+template <>
+__device__ inline void PairVec<float>::load(const float *p, float (&o)[4]) {
+  cc::Vec<float>::unpack(cc::Vec<float>::load(p), o);
+}
+template <>
+__device__ inline void PairVec<float>::store(float *p, const float (&o)[4]) {
+  cc::Vec<float>::store(p, o);
 }
 
 // Pass 1.  Block (n2, signal block, b).  Data mode: signal s of sequence b is
@@ -92,36 +153,53 @@ __global__ void __launch_bounds__(kThreads)
                      float2 *__restrict__ A, const FftParams p) {
   extern __shared__ float2 fsm[];
   const int n1len = p.N1;
-  float2 *b0 = fsm, *b1 = fsm + n1len * kP, *tw = fsm + 2 * n1len * kP;
+  float2 *b0 = fsm, *b1 = fsm + n1len * kP, *tw = fsm + 2 * n1len * kP, *tw2 = tw + n1len;
   const int n2 = blockIdx.x;
   const long long s0 = static_cast<long long>(blockIdx.y) * kP;
   const long long b = blockIdx.z;
   const long long N = static_cast<long long>(p.N1) * p.N2;
-  fill_twiddles(tw, n1len);
-  for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
-    const int n1 = e / kP, sig = e % kP;
-    const long long t = static_cast<long long>(p.N2) * n1 + n2;
-    const long long s = s0 + sig;
-    float2 z = make_float2(0.f, 0.f);
-    if (s < p.PT) {
-      if (kSpectrum) {
-        if (t < p.l_h) z.x = __ldg(h + s * p.l_h + t);
-      } else if (t < p.L) {
-        const long long off = (b * p.L + t) * p.D + 2 * s;
-        z.x = cc::to_f32(k[off]) * cc::to_f32(v[off]);
-        z.y = cc::to_f32(k[off + 1]) * cc::to_f32(v[off + 1]);
-      }
+  fill_twiddles(tw, n1len, tw2, n2, N);
+  if constexpr (kSpectrum) {
+    for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
+      const int n1 = e / kP, sig = e % kP;
+      const long long t = static_cast<long long>(p.N2) * n1 + n2;
+      const long long s = s0 + sig;
+      b0[e] = make_float2(s < p.PT && t < p.l_h ? __ldg(h + s * p.l_h + t) : 0.f, 0.f);
     }
-    b0[e] = z;
+  } else {
+    constexpr int VP = PairVec<T>::VP, NV = kP / VP;
+    for (int e = threadIdx.x; e < n1len * NV; e += blockDim.x) {
+      const int n1 = e / NV, cv = e % NV;
+      const long long t = static_cast<long long>(p.N2) * n1 + n2;
+      const long long s = s0 + cv * VP;
+      float kf[2 * VP], vf[2 * VP];
+#pragma unroll
+      for (int i = 0; i < 2 * VP; ++i) kf[i] = vf[i] = 0.f;
+      if (t < p.L && s < p.PT) {
+        const long long off = (b * p.L + t) * p.D + 2 * s;
+        if (p.vec && s + VP <= p.PT) {
+          PairVec<T>::load(k + off, kf);
+          PairVec<T>::load(v + off, vf);
+        } else {
+          for (int i = 0; i < VP && s + i < p.PT; ++i) {
+            kf[2 * i] = cc::to_f32(k[off + 2 * i]);
+            kf[2 * i + 1] = cc::to_f32(k[off + 2 * i + 1]);
+            vf[2 * i] = cc::to_f32(v[off + 2 * i]);
+            vf[2 * i + 1] = cc::to_f32(v[off + 2 * i + 1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < VP; ++i)
+        b0[n1 * kP + cv * VP + i] = make_float2(kf[2 * i] * vf[2 * i], kf[2 * i + 1] * vf[2 * i + 1]);
+    }
   }
   __syncthreads();
-  const float2 *r = fft_smem<false>(b0, b1, n1len, p.log1, tw);
+  const float2 *r = fft_smem<false>(b0, b1, n1len, tw);
   for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
     const int k1 = e / kP, sig = e % kP;
     const long long s = s0 + sig;
-    if (s < p.PT)
-      A[((b * p.N1 + k1) * p.N2 + n2) * p.PT + s] =
-          cmul(r[e], twiddle((static_cast<long long>(n2) * k1) % N, N));
+    if (s < p.PT) A[((b * p.N1 + k1) * p.N2 + n2) * p.PT + s] = cmul(r[e], tw2[k1]);
   }
 }
 
@@ -145,7 +223,7 @@ __global__ void __launch_bounds__(kThreads)
     b0[e] = s < p.PT ? row[n2 * p.PT + s] : make_float2(0.f, 0.f);
   }
   __syncthreads();
-  float2 *r = fft_smem<false>(b0, b1, n2len, p.log2, tw);
+  float2 *r = fft_smem<false>(b0, b1, n2len, tw);
   float2 *o = r == b0 ? b1 : b0;
   if constexpr (kSpectrum) {
     for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
@@ -161,7 +239,7 @@ __global__ void __launch_bounds__(kThreads)
       r[e] = cmul(r[e], H[(static_cast<long long>(k1) * p.N2 + k2) * p.G + g]);
     }
     __syncthreads();
-    const float2 *y = fft_smem<true>(r, o, n2len, p.log2, tw);
+    const float2 *y = fft_smem<true>(r, o, n2len, tw);
     for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
       const int n2 = e / kP, sig = e % kP;
       const long long s = s0 + sig;
@@ -178,34 +256,48 @@ __global__ void __launch_bounds__(kThreads)
                      const FftParams p) {
   extern __shared__ float2 fsm[];
   const int n1len = p.N1;
-  float2 *b0 = fsm, *b1 = fsm + n1len * kP, *tw = fsm + 2 * n1len * kP;
+  float2 *b0 = fsm, *b1 = fsm + n1len * kP, *tw = fsm + 2 * n1len * kP, *tw2 = tw + n1len;
   const int n2 = blockIdx.x;
   const long long s0 = static_cast<long long>(blockIdx.y) * kP;
   const long long b = blockIdx.z;
   const long long N = static_cast<long long>(p.N1) * p.N2;
-  fill_twiddles(tw, n1len);
+  fill_twiddles(tw, n1len, tw2, n2, N);
+  __syncthreads();
   for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
     const int k1 = e / kP, sig = e % kP;
     const long long s = s0 + sig;
     float2 z = make_float2(0.f, 0.f);
     if (s < p.PT) {
-      float2 w = twiddle((static_cast<long long>(n2) * k1) % N, N);
-      w.y = -w.y;
-      z = cmul(A[((b * p.N1 + k1) * p.N2 + n2) * p.PT + s], w);
+      const float2 w = tw2[k1];
+      z = cmul(A[((b * p.N1 + k1) * p.N2 + n2) * p.PT + s], make_float2(w.x, -w.y));
     }
     b0[e] = z;
   }
   __syncthreads();
-  const float2 *r = fft_smem<true>(b0, b1, n1len, p.log1, tw);
+  const float2 *r = fft_smem<true>(b0, b1, n1len, tw);
   const float inv = 1.0f / static_cast<float>(N);
-  for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
-    const int n1 = e / kP, sig = e % kP;
+  constexpr int VP = PairVec<T>::VP, NV = kP / VP;
+  for (int e = threadIdx.x; e < n1len * NV; e += blockDim.x) {
+    const int n1 = e / NV, cv = e % NV;
     const long long t = static_cast<long long>(p.N2) * n1 + n2;
-    const long long s = s0 + sig;
-    if (s < p.PT && t < p.L) {
-      const long long off = (b * p.L + t) * p.D + 2 * s;
-      cc::from_f32(cc::to_f32(q[off]) * (r[e].x * inv), y + off);
-      cc::from_f32(cc::to_f32(q[off + 1]) * (r[e].y * inv), y + off + 1);
+    const long long s = s0 + cv * VP;
+    if (t >= p.L || s >= p.PT) continue;
+    const long long off = (b * p.L + t) * p.D + 2 * s;
+    const float2 *rr = r + n1 * kP + cv * VP;
+    if (p.vec && s + VP <= p.PT) {
+      float qf[2 * VP], o[2 * VP];
+      PairVec<T>::load(q + off, qf);
+#pragma unroll
+      for (int i = 0; i < VP; ++i) {
+        o[2 * i] = qf[2 * i] * (rr[i].x * inv);
+        o[2 * i + 1] = qf[2 * i + 1] * (rr[i].y * inv);
+      }
+      PairVec<T>::store(y + off, o);
+    } else {
+      for (int i = 0; i < VP && s + i < p.PT; ++i) {
+        cc::from_f32(cc::to_f32(q[off + 2 * i]) * (rr[i].x * inv), y + off + 2 * i);
+        cc::from_f32(cc::to_f32(q[off + 2 * i + 1]) * (rr[i].y * inv), y + off + 2 * i + 1);
+      }
     }
   }
 }

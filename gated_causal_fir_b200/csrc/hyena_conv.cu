@@ -35,9 +35,10 @@ constexpr int kMaxDevices = 64;
 constexpr int kDhSmemMax =
     (2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (64 + 1) * static_cast<int>(sizeof(float));
 constexpr int kMaxWindowTaps = 16;
-// Shared memory of an FFT pass over n points: two buffers of n x kP complex and n / 2 twiddles.
+// Shared memory of an FFT pass over n points: two buffers of n x kP complex, n twiddles W_n^k
+// and n inter-factor twiddles.
 constexpr int fft_smem_bytes(int n) {
-  return (2 * n * hyena::fft::kP + n / 2) * static_cast<int>(sizeof(float2));
+  return (2 * n * hyena::fft::kP + 2 * n) * static_cast<int>(sizeof(float2));
 }
 constexpr int kFftSmemMax = fft_smem_bytes(hyena::fft::kMaxLen);
 #ifndef HYENA_WINDOW_ROWS
@@ -631,9 +632,10 @@ int launch_fft(const Problem &P, const FftPlan &f, uint8_t *ws, cudaStream_t s) 
   p.l_h = P.l_h;
   p.N1 = f.N1;
   p.N2 = f.N2;
-  p.log1 = f.log1;
-  p.log2 = f.log2;
   p.G = static_cast<int>(P.G());
+  const int vec_ch = 16 / static_cast<int>(P.elem());  // channels per 16-byte vector
+  p.vec = P.D % vec_ch == 0 && aligned(P.q, 16) && aligned(P.k, 16) && aligned(P.v, 16) &&
+          aligned(P.y, 16);
   // the filters' spectrum H[k1][k2][g]
   hf::FftParams ph = p;
   ph.PT = P.G();
