@@ -34,11 +34,12 @@ constexpr int kP = 16;          // signals (channel pairs) per CTA
 constexpr int kThreads = 256;
 constexpr int kMaxLen = 256;    // N1, N2 <= 256: N <= 65536
 
+// Sizes as 32-bit ints: the host checks that every per-sequence offset fits (L D and N PT below
+// 2^31); the batch offsets are formed once per CTA in 64 bits.
 struct FftParams {
-  long long B, L, D;
-  int d_g, l_h;
+  int L, D, d_g, l_h;
   int N1, N2;
-  long long PT;      // signals per sequence: D / 2 (data) or G (spectrum)
+  int PT;            // signals per sequence: D / 2 (data) or G (spectrum)
   int G;
   int vec;           // q, k, v, y 16-byte aligned and D a multiple of one 16-byte vector
 };
@@ -47,8 +48,8 @@ __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
   return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
 }
 
-// exp(-2 pi i num / den) (den a power of two, |num| < den), accurate to a few ulp.
-__device__ __forceinline__ float2 twiddle(long long num, long long den) {
+// exp(-2 pi i num / den) (den a power of two, 0 <= num < den), accurate to a few ulp.
+__device__ __forceinline__ float2 twiddle(int num, int den) {
   float s, c;
   sincospif(-2.0f * static_cast<float>(num) / static_cast<float>(den), &s, &c);
   return make_float2(c, s);
@@ -112,11 +113,11 @@ __device__ float2 *fft_smem(float2 *a, float2 *b, int n, const float2 *tw) {
 
 // tw[k] = W_n^k for k < n; with n2 >= 0 also tw2[k1] = W_N^{n2 k1} for k1 < n (the twiddles
 // between the two factors of the four-step transform, for this CTA's n2).
-__device__ __forceinline__ void fill_twiddles(float2 *tw, int n, float2 *tw2 = nullptr,
-                                              long long n2 = 0, long long N = 1) {
+__device__ __forceinline__ void fill_twiddles(float2 *tw, int n, float2 *tw2 = nullptr, int n2 = 0,
+                                              int N = 1) {
   for (int k = threadIdx.x; k < n; k += blockDim.x) {
     tw[k] = twiddle(k, n);
-    if (tw2) tw2[k] = twiddle((n2 * k) % N, N);
+    if (tw2) tw2[k] = twiddle((n2 * k) & (N - 1), N);
   }
 }
 
@@ -155,37 +156,36 @@ __global__ void __launch_bounds__(kThreads)
   const int n1len = p.N1;
   float2 *b0 = fsm, *b1 = fsm + n1len * kP, *tw = fsm + 2 * n1len * kP, *tw2 = tw + n1len;
   const int n2 = blockIdx.x;
-  const long long s0 = static_cast<long long>(blockIdx.y) * kP;
+  const int s0 = blockIdx.y * kP;
   const long long b = blockIdx.z;
-  const long long N = static_cast<long long>(p.N1) * p.N2;
+  const int N = p.N1 * p.N2;
   fill_twiddles(tw, n1len, tw2, n2, N);
   if constexpr (kSpectrum) {
     for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
       const int n1 = e / kP, sig = e % kP;
-      const long long t = static_cast<long long>(p.N2) * n1 + n2;
-      const long long s = s0 + sig;
+      const int t = p.N2 * n1 + n2, s = s0 + sig;
       b0[e] = make_float2(s < p.PT && t < p.l_h ? __ldg(h + s * p.l_h + t) : 0.f, 0.f);
     }
   } else {
     constexpr int VP = PairVec<T>::VP, NV = kP / VP;
+    const T *kb = k + b * p.L * p.D + 2 * s0, *vb = v + b * p.L * p.D + 2 * s0;
     for (int e = threadIdx.x; e < n1len * NV; e += blockDim.x) {
       const int n1 = e / NV, cv = e % NV;
-      const long long t = static_cast<long long>(p.N2) * n1 + n2;
-      const long long s = s0 + cv * VP;
+      const int t = p.N2 * n1 + n2, s = s0 + cv * VP;
       float kf[2 * VP], vf[2 * VP];
 #pragma unroll
       for (int i = 0; i < 2 * VP; ++i) kf[i] = vf[i] = 0.f;
       if (t < p.L && s < p.PT) {
-        const long long off = (b * p.L + t) * p.D + 2 * s;
+        const int off = t * p.D + 2 * cv * VP;
         if (p.vec && s + VP <= p.PT) {
-          PairVec<T>::load(k + off, kf);
-          PairVec<T>::load(v + off, vf);
+          PairVec<T>::load(kb + off, kf);
+          PairVec<T>::load(vb + off, vf);
         } else {
           for (int i = 0; i < VP && s + i < p.PT; ++i) {
-            kf[2 * i] = cc::to_f32(k[off + 2 * i]);
-            kf[2 * i + 1] = cc::to_f32(k[off + 2 * i + 1]);
-            vf[2 * i] = cc::to_f32(v[off + 2 * i]);
-            vf[2 * i + 1] = cc::to_f32(v[off + 2 * i + 1]);
+            kf[2 * i] = cc::to_f32(kb[off + 2 * i]);
+            kf[2 * i + 1] = cc::to_f32(kb[off + 2 * i + 1]);
+            vf[2 * i] = cc::to_f32(vb[off + 2 * i]);
+            vf[2 * i + 1] = cc::to_f32(vb[off + 2 * i + 1]);
           }
         }
       }
@@ -196,10 +196,12 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   const float2 *r = fft_smem<false>(b0, b1, n1len, tw);
+  // A[b][k1][n2][s]: this CTA's signals at k1 lie k1 N2 PT apart
+  float2 *ab = A + b * N * p.PT + n2 * p.PT + s0;
+  const int kstride = p.N2 * p.PT;
   for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
     const int k1 = e / kP, sig = e % kP;
-    const long long s = s0 + sig;
-    if (s < p.PT) A[((b * p.N1 + k1) * p.N2 + n2) * p.PT + s] = cmul(r[e], tw2[k1]);
+    if (s0 + sig < p.PT) ab[k1 * kstride + sig] = cmul(r[e], tw2[k1]);
   }
 }
 
@@ -213,37 +215,36 @@ __global__ void __launch_bounds__(kThreads)
   const int n2len = p.N2;
   float2 *b0 = fsm, *b1 = fsm + n2len * kP, *tw = fsm + 2 * n2len * kP;
   const int k1 = blockIdx.x;
-  const long long s0 = static_cast<long long>(blockIdx.y) * kP;
+  const int s0 = blockIdx.y * kP;
   const long long b = blockIdx.z;
   fill_twiddles(tw, n2len);
-  float2 *row = A + (b * p.N1 + k1) * p.N2 * p.PT;
+  // A[b][k1][n2][s0 + sig] at row[n2 PT + sig]
+  float2 *row = A + (b * p.N1 + k1) * p.N2 * p.PT + s0;
   for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
     const int n2 = e / kP, sig = e % kP;
-    const long long s = s0 + sig;
-    b0[e] = s < p.PT ? row[n2 * p.PT + s] : make_float2(0.f, 0.f);
+    b0[e] = s0 + sig < p.PT ? row[n2 * p.PT + sig] : make_float2(0.f, 0.f);
   }
   __syncthreads();
   float2 *r = fft_smem<false>(b0, b1, n2len, tw);
   float2 *o = r == b0 ? b1 : b0;
+  const float2 *hk = H + k1 * p.N2 * p.G;  // H[k1][k2][g] at hk[k2 G + g]
   if constexpr (kSpectrum) {
     for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
       const int k2 = e / kP, sig = e % kP;
-      const long long s = s0 + sig;
-      if (s < p.PT) H[(static_cast<long long>(k1) * p.N2 + k2) * p.G + s] = r[e];
+      if (s0 + sig < p.PT) H[k1 * p.N2 * p.G + k2 * p.G + s0 + sig] = r[e];
     }
   } else {
     for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
       const int k2 = e / kP, sig = e % kP;
-      const long long s = s0 + sig;
-      const long long g = s < p.PT ? (2 * s) / p.d_g : 0;
-      r[e] = cmul(r[e], H[(static_cast<long long>(k1) * p.N2 + k2) * p.G + g]);
+      const int s = s0 + sig;
+      const int g = s < p.PT ? (2 * s) / p.d_g : 0;
+      r[e] = cmul(r[e], hk[k2 * p.G + g]);
     }
     __syncthreads();
     const float2 *y = fft_smem<true>(r, o, n2len, tw);
     for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
       const int n2 = e / kP, sig = e % kP;
-      const long long s = s0 + sig;
-      if (s < p.PT) row[n2 * p.PT + s] = y[e];
+      if (s0 + sig < p.PT) row[n2 * p.PT + sig] = y[e];
     }
   }
 }
@@ -258,18 +259,19 @@ __global__ void __launch_bounds__(kThreads)
   const int n1len = p.N1;
   float2 *b0 = fsm, *b1 = fsm + n1len * kP, *tw = fsm + 2 * n1len * kP, *tw2 = tw + n1len;
   const int n2 = blockIdx.x;
-  const long long s0 = static_cast<long long>(blockIdx.y) * kP;
+  const int s0 = blockIdx.y * kP;
   const long long b = blockIdx.z;
-  const long long N = static_cast<long long>(p.N1) * p.N2;
+  const int N = p.N1 * p.N2;
   fill_twiddles(tw, n1len, tw2, n2, N);
   __syncthreads();
+  const float2 *ab = A + b * N * p.PT + n2 * p.PT + s0;
+  const int kstride = p.N2 * p.PT;
   for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
     const int k1 = e / kP, sig = e % kP;
-    const long long s = s0 + sig;
     float2 z = make_float2(0.f, 0.f);
-    if (s < p.PT) {
+    if (s0 + sig < p.PT) {
       const float2 w = tw2[k1];
-      z = cmul(A[((b * p.N1 + k1) * p.N2 + n2) * p.PT + s], make_float2(w.x, -w.y));
+      z = cmul(ab[k1 * kstride + sig], make_float2(w.x, -w.y));
     }
     b0[e] = z;
   }
@@ -277,26 +279,27 @@ __global__ void __launch_bounds__(kThreads)
   const float2 *r = fft_smem<true>(b0, b1, n1len, tw);
   const float inv = 1.0f / static_cast<float>(N);
   constexpr int VP = PairVec<T>::VP, NV = kP / VP;
+  const T *qb = q + b * p.L * p.D + 2 * s0;
+  T *yb = y + b * p.L * p.D + 2 * s0;
   for (int e = threadIdx.x; e < n1len * NV; e += blockDim.x) {
     const int n1 = e / NV, cv = e % NV;
-    const long long t = static_cast<long long>(p.N2) * n1 + n2;
-    const long long s = s0 + cv * VP;
+    const int t = p.N2 * n1 + n2, s = s0 + cv * VP;
     if (t >= p.L || s >= p.PT) continue;
-    const long long off = (b * p.L + t) * p.D + 2 * s;
+    const int off = t * p.D + 2 * cv * VP;
     const float2 *rr = r + n1 * kP + cv * VP;
     if (p.vec && s + VP <= p.PT) {
       float qf[2 * VP], o[2 * VP];
-      PairVec<T>::load(q + off, qf);
+      PairVec<T>::load(qb + off, qf);
 #pragma unroll
       for (int i = 0; i < VP; ++i) {
         o[2 * i] = qf[2 * i] * (rr[i].x * inv);
         o[2 * i + 1] = qf[2 * i + 1] * (rr[i].y * inv);
       }
-      PairVec<T>::store(y + off, o);
+      PairVec<T>::store(yb + off, o);
     } else {
       for (int i = 0; i < VP && s + i < p.PT; ++i) {
-        cc::from_f32(cc::to_f32(q[off + 2 * i]) * (rr[i].x * inv), y + off + 2 * i);
-        cc::from_f32(cc::to_f32(q[off + 2 * i + 1]) * (rr[i].y * inv), y + off + 2 * i + 1);
+        cc::from_f32(cc::to_f32(qb[off + 2 * i]) * (rr[i].x * inv), yb + off + 2 * i);
+        cc::from_f32(cc::to_f32(qb[off + 2 * i + 1]) * (rr[i].y * inv), yb + off + 2 * i + 1);
       }
     }
   }

@@ -611,8 +611,10 @@ FftLayout fft_layout(int64_t B, int64_t D, int64_t G, int64_t N) {
 int fft_supported(const Problem &P, FftPlan &f) {
   if (P.D % 2 != 0 || P.d_g % 2 != 0) return HYENA_ERR_UNSUPPORTED;
   f = fft_plan(P.L, P.l_h);
+  const int64_t i32 = std::numeric_limits<int32_t>::max();
   if (!f.ok || P.B > 65535 || (P.D / 2 + hyena::fft::kP - 1) / hyena::fft::kP > 65535 ||
-      (P.G() + hyena::fft::kP - 1) / hyena::fft::kP > 65535)
+      (P.G() + hyena::fft::kP - 1) / hyena::fft::kP > 65535 || P.L * P.D > i32 ||
+      f.N * (P.D / 2) > i32 || f.N * P.G() > i32 || P.G() * static_cast<int64_t>(P.l_h) > i32)
     return HYENA_ERR_UNSUPPORTED;
   return HYENA_OK;
 }
@@ -625,9 +627,8 @@ int launch_fft(const Problem &P, const FftPlan &f, uint8_t *ws, cudaStream_t s) 
   float2 *Hs = reinterpret_cast<float2 *>(ws + lay.off_hspec);
   float2 *Hh = reinterpret_cast<float2 *>(ws + lay.off_h);
   hf::FftParams p;
-  p.B = P.B;
-  p.L = P.L;
-  p.D = P.D;
+  p.L = static_cast<int>(P.L);
+  p.D = static_cast<int>(P.D);
   p.d_g = P.d_g;
   p.l_h = P.l_h;
   p.N1 = f.N1;
@@ -638,15 +639,14 @@ int launch_fft(const Problem &P, const FftPlan &f, uint8_t *ws, cudaStream_t s) 
           aligned(P.y, 16);
   // the filters' spectrum H[k1][k2][g]
   hf::FftParams ph = p;
-  ph.PT = P.G();
-  ph.B = 1;
+  ph.PT = static_cast<int>(P.G());
   const unsigned gb = static_cast<unsigned>((ph.PT + hf::kP - 1) / hf::kP);
   hf::fft_pass1_kernel<float, true><<<dim3(f.N2, gb, 1), hf::kThreads, fft_smem_bytes(f.N1), s>>>(
       nullptr, nullptr, P.h, Hh, ph);
   hf::fft_pass2_kernel<true><<<dim3(f.N1, gb, 1), hf::kThreads, fft_smem_bytes(f.N2), s>>>(
       Hh, Hs, ph);
   // the data: pass 1, pass 2 (times H, inverse), pass 3 (inverse, q gate)
-  p.PT = P.D / 2;
+  p.PT = static_cast<int>(P.D / 2);
   const unsigned db = static_cast<unsigned>((p.PT + hf::kP - 1) / hf::kP);
   const unsigned nb = static_cast<unsigned>(P.B);
   hf::fft_pass1_kernel<T, false><<<dim3(f.N2, db, nb), hf::kThreads, fft_smem_bytes(f.N1), s>>>(
