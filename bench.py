@@ -15,8 +15,10 @@ Rank 0 prints one JSON line.  Besides the throughput it reports the roofline of 
 (algorithmic bytes / mean launch time vs the measured HBM copy bandwidth), SM clocks sampled
 through NVML during the timed region, an end-to-end figure through
 ``hyena_conv_fwd_from_host`` (pinned host buffers, copies inside the timed region) and the
-fp64 oracle timed on the host cores as a CPU baseline.  ``--impl reference`` times only the
-oracle, one l_b-row chunk of the workload per step.
+fp64 oracle timed on the host cores as a CPU baseline.  Beside the forward it reports the
+backward (``backward``) and two longer-filter cases (``long_filters``: the Hyena-LI-shaped
+workload through the FFT entry point, and l_h = 513 on the tensor-core path).
+``--impl reference`` times only the oracle, one l_b-row chunk of the workload per step.
 """
 import argparse
 import ctypes
@@ -51,6 +53,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--bwd-steps", type=int, default=200,
                    help="timed steps of the backward (hyena_conv_bwd); 0 skips it")
+    p.add_argument("--long-steps", type=int, default=20,
+                   help="timed steps of the long-filter measurements (FFT, l_h = 513); 0 skips")
     return p.parse_args()
 
 
@@ -197,6 +201,68 @@ def run_reference(args, wl, rank, world):
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
     del torch
+
+
+def time_long_filters(args, stream, dev, D, g, _native, peak, peak_kind):
+    """Filters longer than the MR workload's, on one GPU, timed like the forward (CUDA events on
+    the launching stream over back-to-back calls, two rotating input sets):
+
+    * ``li_fft``: the Hyena-LI-shaped workload (B=1, L=8192, D=4096, d_g=64, l_h=8192) through
+      hyena_conv_fwd_fft (four-step FFT, caller workspace);
+    * ``mr_lh513``: the MR shape with l_h = 513, the longest filter of the tensor-core path
+      (hyena_conv_fwd, AUTO).
+
+    Algorithmic bytes per call: q, k, v read and y written (4 B L D bf16 elements); the FFT's
+    spectra in the workspace are overhead, not counted."""
+    import torch
+    from gated_causal_fir_b200.workloads import WORKLOADS, custom, make_inputs
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    out = {}
+    for name, wl, fft in (("li_fft", WORKLOADS["li"], True),
+                          ("mr_lh513", custom("mr_lh513", 1, 8192, 4096, 64, 513, 64, "bf16",
+                                              "mr", seed=6), False)):
+        sets = [make_inputs(wl, device=dev, seed=wl.seed + 101 * s) for s in range(2)]
+        ys = [torch.empty_like(x[0]) for x in sets]
+        if fft:
+            need = g.hyena_conv_fwd_fft_workspace_bytes(wl.B, wl.L, wl.D, wl.d_g, wl.l_h)
+            ws = torch.empty(need, dtype=torch.uint8, device=dev)
+            cfn = _native.lib().hyena_conv_fwd_fft
+            cargs = [(x[0].data_ptr(), x[1].data_ptr(), x[2].data_ptr(), x[3].data_ptr(),
+                      y.data_ptr(), wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, 0, ws.data_ptr(),
+                      need, sh) for x, y in zip(sets, ys)]
+            kernels = ["fft_pass1_kernel (filters)", "fft_pass2_kernel (filters)",
+                       "fft_pass1_kernel", "fft_pass2_kernel", "fft_pass3_kernel"]
+        else:
+            cfn = _native.lib().hyena_conv_fwd
+            cargs = [(x[0].data_ptr(), x[1].data_ptr(), x[2].data_ptr(), x[3].data_ptr(),
+                      y.data_ptr(), wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, sh)
+                     for x, y in zip(sets, ys)]
+            kernels = ["fir_tc_kernel"]
+        for i in range(max(3, args.warmup)):
+            if cfn(*cargs[i % 2]) != 0:
+                raise _native.HyenaError(name, cfn(*cargs[i % 2]))
+        torch.cuda.synchronize()
+        K = args.long_steps
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        D.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(K):
+            cfn(*cargs[i % 2])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = D.max_over_ranks(e0.elapsed_time(e1), device=dev) / K
+        nbytes = 4 * wl.B * wl.L * wl.D * 2
+        achieved = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"workload": wl.describe(), "ms_per_step": ms, "steps": K,
+                     "value": D.env_world()[2] * wl.tokens / (ms / 1e3), "unit": UNIT,
+                     "gpu_launches": len(kernels) * K, "kernels": kernels,
+                     "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
+                                  "unit": "GB/s", "frac": achieved / peak,
+                                  "algorithmic_bytes_per_step": nbytes,
+                                  "peak_source": peak_kind}}
+        del sets, ys
+    return out
 
 
 def time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind):
@@ -369,6 +435,11 @@ def main():
         peak, peak_kind = measured_peak_hbm()
         bwd = time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind)
 
+    long_filters = None
+    if args.long_steps > 0 and wl.name == "mr":
+        peak, peak_kind = measured_peak_hbm()
+        long_filters = time_long_filters(args, stream, dev, D, g, _native, peak, peak_kind)
+
     cpu, parity = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu, y_ref = cpu_baseline(wl, *sets[0][:4], target_s=args.cpu_seconds)
@@ -404,7 +475,7 @@ def main():
                          "mean_launch_us": 1e3 * mean_launch_ms, "kernel": kernel},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K,
             "clocks": clocks.summary(t_wall0, t_wall1),
-            "backward": bwd, "kernel_algo": g.ALGO_NAMES[algo], "device_status": status, "parity": parity,
+            "backward": bwd, "long_filters": long_filters, "kernel_algo": g.ALGO_NAMES[algo], "device_status": status, "parity": parity,
             "wall_s_timed_region": t_wall1 - t_wall0,
         }
         print(json.dumps(line), flush=True)
