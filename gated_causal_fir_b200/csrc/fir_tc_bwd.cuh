@@ -30,8 +30,8 @@
 //    segment.
 //  * Tensor memory (512 columns): two dx accumulators [0, 128) (the MMA issuer fills one while
 //    the epilogue drains the other), band [128, 256), C [256, 512).
-//  * Warp roles as the forward: 0 TMA k/v, 10 TMA q/dy (both fetch their tiles into L2 a few
-//    items ahead, then into shared memory), 1 MMA issuer + TMEM owner, 2-5 operand build
+//  * Warp roles as the forward: 0 TMA k/v, 10 TMA q/dy (fetching into L2 ahead of the loads
+//    as well measured slower: prefetched tiles were evicted before use), 1 MMA issuer + TMEM owner, 2-5 operand build
 //    (x = k v; dz = q dy written over the q tile; the band), 6-9 epilogue.  The epilogue copies
 //    its k, v rows from the stage into registers, releases it, and stores dk, dv rows directly;
 //    it also sums the dh anti-diagonals.  Every wait is bounded; a timeout raises
@@ -56,7 +56,6 @@ constexpr int kNKV = 3;   // k/v stages (32 KB each)
 constexpr int kNQ = 3;    // q stages; each becomes the tile's fp16 dz (channel-major, reversed)
 constexpr int kNDY = 2;   // dy stages (free once dz is built)
 constexpr int kNX = 2;    // fp16 x tiles, channel-major (free once the tile's dh product ran)
-constexpr int kPrefetch = 3;  // items a producer fetches into L2 ahead of its loads
 
 constexpr uint32_t kColDX = 0, kColBand = 128, kColC = 256;
 constexpr int kTmemCols = 512;
@@ -383,9 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  // Nothing above touches global memory: under a programmatic dependent launch it overlaps the
-  // previous kernel (the dq forward).  From here on the inputs may be read.
-  griddep_wait();
+  // Launched with programmatic stream serialisation after the dq forward, which only starts
+  // its dependents once it has itself waited for every earlier kernel of the stream: the
+  // inputs are complete when this grid starts, and nothing here reads what the forward writes
+  // (dq), so the work overlaps the forward's last tiles without a grid-dependency wait.
   griddep_launch_dependents();
   // The gate threads issue the loads of the first segment's filter taps before the barrier.
   bool over = false;
@@ -405,22 +405,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      BwdWalk it(w_begin, w_end, p.nT, p.B), pf(w_begin, w_end, p.nT, p.B);
-      BItem t, u;
-      // L2 prefetch runs kPrefetch loads ahead: the loads then find their tiles in L2.
-      auto prefetch_next = [&]() {
-        while (pf.next(u)) {
-          if (u.kind != kMain) continue;
-          tma_prefetch_l2_3d(&tm_k, u.g * kNC, u.i * kTM, u.b);
-          tma_prefetch_l2_3d(&tm_v, u.g * kNC, u.i * kTM, u.b);
-          return;
-        }
-      };
-      for (int n = 0; n < kPrefetch; ++n) prefetch_next();
+      BwdWalk it(w_begin, w_end, p.nT, p.B);
+      BItem t;
       uint32_t kc = 0;
       while (it.next(t)) {
         if (t.kind != kMain) continue;
-        prefetch_next();
         const int ks = kc % kNKV;
         if (!tc::thread_wait(&bars[kBarKVEmpty + ks], ((kc / kNKV) & 1) ^ 1, abort)) break;
         mbar_arrive_expect_tx(&bars[kBarKVFull + ks], 2 * kTileBytes);
@@ -437,18 +426,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_dy);
-      BwdWalk it(w_begin, w_end, p.nT, p.B), pf(w_begin, w_end, p.nT, p.B);
-      BItem t, u;
-      auto prefetch_next = [&]() {
-        if (pf.next(u)) {
-          tma_prefetch_l2_3d(&tm_q, u.g * kNC, u.i * kTM, u.b);
-          tma_prefetch_l2_3d(&tm_dy, u.g * kNC, u.i * kTM, u.b);
-        }
-      };
-      for (int n = 0; n < kPrefetch; ++n) prefetch_next();
+      BwdWalk it(w_begin, w_end, p.nT, p.B);
+      BItem t;
       uint32_t qc = 0, dc = 0;
       while (it.next(t)) {
-        prefetch_next();
         const int qs = qc % kNQ, ds = dc % kNDY;
         if (!tc::thread_wait(&bars[kBarQEmpty + qs], ((qc / kNQ) & 1) ^ 1, abort)) break;
         mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes);
