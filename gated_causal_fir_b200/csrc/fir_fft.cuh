@@ -16,11 +16,13 @@
 // so its spectrum) is the same and both signals are real, so the inverse transform of
 // H (X_c + i X_{c+1}) is y_c + i y_{c+1} exactly -- no separation step.
 //
-// Every FFT runs in shared memory: P signals (channel pairs) side by side, radix-4 (and one
-// radix-2) Stockham stages (self-sorting: natural order in, natural order out), twiddles from
-// sincospif tabled once per CTA.  The
-// intermediate spectra live in a caller-owned fp32 workspace laid out [b][k1][n2][pair], so
-// every pass reads and writes P contiguous complex values (128 bytes) per index.
+// Each length-n transform (n = R1 R2, both at most 16) runs as two in-register DFTs joined by one
+// exchange through shared memory: a thread holds R1 points of one signal (stride R2), transforms
+// them, applies W_n^{j k1} and stores them; then a thread holds R2 points (one k1) and
+// transforms those.  16 signals (channel pairs) per CTA, 16 threads per signal.  Twiddles come
+// from sincospif, tabled once per CTA.  The intermediate spectra live in a caller-owned fp32
+// workspace laid out [b][k1][n2][pair]: every pass moves 16 contiguous complex values (128
+// bytes) per index.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -31,8 +33,8 @@ namespace hyena {
 namespace fft {
 
 constexpr int kP = 16;          // signals (channel pairs) per CTA
-constexpr int kThreads = 256;
-constexpr int kMaxLen = 256;    // N1, N2 <= 256: N <= 65536
+constexpr int kThreads = 256;   // 16 threads per signal
+constexpr int kMinLen = 16, kMaxLen = 256;  // N1, N2 in [16, 256]: N in [256, 65536]
 
 // Sizes as 32-bit ints: the host checks that every per-sequence offset fits (L D and N PT below
 // 2^31); the batch offsets are formed once per CTA in 64 bits.
@@ -47,6 +49,7 @@ struct FftParams {
 __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
   return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
 }
+__device__ __forceinline__ float2 cconj(float2 a) { return make_float2(a.x, -a.y); }
 
 // exp(-2 pi i num / den) (den a power of two, 0 <= num < den), accurate to a few ulp.
 __device__ __forceinline__ float2 twiddle(int num, int den) {
@@ -55,64 +58,127 @@ __device__ __forceinline__ float2 twiddle(int num, int den) {
   return make_float2(c, s);
 }
 
-__device__ __forceinline__ float2 times_i(float2 a, bool neg) {  // +i a, or -i a when neg
-  return neg ? make_float2(a.y, -a.x) : make_float2(-a.y, a.x);
-}
-
-// Stockham FFT (self-sorting) of n = 2^k points for kP signals laid out a[point * kP + signal]:
-// radix-4 stages while four or more points per sub-transform remain, then one radix-2 stage
-// when log2 n is odd.  b is scratch of the same size; tw[k] = W_n^k for k < n.  Forward (W)
-// or inverse (W^-1, unscaled).  Returns the buffer holding the result.  All threads take part.
-template <bool kInverse>
-__device__ float2 *fft_smem(float2 *a, float2 *b, int n, const float2 *tw) {
-  for (int ns = 1; ns < n;) {
-    const bool r4 = n / ns >= 4;
-    const int R = r4 ? 4 : 2;
-    const int m = n / R;
-    const int step = n / (R * ns);
-    for (int e = threadIdx.x; e < m * kP; e += blockDim.x) {
-      const int j = e / kP, sig = e % kP;
-      const int k = j & (ns - 1);
-      const int d = (j - k) * R + k;
-      if (r4) {
-        float2 w1 = tw[k * step], w2 = tw[2 * k * step], w3 = tw[3 * k * step];
-        if (kInverse) {
-          w1.y = -w1.y;
-          w2.y = -w2.y;
-          w3.y = -w3.y;
-        }
-        const float2 v0 = a[j * kP + sig];
-        const float2 v1 = cmul(a[(j + m) * kP + sig], w1);
-        const float2 v2 = cmul(a[(j + 2 * m) * kP + sig], w2);
-        const float2 v3 = cmul(a[(j + 3 * m) * kP + sig], w3);
-        const float2 a0 = make_float2(v0.x + v2.x, v0.y + v2.y);
-        const float2 a1 = make_float2(v0.x - v2.x, v0.y - v2.y);
-        const float2 b0 = make_float2(v1.x + v3.x, v1.y + v3.y);
-        const float2 b1 = times_i(make_float2(v1.x - v3.x, v1.y - v3.y), !kInverse);
-        b[d * kP + sig] = make_float2(a0.x + b0.x, a0.y + b0.y);
-        b[(d + ns) * kP + sig] = make_float2(a1.x + b1.x, a1.y + b1.y);
-        b[(d + 2 * ns) * kP + sig] = make_float2(a0.x - b0.x, a0.y - b0.y);
-        b[(d + 3 * ns) * kP + sig] = make_float2(a1.x - b1.x, a1.y - b1.y);
-      } else {
-        float2 w = tw[k * step];
-        if (kInverse) w.y = -w.y;
-        const float2 u = a[j * kP + sig];
-        const float2 t = cmul(a[(j + m) * kP + sig], w);
-        b[d * kP + sig] = make_float2(u.x + t.x, u.y + t.y);
-        b[(d + ns) * kP + sig] = make_float2(u.x - t.x, u.y - t.y);
-      }
-    }
-    __syncthreads();
-    float2 *x = a;
-    a = b;
-    b = x;
-    ns *= R;
+// d * W_16^w (or its conjugate) for a compile-time w < 8; W_16^w = cos(pi w / 8) - i sin(pi w / 8).
+template <int w, bool kInv>
+__device__ __forceinline__ float2 w16mul(float2 d) {
+  constexpr float c8 = 0.92387953251128674f, s8 = 0.38268343236508978f, r2 = 0.70710678118654752f;
+  constexpr float cs[8] = {1.f, c8, r2, s8, 0.f, -s8, -r2, -c8};
+  constexpr float sn[8] = {0.f, s8, r2, c8, 1.f, c8, r2, s8};  // sin(pi w / 8) >= 0
+  if constexpr (w == 0) {
+    return d;
+  } else if constexpr (w == 4) {  // -i (forward) or +i (inverse)
+    return kInv ? make_float2(-d.y, d.x) : make_float2(d.y, -d.x);
+  } else {
+    const float c = cs[w], s = kInv ? sn[w] : -sn[w];
+    return make_float2(d.x * c - d.y * s, d.x * s + d.y * c);
   }
-  return a;
 }
 
-// tw[k] = W_n^k for k < n; with n2 >= 0 also tw2[k1] = W_N^{n2 k1} for k1 < n (the twiddles
-// between the two factors of the four-step transform, for this CTA's n2).
+__host__ __device__ constexpr int brev(int i, int bits) {
+  int r = 0;
+  for (int b = 0; b < bits; ++b) r |= ((i >> b) & 1) << (bits - 1 - b);
+  return r;
+}
+__host__ __device__ constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n / 2); }
+
+// t[bit-reverse(i)] = v[i] for every i, with compile-time indices.
+template <int R, int i = 0>
+__device__ __forceinline__ void brev_copy(float2 (&t)[R], const float2 (&v)[R]) {
+  if constexpr (i < R) {
+    t[brev(i, ilog2(R))] = v[i];
+    brev_copy<R, i + 1>(t, v);
+  }
+}
+
+// One radix-2 decimation-in-frequency stage of span h over R registers.
+template <int R, int h, bool kInv, int i = 0, int j = 0>
+__device__ __forceinline__ void dif_stage(float2 (&v)[R]) {
+  if constexpr (i < R) {
+    if constexpr (j < h) {
+      const float2 a = v[i + j], b = v[i + j + h];
+      v[i + j] = make_float2(a.x + b.x, a.y + b.y);
+      v[i + j + h] = w16mul<j * (16 / (2 * h)), kInv>(make_float2(a.x - b.x, a.y - b.y));
+      dif_stage<R, h, kInv, i, j + 1>(v);
+    } else {
+      dif_stage<R, h, kInv, i + 2 * h, 0>(v);
+    }
+  }
+}
+
+template <int R, int h, bool kInv>
+__device__ __forceinline__ void dif_all(float2 (&v)[R]) {
+  if constexpr (h >= 1) {
+    dif_stage<R, h, kInv>(v);
+    dif_all<R, h / 2, kInv>(v);
+  }
+}
+
+// In-register DFT of R (2..16) points, natural order in and out, forward or inverse (unscaled).
+template <int R, bool kInv>
+__device__ __forceinline__ void dft_reg(float2 (&v)[R]) {
+  dif_all<R, R / 2, kInv>(v);
+  float2 t[R];
+  brev_copy<R>(t, v);
+#pragma unroll
+  for (int i = 0; i < R; ++i) v[i] = t[i];
+}
+
+// The split n = R1 R2 of a transform length (R1, R2 <= 16).
+template <int n> struct Split;
+template <> struct Split<16> { static constexpr int R1 = 4, R2 = 4; };
+template <> struct Split<32> { static constexpr int R1 = 4, R2 = 8; };
+template <> struct Split<64> { static constexpr int R1 = 8, R2 = 8; };
+template <> struct Split<128> { static constexpr int R1 = 8, R2 = 16; };
+template <> struct Split<256> { static constexpr int R1 = 16, R2 = 16; };
+
+// Length-n transforms of 16 signals by the CTA.  Layouts (per signal; sig = thread % 16,
+// idx = thread / 16):
+//   "A" layout: thread idx = j < R2 holds x[j + R2 m], m < R1   (natural time order)
+//   "B" layout: thread idx = k1 < R1 holds X[k1 + R1 k2], k2 < R2 (natural frequency order)
+// ex is n x 16 complex of shared memory, tw[k] = W_n^k.  Both functions end with the result
+// in registers; they synchronise the CTA around their use of ex.
+template <int n, bool kInv>
+__device__ __forceinline__ void a_to_b(float2 (&va)[Split<n>::R1], float2 (&vb)[Split<n>::R2],
+                                       float2 *ex, const float2 *tw, int idx, int sig) {
+  constexpr int R1 = Split<n>::R1, R2 = Split<n>::R2;
+  __syncthreads();  // ex is free
+  if (idx < R2) {
+    dft_reg<R1, kInv>(va);
+#pragma unroll
+    for (int k1 = 0; k1 < R1; ++k1) {
+      const float2 w = tw[(idx * k1) & (n - 1)];
+      ex[(k1 * R2 + idx) * kP + sig] = cmul(va[k1], kInv ? cconj(w) : w);
+    }
+  }
+  __syncthreads();
+  if (idx < R1) {
+#pragma unroll
+    for (int j = 0; j < R2; ++j) vb[j] = ex[(idx * R2 + j) * kP + sig];
+    dft_reg<R2, kInv>(vb);
+  }
+}
+
+template <int n, bool kInv>
+__device__ __forceinline__ void b_to_a(float2 (&vb)[Split<n>::R2], float2 (&va)[Split<n>::R1],
+                                       float2 *ex, const float2 *tw, int idx, int sig) {
+  constexpr int R1 = Split<n>::R1, R2 = Split<n>::R2;
+  __syncthreads();
+  if (idx < R1) {
+    dft_reg<R2, kInv>(vb);
+#pragma unroll
+    for (int j = 0; j < R2; ++j) {
+      const float2 w = tw[(idx * j) & (n - 1)];
+      ex[(idx * R2 + j) * kP + sig] = cmul(vb[j], kInv ? cconj(w) : w);
+    }
+  }
+  __syncthreads();
+  if (idx < R2) {
+#pragma unroll
+    for (int k1 = 0; k1 < R1; ++k1) va[k1] = ex[(k1 * R2 + idx) * kP + sig];
+    dft_reg<R1, kInv>(va);
+  }
+}
+
 __device__ __forceinline__ void fill_twiddles(float2 *tw, int n, float2 *tw2 = nullptr, int n2 = 0,
                                               int N = 1) {
   for (int k = threadIdx.x; k < n; k += blockDim.x) {
@@ -145,31 +211,32 @@ __device__ inline void PairVec<float>::store(float *p, const float (&o)[4]) {
   cc::Vec<float>::store(p, o);
 }
 
-// Pass 1.  Block (n2, signal block, b).  Data mode: signal s of sequence b is
-// k v at channels 2s, 2s+1 (real, imaginary); spectrum mode: signal s is filter s (real).
-// Writes A[b][k1][n2][s] = W_N^{n2 k1} * sum_{n1} z[N2 n1 + n2] W_N1^{n1 k1}.
-template <typename T, bool kSpectrum>
+// Pass 1.  Block (n2, signal block, b): signal s of sequence b is k v at channels 2s, 2s+1
+// (real, imaginary) -- or, in spectrum mode, filter s (real).  Writes
+// A[b][k][n2][s] = W_N^{n2 k} * sum_{n1} z[N2 n1 + n2] W_N1^{n1 k}, k < N1.
+template <typename T, bool kSpectrum, int N1>
 __global__ void __launch_bounds__(kThreads)
     fft_pass1_kernel(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ h,
                      float2 *__restrict__ A, const FftParams p) {
-  extern __shared__ float2 fsm[];
-  const int n1len = p.N1;
-  float2 *b0 = fsm, *b1 = fsm + n1len * kP, *tw = fsm + 2 * n1len * kP, *tw2 = tw + n1len;
-  const int n2 = blockIdx.x;
-  const int s0 = blockIdx.y * kP;
+  constexpr int R1 = Split<N1>::R1, R2 = Split<N1>::R2;
+  __shared__ float2 ex[N1 * kP];
+  __shared__ float2 tw[N1], tw2[N1];
+  const int n2 = blockIdx.x, s0 = blockIdx.y * kP;
   const long long b = blockIdx.z;
-  const int N = p.N1 * p.N2;
-  fill_twiddles(tw, n1len, tw2, n2, N);
+  const int N = N1 * p.N2;
+  const int idx = threadIdx.x / kP, sig = threadIdx.x % kP;
+  fill_twiddles(tw, N1, tw2, n2, N);
+  // stage the rows t = N2 n1 + n2 of the CTA's 16 signals: ex[n1 * 16 + signal]
   if constexpr (kSpectrum) {
-    for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
-      const int n1 = e / kP, sig = e % kP;
-      const int t = p.N2 * n1 + n2, s = s0 + sig;
-      b0[e] = make_float2(s < p.PT && t < p.l_h ? __ldg(h + s * p.l_h + t) : 0.f, 0.f);
+    for (int e = threadIdx.x; e < N1 * kP; e += blockDim.x) {
+      const int n1 = e / kP, sg = e % kP;
+      const int t = p.N2 * n1 + n2, s = s0 + sg;
+      ex[e] = make_float2(s < p.PT && t < p.l_h ? __ldg(h + s * p.l_h + t) : 0.f, 0.f);
     }
   } else {
     constexpr int VP = PairVec<T>::VP, NV = kP / VP;
     const T *kb = k + b * p.L * p.D + 2 * s0, *vb = v + b * p.L * p.D + 2 * s0;
-    for (int e = threadIdx.x; e < n1len * NV; e += blockDim.x) {
+    for (int e = threadIdx.x; e < N1 * NV; e += blockDim.x) {
       const int n1 = e / NV, cv = e % NV;
       const int t = p.N2 * n1 + n2, s = s0 + cv * VP;
       float kf[2 * VP], vf[2 * VP];
@@ -191,102 +258,114 @@ __global__ void __launch_bounds__(kThreads)
       }
 #pragma unroll
       for (int i = 0; i < VP; ++i)
-        b0[n1 * kP + cv * VP + i] = make_float2(kf[2 * i] * vf[2 * i], kf[2 * i + 1] * vf[2 * i + 1]);
+        ex[n1 * kP + cv * VP + i] = make_float2(kf[2 * i] * vf[2 * i], kf[2 * i + 1] * vf[2 * i + 1]);
     }
   }
   __syncthreads();
-  const float2 *r = fft_smem<false>(b0, b1, n1len, tw);
-  // A[b][k1][n2][s]: this CTA's signals at k1 lie k1 N2 PT apart
-  float2 *ab = A + b * N * p.PT + n2 * p.PT + s0;
-  const int kstride = p.N2 * p.PT;
-  for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
-    const int k1 = e / kP, sig = e % kP;
-    if (s0 + sig < p.PT) ab[k1 * kstride + sig] = cmul(r[e], tw2[k1]);
+  float2 va[R1], vb[R2];
+  if (idx < R2) {
+#pragma unroll
+    for (int m = 0; m < R1; ++m) va[m] = ex[(idx + R2 * m) * kP + sig];
+  }
+  a_to_b<N1, false>(va, vb, ex, tw, idx, sig);
+  if (idx < R1 && s0 + sig < p.PT) {
+    float2 *ab = A + b * N * p.PT + n2 * p.PT + s0 + sig;
+    const int kstride = p.N2 * p.PT;
+#pragma unroll
+    for (int k2 = 0; k2 < R2; ++k2) {
+      const int kk = idx + R1 * k2;
+      ab[kk * kstride] = cmul(vb[k2], tw2[kk]);
+    }
   }
 }
 
-// Pass 2.  Block (k1, signal block, b): length-N2 FFT over n2 of A[b][k1][.][s].  Spectrum
+// Pass 2.  Block (k1, signal block, b): length-N2 transform over n2 of A[b][k1][.][s].  Spectrum
 // mode writes the spectrum H[k1][k2][g] (signal = group); data mode multiplies by the group's
-// H, inverse-transforms over k2 and writes the result back in place.
-template <bool kSpectrum>
+// H, transforms back and writes the result in place.
+template <bool kSpectrum, int N2>
 __global__ void __launch_bounds__(kThreads)
     fft_pass2_kernel(float2 *__restrict__ A, float2 *__restrict__ H, const FftParams p) {
-  extern __shared__ float2 fsm[];
-  const int n2len = p.N2;
-  float2 *b0 = fsm, *b1 = fsm + n2len * kP, *tw = fsm + 2 * n2len * kP;
-  const int k1 = blockIdx.x;
-  const int s0 = blockIdx.y * kP;
+  constexpr int R1 = Split<N2>::R1, R2 = Split<N2>::R2;
+  __shared__ float2 ex[N2 * kP];
+  __shared__ float2 tw[N2];
+  const int k1 = blockIdx.x, s0 = blockIdx.y * kP;
   const long long b = blockIdx.z;
-  fill_twiddles(tw, n2len);
-  // A[b][k1][n2][s0 + sig] at row[n2 PT + sig]
-  float2 *row = A + (b * p.N1 + k1) * p.N2 * p.PT + s0;
-  for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
-    const int n2 = e / kP, sig = e % kP;
-    b0[e] = s0 + sig < p.PT ? row[n2 * p.PT + sig] : make_float2(0.f, 0.f);
+  const int idx = threadIdx.x / kP, sig = threadIdx.x % kP;
+  const bool live = s0 + sig < p.PT;
+  fill_twiddles(tw, N2);
+  // A[b][k1][n2][s0 + sig] at row[n2 PT]
+  float2 *row = A + (b * p.N1 + k1) * N2 * p.PT + s0 + sig;
+  float2 va[R1], vb[R2];
+  if (idx < R2) {
+#pragma unroll
+    for (int m = 0; m < R1; ++m)
+      va[m] = live ? row[(idx + R2 * m) * p.PT] : make_float2(0.f, 0.f);
   }
-  __syncthreads();
-  float2 *r = fft_smem<false>(b0, b1, n2len, tw);
-  float2 *o = r == b0 ? b1 : b0;
-  const float2 *hk = H + k1 * p.N2 * p.G;  // H[k1][k2][g] at hk[k2 G + g]
+  a_to_b<N2, false>(va, vb, ex, tw, idx, sig);  // synchronises before using ex (tw is filled)
   if constexpr (kSpectrum) {
-    for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
-      const int k2 = e / kP, sig = e % kP;
-      if (s0 + sig < p.PT) H[k1 * p.N2 * p.G + k2 * p.G + s0 + sig] = r[e];
+    if (idx < R1 && live) {
+#pragma unroll
+      for (int k2 = 0; k2 < R2; ++k2) H[(k1 * N2 + idx + R1 * k2) * p.G + s0 + sig] = vb[k2];
     }
   } else {
-    for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
-      const int k2 = e / kP, sig = e % kP;
-      const int s = s0 + sig;
-      const int g = s < p.PT ? (2 * s) / p.d_g : 0;
-      r[e] = cmul(r[e], hk[k2 * p.G + g]);
+    if (idx < R1) {
+      const int g = live ? (2 * (s0 + sig)) / p.d_g : 0;
+      const float2 *hk = H + k1 * N2 * p.G + g;
+#pragma unroll
+      for (int k2 = 0; k2 < R2; ++k2) vb[k2] = cmul(vb[k2], hk[(idx + R1 * k2) * p.G]);
     }
-    __syncthreads();
-    const float2 *y = fft_smem<true>(r, o, n2len, tw);
-    for (int e = threadIdx.x; e < n2len * kP; e += blockDim.x) {
-      const int n2 = e / kP, sig = e % kP;
-      if (s0 + sig < p.PT) row[n2 * p.PT + sig] = y[e];
+    b_to_a<N2, true>(vb, va, ex, tw, idx, sig);
+    if (idx < R2 && live) {
+#pragma unroll
+      for (int m = 0; m < R1; ++m) row[(idx + R2 * m) * p.PT] = va[m];
     }
   }
 }
 
-// Pass 3.  Block (n2, signal block, b): W_N^{-n2 k1} times A[b][.][n2][s], inverse length-N1
-// FFT over k1, scaled by 1/N: the convolution at t = N2 n1 + n2; y = q * conv for t < L.
-template <typename T>
+// Pass 3.  Block (n2, signal block, b): W_N^{-n2 k} times A[b][k][n2][s], inverse length-N1
+// transform over k, scaled by 1/N: the convolution at t = N2 n1 + n2; y = q * conv for t < L.
+template <typename T, int N1>
 __global__ void __launch_bounds__(kThreads)
     fft_pass3_kernel(const float2 *__restrict__ A, const T *__restrict__ q, T *__restrict__ y,
                      const FftParams p) {
-  extern __shared__ float2 fsm[];
-  const int n1len = p.N1;
-  float2 *b0 = fsm, *b1 = fsm + n1len * kP, *tw = fsm + 2 * n1len * kP, *tw2 = tw + n1len;
-  const int n2 = blockIdx.x;
-  const int s0 = blockIdx.y * kP;
+  constexpr int R1 = Split<N1>::R1, R2 = Split<N1>::R2;
+  __shared__ float2 ex[N1 * kP];
+  __shared__ float2 tw[N1], tw2[N1];
+  const int n2 = blockIdx.x, s0 = blockIdx.y * kP;
   const long long b = blockIdx.z;
-  const int N = p.N1 * p.N2;
-  fill_twiddles(tw, n1len, tw2, n2, N);
+  const int N = N1 * p.N2;
+  const int idx = threadIdx.x / kP, sig = threadIdx.x % kP;
+  fill_twiddles(tw, N1, tw2, n2, N);
   __syncthreads();
-  const float2 *ab = A + b * N * p.PT + n2 * p.PT + s0;
-  const int kstride = p.N2 * p.PT;
-  for (int e = threadIdx.x; e < n1len * kP; e += blockDim.x) {
-    const int k1 = e / kP, sig = e % kP;
-    float2 z = make_float2(0.f, 0.f);
-    if (s0 + sig < p.PT) {
-      const float2 w = tw2[k1];
-      z = cmul(ab[k1 * kstride + sig], make_float2(w.x, -w.y));
+  float2 va[R1], vb[R2];
+  if (idx < R1) {
+    const bool live = s0 + sig < p.PT;
+    const float2 *ab = A + b * N * p.PT + n2 * p.PT + s0 + sig;
+    const int kstride = p.N2 * p.PT;
+#pragma unroll
+    for (int k2 = 0; k2 < R2; ++k2) {
+      const int kk = idx + R1 * k2;
+      vb[k2] = live ? cmul(ab[kk * kstride], cconj(tw2[kk])) : make_float2(0.f, 0.f);
     }
-    b0[e] = z;
+  }
+  b_to_a<N1, true>(vb, va, ex, tw, idx, sig);
+  // x[n1 = idx + R2 m] * N1 N2 in va: through ex to rows of 16 signals
+  __syncthreads();
+  if (idx < R2) {
+#pragma unroll
+    for (int m = 0; m < R1; ++m) ex[(idx + R2 * m) * kP + sig] = va[m];
   }
   __syncthreads();
-  const float2 *r = fft_smem<true>(b0, b1, n1len, tw);
   const float inv = 1.0f / static_cast<float>(N);
   constexpr int VP = PairVec<T>::VP, NV = kP / VP;
   const T *qb = q + b * p.L * p.D + 2 * s0;
   T *yb = y + b * p.L * p.D + 2 * s0;
-  for (int e = threadIdx.x; e < n1len * NV; e += blockDim.x) {
+  for (int e = threadIdx.x; e < N1 * NV; e += blockDim.x) {
     const int n1 = e / NV, cv = e % NV;
     const int t = p.N2 * n1 + n2, s = s0 + cv * VP;
     if (t >= p.L || s >= p.PT) continue;
     const int off = t * p.D + 2 * cv * VP;
-    const float2 *rr = r + n1 * kP + cv * VP;
+    const float2 *rr = ex + n1 * kP + cv * VP;
     if (p.vec && s + VP <= p.PT) {
       float qf[2 * VP], o[2 * VP];
       PairVec<T>::load(qb + off, qf);

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <limits>
 #include <mutex>
+#include <type_traits>
 
 #include "hyena_conv.h"
 #include "fir_bwd.cuh"
@@ -35,12 +36,6 @@ constexpr int kMaxDevices = 64;
 constexpr int kDhSmemMax =
     (2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (64 + 1) * static_cast<int>(sizeof(float));
 constexpr int kMaxWindowTaps = 16;
-// Shared memory of an FFT pass over n points: two buffers of n x kP complex, n twiddles W_n^k
-// and n inter-factor twiddles.
-constexpr int fft_smem_bytes(int n) {
-  return (2 * n * hyena::fft::kP + 2 * n) * static_cast<int>(sizeof(float2));
-}
-constexpr int kFftSmemMax = fft_smem_bytes(hyena::fft::kMaxLen);
 #ifndef HYENA_WINDOW_ROWS
 #define HYENA_WINDOW_ROWS 128
 #endif
@@ -82,17 +77,6 @@ int current_device(DeviceState *&ds) {
     for (const void *k : dh_kernels)
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kDhSmemMax);
-    const void *fft_kernels[] = {
-        reinterpret_cast<const void *>(hyena::fft::fft_pass1_kernel<float, true>),
-        reinterpret_cast<const void *>(hyena::fft::fft_pass1_kernel<float, false>),
-        reinterpret_cast<const void *>(hyena::fft::fft_pass1_kernel<__nv_bfloat16, false>),
-        reinterpret_cast<const void *>(hyena::fft::fft_pass2_kernel<true>),
-        reinterpret_cast<const void *>(hyena::fft::fft_pass2_kernel<false>),
-        reinterpret_cast<const void *>(hyena::fft::fft_pass3_kernel<float>),
-        reinterpret_cast<const void *>(hyena::fft::fft_pass3_kernel<__nv_bfloat16>)};
-    for (const void *k : fft_kernels)
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kFftSmemMax);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(reinterpret_cast<const void *>(hyena::tcb::fir_tc_bwd_kernel),
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -572,7 +556,7 @@ int launch_tensor_bwd(const Problem &P, const void *dy, void *dq, void *dk, void
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
-// FFT path: N = N1 N2 >= L + l_h - 1 (power of two, >= 64), N1 >= N2, both <= 256.
+// FFT path: N = N1 N2 >= L + l_h - 1 (power of two, >= 256), N1 >= N2, both in [16, 256].
 struct FftPlan {
   int N1, N2, log1, log2;
   int64_t N;
@@ -582,7 +566,7 @@ struct FftPlan {
 FftPlan fft_plan(int64_t L, int l_h) {
   FftPlan f{0, 0, 0, 0, 0, false};
   const int64_t need = L + l_h - 1;
-  int m = 6;
+  int m = 8;
   while ((int64_t{1} << m) < need && m < 40) ++m;
   f.log1 = (m + 1) / 2;
   f.log2 = m / 2;
@@ -619,6 +603,46 @@ int fft_supported(const Problem &P, FftPlan &f) {
   return HYENA_OK;
 }
 
+template <typename T, int N1>
+void launch_fft_p1(const Problem &P, const hyena::fft::FftParams &p, dim3 grid, float2 *A,
+                   cudaStream_t s) {
+  hyena::fft::fft_pass1_kernel<T, false, N1><<<grid, hyena::fft::kThreads, 0, s>>>(
+      static_cast<const T *>(P.k), static_cast<const T *>(P.v), nullptr, A, p);
+}
+
+template <int N1>
+void launch_fft_spec1(const Problem &P, const hyena::fft::FftParams &p, dim3 grid, float2 *A,
+                      cudaStream_t s) {
+  hyena::fft::fft_pass1_kernel<float, true, N1><<<grid, hyena::fft::kThreads, 0, s>>>(
+      nullptr, nullptr, P.h, A, p);
+}
+
+template <typename T, int N1>
+void launch_fft_p3(const Problem &P, const hyena::fft::FftParams &p, dim3 grid, const float2 *A,
+                   cudaStream_t s) {
+  hyena::fft::fft_pass3_kernel<T, N1><<<grid, hyena::fft::kThreads, 0, s>>>(
+      A, static_cast<const T *>(P.q), static_cast<T *>(P.y), p);
+}
+
+template <bool kSpectrum, int N2>
+void launch_fft_p2(const hyena::fft::FftParams &p, dim3 grid, float2 *A, float2 *H,
+                   cudaStream_t s) {
+  hyena::fft::fft_pass2_kernel<kSpectrum, N2><<<grid, hyena::fft::kThreads, 0, s>>>(A, H, p);
+}
+
+// Calls F<n>() for the transform length n in {16, ..., 256}.
+template <typename F>
+bool with_len(int n, F &&f) {
+  switch (n) {
+    case 16: f(std::integral_constant<int, 16>()); return true;
+    case 32: f(std::integral_constant<int, 32>()); return true;
+    case 64: f(std::integral_constant<int, 64>()); return true;
+    case 128: f(std::integral_constant<int, 128>()); return true;
+    case 256: f(std::integral_constant<int, 256>()); return true;
+    default: return false;
+  }
+}
+
 template <typename T>
 int launch_fft(const Problem &P, const FftPlan &f, uint8_t *ws, cudaStream_t s) {
   namespace hf = hyena::fft;
@@ -641,20 +665,17 @@ int launch_fft(const Problem &P, const FftPlan &f, uint8_t *ws, cudaStream_t s) 
   hf::FftParams ph = p;
   ph.PT = static_cast<int>(P.G());
   const unsigned gb = static_cast<unsigned>((ph.PT + hf::kP - 1) / hf::kP);
-  hf::fft_pass1_kernel<float, true><<<dim3(f.N2, gb, 1), hf::kThreads, fft_smem_bytes(f.N1), s>>>(
-      nullptr, nullptr, P.h, Hh, ph);
-  hf::fft_pass2_kernel<true><<<dim3(f.N1, gb, 1), hf::kThreads, fft_smem_bytes(f.N2), s>>>(
-      Hh, Hs, ph);
   // the data: pass 1, pass 2 (times H, inverse), pass 3 (inverse, q gate)
   p.PT = static_cast<int>(P.D / 2);
   const unsigned db = static_cast<unsigned>((p.PT + hf::kP - 1) / hf::kP);
   const unsigned nb = static_cast<unsigned>(P.B);
-  hf::fft_pass1_kernel<T, false><<<dim3(f.N2, db, nb), hf::kThreads, fft_smem_bytes(f.N1), s>>>(
-      static_cast<const T *>(P.k), static_cast<const T *>(P.v), nullptr, A, p);
-  hf::fft_pass2_kernel<false><<<dim3(f.N1, db, nb), hf::kThreads, fft_smem_bytes(f.N2), s>>>(
-      A, Hs, p);
-  hf::fft_pass3_kernel<T><<<dim3(f.N2, db, nb), hf::kThreads, fft_smem_bytes(f.N1), s>>>(
-      A, static_cast<const T *>(P.q), static_cast<T *>(P.y), p);
+  const dim3 g1h(f.N2, gb, 1), g2h(f.N1, gb, 1), g1(f.N2, db, nb), g2(f.N1, db, nb);
+  bool ok = with_len(f.N1, [&](auto n1) { launch_fft_spec1<decltype(n1)::value>(P, ph, g1h, Hh, s); });
+  ok = ok && with_len(f.N2, [&](auto n2) { launch_fft_p2<true, decltype(n2)::value>(ph, g2h, Hh, Hs, s); });
+  ok = ok && with_len(f.N1, [&](auto n1) { launch_fft_p1<T, decltype(n1)::value>(P, p, g1, A, s); });
+  ok = ok && with_len(f.N2, [&](auto n2) { launch_fft_p2<false, decltype(n2)::value>(p, g2, A, Hs, s); });
+  ok = ok && with_len(f.N1, [&](auto n1) { launch_fft_p3<T, decltype(n1)::value>(P, p, g1, A, s); });
+  if (!ok) return HYENA_ERR_UNSUPPORTED;
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 

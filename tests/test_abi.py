@@ -165,7 +165,7 @@ def test_fft_workspace_bytes(lib):
     f = lib.hyena_conv_fwd_fft_workspace_bytes
     # L = l_h = 8192, D = 4096, d_g = 64: N = 16384; 4 B N D of data spectra + 2 x 8 N G
     assert f(1, 8192, 4096, 64, 8192) == 4 * 16384 * 4096 + 2 * 8 * 16384 * 64
-    assert f(2, 8, 4, 2, 3) == 2 * 64 * 2 * 8 + 2 * 64 * 2 * 8   # N = 64, the smallest
+    assert f(2, 8, 4, 2, 3) == 2 * 256 * 2 * 8 + 2 * 256 * 2 * 8   # N = 256, the smallest
     assert f(1, 8192, 4096, 63, 8192) == -1                  # D % d_g
     assert f(1, 8192, 4095, 4095, 10) == -2                  # odd D: channel pairs
     assert f(1, 100, 96, 3, 10) == -2                        # odd d_g

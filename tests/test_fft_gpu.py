@@ -34,9 +34,12 @@ SHAPES = [
     ("mr_filter", 1, 777, 128, 64, 128, "bf16"),
     ("filter_past_L", 1, 500, 32, 2, 600, "f32"),
     ("ragged_signals", 3, 2048, 40, 4, 2048, "bf16"),  # 20 channel pairs: a partial block
-    ("tiny", 1, 8, 4, 2, 3, "bf16"),                   # the smallest transform, N = 64
+    ("tiny", 1, 8, 4, 2, 3, "bf16"),                   # the smallest transform, N = 256
     ("single_tap", 2, 300, 64, 8, 1, "f32"),
     ("f32_long", 2, 1500, 64, 32, 1500, "f32"),
+    ("n512", 1, 300, 64, 16, 200, "bf16"),            # N = 512: 32 x 16 (R = 4 x 8 / 4 x 4)
+    ("n2048", 2, 1500, 32, 8, 500, "bf16"),           # N = 2048: 64 x 32
+    ("n32768_odd", 1, 20000, 32, 32, 10000, "f32"),   # N = 32768: 256 x 128
 ]
 
 
