@@ -114,14 +114,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
 }
 
 // 3-D tiled store from shared memory; rows outside the tensor are clipped by the hardware.
-// Fetch a tile into L2 ahead of its load (no shared memory, no completion signal).
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1), "r"(c2)
-               : "memory");
-}
-
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int c0,
                                              int c1, int c2) {
   asm volatile(
