@@ -16,11 +16,13 @@
 // so its spectrum) is the same and both signals are real, so the inverse transform of
 // H (X_c + i X_{c+1}) is y_c + i y_{c+1} exactly -- no separation step.
 //
-// Each length-n transform (n = R1 R2, both at most 16) runs as two in-register DFTs joined by one
+// Each length-n transform (n = R1 R2, both at most 16) runs as in-register DFTs joined by one
 // exchange through shared memory: a thread holds R1 points of one signal (stride R2), transforms
-// them, applies W_n^{j k1} and stores them; then a thread holds R2 points (one k1) and
-// transforms those.  16 signals (channel pairs) per CTA, 16 threads per signal.  Twiddles come
-// from sincospif, tabled once per CTA.  The intermediate spectra live in a caller-owned fp32
+// them, applies W_n^{j k1} and stores them; then the R2 points of each k1 are shared by
+// P = 16 / R1 threads, each taking the first radix-P step over all of them on the way out of
+// shared memory and an (R2 / P)-point DFT in registers, so that every thread works in both
+// halves and holds at most max(R1, R2 / P) values.  16 signals (channel pairs) per CTA, 16
+// threads per signal.  Twiddles come from sincospif, tabled once per CTA.  The intermediate spectra live in a caller-owned fp32
 // workspace laid out [b][k1][n2][pair]: every pass moves 16 contiguous complex values (128
 // bytes) per index.
 #pragma once
@@ -131,16 +133,44 @@ template <> struct Split<64> { static constexpr int R1 = 8, R2 = 8; };
 template <> struct Split<128> { static constexpr int R1 = 8, R2 = 16; };
 template <> struct Split<256> { static constexpr int R1 = 16, R2 = 16; };
 
-// Length-n transforms of 16 signals by the CTA.  Layouts (per signal; sig = thread % 16,
-// idx = thread / 16):
+// z * W_4^e (e in 0..3; W_4 = -i), or its conjugate, for a run-time e.
+template <bool kInv>
+__device__ __forceinline__ float2 w4mul(float2 z, int e) {
+  if (e & 2) z = make_float2(-z.x, -z.y);
+  if (e & 1) z = kInv ? make_float2(-z.y, z.x) : make_float2(z.y, -z.x);
+  return z;
+}
+
+// Length-n transforms of 16 signals by the CTA, 16 threads per signal (sig = thread % 16,
+// idx = thread / 16).  n = R1 R2; the R2-point half is shared by P = 16 / R1 threads per k1,
+// each computing M = R2 / P of its outputs, so that all 16 threads hold values in both halves.
+// Layouts (per signal):
 //   "A" layout: thread idx = j < R2 holds x[j + R2 m], m < R1   (natural time order)
-//   "B" layout: thread idx = k1 < R1 holds X[k1 + R1 k2], k2 < R2 (natural frequency order)
+//   "B" layout: thread idx = P k1 + q holds X[k1 + R1 (P r + q)], r < M  (see bfreq)
 // ex is n x 16 complex of shared memory, tw[k] = W_n^k.  Both functions end with the result
 // in registers; they synchronise the CTA around their use of ex.
+template <int n>
+struct BLay {
+  static constexpr int R1 = Split<n>::R1, R2 = Split<n>::R2;
+  static constexpr int P = 16 / R1, M = R2 / P;
+  static_assert(P * R1 == 16 && M * P == R2, "split of the R2-point half");
+};
+
+// Frequency index held in register r of B-layout thread idx.
+template <int n>
+__device__ __forceinline__ int bfreq(int idx, int r) {
+  using BL = BLay<n>;
+  return idx / BL::P + BL::R1 * (BL::P * r + idx % BL::P);
+}
+
+// A -> B: R1-point DFTs, twiddles W_n^{j k1}, exchange, then the R2-point DFT over j split
+// four-step style: X[k1 + R1 (P r + q)] = sum_{j < M} W_M^{j r} W_R2^{j q}
+// sum_{p < P} W_P^{p q} y_k1[j + p M].
 template <int n, bool kInv>
-__device__ __forceinline__ void a_to_b(float2 (&va)[Split<n>::R1], float2 (&vb)[Split<n>::R2],
+__device__ __forceinline__ void a_to_b(float2 (&va)[Split<n>::R1], float2 (&vb)[BLay<n>::M],
                                        float2 *ex, const float2 *tw, int idx, int sig) {
-  constexpr int R1 = Split<n>::R1, R2 = Split<n>::R2;
+  using BL = BLay<n>;
+  constexpr int R1 = BL::R1, R2 = BL::R2, P = BL::P, M = BL::M;
   __syncthreads();  // ex is free
   if (idx < R2) {
     dft_reg<R1, kInv>(va);
@@ -151,30 +181,57 @@ __device__ __forceinline__ void a_to_b(float2 (&va)[Split<n>::R1], float2 (&vb)[
     }
   }
   __syncthreads();
-  if (idx < R1) {
+  const int k1 = idx / P, q = idx % P;
 #pragma unroll
-    for (int j = 0; j < R2; ++j) vb[j] = ex[(idx * R2 + j) * kP + sig];
-    dft_reg<R2, kInv>(vb);
+  for (int j = 0; j < M; ++j) {
+    float2 z = ex[(k1 * R2 + j) * kP + sig];
+#pragma unroll
+    for (int p = 1; p < P; ++p) {
+      const float2 t = w4mul<kInv>(ex[(k1 * R2 + j + p * M) * kP + sig], ((4 / P) * p * q) & 3);
+      z = make_float2(z.x + t.x, z.y + t.y);
+    }
+    if (P > 1 && j > 0) {
+      const float2 w = tw[(R1 * j * q) & (n - 1)];
+      z = cmul(z, kInv ? cconj(w) : w);
+    }
+    vb[j] = z;
   }
+  dft_reg<M, kInv>(vb);
 }
 
+// B -> A, the mirror of a_to_b: M-point DFTs, W_R2^{j q}, exchange, the P-point combination
+// and W_n^{k1 j'} (j' = j + p M), then R1-point DFTs.
 template <int n, bool kInv>
-__device__ __forceinline__ void b_to_a(float2 (&vb)[Split<n>::R2], float2 (&va)[Split<n>::R1],
+__device__ __forceinline__ void b_to_a(float2 (&vb)[BLay<n>::M], float2 (&va)[Split<n>::R1],
                                        float2 *ex, const float2 *tw, int idx, int sig) {
-  constexpr int R1 = Split<n>::R1, R2 = Split<n>::R2;
+  using BL = BLay<n>;
+  constexpr int R1 = BL::R1, R2 = BL::R2, P = BL::P, M = BL::M;
   __syncthreads();
-  if (idx < R1) {
-    dft_reg<R2, kInv>(vb);
+  const int k1 = idx / P, q = idx % P;
+  dft_reg<M, kInv>(vb);
 #pragma unroll
-    for (int j = 0; j < R2; ++j) {
-      const float2 w = tw[(idx * j) & (n - 1)];
-      ex[(idx * R2 + j) * kP + sig] = cmul(vb[j], kInv ? cconj(w) : w);
+  for (int j = 0; j < M; ++j) {
+    float2 z = vb[j];
+    if (P > 1 && j > 0) {
+      const float2 w = tw[(R1 * j * q) & (n - 1)];
+      z = cmul(z, kInv ? cconj(w) : w);
     }
+    ex[((k1 * P + q) * M + j) * kP + sig] = z;
   }
   __syncthreads();
   if (idx < R2) {
+    const int j = idx % M, p = idx / M;
 #pragma unroll
-    for (int k1 = 0; k1 < R1; ++k1) va[k1] = ex[(k1 * R2 + idx) * kP + sig];
+    for (int kk = 0; kk < R1; ++kk) {
+      float2 z = ex[((kk * P) * M + j) * kP + sig];
+#pragma unroll
+      for (int qq = 1; qq < P; ++qq) {
+        const float2 t = w4mul<kInv>(ex[((kk * P + qq) * M + j) * kP + sig], ((4 / P) * p * qq) & 3);
+        z = make_float2(z.x + t.x, z.y + t.y);
+      }
+      const float2 w = tw[(idx * kk) & (n - 1)];
+      va[kk] = cmul(z, kInv ? cconj(w) : w);
+    }
     dft_reg<R1, kInv>(va);
   }
 }
@@ -262,19 +319,19 @@ __global__ void __launch_bounds__(kThreads)
     }
   }
   __syncthreads();
-  float2 va[R1], vb[R2];
+  float2 va[R1], vb[BLay<N1>::M];
   if (idx < R2) {
 #pragma unroll
     for (int m = 0; m < R1; ++m) va[m] = ex[(idx + R2 * m) * kP + sig];
   }
   a_to_b<N1, false>(va, vb, ex, tw, idx, sig);
-  if (idx < R1 && s0 + sig < p.PT) {
+  if (s0 + sig < p.PT) {
     float2 *ab = A + b * N * p.PT + n2 * p.PT + s0 + sig;
     const int kstride = p.N2 * p.PT;
 #pragma unroll
-    for (int k2 = 0; k2 < R2; ++k2) {
-      const int kk = idx + R1 * k2;
-      ab[kk * kstride] = cmul(vb[k2], tw2[kk]);
+    for (int r = 0; r < BLay<N1>::M; ++r) {
+      const int kk = bfreq<N1>(idx, r);
+      ab[kk * kstride] = cmul(vb[r], tw2[kk]);
     }
   }
 }
@@ -283,9 +340,10 @@ __global__ void __launch_bounds__(kThreads)
 // mode writes the spectrum H[k1][k2][g] (signal = group); data mode multiplies by the group's
 // H, transforms back and writes the result in place.
 template <bool kSpectrum, int N2>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, N2 <= 128 ? 6 : (kSpectrum ? 1 : 4))
     fft_pass2_kernel(float2 *__restrict__ A, float2 *__restrict__ H, const FftParams p) {
   constexpr int R1 = Split<N2>::R1, R2 = Split<N2>::R2;
+  constexpr int M = BLay<N2>::M;
   __shared__ float2 ex[N2 * kP];
   __shared__ float2 tw[N2];
   const int k1 = blockIdx.x, s0 = blockIdx.y * kP;
@@ -295,7 +353,7 @@ __global__ void __launch_bounds__(kThreads)
   fill_twiddles(tw, N2);
   // A[b][k1][n2][s0 + sig] at row[n2 PT]
   float2 *row = A + (b * p.N1 + k1) * N2 * p.PT + s0 + sig;
-  float2 va[R1], vb[R2];
+  float2 va[R1], vb[BLay<N2>::M];
   if (idx < R2) {
 #pragma unroll
     for (int m = 0; m < R1; ++m)
@@ -303,17 +361,16 @@ __global__ void __launch_bounds__(kThreads)
   }
   a_to_b<N2, false>(va, vb, ex, tw, idx, sig);  // synchronises before using ex (tw is filled)
   if constexpr (kSpectrum) {
-    if (idx < R1 && live) {
+    if (live) {
 #pragma unroll
-      for (int k2 = 0; k2 < R2; ++k2) H[(k1 * N2 + idx + R1 * k2) * p.G + s0 + sig] = vb[k2];
+      for (int r = 0; r < BLay<N2>::M; ++r)
+        H[(k1 * N2 + bfreq<N2>(idx, r)) * p.G + s0 + sig] = vb[r];
     }
   } else {
-    if (idx < R1) {
-      const int g = live ? (2 * (s0 + sig)) / p.d_g : 0;
-      const float2 *hk = H + k1 * N2 * p.G + g;
+    // the group's filter spectrum at this thread's frequencies (L2-resident)
+    const float2 *hk = H + k1 * N2 * p.G + (live ? (2 * (s0 + sig)) / p.d_g : 0);
 #pragma unroll
-      for (int k2 = 0; k2 < R2; ++k2) vb[k2] = cmul(vb[k2], hk[(idx + R1 * k2) * p.G]);
-    }
+    for (int r = 0; r < M; ++r) vb[r] = cmul(vb[r], hk[bfreq<N2>(idx, r) * p.G]);
     b_to_a<N2, true>(vb, va, ex, tw, idx, sig);
     if (idx < R2 && live) {
 #pragma unroll
@@ -337,15 +394,15 @@ __global__ void __launch_bounds__(kThreads)
   const int idx = threadIdx.x / kP, sig = threadIdx.x % kP;
   fill_twiddles(tw, N1, tw2, n2, N);
   __syncthreads();
-  float2 va[R1], vb[R2];
-  if (idx < R1) {
+  float2 va[R1], vb[BLay<N1>::M];
+  {
     const bool live = s0 + sig < p.PT;
     const float2 *ab = A + b * N * p.PT + n2 * p.PT + s0 + sig;
     const int kstride = p.N2 * p.PT;
 #pragma unroll
-    for (int k2 = 0; k2 < R2; ++k2) {
-      const int kk = idx + R1 * k2;
-      vb[k2] = live ? cmul(ab[kk * kstride], cconj(tw2[kk])) : make_float2(0.f, 0.f);
+    for (int r = 0; r < BLay<N1>::M; ++r) {
+      const int kk = bfreq<N1>(idx, r);
+      vb[r] = live ? cmul(ab[kk * kstride], cconj(tw2[kk])) : make_float2(0.f, 0.f);
     }
   }
   b_to_a<N1, true>(vb, va, ex, tw, idx, sig);

@@ -126,7 +126,7 @@ int hyena_conv_fwd_hist(const void *q, const void *k, const void *v, const float
  * 256), minus HYENA_ERR_INVALID_ARG for a bad shape, or minus HYENA_ERR_UNSUPPORTED where the
  * FFT path does not apply (odd D or d_g, or L + l_h - 1 > 65536).  Touches no device.  The
  * workspace holds the fp32 spectra: 4 B L_fft D bytes for the data plus 16 L_fft D / d_g for
- * the filters, L_fft the power of two >= max(64, L + l_h - 1) (256 MiB of data spectra at
+ * the filters, L_fft the power of two >= max(256, L + l_h - 1) (256 MiB of data spectra at
  * B = 1, L = l_h = 8192, D = 4096).
  */
 int64_t hyena_conv_fwd_fft_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h);
