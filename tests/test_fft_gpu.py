@@ -85,6 +85,18 @@ def test_fft_largest_transform_sampled():
     _sampled_rows(y.cpu(), q.cpu(), k.cpu(), v.cpu(), h.cpu(), 64, rows)
 
 
+def test_fft_ragged_signal_block_and_split_group_at_the_largest_transform():
+    """B = 4 at N = 65536 (256 x 256): D = 80 is 40 channel pairs, two full 16-pair blocks and a
+    ragged one of 8, and d_g = 10 puts the group of pairs 15..19 across the first block
+    boundary (the pass-2 filter lookup per signal)."""
+    wl = custom("ragged", 4, 32768, 80, 10, 32768, 64, "bf16", "mr", seed=12)
+    q, k, v, h = make_inputs(wl, device="cuda")
+    y = g.hyena_conv_fwd_fft(q, k, v, h, 10, 64)
+    torch.cuda.synchronize()
+    rows = [(0, 0), (1, 32767), (2, 4097), (3, 20000), (3, 32766)]
+    _sampled_rows(y.cpu(), q.cpu(), k.cpu(), v.cpu(), h.cpu(), 10, rows)
+
+
 def test_fft_li_workload_sampled():
     """The Hyena-LI-shaped workload (B=1, L=8192, D=4096, d_g=64, l_h=8192) on sampled rows."""
     wl = WORKLOADS["li"]
