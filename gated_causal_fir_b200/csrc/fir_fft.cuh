@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kThreads)
 // mode writes the spectrum H[k1][k2][g] (signal = group); data mode multiplies by the group's
 // H, transforms back and writes the result in place.
 template <bool kSpectrum, int N2>
-__global__ void __launch_bounds__(kThreads, N2 <= 128 ? 6 : (kSpectrum ? 1 : 4))
+__global__ void __launch_bounds__(kThreads, N2 <= 128 ? 8 : (kSpectrum ? 1 : 4))
     fft_pass2_kernel(float2 *__restrict__ A, float2 *__restrict__ H, const FftParams p) {
   constexpr int R1 = Split<N2>::R1, R2 = Split<N2>::R2;
   constexpr int M = BLay<N2>::M;

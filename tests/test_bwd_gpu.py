@@ -98,6 +98,7 @@ SHAPES = [
     ("runs_across_seqs", 3, 3000, 512, 64, 100, 64, "bf16"),
     ("long_seq_one_group", 1, 40000, 64, 64, 128, 64, "bf16"),
     ("batched_halo16", 4, 2048, 128, 64, 17, 16, "bf16"),
+    ("three_blocks", 2, 900, 192, 64, 64, 64, "bf16"),  # odd block count: unpaired walk
 ]
 CASES = [(s, a) for s in SHAPES for a in ALGOS if a == "direct" or _tensor_fits(*s[1:6], s[7])]
 
