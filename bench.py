@@ -17,7 +17,9 @@ through NVML during the timed region, an end-to-end figure through
 ``hyena_conv_fwd_from_host`` (pinned host buffers, copies inside the timed region) and the
 fp64 oracle timed on the host cores as a CPU baseline.  Beside the forward it reports the
 backward (``backward``) and two longer-filter cases (``long_filters``: the Hyena-LI-shaped
-workload through the FFT entry point, and l_h = 513 on the tensor-core path).
+workload through the FFT entry point, and l_h = 513 on the tensor-core path) and, as context,
+the pages' naive baseline (``comparator``: PyTorch's depthwise F.conv1d with the gating
+products, on the same inputs).
 ``--impl reference`` times only the oracle, one l_b-row chunk of the workload per step.
 """
 import argparse
@@ -53,6 +55,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--bwd-steps", type=int, default=200,
                    help="timed steps of the backward (hyena_conv_bwd); 0 skips it")
+    p.add_argument("--comparator-steps", type=int, default=5,
+                   help="timed steps of the torch F.conv1d comparator; 0 skips")
     p.add_argument("--long-steps", type=int, default=20,
                    help="timed steps of the long-filter measurements (FFT, l_h = 513); 0 skips")
     return p.parse_args()
@@ -161,7 +165,52 @@ def cpu_baseline(wl, q, k, v, h, target_s):
            "kind": "oracle",
            "sample": "whole %s workload x%d (%.1f s of fp64 direct sums, OpenMP)"
                      % (wl.name, reps, t_total)}
+    # the same oracle on one thread, over the last rows of the first sequence (full sums)
+    n_rows = min(256, wl.L)
+    rows = [(0, t) for t in range(wl.L - n_rows, wl.L)]
+    t = time.perf_counter()
+    oracle.gated_fir_rows(qh, kh, vh, hh, wl.d_g, rows, nthreads=1)
+    dt = time.perf_counter() - t
+    rec["single_thread"] = {"value": n_rows / dt, "unit": UNIT, "cores": 1,
+                            "sample": "rows %d..%d of sequence 0, all %d channels"
+                                      % (wl.L - n_rows, wl.L - 1, wl.D)}
     return rec, y_ref
+
+
+def time_conv1d_comparator(args, wl, sets, stream, y_ours):
+    """Context, not the product: the pages' naive baseline, PyTorch's depthwise F.conv1d
+    (cuDNN; weight = each channel's filter reversed, left padding l_h - 1) with the two gating
+    products around it, in the I/O dtype on the same inputs, timed with CUDA events over
+    rotating input sets.  Its transposes to and from the [B, D, L] layout conv1d wants are part
+    of the step."""
+    import torch
+    import torch.nn.functional as F
+    h = sets[0][3]
+    w = h.repeat_interleave(wl.d_g, dim=0).flip(-1).unsqueeze(1).to(sets[0][0].dtype)
+
+    def step(q, k, v):
+        x = (k * v).transpose(1, 2)
+        z = F.conv1d(F.pad(x, (wl.l_h - 1, 0)), w, groups=wl.D)
+        return q * z.transpose(1, 2)
+
+    with torch.cuda.stream(stream):
+        y = step(*sets[0][:3])
+        for i in range(2):
+            step(*sets[i % len(sets)][:3])
+        torch.cuda.synchronize()
+        diff = float((y.float() - y_ours.float()).abs().max())
+        scale = float(y_ours.float().abs().max())
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        K = args.comparator_steps
+        e0.record(stream)
+        for i in range(K):
+            step(*sets[i % len(sets)][:3])
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    return {"kind": "torch F.conv1d depthwise (cuDNN) + gating, %s" % wl.dtype,
+            "ms_per_step": ms, "value": wl.tokens / (ms / 1e3), "unit": UNIT, "steps": K,
+            "max_abs_diff_vs_kernel": diff, "max_abs_kernel_output": scale}
 
 
 def run_reference(args, wl, rank, world):
@@ -435,6 +484,12 @@ def main():
         peak, peak_kind = measured_peak_hbm()
         bwd = time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind)
 
+    comparator = None
+    if args.comparator_steps > 0 and rank == 0 and world == 1 and wl.B * wl.L * wl.D <= 1 << 26:
+        q, k, v, h, y = sets[0]
+        fwd(q, k, v, h, wl.d_g, wl.l_b, y=y, stream=stream)
+        comparator = time_conv1d_comparator(args, wl, sets, stream, y)
+
     long_filters = None
     if args.long_steps > 0 and wl.name == "mr":
         peak, peak_kind = measured_peak_hbm()
@@ -475,7 +530,8 @@ def main():
                          "mean_launch_us": 1e3 * mean_launch_ms, "kernel": kernel},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K,
             "clocks": clocks.summary(t_wall0, t_wall1),
-            "backward": bwd, "long_filters": long_filters, "kernel_algo": g.ALGO_NAMES[algo], "device_status": status, "parity": parity,
+            "backward": bwd, "long_filters": long_filters, "comparator": comparator,
+            "kernel_algo": g.ALGO_NAMES[algo], "device_status": status, "parity": parity,
             "wall_s_timed_region": t_wall1 - t_wall0,
         }
         print(json.dumps(line), flush=True)
