@@ -82,7 +82,7 @@ struct WindowParams {
 
 // Unroll factor of the time loop: loads of U rows are issued before their arithmetic.
 #ifndef HYENA_WINDOW_UNROLL
-#define HYENA_WINDOW_UNROLL 8
+#define HYENA_WINDOW_UNROLL 4
 #endif
 constexpr int kWindowUnroll = HYENA_WINDOW_UNROLL;
 
@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(kWindowBlock, HYENA_WINDOW_MIN_BLOCKS)
     fir_window_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                       const float *__restrict__ h, T *__restrict__ y, const WindowParams p) {
   constexpr int VN = Vec<T>::N;
-  // Longer windows hold more registers: they unroll less so the loaded rows still fit.
-  constexpr int U = LH <= 8 ? kWindowUnroll : 4;
+  // Longer windows hold more registers: they unroll no further than 4 rows.
+  constexpr int U = LH <= 8 ? kWindowUnroll : (kWindowUnroll < 4 ? kWindowUnroll : 4);
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (gid >= p.B * p.n_tb * p.cv) return;
   const long long cvi = gid % p.cv;

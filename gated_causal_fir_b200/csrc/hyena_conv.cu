@@ -291,22 +291,56 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
   return le == cudaSuccess && cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
+// Time steps per thread of the window kernel: as many as make the whole problem one full wave
+// of resident threads (SMs x resident blocks x block), so that every SM gets the same number of
+// rows, within [kWindowMinRows, kWindowRows] (a longer run where even kWindowRows per thread
+// needs more than one wave).
+#ifndef HYENA_WINDOW_WAVE
+#define HYENA_WINDOW_WAVE 1
+#endif
+constexpr int kWindowMinRows = 32;  // halo (l_h - 1 rows) at most ~half a run at l_h = 16
+
 template <typename T, int LH>
-void launch_window_lh(const Problem &P, const WindowParams &wp, unsigned blocks, cudaStream_t s) {
-  hyena::cc::fir_window_kernel<T, LH><<<blocks, hyena::cc::kWindowBlock, 0, s>>>(
+int launch_window_lh(const Problem &P, WindowParams wp, int sm_count, cudaStream_t s) {
+  const auto kernel = hyena::cc::fir_window_kernel<T, LH>;
+  static int resident[kMaxDevices];  // blocks per SM, per device (0: not yet queried)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYENA_ERR_CUDA;
+  if (resident[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, hyena::cc::kWindowBlock, 0) !=
+        cudaSuccess)
+      return HYENA_ERR_CUDA;
+    resident[dev] = n > 0 ? n : 1;
+  }
+  const long long wave = static_cast<long long>(sm_count) * resident[dev] * hyena::cc::kWindowBlock;
+  const long long units = wp.B * wp.cv;  // thread columns per time block
+  long long rows = kWindowRows;
+  const long long tb_per_wave = wave / units;  // time blocks one wave holds
+  if (HYENA_WINDOW_WAVE && tb_per_wave >= 1 && units * ((wp.L + kWindowRows - 1) / kWindowRows) <= wave) {
+    rows = (wp.L + tb_per_wave - 1) / tb_per_wave;  // ceil(L / rows) <= tb_per_wave
+    rows = std::max<long long>(rows, kWindowMinRows);
+    rows = std::min<long long>(rows, kWindowRows);
+  }
+  wp.rows = static_cast<int>(rows);
+  wp.n_tb = (wp.L + rows - 1) / rows;
+  const long long threads = units * wp.n_tb;
+  const long long blocks = (threads + hyena::cc::kWindowBlock - 1) / hyena::cc::kWindowBlock;
+  if (blocks > std::numeric_limits<int32_t>::max()) return HYENA_ERR_UNSUPPORTED;
+  kernel<<<static_cast<unsigned>(blocks), hyena::cc::kWindowBlock, 0, s>>>(
       static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v), P.h,
       static_cast<T *>(P.y), wp);
+  return HYENA_OK;
 }
 
 template <typename T, int LH = 1>
-void launch_window_dispatch(const Problem &P, const WindowParams &wp, unsigned blocks,
-                            cudaStream_t s) {
+int launch_window_dispatch(const Problem &P, const WindowParams &wp, int sm_count,
+                           cudaStream_t s) {
   if constexpr (LH <= kMaxWindowTaps) {
-    if (P.l_h == LH)
-      launch_window_lh<T, LH>(P, wp, blocks, s);
-    else
-      launch_window_dispatch<T, LH + 1>(P, wp, blocks, s);
+    if (P.l_h == LH) return launch_window_lh<T, LH>(P, wp, sm_count, s);
+    return launch_window_dispatch<T, LH + 1>(P, wp, sm_count, s);
   }
+  return HYENA_ERR_UNSUPPORTED;
 }
 
 int launch_window(const Problem &P, cudaStream_t s) {
@@ -316,19 +350,16 @@ int launch_window(const Problem &P, cudaStream_t s) {
   wp.L = P.L;
   wp.D = P.D;
   wp.d_g = P.d_g;
-  wp.rows = kWindowRows;
-  wp.n_tb = (P.L + kWindowRows - 1) / kWindowRows;
   wp.cv = P.D / vec;
   wp.kh = P.kh;
   wp.vh = P.vh;
   wp.Lh = P.Lh;
-  const long long threads = wp.B * wp.n_tb * wp.cv;
-  const long long blocks = (threads + hyena::cc::kWindowBlock - 1) / hyena::cc::kWindowBlock;
-  if (blocks > std::numeric_limits<int32_t>::max()) return HYENA_ERR_UNSUPPORTED;
-  if (P.dtype == HYENA_DTYPE_F32)
-    launch_window_dispatch<float>(P, wp, static_cast<unsigned>(blocks), s);
-  else
-    launch_window_dispatch<__nv_bfloat16>(P, wp, static_cast<unsigned>(blocks), s);
+  DeviceState *ds = nullptr;
+  if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
+  const int rc = P.dtype == HYENA_DTYPE_F32
+                     ? launch_window_dispatch<float>(P, wp, ds->sm_count, s)
+                     : launch_window_dispatch<__nv_bfloat16>(P, wp, ds->sm_count, s);
+  if (rc != HYENA_OK) return rc;
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
