@@ -515,7 +515,9 @@ def main():
                   g.HYENA_ALGO_DIRECT: "fir_direct_kernel"}[algo]
         traffic = committed_traffic(kernel, wl.name)
         line = {
-            "metric": METRIC, "value": world * wl.tokens * K / (max_ms / 1e3), "unit": UNIT,
+            "metric": METRIC if wl.name == "mr" else
+            "gated causal FIR fwd tokens/s (%s); HBM GB/s vs peak" % wl.describe(),
+            "value": world * wl.tokens * K / (max_ms / 1e3), "unit": UNIT,
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": max_ms / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic", "config": dict(
