@@ -462,7 +462,7 @@ def main():
         qh, kh, vh, hh = (x.cpu().pin_memory() for x in sets[0][:4])
         yh = torch.empty_like(qh).pin_memory()
         g.hyena_conv_fwd_from_host(qh, kh, vh, hh, wl.d_g, wl.l_b, out=yh, device=dev,
-                                   stream=stream)
+                                   stream=stream, chunk=2048)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         D.barrier()
@@ -470,14 +470,20 @@ def main():
         e0.record(stream)
         for _ in range(args.e2e_steps):
             g.hyena_conv_fwd_from_host(qh, kh, vh, hh, wl.d_g, wl.l_b, out=yh, device=dev,
-                                       stream=stream)
+                                       stream=stream, chunk=2048)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = D.max_over_ranks(e0.elapsed_time(e1), device=dev)
+        # bytes the call copies: h once; q, k, v of every chunk with its l_h - 1 history rows
+        chunk, es = 2048, qh.element_size()
+        rows_in = sum(min(wl.L, t0 + chunk) - max(0, t0 - (wl.l_h - 1))
+                      for t0 in range(0, wl.L, chunk))
         e2e = {"value": world * wl.tokens * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (qh, kh, vh, hh)),
+               "h2d_bytes_per_step": hh.numel() * hh.element_size()
+               + 3 * wl.B * rows_in * wl.D * es,
                "d2h_bytes_per_step": yh.numel() * yh.element_size(),
-               "steps": args.e2e_steps, "api": "hyena_conv_fwd_from_host"}
+               "steps": args.e2e_steps,
+               "api": "hyena_conv_fwd_from_host (C ABI; 2048-row chunks, three streams)"}
 
     bwd = None
     if args.bwd_steps > 0:

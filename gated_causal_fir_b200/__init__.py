@@ -27,6 +27,7 @@ __all__ = [
     "HYENA_DEVICE_F16_RANGE", "ALGO_NAMES", "hyena_conv_fwd_from_host",
     "hyena_toeplitz_stages", "hyena_build_toeplitz_blocks", "hyena_conv_fwd_hist",
     "hyena_conv_fwd_fft", "hyena_conv_fwd_fft_workspace_bytes",
+    "hyena_conv_fwd_from_host_workspace_bytes",
 ]
 
 
@@ -312,80 +313,57 @@ def hyena_abi_version():
     return int(_native.lib().hyena_abi_version())
 
 
-class _Pipeline:
-    """Device slots and streams of hyena_conv_fwd_from_host, reused across calls."""
-
-    def __init__(self, torch, rows, D, dtype, hshape, device, nslots=3):
-        dev = torch.device(device)
-        self.slots = [[torch.empty((1, rows, D), dtype=dtype, device=dev) for _ in range(4)]
-                      for _ in range(nslots)]
-        self.h = torch.empty(hshape, dtype=torch.float32, device=dev)
-        self.h2d, self.comp, self.d2h = (torch.cuda.Stream(device=dev) for _ in range(3))
-        self.free = [torch.cuda.Event() for _ in range(nslots)]
-        self.used = [False] * nslots
+_HOST_WS = {}
 
 
-_PIPES = {}
+def hyena_conv_fwd_from_host_workspace_bytes(B, L, D, d_g, l_h, dtype="bf16", chunk=2048):
+    code = HYENA_DTYPE_F32 if dtype in ("f32", "float32") else HYENA_DTYPE_BF16
+    n = int(_native.lib().hyena_conv_fwd_from_host_workspace_bytes(B, L, D, d_g, l_h, code,
+                                                                   chunk))
+    if n < 0:
+        raise _native.HyenaError("hyena_conv_fwd_from_host_workspace_bytes", -n)
+    return n
 
 
 def hyena_conv_fwd_from_host(q, k, v, h, d_g, l_b, out=None, device="cuda", stream=None,
-                             chunk=2048):
-    """End-to-end forward for host tensors: q, k, v (bf16 or fp32 [B, L, D]) and h go to
-    ``device``, the forward runs there, and y comes back into ``out`` (a host tensor).
-
-    The sequence is cut into chunks of ``chunk`` rows.  Chunk c is copied to the device
-    together with the l_h - 1 rows before it (its history), computed as its own sequence, and
-    its rows after the history are copied back: the result is the same as one call on the
-    whole sequence, and the host-to-device copy of one chunk overlaps the kernel and the
-    device-to-host copy of the previous ones (separate streams; PCIe is full duplex).  With
-    pinned host memory every copy is asynchronous.  The call is ordered after the work queued
-    on ``stream`` (default: current stream) and ``stream`` waits for it on return; synchronise
-    ``stream`` before reading ``out``.
-    """
+                             chunk=2048, workspace=None):
+    """End-to-end forward for HOST tensors through the C entry point of the same name: q, k, v
+    (bf16 or fp32 [B, L, D], contiguous; pinned for overlapped copies) and h (fp32
+    [D / d_g, l_h]) go to ``device`` chunk by chunk, the forward runs there and y comes back
+    into ``out`` (a host tensor, pinned when created here).  The library queues every copy and
+    kernel; this wrapper only supplies the device workspace (cached per shape when not given)
+    and the stream.  Synchronise ``stream`` (default: the current stream) before reading
+    ``out``."""
     torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v), ("h", h)):
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise TypeError("%s must be a contiguous host tensor" % name)
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share shape and dtype")
+    if h.dtype != torch.float32:
+        raise TypeError("h must be float32")
     B, L, D = q.shape
-    hist = h.shape[1] - 1
-    rows = min(L, chunk) + hist
-    key = (rows, D, q.dtype, tuple(h.shape), str(device))
-    pipe = _PIPES.get(key)
-    if pipe is None:
-        _PIPES.clear()
-        pipe = _PIPES[key] = _Pipeline(torch, rows, D, q.dtype, h.shape, device)
+    dt = _dtype_code(q)
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-    caller = torch.cuda.current_stream(device) if stream is None else stream
-    start = torch.cuda.Event()
-    start.record(caller)
-    pipe.h2d.wait_event(start)
-    with torch.cuda.stream(pipe.h2d):
-        pipe.h.copy_(h, non_blocking=True)
-    n = 0
-    for b in range(B):
-        for t0 in range(0, L, chunk):
-            t1 = min(L, t0 + chunk)
-            s0 = max(0, t0 - hist)           # first row copied (history included)
-            nr = t1 - s0
-            si = n % len(pipe.slots)
-            qd, kd, vd, yd = (x[:, :nr] for x in pipe.slots[si])
-            if pipe.used[si]:                # the slot's previous chunk is back on the host
-                pipe.h2d.wait_event(pipe.free[si])
-            with torch.cuda.stream(pipe.h2d):
-                qd[0].copy_(q[b, s0:t1], non_blocking=True)
-                kd[0].copy_(k[b, s0:t1], non_blocking=True)
-                vd[0].copy_(v[b, s0:t1], non_blocking=True)
-            loaded = torch.cuda.Event()
-            loaded.record(pipe.h2d)
-            pipe.comp.wait_event(loaded)
-            hyena_conv_fwd_ex(qd, kd, vd, pipe.h, d_g, l_b, y=yd, stream=pipe.comp)
-            done = torch.cuda.Event()
-            done.record(pipe.comp)
-            pipe.d2h.wait_event(done)
-            with torch.cuda.stream(pipe.d2h):
-                out[b, t0:t1].copy_(yd[0, t0 - s0:], non_blocking=True)
-            pipe.free[si].record(pipe.d2h)
-            pipe.used[si] = True
-            n += 1
-    finish = torch.cuda.Event()
-    finish.record(pipe.d2h)
-    caller.wait_event(finish)
+    elif out.device.type != "cpu" or not out.is_contiguous() or out.shape != q.shape or \
+            out.dtype != q.dtype:
+        raise TypeError("out must be a contiguous host tensor like q")
+    dev = torch.device(device)
+    if workspace is None:
+        need = int(_native.lib().hyena_conv_fwd_from_host_workspace_bytes(
+            B, L, D, d_g, h.shape[1], dt, chunk))
+        if need < 0:
+            raise _native.HyenaError("hyena_conv_fwd_from_host", -need)
+        key = (str(dev), need)
+        workspace = _HOST_WS.get(key)
+        if workspace is None:
+            _HOST_WS.clear()
+            workspace = _HOST_WS[key] = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream(dev) if stream is None else stream
+    with torch.cuda.device(dev):
+        _native.check("hyena_conv_fwd_from_host", _native.lib().hyena_conv_fwd_from_host(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), h.data_ptr(), out.data_ptr(), B, L, D,
+            d_g, h.shape[1], l_b, dt, chunk, workspace.data_ptr(), workspace.numel(),
+            st.cuda_stream))
     return out

@@ -48,6 +48,10 @@ SIGNATURES = {
     "hyena_conv_fwd_fft_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32, _i32]),
     "hyena_conv_fwd_fft": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32,
                                   _i32, _vp, ctypes.c_size_t, _vp]),
+    "hyena_conv_fwd_from_host_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32, _i32, _i32,
+                                                         _i64]),
+    "hyena_conv_fwd_from_host": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32,
+                                        _i32, _i32, _i64, _vp, ctypes.c_size_t, _vp]),
     "hyena_select_algo": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32,
                                  _i32]),
     "hyena_conv_bwd_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32, _i32]),

@@ -799,6 +799,127 @@ int static_scratch(void *&ptr) {
 
 }  // namespace
 
+// ------------------------------------------------------------------------------ from host
+// hyena_conv_fwd_from_host: the forward of host-resident q, k, v, h into host y.  Each
+// sequence is cut into chunks of `chunk` rows; chunk [t0, t1) travels to the device with the
+// l_h - 1 rows before it (rows [s0, t1), s0 = max(0, t0 - l_h + 1)), is computed as a sequence
+// of its own (rows from t0 on then equal the whole sequence's), and rows [t0, t1) come back.
+// Three device slots rotate over three streams (copy in, compute, copy out) so that the
+// host-to-device copy of one chunk, the kernel of the previous one and the copy back of the one
+// before overlap (PCIe is full duplex).
+constexpr int kHostSlots = 3;
+
+struct HostPipe {
+  std::once_flag once;
+  std::mutex mu;  // one call at a time per device: the streams and events are shared
+  cudaError_t err = cudaSuccess;
+  cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, loaded[kHostSlots] = {}, done[kHostSlots] = {},
+              freed[kHostSlots] = {}, finish = nullptr;
+};
+HostPipe g_host_pipes[kMaxDevices];
+
+struct HostLayout {
+  int64_t rows, slot_bytes, off_h, bytes;
+};
+
+// Device workspace: kHostSlots slots of (q, k, v, y) chunk buffers, then h.
+HostLayout host_layout(int64_t L, int64_t D, int64_t G, int l_h, int64_t elem, int64_t chunk) {
+  HostLayout o;
+  o.rows = std::min(L, chunk) + l_h - 1;
+  o.slot_bytes = 4 * round256(o.rows * D * elem);
+  o.off_h = kHostSlots * o.slot_bytes;
+  o.bytes = o.off_h + round256(G * l_h * 4);
+  return o;
+}
+
+int host_pipe(HostPipe *&hp) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYENA_ERR_CUDA;
+  hp = &g_host_pipes[dev];
+  HostPipe *h = hp;
+  std::call_once(h->once, [h]() {
+    cudaError_t e = cudaSuccess;
+    for (cudaStream_t *st : {&h->in, &h->comp, &h->out})
+      if (e == cudaSuccess) e = cudaStreamCreateWithFlags(st, cudaStreamNonBlocking);
+    const unsigned fl = cudaEventDisableTiming;
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->start, fl);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->finish, fl);
+    for (int i = 0; i < kHostSlots && e == cudaSuccess; ++i) {
+      e = cudaEventCreateWithFlags(&h->loaded[i], fl);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->done[i], fl);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->freed[i], fl);
+      // a recorded "freed" event lets the first chunk of every slot wait on it unconditionally
+      if (e == cudaSuccess) e = cudaEventRecord(h->freed[i], h->out);
+    }
+    h->err = e;
+  });
+  return h->err == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+int fwd_from_host(const Problem &P, int64_t chunk, void *workspace, size_t workspace_bytes,
+                  cudaStream_t stream) {
+  const int64_t es = P.elem(), D = P.D, hist = P.l_h - 1;
+  const HostLayout lay = host_layout(P.L, D, P.G(), P.l_h, es, chunk);
+  if (!workspace || static_cast<int64_t>(workspace_bytes) < lay.bytes) return HYENA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return HYENA_ERR_MISALIGNED;
+  DeviceState *ds = nullptr;
+  HostPipe *hp = nullptr;
+  if (current_device(ds) != HYENA_OK || host_pipe(hp) != HYENA_OK) return HYENA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(hp->mu);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  float *hd = reinterpret_cast<float *>(ws + lay.off_h);
+  const int64_t tensor_bytes = round256(lay.rows * D * es);
+  const uint8_t *src[3] = {static_cast<const uint8_t *>(P.q), static_cast<const uint8_t *>(P.k),
+                           static_cast<const uint8_t *>(P.v)};
+  uint8_t *yh = static_cast<uint8_t *>(P.y);
+  cudaError_t e = cudaEventRecord(hp->start, stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->in, hp->start, 0);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(hd, P.h, static_cast<size_t>(P.G() * P.l_h * 4), cudaMemcpyHostToDevice,
+                        hp->in);
+  int64_t n = 0;
+  for (int64_t b = 0; b < P.B && e == cudaSuccess; ++b) {
+    for (int64_t t0 = 0; t0 < P.L && e == cudaSuccess; t0 += chunk, ++n) {
+      const int64_t t1 = std::min(P.L, t0 + chunk), s0 = std::max<int64_t>(0, t0 - hist);
+      const int64_t nr = t1 - s0;
+      const int si = static_cast<int>(n % kHostSlots);
+      uint8_t *slot = ws + si * lay.slot_bytes;
+      uint8_t *dev[4] = {slot, slot + tensor_bytes, slot + 2 * tensor_bytes,
+                         slot + 3 * tensor_bytes};
+      const size_t nbytes = static_cast<size_t>(nr * D * es);
+      const int64_t row0 = (b * P.L + s0) * D * es;
+      // copy in once the slot's previous chunk has been copied out
+      e = cudaStreamWaitEvent(hp->in, hp->freed[si], 0);
+      for (int i = 0; i < 3 && e == cudaSuccess; ++i)
+        e = cudaMemcpyAsync(dev[i], src[i] + row0, nbytes, cudaMemcpyHostToDevice, hp->in);
+      if (e == cudaSuccess) e = cudaEventRecord(hp->loaded[si], hp->in);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->comp, hp->loaded[si], 0);
+      if (e != cudaSuccess) break;
+      Problem C = P;
+      C.q = dev[0];
+      C.k = dev[1];
+      C.v = dev[2];
+      C.y = dev[3];
+      C.h = hd;
+      C.B = 1;
+      C.L = nr;
+      const int rc = run(C, HYENA_ALGO_AUTO, hp->comp);
+      if (rc != HYENA_OK) return rc;
+      e = cudaEventRecord(hp->done[si], hp->comp);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->out, hp->done[si], 0);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(yh + (b * P.L + t0) * D * es, dev[3] + (t0 - s0) * D * es,
+                            static_cast<size_t>((t1 - t0) * D * es), cudaMemcpyDeviceToHost,
+                            hp->out);
+      if (e == cudaSuccess) e = cudaEventRecord(hp->freed[si], hp->out);
+    }
+  }
+  if (e == cudaSuccess) e = cudaEventRecord(hp->finish, hp->out);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, hp->finish, 0);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
 extern "C" {
 
 int hyena_conv_fwd(const void *q, const void *k, const void *v, const float *h, void *y,
@@ -991,5 +1112,27 @@ const char *hyena_status_string(int status) {
 }
 
 int hyena_abi_version(void) { return 1; }
+
+int64_t hyena_conv_fwd_from_host_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g,
+                                                 int l_h, int dtype, int64_t chunk) {
+  if (B < 0 || L < 0 || D < 1 || d_g < 1 || D % d_g != 0 || l_h < 1 || chunk < 1 ||
+      (dtype != HYENA_DTYPE_BF16 && dtype != HYENA_DTYPE_F32))
+    return -HYENA_ERR_INVALID_ARG;
+  if (B == 0 || L == 0) return 0;
+  const int64_t es = dtype == HYENA_DTYPE_F32 ? 4 : 2;
+  return host_layout(L, D, D / d_g, l_h, es, chunk).bytes;
+}
+
+int hyena_conv_fwd_from_host(const void *q, const void *k, const void *v, const float *h,
+                             void *y, int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                             int dtype, int64_t chunk, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
+  const Problem P{q, k, v, h, y, B, L, D, d_g, l_h, l_b, dtype};
+  const int rc = validate(P);  // shapes, null pointers, element alignment, y against the inputs
+  if (rc == kEmpty) return HYENA_OK;
+  if (rc != HYENA_OK) return rc;
+  if (chunk < 1) return HYENA_ERR_INVALID_ARG;
+  return fwd_from_host(P, chunk, workspace, workspace_bytes, stream);
+}
 
 }  // extern "C"

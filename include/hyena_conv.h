@@ -150,6 +150,42 @@ int hyena_conv_fwd_fft(const void *q, const void *k, const void *v, const float 
                        void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Host-only: bytes of device workspace hyena_conv_fwd_from_host needs (a multiple of 256), or
+ * minus HYENA_ERR_INVALID_ARG for a bad shape, dtype or chunk < 1.  Touches no device.  The
+ * workspace holds three chunk slots of q, k, v and y, (min(L, chunk) + l_h - 1) rows of D
+ * elements each, and the filters: 12 (min(L, chunk) + l_h - 1) D elem + 4 (D / d_g) l_h
+ * bytes, each buffer rounded up to 256 bytes.
+ */
+int64_t hyena_conv_fwd_from_host_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g,
+                                                 int l_h, int dtype, int64_t chunk);
+
+/*
+ * The forward of hyena_conv_fwd_ex (AUTO) with q, k, v, h and y in HOST memory: the
+ * end-to-end call, host-to-device copies, kernels and device-to-host copies queued by the
+ * library.  Each sequence is processed in chunks of `chunk` rows: rows [t0, t1) travel to the
+ * device with the l_h - 1 rows before them (page 04, Sec. 3: output chunk n needs only input
+ * chunk n-1), are computed as a sequence of their own, which gives exactly the whole
+ * sequence's rows t0 .. t1-1, and come back into y.  Three chunk slots of the workspace rotate
+ * over three library streams (copy in, compute, copy out) so that the copies in both
+ * directions overlap the kernels; with page-locked (pinned) host buffers every copy is
+ * asynchronous, with pageable ones the copies still complete correctly but may serialise.
+ *
+ * q, k, v, y: HOST [B, L, D] of `dtype`; h: HOST [D / d_g, l_h] fp32.  workspace: DEVICE,
+ * 256-byte aligned, at least hyena_conv_fwd_from_host_workspace_bytes() bytes, owned by the
+ * caller.  The call is ordered after the work already queued on `stream`, and `stream` waits
+ * for its last copy: synchronise `stream` before reading y, and keep the host buffers and the
+ * workspace alive until then.  The library's streams and events are created once per device;
+ * calls on one device are serialised on the host.  Errors: as hyena_conv_fwd_ex for the
+ * shape and pointers, HYENA_ERR_INVALID_ARG for chunk < 1 or a missing or short workspace,
+ * HYENA_ERR_MISALIGNED for a workspace not 256-byte aligned, HYENA_ERR_CUDA when a copy or
+ * launch fails (work queued before the failure stays queued).
+ */
+int hyena_conv_fwd_from_host(const void *q, const void *k, const void *v, const float *h,
+                             void *y, int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
+                             int dtype, int64_t chunk, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
+
+/*
  * Host-only: the algorithm (enum hyena_algo, > 0) that HYENA_ALGO_AUTO would run for this
  * problem and these pointers, or minus an error code.  Touches no device.
  */

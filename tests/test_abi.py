@@ -186,6 +186,34 @@ def test_fft_validation(lib):
     assert f(q, k, v, h, y, 0, 64, 128, 64, 16, 16, 0, None, 0, None) == 0  # empty: no launch
 
 
+def test_from_host_workspace_bytes(lib):
+    f = lib.hyena_conv_fwd_from_host_workspace_bytes
+    # MR, 2048-row chunks: 3 slots x 4 tensors x (2048 + 127) rows x 4096 x 2 B, plus h
+    assert f(1, 8192, 4096, 64, 128, 0, 2048) == 3 * 4 * 2175 * 4096 * 2 + 64 * 128 * 4
+    # chunk longer than L: a slot tensor holds L + l_h - 1 = 104 rows of 12 fp32 (4992 B,
+    # rounded up to 5120); h (2 x 5 floats) rounds up to 256
+    assert f(2, 100, 12, 6, 5, 1, 4096) == 3 * 4 * 5120 + 256
+    assert f(1, 100, 64, 63, 5, 0, 64) == -1        # D % d_g
+    assert f(1, 100, 64, 64, 5, 0, 0) == -1         # chunk < 1
+    assert f(1, 100, 64, 64, 5, 7, 64) == -1        # dtype
+    assert f(0, 100, 64, 64, 5, 0, 64) == 0
+
+
+def test_from_host_validation(lib):
+    f = lib.hyena_conv_fwd_from_host
+    q, k, v, h, y = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+    need = lib.hyena_conv_fwd_from_host_workspace_bytes(1, 64, 128, 64, 16, 0, 32)
+    a = (1, 64, 128, 64, 16, 16, 0, 32)               # B, L, D, d_g, l_h, l_b, dtype, chunk
+    assert f(q, k, v, h, y, *a, None, need, None) == 1              # no workspace
+    assert f(q, k, v, h, y, *a, 0x600000, need - 1, None) == 1      # short workspace
+    assert f(q, k, v, h, y, *a, 0x600010, need, None) == 3          # workspace not 256-aligned
+    assert f(q, k, v, h, y, 1, 64, 128, 64, 16, 16, 0, 0, 0x600000, need, None) == 1  # chunk 0
+    assert f(None, k, v, h, y, *a, 0x600000, need, None) == 1       # null input
+    assert f(q, k, v, h, q, *a, 0x600000, need, None) == 1          # y aliases q
+    assert f(q + 1, k, v, h, y, *a, 0x600000, need, None) == 3      # misaligned element
+    assert f(q, k, v, h, y, 0, 64, 128, 64, 16, 16, 0, 32, None, 0, None) == 0  # empty
+
+
 def test_device_status_needs_out(lib):
     assert lib.hyena_device_status(None, 0) == 1
 

@@ -280,16 +280,32 @@ def test_mr_1m_sampled():
     _sampled(WORKLOADS["mr_1m"], 64, l_slice=1 << 16)
 
 
-@pytest.mark.parametrize("chunk", [300, 2048])
-def test_from_host_pipeline(chunk):
-    """Host tensors in, host tensor out: sequence chunks with l_h - 1 history rows each, copies
-    overlapped with compute; the result matches the oracle like the device path."""
-    wl = custom("host", 2, 1000, 128, 64, 128, 64, "bf16", "mr", seed=12)
+HOST_CASES = [
+    # name, B, L, D, d_g, l_h, l_b, dtype, chunk, pinned
+    ("mr_chunks", 2, 1000, 128, 64, 128, 64, "bf16", 300, True),
+    ("mr_one_chunk", 2, 1000, 128, 64, 128, 64, "bf16", 2048, True),
+    ("f32_ragged", 3, 777, 96, 32, 33, 32, "f32", 250, True),
+    ("se_window", 1, 5000, 256, 16, 7, 16, "bf16", 1024, True),
+    ("chunk_shorter_than_halo", 1, 400, 64, 64, 100, 64, "bf16", 40, True),
+    ("pageable", 2, 600, 128, 64, 64, 64, "bf16", 256, False),
+]
+
+
+@pytest.mark.parametrize("case", HOST_CASES, ids=[c[0] for c in HOST_CASES])
+def test_from_host_pipeline(case):
+    """Host tensors in, host tensor out through the C entry point: sequence chunks with l_h - 1
+    history rows each, copies overlapped with compute over three rotating device slots; the
+    result matches the oracle like the device path, and a second call (slots and events
+    reused) gives the same bits."""
+    name, B, L, D, d_g, l_h, l_b, dt, chunk, pinned = case
+    wl = custom(name, B, L, D, d_g, l_h, l_b, dt, "mr" if l_h > 16 else "se", seed=12)
     q, k, v, h = (x.cpu() for x in make_inputs(wl, device="cuda"))
-    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
-    y = g.hyena_conv_fwd_from_host(qh, kh, vh, h, wl.d_g, wl.l_b, chunk=chunk)
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v)) if pinned else (q, k, v)
+    out = None if pinned else torch.empty_like(q)
+    y = g.hyena_conv_fwd_from_host(qh, kh, vh, h, wl.d_g, wl.l_b, chunk=chunk, out=out)
     torch.cuda.synchronize()
     U.assert_parity(y, U.oracle_full(q, k, v, h, wl.d_g), q.dtype)
-    y2 = g.hyena_conv_fwd_from_host(qh, kh, vh, h, wl.d_g, wl.l_b, chunk=chunk)  # slots reused
+    y2 = g.hyena_conv_fwd_from_host(qh, kh, vh, h, wl.d_g, wl.l_b, chunk=chunk)
     torch.cuda.synchronize()
     assert torch.equal(y, y2)
+    assert g.hyena_device_status(clear=True) == 0
