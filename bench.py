@@ -474,13 +474,10 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = D.max_over_ranks(e0.elapsed_time(e1), device=dev)
-        # bytes the call copies: h once; q, k, v of every chunk with its l_h - 1 history rows
-        chunk, es = 2048, qh.element_size()
-        rows_in = sum(min(wl.L, t0 + chunk) - max(0, t0 - (wl.l_h - 1))
-                      for t0 in range(0, wl.L, chunk))
+        # bytes the call copies: h once, every row of q, k, v once (a chunk's history rows
+        # are copied on the device from the previous chunk), every row of y once
         e2e = {"value": world * wl.tokens * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": hh.numel() * hh.element_size()
-               + 3 * wl.B * rows_in * wl.D * es,
+               "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (qh, kh, vh, hh)),
                "d2h_bytes_per_step": yh.numel() * yh.element_size(),
                "steps": args.e2e_steps,
                "api": "hyena_conv_fwd_from_host (C ABI; 2048-row chunks, three streams)"}

@@ -882,17 +882,33 @@ int fwd_from_host(const Problem &P, int64_t chunk, void *workspace, size_t works
   for (int64_t b = 0; b < P.B && e == cudaSuccess; ++b) {
     for (int64_t t0 = 0; t0 < P.L && e == cudaSuccess; t0 += chunk, ++n) {
       const int64_t t1 = std::min(P.L, t0 + chunk), s0 = std::max<int64_t>(0, t0 - hist);
-      const int64_t nr = t1 - s0;
+      const int64_t nr = t1 - s0, nh = t0 - s0;  // rows in the slot, of which history
       const int si = static_cast<int>(n % kHostSlots);
       uint8_t *slot = ws + si * lay.slot_bytes;
       uint8_t *dev[4] = {slot, slot + tensor_bytes, slot + 2 * tensor_bytes,
                          slot + 3 * tensor_bytes};
-      const size_t nbytes = static_cast<size_t>(nr * D * es);
-      const int64_t row0 = (b * P.L + s0) * D * es;
-      // copy in once the slot's previous chunk has been copied out
+      const size_t row_bytes = static_cast<size_t>(D * es), hbytes = nh * row_bytes;
+      const size_t nbytes = static_cast<size_t>(t1 - t0) * row_bytes;
+      const int64_t row0 = (b * P.L + t0) * D * es;
+      // copy in once the slot's previous chunk has been copied out: rows [t0, t1) from the
+      // host; the history rows of k and v from the previous chunk's slot (already on the device,
+      // queued earlier on the same stream); the history rows of q only feed outputs that are
+      // dropped, so they are zeroed
       e = cudaStreamWaitEvent(hp->in, hp->freed[si], 0);
       for (int i = 0; i < 3 && e == cudaSuccess; ++i)
-        e = cudaMemcpyAsync(dev[i], src[i] + row0, nbytes, cudaMemcpyHostToDevice, hp->in);
+        e = cudaMemcpyAsync(dev[i] + hbytes, src[i] + row0, nbytes, cudaMemcpyHostToDevice,
+                            hp->in);
+      if (nh > 0 && e == cudaSuccess) {
+        // the previous chunk of this sequence (t0 > 0) sits in slot n - 1, its rows from s0p
+        const int sp = static_cast<int>((n + kHostSlots - 1) % kHostSlots);
+        const int64_t s0p = std::max<int64_t>(0, t0 - chunk - hist);
+        uint8_t *prev = ws + sp * lay.slot_bytes;
+        const size_t off = static_cast<size_t>(s0 - s0p) * row_bytes;
+        e = cudaMemsetAsync(dev[0], 0, hbytes, hp->in);
+        for (int i = 1; i < 3 && e == cudaSuccess; ++i)
+          e = cudaMemcpyAsync(dev[i], prev + i * tensor_bytes + off, hbytes,
+                              cudaMemcpyDeviceToDevice, hp->in);
+      }
       if (e == cudaSuccess) e = cudaEventRecord(hp->loaded[si], hp->in);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->comp, hp->loaded[si], 0);
       if (e != cudaSuccess) break;

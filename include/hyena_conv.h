@@ -162,10 +162,11 @@ int64_t hyena_conv_fwd_from_host_workspace_bytes(int64_t B, int64_t L, int64_t D
 /*
  * The forward of hyena_conv_fwd_ex (AUTO) with q, k, v, h and y in HOST memory: the
  * end-to-end call, host-to-device copies, kernels and device-to-host copies queued by the
- * library.  Each sequence is processed in chunks of `chunk` rows: rows [t0, t1) travel to the
- * device with the l_h - 1 rows before them (page 04, Sec. 3: output chunk n needs only input
- * chunk n-1), are computed as a sequence of their own, which gives exactly the whole
- * sequence's rows t0 .. t1-1, and come back into y.  Three chunk slots of the workspace rotate
+ * library.  Each sequence is processed in chunks of `chunk` rows: rows [t0, t1) of q, k, v
+ * travel to the device once, the l_h - 1 rows of k and v before them (page 04, Sec. 3: output
+ * chunk n needs only input chunk n-1) are copied on the device from the previous chunk, the
+ * block is computed as a sequence of its own, which gives exactly the whole sequence's rows
+ * t0 .. t1-1, and those rows come back into y.  Three chunk slots of the workspace rotate
  * over three library streams (copy in, compute, copy out) so that the copies in both
  * directions overlap the kernels; with page-locked (pinned) host buffers every copy is
  * asynchronous, with pageable ones the copies still complete correctly but may serialise.
