@@ -361,6 +361,9 @@ def hyena_conv_fwd_from_host(q, k, v, h, d_g, l_b, out=None, device="cuda", stre
             _HOST_WS.clear()
             workspace = _HOST_WS[key] = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream(dev) if stream is None else stream
+    # the library's streams finish before `st` goes on: the allocator must not hand the
+    # workspace out again before `st` has passed this call
+    workspace.record_stream(st)
     with torch.cuda.device(dev):
         _native.check("hyena_conv_fwd_from_host", _native.lib().hyena_conv_fwd_from_host(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), h.data_ptr(), out.data_ptr(), B, L, D,

@@ -4,6 +4,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <limits>
 #include <mutex>
@@ -303,17 +305,18 @@ constexpr int kWindowMinRows = 32;  // halo (l_h - 1 rows) at most ~half a run a
 template <typename T, int LH>
 int launch_window_lh(const Problem &P, WindowParams wp, int sm_count, cudaStream_t s) {
   const auto kernel = hyena::cc::fir_window_kernel<T, LH>;
-  static int resident[kMaxDevices];  // blocks per SM, per device (0: not yet queried)
+  static std::atomic<int> resident[kMaxDevices];  // blocks per SM per device (0: not queried)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYENA_ERR_CUDA;
-  if (resident[dev] == 0) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, hyena::cc::kWindowBlock, 0) !=
-        cudaSuccess)
+  int per_sm = resident[dev].load(std::memory_order_relaxed);
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, hyena::cc::kWindowBlock,
+                                                      0) != cudaSuccess)
       return HYENA_ERR_CUDA;
-    resident[dev] = n > 0 ? n : 1;
+    per_sm = per_sm > 0 ? per_sm : 1;
+    resident[dev].store(per_sm, std::memory_order_relaxed);
   }
-  const long long wave = static_cast<long long>(sm_count) * resident[dev] * hyena::cc::kWindowBlock;
+  const long long wave = static_cast<long long>(sm_count) * per_sm * hyena::cc::kWindowBlock;
   const long long units = wp.B * wp.cv;  // thread columns per time block
   long long rows = kWindowRows;
   const long long tb_per_wave = wave / units;  // time blocks one wave holds
@@ -815,7 +818,7 @@ struct HostPipe {
   cudaError_t err = cudaSuccess;
   cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
   cudaEvent_t start = nullptr, loaded[kHostSlots] = {}, done[kHostSlots] = {},
-              freed[kHostSlots] = {}, finish = nullptr;
+              freed[kHostSlots] = {}, tail_in = nullptr, tail_comp = nullptr, finish = nullptr;
 };
 HostPipe g_host_pipes[kMaxDevices];
 
@@ -844,7 +847,8 @@ int host_pipe(HostPipe *&hp) {
       if (e == cudaSuccess) e = cudaStreamCreateWithFlags(st, cudaStreamNonBlocking);
     const unsigned fl = cudaEventDisableTiming;
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->start, fl);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->finish, fl);
+    for (cudaEvent_t *ev : {&h->finish, &h->tail_in, &h->tail_comp})
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, fl);
     for (int i = 0; i < kHostSlots && e == cudaSuccess; ++i) {
       e = cudaEventCreateWithFlags(&h->loaded[i], fl);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->done[i], fl);
@@ -879,7 +883,8 @@ int fwd_from_host(const Problem &P, int64_t chunk, void *workspace, size_t works
     e = cudaMemcpyAsync(hd, P.h, static_cast<size_t>(P.G() * P.l_h * 4), cudaMemcpyHostToDevice,
                         hp->in);
   int64_t n = 0;
-  for (int64_t b = 0; b < P.B && e == cudaSuccess; ++b) {
+  int status = HYENA_OK;
+  for (int64_t b = 0; b < P.B && e == cudaSuccess && status == HYENA_OK; ++b) {
     for (int64_t t0 = 0; t0 < P.L && e == cudaSuccess; t0 += chunk, ++n) {
       const int64_t t1 = std::min(P.L, t0 + chunk), s0 = std::max<int64_t>(0, t0 - hist);
       const int64_t nr = t1 - s0, nh = t0 - s0;  // rows in the slot, of which history
@@ -920,8 +925,8 @@ int fwd_from_host(const Problem &P, int64_t chunk, void *workspace, size_t works
       C.h = hd;
       C.B = 1;
       C.L = nr;
-      const int rc = run(C, HYENA_ALGO_AUTO, hp->comp);
-      if (rc != HYENA_OK) return rc;
+      status = run(C, HYENA_ALGO_AUTO, hp->comp);
+      if (status != HYENA_OK) break;
       e = cudaEventRecord(hp->done[si], hp->comp);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->out, hp->done[si], 0);
       if (e == cudaSuccess)
@@ -931,9 +936,18 @@ int fwd_from_host(const Problem &P, int64_t chunk, void *workspace, size_t works
       if (e == cudaSuccess) e = cudaEventRecord(hp->freed[si], hp->out);
     }
   }
-  if (e == cudaSuccess) e = cudaEventRecord(hp->finish, hp->out);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, hp->finish, 0);
-  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+  // `stream` waits for everything queued on the three streams, also after an error, so that
+  // synchronising it covers every copy that still reads the caller's buffers
+  cudaError_t t = cudaEventRecord(hp->tail_in, hp->in);
+  if (t == cudaSuccess) t = cudaEventRecord(hp->tail_comp, hp->comp);
+  if (t == cudaSuccess) t = cudaStreamWaitEvent(hp->out, hp->tail_in, 0);
+  if (t == cudaSuccess) t = cudaStreamWaitEvent(hp->out, hp->tail_comp, 0);
+  if (t == cudaSuccess) t = cudaEventRecord(hp->finish, hp->out);
+  if (t == cudaSuccess) t = cudaStreamWaitEvent(stream, hp->finish, 0);
+  if (status != HYENA_OK) return status;
+  return e == cudaSuccess && t == cudaSuccess && cudaGetLastError() == cudaSuccess
+             ? HYENA_OK
+             : HYENA_ERR_CUDA;
 }
 
 extern "C" {
