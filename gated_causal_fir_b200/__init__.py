@@ -177,7 +177,7 @@ def hyena_conv_fwd_f32(q, k, v, h, d_g, l_b, y=None, stream=None):
 def hyena_select_algo(B, L, D, d_g, l_h, l_b, dtype=HYENA_DTYPE_BF16, ptrs=(16, 16, 16, 16, 16)):
     """Host-only: the algorithm AUTO would run (HYENA_ALGO_*), or raises HyenaError.
 
-    ``ptrs`` are the (q, k, v, h, y) addresses to judge alignment by (plain integers); the
+    ``ptrs`` are the (q, k, v, h, y) addresses whose alignment counts (plain integers); the
     defaults stand for distinct 16-byte aligned buffers.
     """
     n = B * L * D * (4 if dtype == HYENA_DTYPE_F32 else 2)
