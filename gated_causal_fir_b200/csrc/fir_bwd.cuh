@@ -6,8 +6,8 @@
 //   dz = q * dy,  dx[t] = sum_j h[j] dz[t + j]   (transposed Toeplitz: anti-causal)
 //   dk = dx * v,  dv = dx * k                      -- fir_bwd_dx_kernel (one pass, both outputs)
 //   dh[g][j] = sum_{b, t, c in g} dz[b,t,c] x[b,t-j,c]
-//                            -- two passes as on the page: fir_bwd_dh_partial_kernel writes one
-//                               partial per (sequence, 64-row chunk, channel piece), coalesced
+//                            -- two passes as on the page: fir_bwd_dh_partial_kernel (or, for
+//                               short filters, fir_bwd_window_kernel) writes partials, coalesced
 //                               along j; fir_bwd_dh_reduce_kernel sums them in a fixed order.
 // All arithmetic is fp32 with products formed before rounding (exact for bf16 inputs).
 #pragma once
@@ -118,22 +118,148 @@ __global__ void __launch_bounds__(kDhTaps)
   }
 }
 
-// Pass 2.  dh[g][j] = sum over b, chunk and the group's pieces of the partials, in that order.
-__global__ void __launch_bounds__(256)
+// Short filters (l_h <= 16): dk, dv and the dh partials in one pass over q, k, v, dy, the
+// backward counterpart of cc::fir_window_kernel.  A thread owns VN channels (16 bytes, all in one
+// group) over a run of rows [t0, t1) and walks it in DECREASING time with a register window of
+// dz = q dy over rows t .. t + l_h - 1 (the l_h - 1 rows after the run are its halo, zero past
+// L):
+//   dx[t] = sum_j h[j] dz[t + j]       (the transposed Toeplitz product, taps in order j = 0 ..)
+//   dk[t] = dx[t] v[t],  dv[t] = dx[t] k[t]
+//   dh[j] += sum_{c in thread} dz[t + j, c] x[t, c],  x = k v
+// so every (t, j) pair of the filter gradient is met once, at the run that owns row t.  The
+// thread's l_h partial sums go to partial[gid][j] (gid = (b n_tb + tb) cv + channel vector):
+// the layout fir_bwd_dh_reduce_kernel reads with one piece per channel vector.
+#ifndef HYENA_BWD_WINDOW_BLOCK
+#define HYENA_BWD_WINDOW_BLOCK 128
+#endif
+constexpr int kBwdWindowBlock = HYENA_BWD_WINDOW_BLOCK;
+
+template <typename T, int LH>
+__global__ void __launch_bounds__(kBwdWindowBlock)
+    fir_bwd_window_kernel(const T *__restrict__ q, const T *__restrict__ k,
+                          const T *__restrict__ v, const float *__restrict__ h,
+                          const T *__restrict__ dy, T *__restrict__ dk, T *__restrict__ dv,
+                          float *__restrict__ partial, const cc::WindowParams p) {
+  using V = cc::Vec<T>;
+  constexpr int VN = V::N;
+  constexpr int U = LH <= 8 ? 4 : 2;  // rows of loads issued before their arithmetic
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gid >= p.B * p.n_tb * p.cv) return;
+  const long long cvi = gid % p.cv;
+  const long long rest = gid / p.cv;
+  const long long tb = rest % p.n_tb;
+  const long long b = rest / p.n_tb;
+  const long long c0 = cvi * VN;
+  const long long g = c0 / p.d_g;
+
+  float hr[LH];
+#pragma unroll
+  for (int j = 0; j < LH; ++j) hr[j] = __ldg(h + g * LH + j);
+  float zw[LH][VN];  // zw[j] = dz at time t + j
+  float dh[LH];
+#pragma unroll
+  for (int j = 0; j < LH; ++j) {
+    dh[j] = 0.f;
+#pragma unroll
+    for (int e = 0; e < VN; ++e) zw[j][e] = 0.f;
+  }
+  const long long t0 = tb * p.rows;
+  const long long t1 = min(t0 + p.rows, p.L);
+  const long long seq = b * p.L * p.D + c0;
+
+  // Halo: rows t1 + l_h - 2 down to t1 (zero from L on), so that the window is complete at the
+  // first row of the run.
+#pragma unroll
+  for (int s = LH - 2; s >= 0; --s) {
+#pragma unroll
+    for (int j = LH - 1; j >= 1; --j)
+#pragma unroll
+      for (int e = 0; e < VN; ++e) zw[j][e] = zw[j - 1][e];
+    const long long t = t1 + s;
+    if (t < p.L) {
+      float qq[VN], gg[VN];
+      V::unpack(V::load(q + seq + t * p.D), qq);
+      V::unpack(V::load(dy + seq + t * p.D), gg);
+#pragma unroll
+      for (int e = 0; e < VN; ++e) zw[0][e] = qq[e] * gg[e];
+    } else {
+#pragma unroll
+      for (int e = 0; e < VN; ++e) zw[0][e] = 0.f;
+    }
+  }
+
+  for (long long t = t1 - 1; t >= t0; t -= U) {
+    uint4 qr[U], gr[U], kr[U], vr[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (t - u >= t0) {
+        const long long off = seq + (t - u) * p.D;
+        qr[u] = V::load(q + off);
+        gr[u] = V::load(dy + off);
+        kr[u] = V::load(k + off);
+        vr[u] = V::load(v + off);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (t - u >= t0) {
+#pragma unroll
+        for (int j = LH - 1; j >= 1; --j)
+#pragma unroll
+          for (int e = 0; e < VN; ++e) zw[j][e] = zw[j - 1][e];
+        float qq[VN], gg[VN], kk[VN], vv[VN], ok[VN], ov[VN];
+        V::unpack(qr[u], qq);
+        V::unpack(gr[u], gg);
+        V::unpack(kr[u], kk);
+        V::unpack(vr[u], vv);
+#pragma unroll
+        for (int e = 0; e < VN; ++e) zw[0][e] = qq[e] * gg[e];
+#pragma unroll
+        for (int e = 0; e < VN; ++e) {
+          float dx = 0.f;
+#pragma unroll
+          for (int j = 0; j < LH; ++j) dx = fmaf(hr[j], zw[j][e], dx);
+          ok[e] = dx * vv[e];
+          ov[e] = dx * kk[e];
+          const float x = kk[e] * vv[e];
+#pragma unroll
+          for (int j = 0; j < LH; ++j) dh[j] = fmaf(zw[j][e], x, dh[j]);
+        }
+        const long long off = seq + (t - u) * p.D;
+        V::store(dk + off, ok);
+        V::store(dv + off, ov);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < LH; ++j) partial[gid * LH + j] = dh[j];
+}
+
+// Pass 2.  dh[g][j] = sum over b, chunk and the group's pieces of the partials.  One warp per
+// output: lane i adds the terms i, i + 32, ... (term = (b, chunk, piece), piece fastest) in
+// that order, then the 32 lane sums meet in a fixed butterfly (IEEE addition is commutative, so
+// every lane ends with the same bits): deterministic, and the G l_h outputs spread over
+// G l_h warps instead of as many threads.
+constexpr int kReduceBlock = 256;
+__global__ void __launch_bounds__(kReduceBlock)
     fir_bwd_dh_reduce_kernel(const float *__restrict__ partial, float *__restrict__ dh, int B,
                              int nchunk, int npieces, int pieces_per_group, int G, int l_h) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (kReduceBlock / 32);
   const long long n = static_cast<long long>(G) * l_h;
-  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int g = static_cast<int>(e / l_h), j = static_cast<int>(e % l_h);
+  const int terms = B * nchunk * pieces_per_group;  // < 2^31 (checked by the host)
+  for (long long w = static_cast<long long>(blockIdx.x) * (kReduceBlock / 32) + threadIdx.x / 32;
+       w < n; w += warps) {
+    const int g = static_cast<int>(w / l_h), j = static_cast<int>(w % l_h);
+    const float *pg = partial + static_cast<long long>(g) * pieces_per_group * l_h + j;
     float s = 0.f;
-    for (int b = 0; b < B; ++b)
-      for (int ch = 0; ch < nchunk; ++ch) {
-        const float *row = partial + ((static_cast<long long>(b) * nchunk + ch) * npieces +
-                                      static_cast<long long>(g) * pieces_per_group) * l_h + j;
-        for (int pc = 0; pc < pieces_per_group; ++pc) s += row[static_cast<long long>(pc) * l_h];
-      }
-    dh[e] = s;
+    for (int i = lane; i < terms; i += 32) {
+      const int pc = i % pieces_per_group, bc = i / pieces_per_group;  // bc = b nchunk + chunk
+      s += pg[(static_cast<long long>(bc) * npieces + pc) * l_h];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) dh[w] = s;
   }
 }
 

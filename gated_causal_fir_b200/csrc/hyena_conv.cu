@@ -302,29 +302,45 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
 #endif
 constexpr int kWindowMinRows = 32;  // halo (l_h - 1 rows) at most ~half a run at l_h = 16
 
+// Resident blocks per SM of `kernel` at `block` threads on the current device, queried once per
+// (kernel, device) through the caller's cache.
+template <typename K>
+int resident_blocks(K kernel, int block, std::atomic<int> (&cache)[kMaxDevices], int &per_sm) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYENA_ERR_CUDA;
+  per_sm = cache[dev].load(std::memory_order_relaxed);
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, block, 0) != cudaSuccess)
+      return HYENA_ERR_CUDA;
+    per_sm = per_sm > 0 ? per_sm : 1;
+    cache[dev].store(per_sm, std::memory_order_relaxed);
+  }
+  return HYENA_OK;
+}
+
+// Run length of the window kernels: with `units` thread columns per time block and `wave`
+// resident threads, the rows that make the whole problem one full wave.
+long long window_rows(long long units, long long L, long long wave) {
+  long long rows = kWindowRows;
+  const long long tb_per_wave = wave / units;  // time blocks one wave holds
+  if (HYENA_WINDOW_WAVE && tb_per_wave >= 1 && units * ((L + kWindowRows - 1) / kWindowRows) <= wave) {
+    rows = (L + tb_per_wave - 1) / tb_per_wave;  // ceil(L / rows) <= tb_per_wave
+    rows = std::max<long long>(rows, kWindowMinRows);
+    rows = std::min<long long>(rows, kWindowRows);
+  }
+  return rows;
+}
+
 template <typename T, int LH>
 int launch_window_lh(const Problem &P, WindowParams wp, int sm_count, cudaStream_t s) {
   const auto kernel = hyena::cc::fir_window_kernel<T, LH>;
   static std::atomic<int> resident[kMaxDevices];  // blocks per SM per device (0: not queried)
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYENA_ERR_CUDA;
-  int per_sm = resident[dev].load(std::memory_order_relaxed);
-  if (per_sm == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, hyena::cc::kWindowBlock,
-                                                      0) != cudaSuccess)
-      return HYENA_ERR_CUDA;
-    per_sm = per_sm > 0 ? per_sm : 1;
-    resident[dev].store(per_sm, std::memory_order_relaxed);
-  }
+  int per_sm = 0;
+  if (resident_blocks(kernel, hyena::cc::kWindowBlock, resident, per_sm) != HYENA_OK)
+    return HYENA_ERR_CUDA;
   const long long wave = static_cast<long long>(sm_count) * per_sm * hyena::cc::kWindowBlock;
   const long long units = wp.B * wp.cv;  // thread columns per time block
-  long long rows = kWindowRows;
-  const long long tb_per_wave = wave / units;  // time blocks one wave holds
-  if (HYENA_WINDOW_WAVE && tb_per_wave >= 1 && units * ((wp.L + kWindowRows - 1) / kWindowRows) <= wave) {
-    rows = (wp.L + tb_per_wave - 1) / tb_per_wave;  // ceil(L / rows) <= tb_per_wave
-    rows = std::max<long long>(rows, kWindowMinRows);
-    rows = std::min<long long>(rows, kWindowRows);
-  }
+  const long long rows = window_rows(units, wp.L, wave);
   wp.rows = static_cast<int>(rows);
   wp.n_tb = (wp.L + rows - 1) / rows;
   const long long threads = units * wp.n_tb;
@@ -452,10 +468,27 @@ int64_t tc_bwd_bytes_bound(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
   return tc_bwd_layout(B * G + 2 * grid, grid, l_h).bytes;
 }
 
-int64_t bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
+// Partials of fir_bwd_window_kernel for any dtype: one per thread (4 channels at fp32) and time
+// block.  With `min_rows`-row time blocks (the shortest run the launch picks) every run length
+// fits; with one time block the launch lengthens the runs to fit whatever it is given.
+int64_t window_bwd_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h, int64_t min_rows) {
+  if (l_h > kMaxWindowTaps || d_g % 4 != 0) return 0;
+  return round256(B * ((L + min_rows - 1) / min_rows) * (D / 4) * l_h * 4);
+}
+
+// The workspace a backward call needs at least (every algorithm runs in it) ...
+int64_t bwd_required_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
   const int64_t cc = round256(bwd_plan(B, L, D, d_g, l_h).partial_floats * 4);
   const int64_t tc = tc_bwd_bytes_bound(B, L, D, d_g, l_h);
-  return cc > tc ? cc : tc;
+  const int64_t win = window_bwd_bytes(B, L, D, d_g, l_h, std::max<int64_t>(L, 1));
+  return std::max(cc, std::max(tc, win));
+}
+
+// ... and the size hyena_conv_bwd_workspace_bytes reports: enough for the window kernel's
+// shortest runs as well.
+int64_t bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
+  return std::max(bwd_required_bytes(B, L, D, d_g, l_h),
+                  window_bwd_bytes(B, L, D, d_g, l_h, kWindowMinRows));
 }
 
 template <typename T>
@@ -473,7 +506,9 @@ int launch_bwd_cuda_core(const Problem &P, const void *dy, void *dk, void *dv, f
       P.d_g, P.l_h);
   if (cudaGetLastError() != cudaSuccess) return HYENA_ERR_CUDA;
   const BwdPlan b = bwd_plan(P.B, P.L, P.D, P.d_g, P.l_h);
-  if (b.nchunk > 2147483647 || P.B > 65535 || b.npieces > 65535) return HYENA_ERR_UNSUPPORTED;
+  if (b.nchunk > 2147483647 || P.B > 65535 || b.npieces > 65535 ||
+      P.B * b.nchunk * (P.d_g / b.cp) > std::numeric_limits<int32_t>::max())
+    return HYENA_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(b.nchunk), static_cast<unsigned>(b.npieces),
                   static_cast<unsigned>(P.B));
   const int smem = (2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (b.cp + 1) * 4;
@@ -481,13 +516,102 @@ int launch_bwd_cuda_core(const Problem &P, const void *dy, void *dk, void *dv, f
       static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v),
       static_cast<const T *>(dy), partial, P.L, P.D, P.l_h, b.cp);
   if (cudaGetLastError() != cudaSuccess) return HYENA_ERR_CUDA;
-  const long long gn = P.G() * P.l_h;
-  long long rblocks = (gn + 255) / 256;
+  const long long gn = P.G() * P.l_h;  // one warp per output
+  long long rblocks = (gn + hyena::bwd::kReduceBlock / 32 - 1) / (hyena::bwd::kReduceBlock / 32);
   if (rblocks > cap) rblocks = cap;
-  hyena::bwd::fir_bwd_dh_reduce_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
+  hyena::bwd::fir_bwd_dh_reduce_kernel<<<static_cast<unsigned>(rblocks),
+                                         hyena::bwd::kReduceBlock, 0, s>>>(
       partial, dh, static_cast<int>(P.B), b.nchunk, b.npieces, P.d_g / b.cp,
       static_cast<int>(P.G()), P.l_h);
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+// Short filters: fir_bwd_window_kernel (dk, dv and a dh partial per thread) and the fixed-order
+// reduction of the partials (one piece per channel vector).  The run length follows the
+// forward's one-wave rule; it grows where the workspace cannot hold one partial per thread.
+template <typename T, int LH>
+int launch_window_bwd_lh(const Problem &P, WindowParams wp, const void *dy, void *dk, void *dv,
+                         float *dh, float *partial, int64_t partial_floats, int sm_count,
+                         cudaStream_t s) {
+  const auto kernel = hyena::bwd::fir_bwd_window_kernel<T, LH>;
+  static std::atomic<int> resident[kMaxDevices];
+  int per_sm = 0;
+  if (resident_blocks(kernel, hyena::bwd::kBwdWindowBlock, resident, per_sm) != HYENA_OK)
+    return HYENA_ERR_CUDA;
+  const long long wave = static_cast<long long>(sm_count) * per_sm * hyena::bwd::kBwdWindowBlock;
+  const long long units = wp.B * wp.cv;
+  long long rows = window_rows(units, wp.L, wave);
+  const long long max_tb = partial_floats / (units * LH);  // time blocks the workspace holds
+  if (max_tb < 1) return HYENA_ERR_INVALID_ARG;
+  if ((wp.L + rows - 1) / rows > max_tb) rows = (wp.L + max_tb - 1) / max_tb;
+  wp.rows = static_cast<int>(rows);
+  wp.n_tb = (wp.L + rows - 1) / rows;
+  const long long threads = units * wp.n_tb;
+  const long long blocks =
+      (threads + hyena::bwd::kBwdWindowBlock - 1) / hyena::bwd::kBwdWindowBlock;
+  if (blocks > std::numeric_limits<int32_t>::max() || wp.n_tb > std::numeric_limits<int32_t>::max() ||
+      wp.cv > std::numeric_limits<int32_t>::max() ||
+      wp.B * wp.n_tb * (P.d_g / (wp.D / wp.cv)) > std::numeric_limits<int32_t>::max())
+    return HYENA_ERR_UNSUPPORTED;
+  kernel<<<static_cast<unsigned>(blocks), hyena::bwd::kBwdWindowBlock, 0, s>>>(
+      static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v), P.h,
+      static_cast<const T *>(dy), static_cast<T *>(dk), static_cast<T *>(dv), partial, wp);
+  if (cudaGetLastError() != cudaSuccess) return HYENA_ERR_CUDA;
+  const long long gn = P.G() * P.l_h;  // one warp per output
+  long long rblocks = (gn + hyena::bwd::kReduceBlock / 32 - 1) / (hyena::bwd::kReduceBlock / 32);
+  const long long cap = static_cast<long long>(sm_count) * 16;
+  if (rblocks > cap) rblocks = cap;
+  hyena::bwd::fir_bwd_dh_reduce_kernel<<<static_cast<unsigned>(rblocks),
+                                         hyena::bwd::kReduceBlock, 0, s>>>(
+      partial, dh, static_cast<int>(P.B), static_cast<int>(wp.n_tb), static_cast<int>(wp.cv),
+      static_cast<int>(P.d_g / (wp.D / wp.cv)), static_cast<int>(P.G()), P.l_h);
+  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+template <typename T, int LH = 1>
+int launch_window_bwd_dispatch(const Problem &P, const WindowParams &wp, const void *dy,
+                               void *dk, void *dv, float *dh, float *partial,
+                               int64_t partial_floats, int sm_count, cudaStream_t s) {
+  if constexpr (LH <= kMaxWindowTaps) {
+    if (P.l_h == LH)
+      return launch_window_bwd_lh<T, LH>(P, wp, dy, dk, dv, dh, partial, partial_floats,
+                                         sm_count, s);
+    return launch_window_bwd_dispatch<T, LH + 1>(P, wp, dy, dk, dv, dh, partial, partial_floats,
+                                                 sm_count, s);
+  }
+  return HYENA_ERR_UNSUPPORTED;
+}
+
+bool window_bwd_supported(const Problem &P, const void *dy, const void *dk, const void *dv) {
+  const int vec = P.dtype == HYENA_DTYPE_F32 ? 4 : 8;
+  return P.l_h <= kMaxWindowTaps && P.d_g % vec == 0 && aligned(P.q, 16) && aligned(P.k, 16) &&
+         aligned(P.v, 16) && aligned(dy, 16) && aligned(dk, 16) && aligned(dv, 16);
+}
+
+// dq through the forward kernels (dy in the place of q), then fir_bwd_window_kernel and the
+// reduction of its dh partials.
+int run_bwd_window(const Problem &P, const void *dy, void *dq, void *dk, void *dv, float *dh,
+                   void *workspace, size_t workspace_bytes, cudaStream_t s) {
+  Problem F = P;
+  F.q = dy;
+  F.y = dq;
+  const int r = run(F, HYENA_ALGO_AUTO, s);
+  if (r != HYENA_OK) return r;
+  DeviceState *ds = nullptr;
+  if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
+  WindowParams wp{};
+  wp.B = P.B;
+  wp.L = P.L;
+  wp.D = P.D;
+  wp.d_g = P.d_g;
+  wp.cv = P.D / (P.dtype == HYENA_DTYPE_F32 ? 4 : 8);
+  const int64_t floats = static_cast<int64_t>(workspace_bytes / 4);
+  float *partial = static_cast<float *>(workspace);
+  if (P.dtype == HYENA_DTYPE_F32)
+    return launch_window_bwd_dispatch<float>(P, wp, dy, dk, dv, dh, partial, floats,
+                                             ds->sm_count, s);
+  return launch_window_bwd_dispatch<__nv_bfloat16>(P, wp, dy, dk, dv, dh, partial, floats,
+                                                   ds->sm_count, s);
 }
 
 // dq through the forward kernels (dy in the place of q), then the CUDA-core dx/dk/dv and dh
@@ -734,7 +858,7 @@ int validate_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv,
       if (overlaps(outs[i], outs[j], bytes)) return HYENA_ERR_INVALID_ARG;
   }
   if (!workspace ||
-      static_cast<int64_t>(workspace_bytes) < bwd_workspace_bytes(P.B, P.L, P.D, P.d_g, P.l_h))
+      static_cast<int64_t>(workspace_bytes) < bwd_required_bytes(P.B, P.L, P.D, P.d_g, P.l_h))
     return HYENA_ERR_INVALID_ARG;
   return HYENA_OK;
 }
@@ -744,11 +868,13 @@ int validate_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv,
 int select_bwd(const Problem &P, const void *dy, const void *dq, const void *dk, const void *dv,
                int algo) {
   const bool tc = tc_bwd_supported(P, dy, dq, dk, dv);
+  const bool win = window_bwd_supported(P, dy, dk, dv);
   switch (algo) {
-    case HYENA_ALGO_AUTO: return tc ? HYENA_ALGO_TENSOR : HYENA_ALGO_DIRECT;
+    case HYENA_ALGO_AUTO:
+      return tc ? HYENA_ALGO_TENSOR : (win ? HYENA_ALGO_WINDOW : HYENA_ALGO_DIRECT);
     case HYENA_ALGO_TENSOR: return tc ? HYENA_ALGO_TENSOR : -HYENA_ERR_UNSUPPORTED;
+    case HYENA_ALGO_WINDOW: return win ? HYENA_ALGO_WINDOW : -HYENA_ERR_UNSUPPORTED;
     case HYENA_ALGO_DIRECT: return HYENA_ALGO_DIRECT;
-    case HYENA_ALGO_WINDOW: return -HYENA_ERR_UNSUPPORTED;
     default: return -HYENA_ERR_INVALID_ARG;
   }
 }
@@ -765,6 +891,8 @@ int run_bwd(const Problem &P, const void *dy, void *dq, void *dk, void *dv, floa
   if (a < 0) return -a;
   if (a == HYENA_ALGO_TENSOR)
     return launch_tensor_bwd(P, dy, dq, dk, dv, dh, workspace, workspace_bytes, s);
+  if (a == HYENA_ALGO_WINDOW)
+    return run_bwd_window(P, dy, dq, dk, dv, dh, workspace, workspace_bytes, s);
   return run_bwd_cuda_core(P, dy, dq, dk, dv, dh, workspace, s);
 }
 
@@ -1063,7 +1191,7 @@ int hyena_conv_bwd_static_scratch(const void *q, const void *k, const void *v, c
   const int rc = validate(P);
   if (rc != HYENA_OK && rc != kEmpty) return rc;
   if (rc == HYENA_OK &&
-      bwd_workspace_bytes(B, L, D, d_g, l_h) > static_cast<int64_t>(HYENA_BWD_STATIC_SCRATCH_BYTES))
+      bwd_required_bytes(B, L, D, d_g, l_h) > static_cast<int64_t>(HYENA_BWD_STATIC_SCRATCH_BYTES))
     return HYENA_ERR_UNSUPPORTED;
   void *ws = nullptr;
   if (static_scratch(ws) != HYENA_OK) return HYENA_ERR_CUDA;

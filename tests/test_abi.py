@@ -232,6 +232,9 @@ def test_bwd_workspace_bytes(lib):
     assert lib.hyena_conv_bwd_workspace_bytes(1, 8192, 4096, 63, 128) == -1
     assert lib.hyena_conv_bwd_workspace_bytes(0, 8192, 4096, 64, 128) == 0
     assert lib.hyena_conv_bwd_workspace_bytes(1, 1, 6, 6, 5) == 256  # rounded up
+    # SE (l_h = 7, d_g = 16): the window kernel's partials at its shortest runs, one per
+    # 32-row block and 4-channel vector (the fp32 width): 256 x 1024 x 7 floats
+    assert lib.hyena_conv_bwd_workspace_bytes(1, 8192, 4096, 16, 7) == 256 * 1024 * 7 * 4
 
 
 def test_bwd_static_scratch_rejects_oversize_on_host(lib):
@@ -248,10 +251,12 @@ def test_bwd_static_scratch_rejects_oversize_on_host(lib):
 
 
 def test_select_bwd_algo(lib):
-    T, Dd = g.HYENA_ALGO_TENSOR, g.HYENA_ALGO_DIRECT
+    T, Dd, W = g.HYENA_ALGO_TENSOR, g.HYENA_ALGO_DIRECT, g.HYENA_ALGO_WINDOW
     assert g.hyena_select_bwd_algo(1, 8192, 4096, 64, 128, 64) == T   # MR: fused tensor kernel
-    assert g.hyena_select_bwd_algo(1, 8192, 4096, 16, 7, 16) == Dd    # d_g 16: CUDA cores
+    assert g.hyena_select_bwd_algo(1, 8192, 4096, 16, 7, 16) == W     # SE: register window
+    assert g.hyena_select_bwd_algo(1, 8192, 4096, 16, 17, 16) == Dd   # 17 taps: past the window
+    assert g.hyena_select_bwd_algo(1, 8192, 4092, 6, 7, 16) == Dd     # 6-channel groups
     assert g.hyena_select_bwd_algo(1, 8192, 4096, 64, 128, 64, g.HYENA_DTYPE_F32) == Dd
     assert g.hyena_select_bwd_algo(1, 300, 4096, 64, 130, 65) == Dd   # l_h > 129
-    assert g.hyena_select_bwd_algo(1, 300, 96, 32, 16, 16) == Dd
+    assert g.hyena_select_bwd_algo(1, 300, 96, 32, 16, 16) == W
     assert g.hyena_select_bwd_algo(1, 300, 4096, 64, 300, 16) == Dd   # l_h > 2 l_b: block form

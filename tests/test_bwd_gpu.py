@@ -10,6 +10,9 @@ Tolerances:
     u * 64 * sqrt(4096) * sqrt(N / 4096) ~ 2e-6 sqrt(N), i.e. ~2e-6 normwise, so 1e-4 keeps a
     50x margin while a single dropped or doubled term (~1 / sqrt(N) normwise, 1.4e-3 at the MR
     size) still fails.
+  * dh, window path (l_h <= 16): normwise 1e-4, as the CUDA-core path: each thread sums
+    dz[t + j] x[t] over its run (at most 128 rows) and its 4 or 8 channels, a fixed-order sum
+    of those partials follows; the same error estimate holds.
   * dh, tensor path: normwise 2e-3.  Its products take x = k v and dz = q dy rounded to fp16
     (relative error <= 2^-11 each, ~4e-4 rms per product); the sum of N such errors of random
     sign is ~4e-4 sqrt(N), i.e. ~4e-4 / 3.5 ~ 1.2e-4 of max|ref| on average and ~5e-4 at the
@@ -30,12 +33,25 @@ import oracle
 
 pytestmark = pytest.mark.gpu
 
-DH_NORMWISE = {g.HYENA_ALGO_DIRECT: 1e-4, g.HYENA_ALGO_TENSOR: 2e-3}
-ALGOS = {"direct": g.HYENA_ALGO_DIRECT, "tensor": g.HYENA_ALGO_TENSOR}
+DH_NORMWISE = {g.HYENA_ALGO_DIRECT: 1e-4, g.HYENA_ALGO_TENSOR: 2e-3,
+               g.HYENA_ALGO_WINDOW: 1e-4}
+ALGOS = {"direct": g.HYENA_ALGO_DIRECT, "tensor": g.HYENA_ALGO_TENSOR,
+         "window": g.HYENA_ALGO_WINDOW}
 
 
 def _tensor_fits(B, L, D, d_g, l_h, dt):
     return dt == "bf16" and d_g == 64 and D % 64 == 0 and l_h <= 129
+
+
+def _window_fits(B, L, D, d_g, l_h, dt):
+    return l_h <= 16 and d_g % (4 if dt == "f32" else 8) == 0
+
+
+def _fits(algo, shape):
+    if algo == "direct":
+        return True
+    fits = _tensor_fits if algo == "tensor" else _window_fits
+    return fits(*shape[1:6], shape[7])
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -76,7 +92,7 @@ def test_bwd_workload(name):
     dy = make_grad(wl, device="cuda")
     algo = g.hyena_select_bwd_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b,
                                    g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16)
-    assert algo == (g.HYENA_ALGO_TENSOR if name == "mr" else g.HYENA_ALGO_DIRECT)
+    assert algo == (g.HYENA_ALGO_TENSOR if name == "mr" else g.HYENA_ALGO_WINDOW)
     out = g.hyena_conv_bwd(q, k, v, h, dy, wl.d_g, wl.l_b)
     torch.cuda.synchronize()
     ref = oracle.gated_fir_bwd(q, k, v, h, dy, wl.d_g)
@@ -99,8 +115,12 @@ SHAPES = [
     ("long_seq_one_group", 1, 40000, 64, 64, 128, 64, "bf16"),
     ("batched_halo16", 4, 2048, 128, 64, 17, 16, "bf16"),
     ("three_blocks", 2, 900, 192, 64, 64, 64, "bf16"),  # odd block count: unpaired walk
+    ("se_window", 2, 1500, 256, 16, 7, 16, "bf16"),
+    ("window_16_taps", 1, 700, 128, 8, 16, 16, "bf16"),
+    ("window_f32_ragged", 3, 333, 32, 4, 3, 4, "f32"),
+    ("window_runs_short", 2, 20, 64, 16, 7, 16, "bf16"),   # one run shorter than the halo
 ]
-CASES = [(s, a) for s in SHAPES for a in ALGOS if a == "direct" or _tensor_fits(*s[1:6], s[7])]
+CASES = [(s, a) for s in SHAPES for a in ALGOS if _fits(a, s)]
 
 
 @pytest.mark.parametrize("shape,algo", CASES, ids=["%s-%s" % (s[0], a) for s, a in CASES])
@@ -112,6 +132,15 @@ def test_bwd_shapes(shape, algo):
     out = _bwd(q, k, v, h, dy, wl, ALGOS[algo])
     ref = oracle.gated_fir_bwd(q, k, v, h, dy, wl.d_g)
     _check_all(out, ref, q.dtype, ALGOS[algo])
+
+
+def test_bwd_window_unsupported_is_rejected():
+    wl = custom("w17", 1, 300, 128, 16, 17, 16, "bf16")  # 17 taps: past the register window
+    q, k, v, h = make_inputs(wl, device="cuda")
+    dy = make_grad(wl, device="cuda")
+    with pytest.raises(g.HyenaError) as e:
+        _bwd(q, k, v, h, dy, wl, g.HYENA_ALGO_WINDOW)
+    assert e.value.status == 2
 
 
 def test_bwd_tensor_unsupported_is_rejected():
@@ -130,8 +159,7 @@ INT_SHAPES = [
     ("dg32", 1, 1000, 128, 32, 65, 64, "bf16"),
     ("f32", 2, 700, 64, 8, 12, 8, "f32"),
 ]
-INT_CASES = [(s, a) for s in INT_SHAPES for a in ALGOS
-             if a == "direct" or _tensor_fits(*s[1:6], s[7])]
+INT_CASES = [(s, a) for s in INT_SHAPES for a in ALGOS if _fits(a, s)]
 
 
 @pytest.mark.parametrize("shape,algo", INT_CASES,
@@ -152,7 +180,10 @@ def test_integer_exact(shape, algo):
 
 @pytest.mark.parametrize("algo", list(ALGOS))
 def test_bwd_deterministic(algo):
-    wl = custom("det", 2, 1000, 256, 64, 128, 64, "bf16", filt="mr", seed=3)
+    if algo == "window":
+        wl = custom("det_w", 2, 1000, 256, 16, 7, 16, "bf16", seed=3)
+    else:
+        wl = custom("det", 2, 1000, 256, 64, 128, 64, "bf16", filt="mr", seed=3)
     q, k, v, h = make_inputs(wl, device="cuda")
     dy = make_grad(wl, device="cuda")
     a = [t.clone() for t in _bwd(q, k, v, h, dy, wl, ALGOS[algo])]
@@ -176,8 +207,7 @@ def test_bwd_rejects_bad_workspace_and_overlap():
     wl = custom("bad", 1, 300, 128, 64, 16, 16, "bf16")
     q, k, v, h = make_inputs(wl, device="cuda")
     dy = make_grad(wl, device="cuda")
-    need = g.hyena_conv_bwd_workspace_bytes(1, 300, 128, 64, 16)
-    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    small = torch.empty(256, dtype=torch.uint8, device="cuda")  # under any algorithm's need
     with pytest.raises(g.HyenaError) as e:
         g.hyena_conv_bwd(q, k, v, h, dy, 64, 16, workspace=small)
     assert e.value.status == 1
