@@ -198,8 +198,12 @@ int hyena_select_algo(const void *q, const void *k, const void *v, const float *
  * Host-only: the bytes of device workspace the backward entry points need for this shape, on
  * any algorithm and any device (a multiple of 256), or minus HYENA_ERR_INVALID_ARG for a bad
  * shape.  The workspace holds fp32 partial filter gradients: on the CUDA-core path one per
- * sequence, 64-step chunk, channel piece and tap; on the tensor path one per (CTA, sequence
- * run) and tap, with the run's group and a run count per CTA.  Touches no device.
+ * sequence, 64-step chunk, channel piece and tap; on the register-window path (l_h <= 16) one
+ * per thread (a 16-byte channel vector over a run of at least 32 time steps) and tap; on the
+ * tensor path one per (CTA, sequence run) and tap, with the run's group and a run count per CTA.
+ * Touches no device.  A smaller workspace still runs where it holds what the chosen algorithm
+ * needs at least (the window path then takes longer runs); the size returned here runs every
+ * algorithm at full speed.
  */
 int64_t hyena_conv_bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h);
 
@@ -214,12 +218,15 @@ int64_t hyena_conv_bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g,
  *
  * q, k, v, dy, dq, dk, dv: DEVICE [B, L, D] tensors of `dtype`, layout as the forward.
  * h: DEVICE fp32 [D / d_g, l_h].  dh: DEVICE fp32 [D / d_g, l_h], overwritten (not
- * accumulated into).  The forward's shape rules apply (any l_h >= 1).  Algorithm (AUTO): where
- * the tensor path applies (bf16, d_g == 64, D % 64 == 0, l_h <= 129, all seven tensors
- * 16-byte aligned) one fused tcgen05 kernel reads q, k, v, dy once and writes dq, dk, dv once,
- * with fp16 operands (x = k v, dz = q dy, h rounded to fp16) and fp32 accumulation; otherwise
- * dq comes from the forward kernels and dk, dv, dh from CUDA-core kernels in fp32.  dh is
- * summed in a fixed order on either path: results are deterministic on a given device.
+ * accumulated into).  The forward's shape rules apply (any l_h >= 1).  Algorithm (AUTO): dq
+ * comes from the forward kernels (dy in the place of q); where the tensor path applies (bf16,
+ * d_g == 64, D % 64 == 0, l_h <= 129, all seven tensors 16-byte aligned) one tcgen05 kernel
+ * reads q, k, v, dy once and writes dk, dv once, with fp16 operands (x = k v, dz = q dy, h
+ * rounded to fp16) and fp32 accumulation; else, for l_h <= 16 with d_g a multiple of 8 (bf16)
+ * or 4 (fp32) and q, k, v, dy, dk, dv 16-byte aligned, one CUDA-core register-window kernel
+ * (HYENA_ALGO_WINDOW) does the same in fp32; otherwise CUDA-core kernels in fp32 (one for dk,
+ * dv, one for the dh partials).  dh is summed in a fixed order on every path: results are
+ * deterministic on a given device.
  * workspace: DEVICE scratch of at least hyena_conv_bwd_workspace_bytes() bytes, 16-byte
  * aligned, owned by the caller, unused after the queued work ends.  Outputs must not overlap
  * each other or an input.  B == 0 or L == 0 zeroes dh and launches nothing else.
@@ -233,9 +240,9 @@ int hyena_conv_bwd(const void *q, const void *k, const void *v, const float *h, 
 
 /*
  * hyena_conv_bwd with the algorithm chosen by the caller: HYENA_ALGO_AUTO, HYENA_ALGO_TENSOR
- * (the fused tcgen05 kernel; HYENA_ERR_UNSUPPORTED where it does not apply) or
- * HYENA_ALGO_DIRECT (the CUDA-core kernels; any shape).  HYENA_ALGO_WINDOW has no backward
- * and returns HYENA_ERR_UNSUPPORTED.  Nothing is queued when an error is returned.
+ * (the tcgen05 kernel), HYENA_ALGO_WINDOW (the register-window kernel) -- each
+ * HYENA_ERR_UNSUPPORTED where it does not apply -- or HYENA_ALGO_DIRECT (the CUDA-core
+ * kernels; any shape).  Nothing is queued when an error is returned.
  */
 int hyena_conv_bwd_ex(const void *q, const void *k, const void *v, const float *h,
                       const void *dy, void *dq, void *dk, void *dv, float *dh, int64_t B,
@@ -243,8 +250,9 @@ int hyena_conv_bwd_ex(const void *q, const void *k, const void *v, const float *
                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
- * Host-only: the algorithm (HYENA_ALGO_TENSOR or HYENA_ALGO_DIRECT) HYENA_ALGO_AUTO would run
- * for this backward problem and these pointers, or minus an error code.  Touches no device.
+ * Host-only: the algorithm (HYENA_ALGO_TENSOR, HYENA_ALGO_WINDOW or HYENA_ALGO_DIRECT) that
+ * HYENA_ALGO_AUTO would run for this backward problem and these pointers, or minus an error
+ * code.  Touches no device.
  */
 int hyena_select_bwd_algo(const void *q, const void *k, const void *v, const float *h,
                           const void *dy, const void *dq, const void *dk, const void *dv,
@@ -262,9 +270,9 @@ int hyena_select_bwd_algo(const void *q, const void *k, const void *v, const flo
  * device, which a latency-bound loop cannot afford).  The dh partials go to a fixed array of
  * HYENA_BWD_STATIC_SCRATCH_BYTES in the library's device memory (one per device); this call
  * allocates nothing.  Arguments, results and errors are those of hyena_conv_bwd, plus:
- *   - HYENA_ERR_UNSUPPORTED, with nothing queued, when hyena_conv_bwd_workspace_bytes() of the
- *     shape exceeds HYENA_BWD_STATIC_SCRATCH_BYTES (e.g. the D = 4096, d_g = 64, l_h = 128
- *     shape above B * L = 16384 tokens); use hyena_conv_bwd with a workspace there.
+ *   - HYENA_ERR_UNSUPPORTED, with nothing queued, when the least workspace the shape needs
+ *     exceeds HYENA_BWD_STATIC_SCRATCH_BYTES (e.g. the D = 4096, d_g = 64, l_h = 128 shape
+ *     above B * L = 16384 tokens); use hyena_conv_bwd with a workspace there.
  *   - The first call on each device looks up the array's address (cudaGetSymbolAddress) with
  *     that device current; make that first call before any stream capture.
  *   - Calls that overlap in time on one device (different streams, or threads) share the array
