@@ -337,10 +337,13 @@ def time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind):
         bufs.append((q, k, v, h, dy, dq, dk, dv, dh))
     cfn = _native.lib().hyena_conv_bwd
     algo = g.hyena_select_bwd_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, code)
-    kernels = (["fir_tc_kernel (dq)", "fir_tc_bwd_kernel", "fir_bwd_tc_reduce_kernel"]
-               if algo == g.HYENA_ALGO_TENSOR
-               else ["forward kernel (dq)", "fir_bwd_dx_kernel", "fir_bwd_dh_partial_kernel",
-                     "fir_bwd_dh_reduce_kernel"])
+    kernels = {
+        g.HYENA_ALGO_TENSOR: ["fir_tc_kernel (dq)", "fir_tc_bwd_kernel",
+                              "fir_bwd_tc_reduce_kernel"],
+        g.HYENA_ALGO_WINDOW: ["forward kernel (dq)", "fir_bwd_window_kernel",
+                              "fir_bwd_dh_reduce_kernel"],
+    }.get(algo, ["forward kernel (dq)", "fir_bwd_dx_kernel", "fir_bwd_dh_partial_kernel",
+                 "fir_bwd_dh_reduce_kernel"])
     cargs = [tuple(t.data_ptr() for t in b) + (wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, code,
                                                 ws.data_ptr(), ws.numel(), sh) for b in bufs]
 
@@ -366,7 +369,7 @@ def time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind):
     elem = 4 if wl.dtype == "f32" else 2
     nbytes = 7 * wl.B * wl.L * wl.D * elem + 2 * wl.G * wl.l_h * 4
     achieved = nbytes / (ms / 1e3) / 1e9
-    return {"metric": "Hyena-MR bwd tokens/s (dq, dk, dv, dh)",
+    return {"metric": "%s bwd tokens/s (dq, dk, dv, dh)" % wl.describe(),
             "value": world * wl.tokens / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
             "steps": K, "gpu_launches": len(kernels) * K, "kernels": kernels,
             "algo": g.ALGO_NAMES[algo],
