@@ -200,7 +200,7 @@ bool window_supported(const Problem &P) {
 // MMAs one 128-row tile issues on the tensor path (groups per tile x k-steps).  Each costs
 // ~55 cycles of issue at any N <= 64; past ~24 per tile the issuing thread, not HBM, sets the
 // pace, and for short filters the CUDA-core window kernel is faster (measured on the SE
-// workload: 36 MMAs per tile, 80 us on tensor cores vs 56 us in the window kernel).
+// workload: 36 MMAs per tile, 80 us on tensor cores vs 50 us in the window kernel).
 constexpr int kMaxTileMmas = 24;
 
 int select_algo(const Problem &P) {
