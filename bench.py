@@ -342,7 +342,7 @@ def time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind):
                               "fir_bwd_tc_reduce_kernel"],
         g.HYENA_ALGO_WINDOW: ["forward kernel (dq)", "fir_bwd_window_kernel",
                               "fir_bwd_dh_reduce_kernel"],
-    }.get(algo, ["forward kernel (dq)", "fir_bwd_dx_kernel", "fir_bwd_dh_partial_kernel",
+    }.get(algo, ["forward kernel (dq)", "fir_tiled_kernel (dk, dv)", "fir_bwd_dh_partial_kernel",
                  "fir_bwd_dh_reduce_kernel"])
     cargs = [tuple(t.data_ptr() for t in b) + (wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, code,
                                                 ws.data_ptr(), ws.numel(), sh) for b in bufs]

@@ -4,7 +4,8 @@
 // Hardware-aware convolution kernels", Sec. 7 two-pass backward):
 //   dq = dy * z              -- the forward kernels with dy in the place of q
 //   dz = q * dy,  dx[t] = sum_j h[j] dz[t + j]   (transposed Toeplitz: anti-causal)
-//   dk = dx * v,  dv = dx * k                      -- fir_bwd_dx_kernel (one pass, both outputs)
+//   dk = dx * v,  dv = dx * k      -- cc::fir_tiled_kernel<T, true> (one pass, both outputs), or
+//                                     fir_bwd_window_kernel below for short filters
 //   dh[g][j] = sum_{b, t, c in g} dz[b,t,c] x[b,t-j,c]
 //                            -- two passes as on the page: fir_bwd_dh_partial_kernel (or, for
 //                               short filters, fir_bwd_window_kernel) writes partials, coalesced
@@ -21,30 +22,6 @@ namespace bwd {
 
 using cc::from_f32;
 using cc::to_f32;
-
-// dk, dv for every element: dx = sum_{j < l_h, t + j < L} h[g][j] * q[t+j] * dy[t+j].
-template <typename T>
-__global__ void __launch_bounds__(256)
-    fir_bwd_dx_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                      const float *__restrict__ h, const T *__restrict__ dy, T *__restrict__ dk,
-                      T *__restrict__ dv, long long B, long long L, long long D, int d_g,
-                      int l_h) {
-  const long long n = B * L * D;
-  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long c = e % D;
-    const long long t = (e / D) % L;
-    const float *hg = h + (c / d_g) * l_h;
-    const long long jmax = min(static_cast<long long>(l_h - 1), L - 1 - t);
-    float dx = 0.f;
-    for (long long j = 0; j <= jmax; ++j) {
-      const long long src = e + j * D;
-      dx = fmaf(__ldg(hg + j), to_f32(q[src]) * to_f32(dy[src]), dx);
-    }
-    from_f32(dx * to_f32(v[e]), dk + e);
-    from_f32(dx * to_f32(k[e]), dv + e);
-  }
-}
 
 constexpr int kDhRows = 64;     // time rows of one partial
 constexpr int kDhTaps = 128;    // taps per pass over the staged window (= threads per block)

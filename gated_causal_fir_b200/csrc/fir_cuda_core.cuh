@@ -8,8 +8,9 @@
 //    direct causal sum of page "04. Hardware-aware convolution kernels", Sec. 1, evaluated
 //    output by output; for l_h <= 16 it needs ~2 l_h flops per element, far below the HBM
 //    roofline's compute ridge, so no GEMM is needed.
-//  * fir_direct_kernel: one thread per output element, taps read through the cache; any
-//    supported shape, any alignment.  The fallback for shapes the fast kernels do not cover.
+//  * fir_tiled_kernel: the direct sum for any supported shape and alignment, tiled through
+//    shared memory (also the backward's transposed product).  The fallback for shapes the
+//    fast kernels do not cover.
 //
 // Both accumulate in fp32 in tap order j = 0 .. l_h-1; x = k*v is formed in fp32 (exact for
 // bf16 inputs) and y = q * acc is rounded once to the output type.
@@ -186,35 +187,109 @@ __global__ void __launch_bounds__(kWindowBlock, HYENA_WINDOW_MIN_BLOCKS)
   }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(256)
-    fir_direct_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                      const float *__restrict__ h, T *__restrict__ y, long long B, long long L,
-                      long long D, int d_g, int l_h, const T *__restrict__ kh,
-                      const T *__restrict__ vh, long long Lh) {
-  const long long n = B * L * D;
-  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long c = e % D;
-    const long long t = (e / D) % L;
-    const float *hg = h + (c / d_g) * l_h;
-    const long long jmax = min(static_cast<long long>(l_h - 1), t);
-    float acc = 0.f;
-    for (long long j = 0; j <= jmax; ++j) {
-      const long long src = e - j * D;
-      acc = fmaf(__ldg(hg + j), to_f32(k[src]) * to_f32(v[src]), acc);
+// Tiled direct sum, any shape.  A CTA takes 64 channels x 128 rows of one sequence; thread
+// (channel tid % 64, row group tid / 64) owns rows 32 rg .. 32 rg + 31 of its channel as four
+// blocks of 8.  Taps go in chunks of 128: the chunk's source rows (255 x 64, fp32) are staged in
+// shared memory, then every thread slides four 8-row register windows along them, one shared
+// load per 8 FMAs.  Each output sums its taps in the order j = 0, 1, ... (fmaf from 0): taps
+// that reach rows with no data add exact zeros, so the results are those of a plain per-output
+// loop.
+//   kAnti = false: y[t] = q[t] sum_j h[j] x[t - j], x = k v (rows -Lh .. -1 from the history
+//                  k_hist, v_hist, zero before them);
+//   kAnti = true:  dx[t] = sum_j h[j] dz[t + j], dz = q dy (zero from L on); writes
+//                  dk = dx v and dv = dx k (the backward's transposed product).
+constexpr int kTileC = 64, kTileR = 128, kTileJ = 128, kTileThreads = 256;
+constexpr int kTileWin = kTileR + kTileJ - 1;
+constexpr int kTileSmemBytes = kTileWin * kTileC * 4;
+
+template <typename T, bool kAnti>
+__global__ void __launch_bounds__(kTileThreads)
+    fir_tiled_kernel(const T *__restrict__ a0, const T *__restrict__ a1,
+                     const T *__restrict__ k, const T *__restrict__ v,
+                     const float *__restrict__ h, T *__restrict__ o0, T *__restrict__ o1,
+                     long long B, long long L, long long D, int d_g, int l_h,
+                     const T *__restrict__ kh, const T *__restrict__ vh, long long Lh) {
+  // forward: a0 = q, a1 unused, o0 = y;  anti: a0 = q, a1 = dy, o0 = dk, o1 = dv
+  extern __shared__ float xs[];  // [kTileWin][kTileC]
+  const int cl = threadIdx.x % kTileC, rg = threadIdx.x / kTileC;
+  const long long n_ct = (D + kTileC - 1) / kTileC, n_rt = (L + kTileR - 1) / kTileR;
+  const long long n_tiles = B * n_rt * n_ct;
+  // tiles (channel tile fastest, then row tile, then sequence), grid-stride over the CTAs
+  for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+  const long long c0 = (tile % n_ct) * kTileC;
+  const long long t0 = ((tile / n_ct) % n_rt) * kTileR;
+  const long long b = tile / (n_ct * n_rt);
+  const long long c = c0 + cl;
+  const bool live_c = c < D;
+  const float *hg = h + (live_c ? c / d_g : 0) * l_h;
+  const long long seq = b * L * D;
+  float acc[4][8];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[q4][i] = 0.f;
+
+  for (int j0 = 0; j0 < l_h; j0 += kTileJ) {
+    // source row of window row w: base + w
+    const long long base = kAnti ? t0 + j0 : t0 - j0 - (kTileJ - 1);
+    __syncthreads();  // the previous chunk's window has been read
+    for (int e = threadIdx.x; e < kTileWin * kTileC; e += kTileThreads) {
+      const int w = e / kTileC, ce = e % kTileC;
+      const long long sr = base + w, gc = c0 + ce;
+      float val = 0.f;
+      if (gc < D) {
+        if (sr >= 0 && sr < L) {
+          const long long a = seq + sr * D + gc;
+          val = kAnti ? to_f32(a0[a]) * to_f32(a1[a]) : to_f32(k[a]) * to_f32(v[a]);
+        } else if (!kAnti && sr < 0 && sr >= -Lh) {
+          const long long a = (b * Lh + Lh + sr) * D + gc;
+          val = to_f32(kh[a]) * to_f32(vh[a]);
+        }
+      }
+      xs[w * kTileC + ce] = val;
     }
-    // taps that reach before row 0: the history rows [B, Lh, D] (row Lh - 1 precedes row 0)
-    const long long jh = min(static_cast<long long>(l_h - 1), t + Lh);
-    if (jh > t) {
-      const long long hrow = (e / (L * D)) * Lh + Lh + t;  // history row of tap j: hrow - j
-      for (long long j = t + 1; j <= jh; ++j) {
-        const long long src = (hrow - j) * D + c;
-        acc = fmaf(__ldg(hg + j), to_f32(kh[src]) * to_f32(vh[src]), acc);
+    __syncthreads();
+    const int nj = min(kTileJ, l_h - j0);
+    // taps in groups of 8 (past l_h: h = 0, which adds exact zeros): an 8 x 8 block of a row
+    // block's outputs and the group's taps reads 15 window rows, u = i - t + 7 (forward) or
+    // u = i + t (anti) for output i and tap t of the group
+    for (int jj0 = 0; jj0 < nj; jj0 += 8) {
+      float hv[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) hv[t] = jj0 + t < nj ? __ldg(hg + j0 + jj0 + t) : 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int r0 = rg * 32 + q4 * 8;
+        const int w0 = kAnti ? r0 + jj0 : r0 + kTileJ - 8 - jj0;
+        float xw[15];
+#pragma unroll
+        for (int u = 0; u < 15; ++u) xw[u] = xs[(w0 + u) * kTileC + cl];
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            acc[q4][i] = fmaf(hv[t], xw[kAnti ? i + t : i - t + 7], acc[q4][i]);
       }
     }
-    from_f32(to_f32(q[e]) * acc, y + e);
   }
+  if (live_c) {
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const long long t = t0 + rg * 32 + q4 * 8 + i;
+        if (t >= L) continue;
+        const long long a = seq + t * D + c;
+        if (kAnti) {
+          from_f32(acc[q4][i] * to_f32(v[a]), o0 + a);
+          from_f32(acc[q4][i] * to_f32(k[a]), o1 + a);
+        } else {
+          from_f32(to_f32(a0[a]) * acc[q4][i], o0 + a);
+        }
+      }
+    }
+  }
+  }  // tiles
 }
 
 // Toeplitz sub-blocks H_m[g][i][j] = h[g][m*l_b + i - j] (zero outside [0, l_h)), m = 0, 1, 2.

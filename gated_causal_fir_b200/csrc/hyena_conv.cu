@@ -83,6 +83,15 @@ int current_device(DeviceState *&ds) {
       e = cudaFuncSetAttribute(reinterpret_cast<const void *>(hyena::tcb::fir_tc_bwd_kernel),
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                hyena::tcb::kSmemBytes);
+    const void *tiled[] = {
+        reinterpret_cast<const void *>(hyena::cc::fir_tiled_kernel<float, false>),
+        reinterpret_cast<const void *>(hyena::cc::fir_tiled_kernel<float, true>),
+        reinterpret_cast<const void *>(hyena::cc::fir_tiled_kernel<__nv_bfloat16, false>),
+        reinterpret_cast<const void *>(hyena::cc::fir_tiled_kernel<__nv_bfloat16, true>)};
+    for (const void *k : tiled)
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 hyena::cc::kTileSmemBytes);
 
     d->err = e;
   });
@@ -382,25 +391,27 @@ int launch_window(const Problem &P, cudaStream_t s) {
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
-int launch_direct(const Problem &P, cudaStream_t s) {
+// The tiled direct sum (fir_tiled_kernel): forward (y) or, with kAnti, the backward's
+// transposed product (dk, dv from q, dy).  Persistent CTAs over the tiles.
+template <typename T, bool kAnti>
+int launch_tiled(const Problem &P, const void *dy, void *out0, void *out1, cudaStream_t s) {
   DeviceState *ds = nullptr;
   if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
-  const long long n = P.numel();
-  long long blocks = (n + 255) / 256;
-  const long long cap = static_cast<long long>(ds->sm_count) * 16;
-  if (blocks > cap) blocks = cap;
-  if (P.dtype == HYENA_DTYPE_F32)
-    hyena::cc::fir_direct_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-        static_cast<const float *>(P.q), static_cast<const float *>(P.k),
-        static_cast<const float *>(P.v), P.h, static_cast<float *>(P.y), P.B, P.L, P.D, P.d_g,
-        P.l_h, static_cast<const float *>(P.kh), static_cast<const float *>(P.vh), P.Lh);
-  else
-    hyena::cc::fir_direct_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16 *>(P.q), static_cast<const __nv_bfloat16 *>(P.k),
-        static_cast<const __nv_bfloat16 *>(P.v), P.h, static_cast<__nv_bfloat16 *>(P.y), P.B,
-        P.L, P.D, P.d_g, P.l_h, static_cast<const __nv_bfloat16 *>(P.kh),
-        static_cast<const __nv_bfloat16 *>(P.vh), P.Lh);
+  namespace cc = hyena::cc;
+  const long long tiles = P.B * ((P.L + cc::kTileR - 1) / cc::kTileR) *
+                          ((P.D + cc::kTileC - 1) / cc::kTileC);
+  const long long grid = std::min<long long>(tiles, static_cast<long long>(ds->sm_count) * 4);
+  cc::fir_tiled_kernel<T, kAnti><<<static_cast<unsigned>(grid), cc::kTileThreads,
+                                   cc::kTileSmemBytes, s>>>(
+      static_cast<const T *>(P.q), static_cast<const T *>(dy), static_cast<const T *>(P.k),
+      static_cast<const T *>(P.v), P.h, static_cast<T *>(out0), static_cast<T *>(out1), P.B,
+      P.L, P.D, P.d_g, P.l_h, static_cast<const T *>(P.kh), static_cast<const T *>(P.vh), P.Lh);
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+int launch_direct(const Problem &P, cudaStream_t s) {
+  if (P.dtype == HYENA_DTYPE_F32) return launch_tiled<float, false>(P, nullptr, P.y, nullptr, s);
+  return launch_tiled<__nv_bfloat16, false>(P, nullptr, P.y, nullptr, s);
 }
 
 int run(const Problem &P, int algo, cudaStream_t s) {
@@ -496,15 +507,9 @@ int launch_bwd_cuda_core(const Problem &P, const void *dy, void *dk, void *dv, f
                          float *partial, cudaStream_t s) {
   DeviceState *ds = nullptr;
   if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
-  const long long n = P.numel();
-  long long blocks = (n + 255) / 256;
   const long long cap = static_cast<long long>(ds->sm_count) * 16;
-  if (blocks > cap) blocks = cap;
-  hyena::bwd::fir_bwd_dx_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-      static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v), P.h,
-      static_cast<const T *>(dy), static_cast<T *>(dk), static_cast<T *>(dv), P.B, P.L, P.D,
-      P.d_g, P.l_h);
-  if (cudaGetLastError() != cudaSuccess) return HYENA_ERR_CUDA;
+  const int rt = launch_tiled<T, true>(P, dy, dk, dv, s);  // dk, dv
+  if (rt != HYENA_OK) return rt;
   const BwdPlan b = bwd_plan(P.B, P.L, P.D, P.d_g, P.l_h);
   if (b.nchunk > 2147483647 || P.B > 65535 || b.npieces > 65535 ||
       P.B * b.nchunk * (P.d_g / b.cp) > std::numeric_limits<int32_t>::max())
