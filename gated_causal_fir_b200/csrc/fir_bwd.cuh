@@ -35,11 +35,16 @@ __host__ __device__ inline int dh_piece(int d_g) {
 }
 
 // Pass 1.  Block (chunk, piece, b): rows [64 chunk, 64 chunk + 64) of sequence b, channels
-// [piece * cp, piece * cp + cp).  Thread j of a tap block accumulates
+// [piece * cp, piece * cp + cp).  For each tap j of a 128-tap block it forms
 //   sum_{t in rows, c in piece} dz[t, c] * x[t - j, c]
-// from shared memory (dz rows and the x window the tap block needs, rows padded by one float so
-// that the lanes' different rows fall in different banks), and writes
-// partial[((b * nchunk + chunk) * npieces + piece) * l_h + j].
+// from shared memory (the dz rows and the x window of the tap block, rows padded by one float)
+// and writes partial[((b * nchunk + chunk) * npieces + piece) * l_h + j].  Thread (cg, tg) =
+// (tid % 8, tid / 8) takes the 8 taps 8 tg .. 8 tg + 7 over the channels cg, cg + 8, ...: per 8
+// rows of one channel it reads 8 dz values and 15 window values for 64 FMAs; the 8 channel
+// groups' sums then meet in shared memory in a fixed order.
+constexpr int kDhGroups = 8;                                  // channel groups per block
+constexpr int kDhRedFloats = kDhGroups * kDhTaps;             // the reduction buffer
+
 template <typename T>
 __global__ void __launch_bounds__(kDhTaps)
     fir_bwd_dh_partial_kernel(const T *__restrict__ q, const T *__restrict__ k,
@@ -53,8 +58,10 @@ __global__ void __launch_bounds__(kDhTaps)
   const long long c0 = static_cast<long long>(piece) * cp;
   const long long base = static_cast<long long>(b) * L * D;
   const int ld = cp + 1;
-  float *dzs = sm;                       // [kDhRows][ld]
-  float *xs = sm + kDhRows * ld;         // [kDhRows + kDhTaps - 1][ld]
+  const int cg = threadIdx.x % kDhGroups, tg = threadIdx.x / kDhGroups;
+  float *red = sm;                              // [kDhGroups][kDhTaps]
+  float *dzs = sm + kDhRedFloats;               // [kDhRows][ld]
+  float *xs = dzs + kDhRows * ld;               // [kDhRows + kDhTaps - 1][ld]
   for (int e = threadIdx.x; e < kDhRows * cp; e += blockDim.x) {
     const int r = e / cp, c = e % cp;
     const long long t = t0 + r;
@@ -70,7 +77,7 @@ __global__ void __launch_bounds__(kDhTaps)
     // x rows t0 - j0 - (kDhTaps - 1) .. t0 + kDhRows - 1 - j0; window row w holds
     // x[t0 - j0 - (kDhTaps - 1) + w].
     const long long xbase = t0 - j0 - (kDhTaps - 1);
-    __syncthreads();
+    __syncthreads();  // the previous tap block's window and reduction have been read
     for (int e = threadIdx.x; e < (kDhRows + kDhTaps - 1) * cp; e += blockDim.x) {
       const int w = e / cp, c = e % cp;
       const long long t = xbase + w;
@@ -82,16 +89,35 @@ __global__ void __launch_bounds__(kDhTaps)
       xs[w * ld + c] = val;
     }
     __syncthreads();
-    const int j = j0 + threadIdx.x;
-    float acc = 0.f;
-    // row r of dz pairs with x row t0 + r - j = window row r + (kDhTaps - 1) - threadIdx.x
-    const int woff = kDhTaps - 1 - static_cast<int>(threadIdx.x);
-    for (int r = 0; r < kDhRows; ++r) {
-      const float *dzr = dzs + r * ld;
-      const float *xr = xs + (r + woff) * ld;
-      for (int c = 0; c < cp; ++c) acc = fmaf(dzr[c], xr[c], acc);
+    // dz row r pairs with window row r + (kDhTaps - 1) - jj for tap j0 + jj; for rows
+    // r0 + i and taps 8 tg + t that is row w0 + (i - t + 7), w0 = r0 + kDhTaps - 8 - 8 tg
+    float acc[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+    for (int c = cg; c < cp; c += kDhGroups) {
+      for (int r0 = 0; r0 < kDhRows; r0 += 8) {
+        const int w0 = r0 + kDhTaps - 8 - 8 * tg;
+        float dz[8], xw[15];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dz[i] = dzs[(r0 + i) * ld + c];
+#pragma unroll
+        for (int u = 0; u < 15; ++u) xw[u] = xs[(w0 + u) * ld + c];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) acc[t] = fmaf(dz[i], xw[i - t + 7], acc[t]);
+      }
     }
-    if (j < l_h) out[j] = acc;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) red[cg * kDhTaps + tg * 8 + t] = acc[t];
+    __syncthreads();
+    const int j = j0 + threadIdx.x;
+    if (j < l_h) {
+      float s = 0.f;
+#pragma unroll
+      for (int g = 0; g < kDhGroups; ++g) s += red[g * kDhTaps + threadIdx.x];
+      out[j] = s;
+    }
   }
 }
 

@@ -36,7 +36,8 @@ using hyena::cc::WindowParams;
 constexpr int kMaxDevices = 64;
 // Shared memory of the dh partial kernel at 64 channels per piece: dz rows + x window.
 constexpr int kDhSmemMax =
-    (2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (64 + 1) * static_cast<int>(sizeof(float));
+    ((2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (64 + 1) + hyena::bwd::kDhRedFloats) *
+    static_cast<int>(sizeof(float));
 constexpr int kMaxWindowTaps = 16;
 #ifndef HYENA_WINDOW_ROWS
 #define HYENA_WINDOW_ROWS 128
@@ -516,7 +517,8 @@ int launch_bwd_cuda_core(const Problem &P, const void *dy, void *dk, void *dv, f
     return HYENA_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(b.nchunk), static_cast<unsigned>(b.npieces),
                   static_cast<unsigned>(P.B));
-  const int smem = (2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (b.cp + 1) * 4;
+  const int smem = ((2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (b.cp + 1) +
+                    hyena::bwd::kDhRedFloats) * 4;
   hyena::bwd::fir_bwd_dh_partial_kernel<T><<<grid, hyena::bwd::kDhTaps, smem, s>>>(
       static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v),
       static_cast<const T *>(dy), partial, P.L, P.D, P.l_h, b.cp);
