@@ -518,7 +518,7 @@ def main():
         bytes_per_launch = wl.algorithmic_bytes()
         achieved = bytes_per_launch / (mean_launch_ms / 1e3) / 1e9
         kernel = {g.HYENA_ALGO_TENSOR: "fir_tc_kernel", g.HYENA_ALGO_WINDOW: "fir_window_kernel",
-                  g.HYENA_ALGO_DIRECT: "fir_direct_kernel"}[algo]
+                  g.HYENA_ALGO_DIRECT: "fir_tiled_kernel"}[algo]
         traffic = committed_traffic(kernel, wl.name)
         line = {
             "metric": METRIC if wl.name == "mr" else
