@@ -218,6 +218,22 @@ def test_device_status_needs_out(lib):
     assert lib.hyena_device_status(None, 0) == 1
 
 
+def test_from_host_binding_checks_before_any_device_work():
+    """hyena_conv_fwd_from_host takes contiguous host tensors (and fp32 filters) only; the checks
+    run before anything touches a device."""
+    import torch
+    q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
+    h = torch.zeros(1, 4)
+    with pytest.raises(TypeError):
+        g.hyena_conv_fwd_from_host(q.transpose(1, 2), q, q, h, d_g=64, l_b=4)  # not contiguous
+    with pytest.raises(TypeError):
+        g.hyena_conv_fwd_from_host(q, q, q, h.double(), d_g=64, l_b=4)         # fp64 filters
+    with pytest.raises(TypeError):
+        g.hyena_conv_fwd_from_host(q, q.float(), q, h, d_g=64, l_b=4)          # mixed dtypes
+    with pytest.raises(TypeError):
+        g.hyena_conv_fwd_from_host(q, q, q, h, d_g=64, l_b=4, out=torch.zeros(1, 8, 32))
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
