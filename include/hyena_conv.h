@@ -10,7 +10,8 @@
  * two-stage form Yhat_n = H0 Xhat_n + H1 Xhat_{n-1}, Xhat_{-1} = 0).
  *
  * Conventions shared by every entry point:
- *   - q, k, v, y are DEVICE pointers to [B, L, D] row-major tensors (channels contiguous).
+ *   - q, k, v, y are DEVICE pointers to [B, L, D] row-major tensors (channels contiguous),
+ *     except in hyena_conv_fwd_from_host, which takes HOST buffers.
  *   - h is a DEVICE pointer to fp32 [D / d_g, l_h], natural tap order: h[g][0] multiplies the
  *     current token.  Channel c belongs to group c / d_g (contiguous groups).
  *   - Every sequence b starts from zero history; no state is kept between calls.
@@ -58,10 +59,11 @@ enum hyena_algo {
                                     D % 64 == 0, d_g in {16, 32, 64}; l_h <= 513 for
                                     d_g == 64, <= 257 for d_g == 32, <= 65 for d_g == 16;
                                     16-byte aligned tensors) */
-    HYENA_ALGO_WINDOW = 2,       /* CUDA-core register sliding window (l_h <= 16; d_g a
-                                    multiple of 8 channels for bf16, 4 for fp32; 16-byte
-                                    aligned tensors) */
-    HYENA_ALGO_DIRECT = 3        /* CUDA-core direct sum; any supported shape */
+    HYENA_ALGO_WINDOW = 2,       /* CUDA-core register sliding window, forward and backward
+                                    (l_h <= 16; d_g a multiple of 8 channels for bf16, 4 for
+                                    fp32; 16-byte aligned tensors) */
+    HYENA_ALGO_DIRECT = 3        /* CUDA-core direct sum, tiled through shared memory; any
+                                    supported shape */
 };
 
 /* Bits of the per-device status word (hyena_device_status). */
@@ -78,7 +80,7 @@ enum hyena_device_status_bits {
  * every filter length (the two-stage form of Sec. 3 is the case S = 2, l_h <= l_b + 1), so the
  * result does not depend on l_b.  The kernels pick their own internal block size.  Filters
  * longer than the tensor path's limit (HYENA_ALGO_TENSOR above) run on the CUDA-core direct
- * kernel.  All tensors 2-byte aligned.
+ * sum; hyena_conv_fwd_fft is the faster entry point for them.  All tensors 2-byte aligned.
  */
 int hyena_conv_fwd(const void *q, const void *k, const void *v, const float *h, void *y,
                    int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
