@@ -10,6 +10,7 @@ import re
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libhyena_conv.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "hyena_conv.h")
+TESTING_HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "hyena_conv_testing.h")
 
 HYENA_OK = 0
 HYENA_ERR_INVALID_ARG = 1
@@ -71,6 +72,12 @@ SIGNATURES = {
     "hyena_abi_version": (_i32, []),
 }
 
+# include/hyena_conv_testing.h: test hooks, not part of the operation's interface
+TESTING_SIGNATURES = {
+    "hyena_testing_fwd_fault": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32,
+                                       _i32, ctypes.c_uint64, _vp]),
+}
+
 _LIB = None
 
 
@@ -82,9 +89,9 @@ class HyenaError(RuntimeError):
         super().__init__("%s failed: %s (status %d)" % (fn, status_string(status), status))
 
 
-def header_functions():
-    """Names of the functions include/hyena_conv.h declares."""
-    src = open(HEADER_PATH).read()
+def header_functions(path=HEADER_PATH):
+    """Names of the functions a header (default include/hyena_conv.h) declares."""
+    src = open(path).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(hyena_[a-z0-9_]+)\s*\(", src)))
 
@@ -97,7 +104,7 @@ def lib():
             raise ImportError("libhyena_conv.so is not built (%s); run "
                               "`python -m gated_causal_fir_b200.build`" % LIB_PATH)
         handle = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in SIGNATURES.items():
+        for name, (res, args) in list(SIGNATURES.items()) + list(TESTING_SIGNATURES.items()):
             fn = getattr(handle, name)
             fn.restype = res
             fn.argtypes = args

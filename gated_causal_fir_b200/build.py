@@ -13,7 +13,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libhyena_conv.so")
 SOURCES = [os.path.join(CSRC, "hyena_conv.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
-    os.path.join(ROOT, "include", "hyena_conv.h")]
+    os.path.join(ROOT, "include", "hyena_conv.h"), os.path.join(ROOT, "include", "hyena_conv_testing.h")]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared", "-Xptxas", "-warn-spills"]

@@ -35,6 +35,8 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include <type_traits>
 #include "ptx.cuh"
 
 namespace hyena {
@@ -51,6 +53,17 @@ constexpr int kMaxHalo = kMaxHist * kTM;
 #define HYENA_TC_KV_STAGES 3
 #endif
 constexpr int kNKV = HYENA_TC_KV_STAGES;  // k/v stages
+// Unrolling of the gate's and the epilogue's per-tile loops (8 iterations each).  The kernel's
+// warp roles run different code side by side, so hot-loop code size competes for the
+// instruction cache.
+#ifndef HYENA_TC_GATE_UNROLL
+#define HYENA_TC_GATE_UNROLL 8
+#endif
+#ifndef HYENA_TC_EPI_UNROLL
+#define HYENA_TC_EPI_UNROLL 8
+#endif
+constexpr int kGateUnroll = HYENA_TC_GATE_UNROLL;
+constexpr int kEpiUnroll = HYENA_TC_EPI_UNROLL;
 constexpr int kNAcc = 2;             // TMEM accumulator sets (tiles in flight)
 constexpr int kRowBytes = kNC * 2;                              // 128 B
 constexpr int kTileBytes = kTM * kRowBytes;                     // 16 KB
@@ -62,8 +75,11 @@ constexpr int kKBlockBytes = kNC * 128;                         // 64 times x 64
 constexpr int kBandCol0 = kNAcc * kNC;                           // 128
 constexpr int kTmemCols = 512;
 
-constexpr int kThreads = 352;
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGate0 = 2, kWarpEpi0 = 6, kWarpTmaQ = 10;
+constexpr int kThreads = 384;
+// Limit of the recomputation warp's wait, which spans the whole kernel.
+constexpr uint64_t kFixWaitNs = 20000000000ull;  // 20 s
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGate0 = 2, kWarpEpi0 = 6, kWarpTmaQ = 10,
+              kWarpFix = 11;
 constexpr int kGroupThreads = 128;
 
 // Shared-memory layout for a kernel whose tiles read kNH earlier tiles (halo <= 128 kNH rows):
@@ -78,10 +94,21 @@ struct Layout {
   static constexpr int kOffX = kOffQ + kNQ * kTileBytes;
   // fp16 filter taps of the tile's groups, zero-padded: 258 + halo per group (see stage_taps);
   // kPer of them per gate thread
-  static constexpr int kHzBytes = kNH == 1 ? 2688 : (kNH == 2 ? 2064 : 1552);
+  static constexpr int kHzBytes = kNH == 1 ? 2688 : (kNH == 2 ? 2064 : (kNH == 3 ? 1296 : 1552));
   static constexpr int kPer = (kHzBytes / 2 + kGroupThreads - 1) / kGroupThreads;
   static constexpr int kOffHz = kOffX + kNX * kTileBytes;
-  static constexpr int kOffBar = kOffHz + kHzBytes;
+  // Output tiles whose fp16 operands left the range, listed by the gate warps for the
+  // epilogue's fp32 recomputation after its main loop: a count, then up to kNBad walk positions
+  // (more than kNBad: every output tile of the CTA is recomputed).
+  static constexpr int kNBad = kNH <= 2 ? 8 : 4;
+  static constexpr int kOffBad = kOffHz + kHzBytes;
+  // Scale exponents of the sequence run, from the gate to the epilogue (two, by run parity):
+  // byte gg = eh + ex of the tile's group gg.
+  static constexpr int kOffSeg = kOffBad + 8 + kNBad * 8;
+  // Per-segment maxima (two sets, by segment parity): |h| of each group (4 words) and |k v| of
+  // the segment's first tile (1 word), as float bits.
+  static constexpr int kOffMax = kOffSeg + 8;
+  static constexpr int kOffBar = kOffMax + 2 * 8 * 4;
   // barriers
   static constexpr int kBarKVFull = 0;
   static constexpr int kBarKVEmpty = kBarKVFull + kNKV;
@@ -96,7 +123,12 @@ struct Layout {
   static constexpr int kBarAEmpty = kBarAFull + 2;  // up to two band sets
   static constexpr int kBarGate = kBarAEmpty + 2;   // the 128 gate threads among themselves
   static constexpr int kBarDone = kBarGate + 1;
-  static constexpr int kNumBars = kBarDone + 1;
+  static constexpr int kBarSegFull = kBarDone + 1;       // two, by run parity
+  static constexpr int kBarSegEmpty = kBarSegFull + 2;
+  static constexpr int kBarGateDone = kBarSegEmpty + 2;  // the gate warps have left their loop
+  static constexpr int kBarEpiDone = kBarGateDone + 1;   // the epilogue has finished (and, when
+                                                         // tiles were listed, its stores landed)
+  static constexpr int kNumBars = kBarEpiDone + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget of one CTA exceeded");
@@ -106,8 +138,34 @@ struct Layout {
 constexpr unsigned kTimeoutBit = 1u;  // HYENA_DEVICE_TIMEOUT
 constexpr unsigned kF16RangeBit = 2u; // HYENA_DEVICE_F16_RANGE
 
+// fp16 operands with power-of-two scales, chosen per sequence run.  The band holds
+// fp16(h * 2^eh): eh = 0 while the group's largest |h| lies in [2^-4, 2^8) (fp16 holds such
+// taps as they are: a tap far below the largest one keeps an absolute error of at most 2^-25,
+// negligible beside it), else the eh that brings it to [2^7, 2^8).  X holds fp16(k v 2^ex) with
+// ex chosen from the run's first tile: ex = -eh of the tile's first group whenever that puts
+// the tile's largest |k v| in [2^-6, 2^9) (room for later tiles up to 2^7 times larger), so
+// that the product needs no rescaling; otherwise the ex that brings it to [2^8, 2^9).  Scaling
+// by a power of two is exact, so the accumulator is the unscaled sum times 2^(eh + ex), which
+// the epilogue divides out exactly.  For operands of ordinary size eh = ex = 0, and the hot
+// loops carry no scaling; the scaled conversions run out of line.  A tile whose inputs still leave
+// the range (a scaled |k v| above 65504, or a warp's 32 rows all below 2^-12 but not all
+// zero, where most values would be fp16 subnormals) is recomputed in fp32 on the CUDA cores
+// once the CTA's stores have landed, and rewritten.
+// A value below fp16's normal range (2^-14 scaled) keeps an absolute error of at most 2^-25
+// scaled, 2^-(25 + ex) unscaled.
+constexpr int kTapExpTarget = 7;
+constexpr int kXExpTarget = 8;
+constexpr int kXBalancedLo = -6, kXBalancedHi = 8;  // accepted floor(log2 max |k v 2^ex|)
+constexpr float kXTiny = 0.000244140625f;  // 2^-12
+
 struct Params {
   const float *h;   // [D / d_g, l_h]
+  // the tensors as raw pointers, for the fp32 recomputation of out-of-range tiles
+  const __nv_bfloat16 *q, *k, *v, *kh, *vh;
+  __nv_bfloat16 *y;
+  long long D;      // channels (row length)
+  unsigned long long wait_ns;  // limit of the bounded waits between roles
+  int fault;        // test hook: 1 = the MMA issuer withholds the first accumulator arrive
   int B, L, l_h;
   int CB;           // 64-channel blocks across D (tiles per time row) = D / 64
   int halo;         // multiple of 16, >= l_h - 1, <= 128 * (history tiles of the kernel)
@@ -182,16 +240,19 @@ struct WorkIter {
   }
 };
 
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-  const bool ok = mbar_wait(bar, parity, abort, &g_device_status, kTimeoutBit);
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
+  const bool ok = mbar_wait(bar, parity, abort, &g_device_status, kTimeoutBit, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ bool thread_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-  return mbar_wait(bar, parity, abort, &g_device_status, kTimeoutBit);
+__device__ __forceinline__ bool thread_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                            uint64_t limit_ns = kWaitTimeoutNs) {
+  return mbar_wait(bar, parity, abort, &g_device_status, kTimeoutBit, limit_ns);
 }
 
 // Drain wait: bounded by time only (ignores the abort flag), for copies this thread issued.
+// Always the full limit: a CTA must not exit with a copy into its shared memory in flight.
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   int no_abort = 0;
   mbar_wait(bar, parity, &no_abort, &g_device_status, kTimeoutBit);
@@ -205,6 +266,105 @@ __device__ __forceinline__ uint32_t gate_pair(uint32_t kw, uint32_t vw, bool &ov
   over |= (fabsf(x0) > 65504.f) | (fabsf(x1) > 65504.f);
   const __half2 hx = __floats2half2_rn(x0, x1);
   return *reinterpret_cast<const uint32_t *>(&hx);
+}
+
+// 2^e as a float, for -126 <= e <= 127.
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// The power-of-two exponent that brings a maximum |value| (float bits) to [2^target,
+// 2^(target+1)): 0 for an all-zero maximum, clamped to [-60, 60] so that the epilogue's
+// combined factor 2^-(eh + ex) is one normal float.  (Operands beyond what the clamp covers
+// leave fp16's range and take the fp32 recomputation.)
+__device__ __forceinline__ int scale_exp(uint32_t max_bits, int target) {
+  if (max_bits == 0) return 0;
+  const int e = static_cast<int>((max_bits >> 23) & 0xFFu) - 127;  // floor(log2 max)
+  return min(max(target - e, -60), 60);
+}
+
+// eh of a group from its largest |h| (see kTapExpTarget); `clamped` is set when the wanted
+// exponent lay beyond the clamp (the run's operands then leave fp16's range).
+__device__ __forceinline__ int tap_scale_exp(uint32_t max_bits, bool &clamped) {
+  const int e = static_cast<int>((max_bits >> 23) & 0xFFu) - 127;
+  if (max_bits == 0 || (e >= -4 && e <= 7)) return 0;
+  clamped |= (kTapExpTarget - e > 60) | (kTapExpTarget - e < -60);
+  return scale_exp(max_bits, kTapExpTarget);
+}
+
+// ex of a sequence run from the largest |k v| of its first tile and the first group's eh (see
+// kTapExpTarget); `clamped` as above.
+__device__ __forceinline__ int x_scale_exp(uint32_t max_bits, int eh0, bool &clamped) {
+  const int e = static_cast<int>((max_bits >> 23) & 0xFFu) - 127;
+  if (max_bits == 0 || (e - eh0 >= kXBalancedLo && e - eh0 <= kXBalancedHi)) return -eh0;
+  clamped |= (kXExpTarget - e > 60) | (kXExpTarget - e < -60);
+  return scale_exp(max_bits, kXExpTarget);
+}
+
+// x = fp16(k * v * s) for two bf16 lanes packed in a 32-bit word (s = 2^ex when kScaled; k*v
+// and k*v*s are exact in fp32); folds |x| (fp32, before the rounding) into the running
+// maximum mx, so that an fp16 overflow shows as mx > 65504 and a value that rounds to zero
+// still counts.
+template <bool kScaled>
+__device__ __forceinline__ uint32_t gate_pair_x(uint32_t kw, uint32_t vw, float s, float &mx) {
+  const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
+  const float v0 = __uint_as_float(vw << 16), v1 = __uint_as_float(vw & 0xFFFF0000u);
+  float x0 = k0 * v0, x1 = k1 * v1;
+  if (kScaled) {
+    x0 *= s;
+    x1 *= s;
+  }
+  mx = fmaxf(mx, fmaxf(fabsf(x0), fabsf(x1)));
+  const __half2 hx = __floats2half2_rn(x0, x1);
+  return *reinterpret_cast<const uint32_t *>(&hx);
+}
+
+// X^T of gate warp gw's 32 rows (channel rows, 64 times per 128-byte row, two 8 KB K-blocks per
+// tile, 128-byte swizzle) from the time-major k and v tiles: 8 x 8 blocks moved with ldmatrix,
+// k*v (times 2^ex when kScaled) formed in fp32, rounded to fp16 and stored transposed with
+// stmatrix (both bank-conflict-free).  Returns this lane's largest |x| before the rounding.
+template <bool kScaled>
+__device__ __forceinline__ float gate_x_tile(uint32_t kbase, uint32_t vbase, uint32_t xbase,
+                                             int gw, int lane, float s) {
+  const int mat = lane >> 3, rr = lane & 7;
+  float mx = 0.f;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int bw = it * 4 + mat;
+    const int tg = gw * 4 + (bw >> 3), cg = bw & 7;  // 8-time group, 8-channel group
+    const uint32_t src = (tg * 8 + rr) * kRowBytes + ((cg ^ rr) << 4);
+    uint32_t kf[4], vf[4], xf[4];
+    ldsm_x4(kbase + src, kf);
+    ldsm_x4(vbase + src, vf);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) xf[e] = gate_pair_x<kScaled>(kf[e], vf[e], s, mx);
+    const int c = cg * 8 + rr;
+    const uint32_t dst = (tg >> 3) * kKBlockBytes + c * kRowBytes + (((tg & 7) ^ rr) << 4);
+    stsm_x4_trans(xbase + dst, xf);
+  }
+  return mx;
+}
+
+// Largest |k v| (float bits) over the 32 rows x 64 channels gate warp gw converts from the
+// time-major, 128-byte-swizzled k and v tiles (the same fragments as the X build).  Once per
+// sequence run.
+__device__ __forceinline__ uint32_t kv_absmax(uint32_t kbase, uint32_t vbase, int gw, int lane) {
+  const int mat = lane >> 3, rr = lane & 7;
+  uint32_t m = 0;
+#pragma unroll 1
+  for (int it = 0; it < 8; ++it) {
+    const int bw = it * 4 + mat;
+    const int tg = gw * 4 + (bw >> 3), cg = bw & 7;
+    const uint32_t src = (tg * 8 + rr) * kRowBytes + ((cg ^ rr) << 4);
+    uint32_t kf[4], vf[4];
+    ldsm_x4(kbase + src, kf);
+    ldsm_x4(vbase + src, vf);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float p0 = __uint_as_float(kf[e] << 16) * __uint_as_float(vf[e] << 16);
+      const float p1 = __uint_as_float(kf[e] & 0xFFFF0000u) * __uint_as_float(vf[e] & 0xFFFF0000u);
+      m = max(m, max(__float_as_uint(fabsf(p0)), __float_as_uint(fabsf(p1))));
+    }
+  }
+  return __reduce_max_sync(0xffffffffu, m);
 }
 
 // Filter taps of the tile's kNG groups, staged once per sequence run by the 128 gate threads:
@@ -237,6 +397,107 @@ __device__ __forceinline__ void tap_store(uint16_t *hz, const float (&v)[kPer], 
       const __half hv = __float2half_rn(v[k]);
       hz[e] = *reinterpret_cast<const uint16_t *>(&hv);
     }
+  }
+}
+
+// The same staging with group gg's taps scaled by 2^eh[gg] (exact) before the rounding to fp16.
+template <int kNG, int kPer>
+__device__ __forceinline__ void tap_store_scaled(uint16_t *hz, const float (&v)[kPer], int halo,
+                                                 int tid, const int (&eh)[kNG]) {
+  const int stride = 258 + halo, n = kNG * stride;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int e = tid + k * kGroupThreads;
+    if (e < n) {
+      const int gg = e / stride;
+      float s = exp2i(eh[0]);
+#pragma unroll
+      for (int g2 = 1; g2 < kNG; ++g2)
+        if (gg == g2) s = exp2i(eh[g2]);
+      const __half hv = __float2half_rn(v[k] * s);
+      hz[e] = *reinterpret_cast<const uint16_t *>(&hv);
+    }
+  }
+}
+
+// Largest |tap| of each of the tile's groups among this thread's staged taps, merged into
+// hmax[gg] (float bits) with shared-memory atomics.
+template <int kNG, int kPer>
+__device__ __forceinline__ void tap_absmax(uint32_t *hmax, const float (&v)[kPer], int halo,
+                                           int tid) {
+  const int stride = 258 + halo;
+  uint32_t m[kNG];
+#pragma unroll
+  for (int gg = 0; gg < kNG; ++gg) m[gg] = 0;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int e = tid + k * kGroupThreads;
+    const int gg = e / stride;
+    const uint32_t a = __float_as_uint(fabsf(v[k]));
+#pragma unroll
+    for (int g2 = 0; g2 < kNG; ++g2)
+      if (gg == g2) m[g2] = max(m[g2], a);
+  }
+#pragma unroll
+  for (int gg = 0; gg < kNG; ++gg) {
+    const uint32_t w = __reduce_max_sync(0xffffffffu, m[gg]);
+    if ((tid & 31) == 0 && w) atomicMax(&hmax[gg], w);
+  }
+}
+
+// The recomputation warp's work: y of one row of an out-of-range tile on the CUDA cores,
+// y[t][c] = q[t][c] sum_j h[g(c)][j] k[t-j][c] v[t-j][c] for the 64 channels of block `blk`,
+// taps in order, fp32, with the rows before the sequence from the history tensors (or zero),
+// rounded to bf16 and written to y in global memory.  Eight channels at a time, through L2.
+template <int kNG>
+__device__ __forceinline__ void recompute_row_fp32(const Params &p, int blk, int b, long long t) {
+  constexpr int kDG = kNC / kNG;
+  if (t >= p.L) return;  // rows past the end do not exist
+  const long long c0 = static_cast<long long>(blk) * kNC;
+  const long long row = (static_cast<long long>(b) * p.L + t) * p.D + c0;
+#pragma unroll 1
+  for (int c8 = 0; c8 < kNC / 8; ++c8) {
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    const float *hg = p.h + (static_cast<size_t>(blk) * kNG + (8 * c8) / kDG) * p.l_h;
+#pragma unroll 1
+    for (int j = 0; j < p.l_h; ++j) {
+      const long long s = t - j;
+      const __nv_bfloat16 *kr, *vr;
+      if (s >= 0) {
+        const long long off = (static_cast<long long>(b) * p.L + s) * p.D + c0;
+        kr = p.k + off;
+        vr = p.v + off;
+      } else if (p.hist_tiles && p.Lh + s >= 0) {
+        const long long off = (static_cast<long long>(b) * p.Lh + p.Lh + s) * p.D + c0;
+        kr = p.kh + off;
+        vr = p.vh + off;
+      } else {
+        break;
+      }
+      const uint4 kw = __ldg(reinterpret_cast<const uint4 *>(kr) + c8);
+      const uint4 vw = __ldg(reinterpret_cast<const uint4 *>(vr) + c8);
+      const float hj = __ldg(hg + j);
+      const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, vv[4] = {vw.x, vw.y, vw.z, vw.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = __uint_as_float(kk[e] << 16) * __uint_as_float(vv[e] << 16);
+        const float x1 = __uint_as_float(kk[e] & 0xFFFF0000u) * __uint_as_float(vv[e] & 0xFFFF0000u);
+        acc[2 * e] = fmaf(hj, x0, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(hj, x1, acc[2 * e + 1]);
+      }
+    }
+    const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(p.q + row) + c8);
+    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+    uint32_t ow[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float q0 = __uint_as_float(qw[e] << 16), q1 = __uint_as_float(qw[e] & 0xFFFF0000u);
+      const __nv_bfloat162 yv = __floats2bfloat162_rn(q0 * acc[2 * e], q1 * acc[2 * e + 1]);
+      ow[e] = *reinterpret_cast<const uint32_t *>(&yv);
+    }
+    reinterpret_cast<uint4 *>(p.y + row)[c8] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
   }
 }
 
@@ -280,13 +541,15 @@ __device__ __forceinline__ void build_band_tmem(uint32_t band_col, int band_cols
 }
 
 // kNG = 64 / d_g groups per tile (1, 2 or 4); MMA N = d_g.  kNH = ceil(halo / 128) earlier
-// tiles feed each tile's product (1 for l_h <= 129, up to 4 for l_h <= 513).
-template <int kNG, int kNH>
+// tiles feed each tile's product (1 for l_h <= 129, up to 4 for l_h <= 513).  kHooks builds
+// the test instantiation: the waits between roles use p.wait_ns, and p.fault == 1 withholds
+// the first accumulator arrive; the product instantiations carry neither.
+template <int kNG, int kNH, bool kHooks = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fir_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_y,
                   const __grid_constant__ CUtensorMap tm_kh,
-                  const __grid_constant__ CUtensorMap tm_vh, const Params p) {
+                  const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ Params p) {
   using Ly = Layout<kNH>;
   constexpr int kNQ = Ly::kNQ, kNX = Ly::kNX;
   constexpr int kOffKV = Ly::kOffKV, kOffQ = Ly::kOffQ, kOffX = Ly::kOffX, kOffBar = Ly::kOffBar,
@@ -296,7 +559,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 kBarYReady = Ly::kBarYReady, kBarXFull = Ly::kBarXFull,
                 kBarXEmpty = Ly::kBarXEmpty, kBarAccFull = Ly::kBarAccFull,
                 kBarAccEmpty = Ly::kBarAccEmpty, kBarAFull = Ly::kBarAFull,
-                kBarAEmpty = Ly::kBarAEmpty, kBarGate = Ly::kBarGate, kBarDone = Ly::kBarDone;
+                kBarAEmpty = Ly::kBarAEmpty, kBarGate = Ly::kBarGate, kBarDone = Ly::kBarDone,
+                kBarSegFull = Ly::kBarSegFull, kBarSegEmpty = Ly::kBarSegEmpty,
+                kBarGateDone = Ly::kBarGateDone, kBarEpiDone = Ly::kBarEpiDone;
+  constexpr int kNBad = Ly::kNBad;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -304,6 +570,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *q_st = smem + kOffQ;
   uint8_t *x_st = smem + kOffX;
   uint16_t *hz = reinterpret_cast<uint16_t *>(smem + Ly::kOffHz);
+  uint32_t *bad_count = reinterpret_cast<uint32_t *>(smem + Ly::kOffBad);
+  long long *bad_w = reinterpret_cast<long long *>(smem + Ly::kOffBad + 8);
+  uint32_t *segf = reinterpret_cast<uint32_t *>(smem + Ly::kOffSeg);
+  uint32_t *maxw = reinterpret_cast<uint32_t *>(smem + Ly::kOffMax);  // [2][8]: |h| x4, |kv|
+  const uint64_t lim = kHooks ? static_cast<uint64_t>(p.wait_ns) : kWaitTimeoutNs;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
   volatile int *abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
@@ -340,6 +611,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars[kBarGate], kGroupThreads);
     mbar_init(&bars[kBarDone], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[kBarSegFull + i], 1);   // gate warp 0, lane 0
+      mbar_init(&bars[kBarSegEmpty + i], 4);  // lane 0 of each epilogue warp
+    }
+    mbar_init(&bars[kBarGateDone], 4);        // lane 0 of each gate warp
+    mbar_init(&bars[kBarEpiDone], 1);         // the epilogue thread that issued the stores
+    for (int i = 0; i < 16; ++i) maxw[i] = 0;
+    *bad_count = 0;
     *abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
@@ -387,7 +666,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // The gate threads issue the loads of the first run's filter taps now; they land while the
   // CTA-wide barrier below completes and are written to shared memory after it.
-  bool over = false;
   float taps[Ly::kPer];
   const bool gate_role = warp >= kWarpGate0 && warp < kWarpGate0 + 4;
   if (gate_role && w_begin < w_end) {
@@ -407,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (!kv_done && kv_it.next(kv_t)) {
         const Item &t = kv_t;
         const int ks = kc % kNKV;
-        if (!thread_wait(&bars[kBarKVEmpty + ks], ((kc / kNKV) & 1) ^ 1, abort)) break;
+        if (!thread_wait(&bars[kBarKVEmpty + ks], ((kc / kNKV) & 1) ^ 1, abort, lim)) break;
         mbar_arrive_expect_tx(&bars[kBarKVFull + ks], 2 * kTileBytes);
         load_kv(ks, t);
         ++kc;
@@ -425,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (it.next(t)) {
         if (t.halo) continue;
         const int qs = qc % kNQ;
-        if (!thread_wait(&bars[kBarQEmpty + qs], ((qc / kNQ) & 1) ^ 1, abort)) break;
+        if (!thread_wait(&bars[kBarQEmpty + qs], ((qc / kNQ) & 1) ^ 1, abort, lim)) break;
         mbar_arrive_expect_tx(&bars[kBarQFull + qs], kTileBytes);
         tma_load_3d(q_st + qs * kTileBytes, &tm_q, &bars[kBarQFull + qs], t.g * kNC, t.i * kTM,
                     t.b);
@@ -458,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           x_seg = t.seg;
           seg_x0 = xc;
         }
-        if (!thread_wait(&bars[kBarXFull + xs], (xc / kNX) & 1, abort)) break;
+        if (!thread_wait(&bars[kBarXFull + xs], (xc / kNX) & 1, abort, lim)) break;
         if (t.halo) {
           ++xc;
           continue;
@@ -468,10 +746,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t.seg != cur_seg) {
           cur_seg = t.seg;
           const int use = p.nbuf == 2 ? (t.seg >> 1) : t.seg;
-          if (!thread_wait(&bars[kBarAFull + pa], use & 1, abort)) break;
+          if (!thread_wait(&bars[kBarAFull + pa], use & 1, abort, lim)) break;
         }
         const int as = ac % kNAcc;
-        if (!thread_wait(&bars[kBarAccEmpty + as], ((ac / kNAcc) & 1) ^ 1, abort)) break;
+        if (!thread_wait(&bars[kBarAccEmpty + as], ((ac / kNAcc) & 1) ^ 1, abort, lim)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + as * kNC;
         const uint32_t band0 = tmem_base + kBandCol0 + pa * kNG * p.band_cols;
@@ -509,7 +787,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc = 1;
           }
         }
-        umma_commit(&bars[kBarAccFull + as]);
+        // (test hook: withholding the first tile's arrive makes the epilogue's bounded wait
+        // run out, which exercises the timeout path)
+        if (!(kHooks && p.fault == 1 && ac == 0)) umma_commit(&bars[kBarAccFull + as]);
         // X slots go back to the gate warps after their last reader: the slot kNH items back
         // is read by no later tile; at the end of a segment every slot still held is free.
         if (xc >= seg_x0 + kNH) umma_commit(&bars[kBarXEmpty + (xc - kNH) % kNX]);
@@ -528,64 +808,116 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= kWarpGate0 && warp < kWarpGate0 + 4) {
     // ---------------------------------------------------------------- pre-gate + band build
     WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH, p.hist_tiles);
-    Item t;
-    uint32_t kc = 0, xc = 0;
-    int cur_seg = -1;
-    const int gtid = threadIdx.x - kWarpGate0 * 32;
-    uint32_t gphase = 0;  // phases of the gate threads' own barrier
-    while (it.next(t)) {
-      if (t.seg != cur_seg) {
-        cur_seg = t.seg;
-        if (t.seg > 0) {
+    Item t{};
+    uint32_t kc = 0, xc = 0, gphase = 0;
+    const int gtid = threadIdx.x - kWarpGate0 * 32, gw = warp - kWarpGate0;
+    constexpr uint32_t kReadMask = (2u << kNH) - 1u;
+    float sx = 1.f;        // 2^ex of the current run
+    bool run_bad = false;  // the run's scales were clamped: all its tiles go to fp32
+    uint32_t recent = 0;   // this warp's range flags of its last items (bit 0 = the newest)
+    // One item (halo or output tile) of the current run: X^T into its slot, then the range
+    // flags; an output tile reads its own rows and those of the kNH items before it.
+    auto gate_item = [&](auto scaled) -> bool {
+      constexpr bool kScaled = decltype(scaled)::value;
+      const int ks = kc % kNKV, xs = xc % kNX;
+      if (!warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort, lim)) return false;
+      if (!warp_wait(&bars[kBarXEmpty + xs], ((xc / kNX) & 1) ^ 1, abort, lim)) return false;
+      const uint32_t kbase = smem_u32(kv_st + ks * 2 * kTileBytes);
+      float mx = gate_x_tile<kScaled>(kbase, kbase + kTileBytes, smem_u32(x_st + xs * kTileBytes),
+                                      gw, lane, sx);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[kBarKVEmpty + ks]);
+      mbar_arrive(&bars[kBarXFull + xs]);
+      // the flags after the arrives: an fp16 overflow, or every value of some lane tiny but
+      // not zero (fp16 subnormals, or values that rounded to zero)
+      asm volatile("" : "+f"(mx)::"memory");
+      const bool bad = __ballot_sync(0xffffffffu, mx > 65504.f || (mx > 0.f && mx < kXTiny)) != 0u;
+      recent = (recent << 1) | (bad ? 1u : 0u);
+      if (!t.halo && (run_bad || (recent & kReadMask)) && lane == 0) {
+        // list the output tile for the recomputation warp
+        const uint32_t n = atomicAdd(bad_count, 1u);
+        if (n < kNBad) bad_w[n] = (static_cast<long long>(t.g / gmul) * p.B + t.b) * p.nT + t.i;
+      }
+      ++kc;
+      ++xc;
+      return true;
+    };
+    bool have = it.next(t), ok = true;
+    while (have && ok) {
+      // ------------------------------------ start of a sequence run (segment)
+      const int seg = t.seg, par = seg & 1;
+      ok = false;
+      do {
+        if (seg > 0) {
           // every gate thread has finished reading the previous taps ...
           tap_load(taps, p.h + static_cast<size_t>(t.g) * kNG * p.l_h, p.l_h, p.halo, kNG, gtid);
           mbar_arrive(&bars[kBarGate]);
-          if (!warp_wait(&bars[kBarGate], gphase++ & 1, abort)) break;
+          if (!warp_wait(&bars[kBarGate], gphase++ & 1, abort, lim)) break;
         }
-        tap_store(hz, taps, p.halo, kNG, gtid, over);
+        // ... the largest |h| of each group, once all have merged theirs ...
+        tap_absmax<kNG>(maxw + 8 * par, taps, p.halo, gtid);
+        mbar_arrive(&bars[kBarGate]);
+        if (!warp_wait(&bars[kBarGate], gphase++ & 1, abort, lim)) break;
+        int eh[kNG];
+        run_bad = false;
+#pragma unroll
+        for (int gg = 0; gg < kNG; ++gg) eh[gg] = tap_scale_exp(maxw[8 * par + gg], run_bad);
+        tap_store_scaled<kNG>(hz, taps, p.halo, gtid, eh);
         // ... and has written its share of the new ones
         mbar_arrive(&bars[kBarGate]);
-        if (!warp_wait(&bars[kBarGate], gphase++ & 1, abort)) break;
-        const int pa = p.nbuf == 2 ? (t.seg & 1) : 0, use = p.nbuf == 2 ? (t.seg >> 1) : t.seg;
-        if (use > 0 && !warp_wait(&bars[kBarAEmpty + pa], (use - 1) & 1, abort)) break;
+        if (!warp_wait(&bars[kBarGate], gphase++ & 1, abort, lim)) break;
+        const int pa = p.nbuf == 2 ? par : 0, use = p.nbuf == 2 ? (seg >> 1) : seg;
+        if (use > 0 && !warp_wait(&bars[kBarAEmpty + pa], (use - 1) & 1, abort, lim)) break;
 #pragma unroll 1
         for (int gg = 0; gg < kNG; ++gg)
           build_band_tmem(kBandCol0 + (pa * kNG + gg) * p.band_cols, p.band_cols, tmem_base,
                           hz + gg * (258 + p.halo) + 2, p.halo, warp & 3, lane);
         tc_fence_before_sync();
         mbar_arrive(&bars[kBarAFull + pa]);
-      }
-      const int ks = kc % kNKV, xs = xc % kNX;
-      if (!warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort)) break;
-      if (!warp_wait(&bars[kBarXEmpty + xs], ((xc / kNX) & 1) ^ 1, abort)) break;
-      // X^T (channel rows, 64 times per 128-byte row, two 8 KB K-blocks per tile, 128-byte
-      // swizzle) from the time-major k and v tiles: each warp moves 8 x 8 blocks with ldmatrix,
-      // forms k*v in fp32, rounds to fp16 and stores the blocks transposed with stmatrix.
-      const uint32_t kbase = smem_u32(kv_st + ks * 2 * kTileBytes);
-      const uint32_t vbase = kbase + kTileBytes;
-      const uint32_t xbase = smem_u32(x_st + xs * kTileBytes);
-      const int gw = warp - kWarpGate0, mat = lane >> 3, rr = lane & 7;
+        // x's scale from the largest |k v| of the run's first tile, once every warp has merged
+        // its own
+        const int ks = kc % kNKV;
+        if (!warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort, lim)) break;
+        const uint32_t kbase = smem_u32(kv_st + ks * 2 * kTileBytes);
+        const uint32_t xm = kv_absmax(kbase, kbase + kTileBytes, gw, lane);
+        if (lane == 0 && xm) atomicMax(&maxw[8 * par + 4], xm);
+        mbar_arrive(&bars[kBarGate]);
+        if (!warp_wait(&bars[kBarGate], gphase++ & 1, abort, lim)) break;
+        const int ex = x_scale_exp(maxw[8 * par + 4], eh[0], run_bad);
+        sx = exp2i(ex);
+        uint32_t fexp = 0;
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int bw = it * 4 + mat;
-        const int tg = gw * 4 + (bw >> 3), cg = bw & 7;  // 8-time group, 8-channel group
-        const uint32_t src = (tg * 8 + rr) * kRowBytes + ((cg ^ rr) << 4);
-        uint32_t kf[4], vf[4], xf[4];
-        ldsm_x4(kbase + src, kf);
-        ldsm_x4(vbase + src, vf);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) xf[e] = gate_pair(kf[e], vf[e], over);
-        const int c = cg * 8 + rr;
-        const uint32_t dst = (tg >> 3) * kKBlockBytes + c * kRowBytes + (((tg & 7) ^ rr) << 4);
-        stsm_x4_trans(xbase + dst, xf);
+        for (int gg = 0; gg < kNG; ++gg)
+          fexp |= (static_cast<uint32_t>(eh[gg] + ex) & 0xFFu) << (8 * gg);
+        // the other parity's maxima were last read before this run's barriers: reset them
+        if (gtid < 8) maxw[8 * (par ^ 1) + gtid] = 0;
+        // hand the run's scale to the epilogue (its slot was last read for the run two back)
+        if (gw == 0) {
+          if (!warp_wait(&bars[kBarSegEmpty + par], ((seg >> 1) & 1) ^ 1, abort, lim)) break;
+          if (lane == 0) {
+            segf[par] = fexp;
+            mbar_arrive(&bars[kBarSegFull + par]);
+          }
+        }
+        recent = 0;
+        ok = true;
+      } while (false);
+      if (!ok) break;
+      // ------------------------------------ the run's items, with or without x's scale
+      if (sx == 1.f) {
+        do {
+          if (!(ok = gate_item(std::false_type()))) break;
+          have = it.next(t);
+        } while (have && t.seg == seg);
+      } else {
+        do {
+          if (!(ok = gate_item(std::true_type()))) break;
+          have = it.next(t);
+        } while (have && t.seg == seg);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&bars[kBarKVEmpty + ks]);
-      mbar_arrive(&bars[kBarXFull + xs]);
-      ++kc;
-      ++xc;
     }
-    if (over) atomicOr(&g_device_status, kF16RangeBit);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[kBarGateDone]);
   } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
     // ---------------------------------------------------------------- epilogue
     const int et = threadIdx.x - kWarpEpi0 * 32;
@@ -593,12 +925,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_lane = quad * 32 + lane;   // MMA row = TMEM lane
     const int r = kTM - 1 - row_lane;        // tile row (time offset) of that lane
     WorkIter it(w_begin, w_end, p.nT, p.B, gmul, goff, kNH, p.hist_tiles);
-    Item t;
+    Item t{};
     uint32_t ac = 0, qc = 0;
-    while (it.next(t)) {
-      if (t.halo) continue;
+    // One output tile: the accumulator (divided by the run's 2^(eh + ex) when kScaled), times q,
+    // rounded to bf16 over the q stage, and stored.
+    auto epi_item = [&](auto scaled, uint32_t rfexp) -> bool {
+      constexpr bool kScaled = decltype(scaled)::value;
       const int as = ac % kNAcc, qs = qc % kNQ;
-      if (!warp_wait(&bars[kBarAccFull + as], (ac / kNAcc) & 1, abort)) break;
+      if (!warp_wait(&bars[kBarAccFull + as], (ac / kNAcc) & 1, abort, lim)) return false;
       tc_fence_after_sync();
       uint32_t a0[32], a1[32];
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + as * kNC;
@@ -609,9 +943,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       reg_fence(a1);
       tc_fence_before_sync();
       mbar_arrive(&bars[kBarAccEmpty + as]);
-      if (!warp_wait(&bars[kBarQFull + qs], (qc / kNQ) & 1, abort)) break;
-      uint8_t *qrow = q_st + qs * kTileBytes + r * (kNC * 2);
+      if (kScaled) {
+        // group gg's accumulator carries 2^(eh[gg] + ex) (byte gg of rfexp): divided out exactly
+        constexpr int kDG = kNC / kNG;
+        float fs[kNG];
 #pragma unroll
+        for (int gg = 0; gg < kNG; ++gg)
+          fs[gg] = exp2i(-static_cast<int>(static_cast<int8_t>(rfexp >> (8 * gg))));
+#pragma unroll
+        for (int ch = 0; ch < 32; ++ch) {
+          a0[ch] = __float_as_uint(__uint_as_float(a0[ch]) * fs[ch / kDG]);
+          a1[ch] = __float_as_uint(__uint_as_float(a1[ch]) * fs[(ch + 32) / kDG]);
+        }
+      }
+      if (!warp_wait(&bars[kBarQFull + qs], (qc / kNQ) & 1, abort, lim)) return false;
+      uint8_t *qrow = q_st + qs * kTileBytes + r * (kNC * 2);
+#pragma unroll kEpiUnroll
       for (int c = 0; c < 8; ++c) {
         uint4 *ptr = reinterpret_cast<uint4 *>(qrow + ((c ^ (r & 7)) << 4));
         const uint4 qv = *ptr;
@@ -630,10 +977,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[kBarYReady + qs]);
-      bool ok = true;
+      bool sok = true;
       if (et == 0) {
-        ok = thread_wait(&bars[kBarYReady + qs], (qc / kNQ) & 1, abort);
-        if (ok) {
+        sok = thread_wait(&bars[kBarYReady + qs], (qc / kNQ) & 1, abort, lim);
+        if (sok) {
           tma_store_3d(&tm_y, q_st + qs * kTileBytes, t.g * kNC, t.i * kTM, t.b);
           bulk_commit_group();
           // One store stays in flight: once the previous tile's store has read its shared
@@ -642,15 +989,84 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (qc > 0) mbar_arrive(&bars[kBarQEmpty + (qc + kNQ - 1) % kNQ]);
         }
       }
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!__all_sync(0xffffffffu, sok)) return false;
       ++ac;
       ++qc;
+      return true;
+    };
+    bool have = it.next(t), ok = true;
+    while (have && ok) {
+      // the run's scale exponents (eh + ex per group), once per run
+      const int seg = t.seg, sp = seg & 1;
+      if (!warp_wait(&bars[kBarSegFull + sp], (seg >> 1) & 1, abort, lim)) break;
+      const uint32_t rfexp = segf[sp];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarSegEmpty + sp]);
+      if (rfexp == 0) {
+        do {
+          if (!t.halo && !(ok = epi_item(std::false_type(), 0u))) break;
+          have = it.next(t);
+        } while (have && t.seg == seg);
+      } else {
+        do {
+          if (!t.halo && !(ok = epi_item(std::true_type(), rfexp))) break;
+          have = it.next(t);
+        } while (have && t.seg == seg);
+      }
     }
     if (et == 0) {
       // The stores must have read their shared memory before the CTA exits; their global
       // writes complete with the grid.
       bulk_wait_group_read<0>();
       if (qc > 0) mbar_arrive(&bars[kBarQEmpty + (qc + kNQ - 1) % kNQ]);
+      // Where the gate listed tiles for recomputation, their rows are rewritten after this
+      // CTA's stores have landed.
+      if (thread_wait(&bars[kBarGateDone], 0, abort, lim) &&
+          *reinterpret_cast<volatile uint32_t *>(bad_count) > 0) {
+        bulk_wait_group<0>();
+        fence_proxy_async_global();
+      }
+      mbar_arrive(&bars[kBarEpiDone]);
+    }
+  } else if (warp == kWarpFix) {
+    // ---------------------------------------------------------------- recomputation
+    // Sleeps until the epilogue is done (the whole kernel, so with a long limit), then
+    // recomputes in fp32 the tiles the gate listed: 4 rows of each per lane.
+    const uint64_t t0 = global_timer_ns();
+    bool go = false;
+    for (;;) {
+      if (mbar_try_wait(smem_u32(&bars[kBarEpiDone]), 0)) {
+        go = true;
+        break;
+      }
+      if (*abort) break;
+      if (global_timer_ns() - t0 > kFixWaitNs) {
+        *abort = 1;
+        atomicOr(&g_device_status, kTimeoutBit);
+        break;
+      }
+      __nanosleep(4000);
+    }
+    const uint32_t nbad = go ? *reinterpret_cast<volatile uint32_t *>(bad_count) : 0u;
+    if (nbad > 0) {
+      if (nbad <= static_cast<uint32_t>(kNBad)) {
+        for (uint32_t k = 0; k < nbad; ++k) {
+          const long long w = bad_w[k], seq = w / p.nT;
+          const int i = static_cast<int>(w - seq * p.nT);
+          const int g = static_cast<int>(seq / p.B) * gmul + goff;
+          const int b = static_cast<int>(seq % p.B);
+          for (int rr = lane; rr < kTM; rr += 32)
+            recompute_row_fp32<kNG>(p, g, b, static_cast<long long>(i) * kTM + rr);
+        }
+      } else {  // more than the list holds: every output tile of this CTA
+        WorkIter all(w_begin, w_end, p.nT, p.B, gmul, goff, kNH, p.hist_tiles);
+        Item t;
+        while (all.next(t))
+          if (!t.halo)
+            for (int rr = lane; rr < kTM; rr += 32)
+              recompute_row_fp32<kNG>(p, t.g, t.b, static_cast<long long>(t.i) * kTM + rr);
+      }
+      if (lane == 0) atomicOr(&g_device_status, kF16RangeBit);
     }
   }
 

@@ -12,6 +12,7 @@
 #include <type_traits>
 
 #include "hyena_conv.h"
+#include "hyena_conv_testing.h"
 #include "fir_bwd.cuh"
 #include "fir_cuda_core.cuh"
 #include "fir_fft.cuh"
@@ -70,7 +71,8 @@ int current_device(DeviceState *&ds) {
         {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 4>), hyena::tc::Layout<4>::kSmemBytes},
         {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<2, 1>), hyena::tc::Layout<1>::kSmemBytes},
         {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<2, 2>), hyena::tc::Layout<2>::kSmemBytes},
-        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<4, 1>), hyena::tc::Layout<1>::kSmemBytes}};
+        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<4, 1>), hyena::tc::Layout<1>::kSmemBytes},
+        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 1, true>), hyena::tc::Layout<1>::kSmemBytes}};
     for (const auto &k : kernels)
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
@@ -225,7 +227,14 @@ int select_algo(const Problem &P) {
   return HYENA_ALGO_DIRECT;
 }
 
-int launch_tensor(const Problem &P, cudaStream_t s) {
+// Test hooks of the tensor-core forward (hyena_testing_fwd_wait_fault): a shorter limit for the
+// waits between roles, and an arrive the MMA issuer withholds.  Zero = the product behaviour.
+struct TcTestHooks {
+  unsigned long long wait_ns = 0;
+  int fault = 0;
+};
+
+int launch_tensor(const Problem &P, cudaStream_t s, const TcTestHooks &hooks = TcTestHooks()) {
   DeviceState *ds = nullptr;
   if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
   EncodeTiledFn enc = encode_tiled();
@@ -250,6 +259,15 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
   const TcPlan plan = tc_plan(P);
   hyena::tc::Params p;
   p.h = P.h;
+  p.q = static_cast<const __nv_bfloat16 *>(P.q);
+  p.y = static_cast<__nv_bfloat16 *>(P.y);
+  p.k = static_cast<const __nv_bfloat16 *>(P.k);
+  p.v = static_cast<const __nv_bfloat16 *>(P.v);
+  p.kh = static_cast<const __nv_bfloat16 *>(hist ? P.kh : P.k);
+  p.vh = static_cast<const __nv_bfloat16 *>(hist ? P.vh : P.v);
+  p.D = P.D;
+  p.wait_ns = hooks.wait_ns ? hooks.wait_ns : hyena::kWaitTimeoutNs;
+  p.fault = hooks.fault;
   p.B = static_cast<int>(P.B);
   p.L = static_cast<int>(P.L);
   p.CB = static_cast<int>(P.D / hyena::tc::kNC);
@@ -289,6 +307,13 @@ int launch_tensor(const Problem &P, cudaStream_t s) {
   cfg.dynamicSmemBytes = hyena::tc::Layout<NH>::kSmemBytes;                                  \
   le = cudaLaunchKernelEx(&cfg, hyena::tc::fir_tc_kernel<NG, NH>, maps[0], maps[1], maps[2], \
                           maps[3], maps[4], maps[5], p)
+  if (hooks.wait_ns || hooks.fault) {  // the test instantiation (one group, one history tile)
+    if (plan.ng != 1 || plan.nh != 1) return HYENA_ERR_UNSUPPORTED;
+    cfg.dynamicSmemBytes = hyena::tc::Layout<1>::kSmemBytes;
+    le = cudaLaunchKernelEx(&cfg, hyena::tc::fir_tc_kernel<1, 1, true>, maps[0], maps[1], maps[2],
+                            maps[3], maps[4], maps[5], p);
+    return le == cudaSuccess && cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+  }
   switch (plan.ng * 8 + plan.nh) {
     case 9: HYENA_TC_LAUNCH(1, 1); break;
     case 10: HYENA_TC_LAUNCH(1, 2); break;
@@ -914,23 +939,27 @@ static __device__ __align__(256) float g_bwd_static_scratch[HYENA_BWD_STATIC_SCR
 namespace {
 
 struct StaticScratch {
-  std::once_flag once;
-  void *ptr = nullptr;
-  cudaError_t err = cudaSuccess;
+  std::mutex mu;
+  void *ptr = nullptr;  // null until a lookup succeeded
 };
 StaticScratch g_static_scratch[kMaxDevices];
 
-// The current device's address of g_bwd_static_scratch, looked up once per device (with that
-// device current) on the first call.
+// The current device's address of g_bwd_static_scratch.  The first successful lookup (with
+// that device current) is kept for the device; a failed one is not kept, so the next call
+// tries again.
 int static_scratch(void *&ptr) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HYENA_ERR_CUDA;
   StaticScratch *sc = &g_static_scratch[dev];
-  std::call_once(sc->once, [sc]() {
-    sc->err = cudaGetSymbolAddress(&sc->ptr, g_bwd_static_scratch);
-    if (sc->err == cudaSuccess && !sc->ptr) sc->err = cudaErrorInvalidSymbol;
-  });
-  if (sc->err != cudaSuccess) return HYENA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(sc->mu);
+  if (!sc->ptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_static_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();  // clear it, so that a later launch check does not report it
+      return HYENA_ERR_CUDA;
+    }
+    sc->ptr = p;
+  }
   ptr = sc->ptr;
   return HYENA_OK;
 }
@@ -1204,6 +1233,22 @@ int hyena_conv_bwd_static_scratch(const void *q, const void *k, const void *v, c
   if (static_scratch(ws) != HYENA_OK) return HYENA_ERR_CUDA;
   return run_bwd(P, dy, dq, dk, dv, dh, ws, HYENA_BWD_STATIC_SCRATCH_BYTES, stream,
                  HYENA_ALGO_AUTO);
+}
+
+int hyena_testing_fwd_fault(const void *q, const void *k, const void *v, const float *h, void *y,
+                            int64_t B, int64_t L, int64_t D, int d_g, int l_h, int fault,
+                            uint64_t wait_ns, cudaStream_t stream) {
+  const Problem P{q, k, v, h, y, B, L, D, d_g, l_h, 1, HYENA_DTYPE_BF16};
+  const int rc = validate(P);
+  if (rc == kEmpty) return HYENA_OK;
+  if (rc != HYENA_OK) return rc;
+  if ((fault != 0 && fault != 1) || wait_ns < 1000000ull || wait_ns > hyena::kWaitTimeoutNs)
+    return HYENA_ERR_INVALID_ARG;
+  if (!tensor_supported(P)) return HYENA_ERR_UNSUPPORTED;
+  TcTestHooks hooks;
+  hooks.wait_ns = wait_ns;
+  hooks.fault = fault;
+  return launch_tensor(P, stream, hooks);
 }
 
 int hyena_build_toeplitz(const float *h, float *H0, float *H1, float *H2_or_null, int G,

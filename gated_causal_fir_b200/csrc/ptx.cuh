@@ -63,10 +63,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with parity `parity` to complete.  Gives up (returns false)
-// when *abort is set by another role or after kWaitTimeoutNs; on a timeout it sets *abort
-// and ORs `timeout_bit` into *status so that the host can see it.
+// when *abort is set by another role or after limit_ns; on a timeout it sets *abort and ORs
+// `timeout_bit` into *status so that the host can see it.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          unsigned int *status, unsigned int timeout_bit) {
+                                          unsigned int *status, unsigned int timeout_bit,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
@@ -74,13 +75,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((polls & 63u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs || polls >= kWaitMaxPolls) {
+      if (global_timer_ns() - t0 > limit_ns || polls >= kWaitMaxPolls) {
         *abort = 1;
         atomicOr(status, timeout_bit);
         return false;
       }
     }
   }
+}
+
+// ------------------------------------------------------------------------------ packed math
+// Two fp32 products in one instruction (packed fp32 pipe of sm_100): d_i = a_i * b_i, each
+// rounded to nearest like a scalar fp32 multiply.
+__device__ __forceinline__ void mul_f32x2(float &d0, float &d1, float a0, float a1, float b0,
+                                          float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Running maximum of magnitudes of two fp16 lanes: |m| = max(|m|, |x|) per lane (the sign
+// bits of m carry no meaning).
+__device__ __forceinline__ void absmax_f16x2(uint32_t &m, uint32_t x) {
+  asm("max.xorsign.abs.f16x2 %0, %0, %1;" : "+r"(m) : "r"(x));
 }
 
 // ------------------------------------------------------------------------------ launch order
@@ -143,6 +164,12 @@ __device__ __forceinline__ void bulk_wait_group() {
 // (TMA engine, tensor cores).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Orders this thread's earlier async-proxy global accesses (completed bulk stores) before its
+// later generic-proxy ones.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ------------------------------------------------------------------------------ ldmatrix
@@ -285,6 +312,13 @@ template <int N>
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
 #pragma unroll
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i])::"memory");
+}
+
+// The same for fp32 values: each must be computed at this point of the instruction stream.
+template <int N>
+__device__ __forceinline__ void reg_fence_f(float (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+f"(r[i])::"memory");
 }
 
 // Shared-memory matrix descriptor of tcgen05 (version 1).  Byte offsets are given in bytes and

@@ -22,9 +22,13 @@
  *   - B == 0 or L == 0 is an empty problem: nothing is launched and HYENA_OK is returned.
  *   - Return value: HYENA_OK or one of the HYENA_ERR_* codes below.  Argument errors are
  *     detected on the host before anything is queued.  HYENA_ERR_CUDA reports a launch
- *     failure (cudaGetLastError).  Errors that happen inside a running kernel (a bounded wait
- *     that ran out, fp16 operand overflow) are recorded in a per-device status word that
- *     hyena_device_status() reads.
+ *     failure (cudaGetLastError).  Events inside a running kernel (a bounded wait that ran
+ *     out; a tile recomputed in fp32 because an fp16 operand left its range) are recorded in
+ *     a per-device status word that hyena_device_status() reads.
+ *   - The library keeps per-device state from the first call on each device (kernel
+ *     attributes, the host-buffer pipeline's streams, the address of the fixed scratch of
+ *     hyena_conv_bwd_static_scratch).  cudaDeviceReset destroys what it refers to: do not call
+ *     the library on a device after resetting it in the same process.
  */
 #ifndef HYENA_CONV_H
 #define HYENA_CONV_H
@@ -69,8 +73,12 @@ enum hyena_algo {
 /* Bits of the per-device status word (hyena_device_status). */
 enum hyena_device_status_bits {
     HYENA_DEVICE_TIMEOUT = 1u,      /* a bounded wait inside a kernel gave up; output invalid */
-    HYENA_DEVICE_F16_RANGE = 2u     /* |k*v| or |h| exceeded the fp16 operand range (65504)
-                                       in the tensor-core path; affected outputs are inf/nan */
+    HYENA_DEVICE_F16_RANGE = 2u     /* information, not an error: in the tensor-core forward
+                                       an fp16 operand left its range even after the kernel's
+                                       power-of-two scaling (a scaled |k*v| above 65504, or a
+                                       warp's rows all far below the sequence run's first
+                                       tile), and the tiles reading it were recomputed in fp32
+                                       on the CUDA cores; outputs are valid */
 };
 
 /*
@@ -81,6 +89,11 @@ enum hyena_device_status_bits {
  * result does not depend on l_b.  The kernels pick their own internal block size.  Filters
  * longer than the tensor path's limit (HYENA_ALGO_TENSOR above) run on the CUDA-core direct
  * sum; hyena_conv_fwd_fft is the faster entry point for them.  All tensors 2-byte aligned.
+ * Precision: on the tensor-core path the MMA operands are fp16 (x = k v formed exactly in
+ * fp32; h), each scaled by a power of two first (per group for h, per sequence run for x),
+ * with fp32 accumulation; tiles whose scaled operands still leave fp16's range are recomputed
+ * in fp32 on the CUDA cores (HYENA_DEVICE_F16_RANGE).  The CUDA-core paths are fp32.  y is
+ * rounded once to bf16.
  */
 int hyena_conv_fwd(const void *q, const void *k, const void *v, const float *h, void *y,
                    int64_t B, int64_t L, int64_t D, int d_g, int l_h, int l_b,
@@ -276,7 +289,8 @@ int hyena_select_bwd_algo(const void *q, const void *k, const void *v, const flo
  *     exceeds HYENA_BWD_STATIC_SCRATCH_BYTES (e.g. the D = 4096, d_g = 64, l_h = 128 shape
  *     above B * L = 16384 tokens); use hyena_conv_bwd with a workspace there.
  *   - The first call on each device looks up the array's address (cudaGetSymbolAddress) with
- *     that device current; make that first call before any stream capture.
+ *     that device current and keeps it (a failed lookup returns HYENA_ERR_CUDA and is tried
+ *     again on the next call); make that first call before any stream capture.
  *   - Calls that overlap in time on one device (different streams, or threads) share the array
  *     and race: serialise them.  Nothing in the array has to start at zero.
  */

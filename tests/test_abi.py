@@ -26,6 +26,24 @@ def test_exports_every_header_function(lib):
     assert set(declared) == set(_native.SIGNATURES), "binding table out of step with the header"
     for name in declared:
         assert hasattr(lib, name), name
+    testing = _native.header_functions(_native.TESTING_HEADER_PATH)
+    assert set(testing) == set(_native.TESTING_SIGNATURES)
+    for name in testing:
+        assert hasattr(lib, name), name
+
+
+def test_testing_entry_point_rejects_bad_arguments(lib):
+    """The test hook checks its own arguments on the host (nothing is launched)."""
+    fn = lib.hyena_testing_fwd_fault
+    p = 256
+    # fault out of range, wait limit out of [1 ms, 2 s], unsupported shape
+    assert fn(p, p, p, p, 1 << 20, 1, 128, 64, 64, 7, 2, 10 ** 7, None) == _native.HYENA_ERR_INVALID_ARG
+    assert fn(p, p, p, p, 1 << 20, 1, 128, 64, 64, 7, 1, 10 ** 5, None) == _native.HYENA_ERR_INVALID_ARG
+    assert fn(p, p, p, p, 1 << 20, 1, 128, 64, 64, 7, 1, 3 * 10 ** 9, None) == \
+        _native.HYENA_ERR_INVALID_ARG
+    assert fn(p, p, p, p, 1 << 20, 1, 128, 96, 32, 40, 1, 10 ** 7, None) == \
+        _native.HYENA_ERR_UNSUPPORTED
+    assert fn(p, p, p, p, 1 << 20, 0, 128, 64, 64, 7, 1, 10 ** 7, None) == _native.HYENA_OK  # empty
 
 
 def test_status_strings_and_version(lib):
