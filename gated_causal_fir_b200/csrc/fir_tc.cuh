@@ -156,7 +156,8 @@ constexpr unsigned kF16RangeBit = 2u; // HYENA_DEVICE_F16_RANGE
 constexpr int kTapExpTarget = 7;
 constexpr int kXExpTarget = 8;
 constexpr int kXBalancedLo = -6, kXBalancedHi = 8;  // accepted floor(log2 max |k v 2^ex|)
-constexpr float kXTiny = 0.000244140625f;  // 2^-12
+constexpr uint32_t kXTinyBits = 0x39800000u;  // 2^-12 as float bits
+constexpr uint32_t kF16MaxBits = 0x477FE000u;  // 65504 as float bits
 
 struct Params {
   const float *h;   // [D / d_g, l_h]
@@ -811,29 +812,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     Item t{};
     uint32_t kc = 0, xc = 0, gphase = 0;
     const int gtid = threadIdx.x - kWarpGate0 * 32, gw = warp - kWarpGate0;
-    constexpr uint32_t kReadMask = (2u << kNH) - 1u;
+    constexpr uint32_t kReadMask = ((2u << kNH) - 1u) | 0x80000000u;
     float sx = 1.f;        // 2^ex of the current run
-    bool run_bad = false;  // the run's scales were clamped: all its tiles go to fp32
-    uint32_t recent = 0;   // this warp's range flags of its last items (bit 0 = the newest)
+    // This warp's range flags of its last items (bit 0 = the newest); bit 31 stays set for a
+    // run whose scales were clamped (all its tiles go to fp32).
+    uint32_t recent = 0;
     // One item (halo or output tile) of the current run: X^T into its slot, then the range
     // flags; an output tile reads its own rows and those of the kNH items before it.
-    auto gate_item = [&](auto scaled) -> bool {
+    float first_mx = 0.f;  // this lane's largest scaled |x| of the run's first tile
+    auto gate_item = [&](auto scaled, bool built) -> bool {
       constexpr bool kScaled = decltype(scaled)::value;
       const int ks = kc % kNKV, xs = xc % kNX;
-      if (!warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort, lim)) return false;
-      if (!warp_wait(&bars[kBarXEmpty + xs], ((xc / kNX) & 1) ^ 1, abort, lim)) return false;
-      const uint32_t kbase = smem_u32(kv_st + ks * 2 * kTileBytes);
-      float mx = gate_x_tile<kScaled>(kbase, kbase + kTileBytes, smem_u32(x_st + xs * kTileBytes),
-                                      gw, lane, sx);
+      float mx = first_mx;  // the run's first tile was converted at the run's start
+      if (!built) {
+        if (!warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort, lim)) return false;
+        if (!warp_wait(&bars[kBarXEmpty + xs], ((xc / kNX) & 1) ^ 1, abort, lim)) return false;
+        const uint32_t kbase = smem_u32(kv_st + ks * 2 * kTileBytes);
+        mx = gate_x_tile<kScaled>(kbase, kbase + kTileBytes, smem_u32(x_st + xs * kTileBytes),
+                                  gw, lane, sx);
+      }
       fence_proxy_async_smem();
       mbar_arrive(&bars[kBarKVEmpty + ks]);
       mbar_arrive(&bars[kBarXFull + xs]);
-      // the flags after the arrives: an fp16 overflow, or every value of some lane tiny but
-      // not zero (fp16 subnormals, or values that rounded to zero)
-      asm volatile("" : "+f"(mx)::"memory");
-      const bool bad = __ballot_sync(0xffffffffu, mx > 65504.f || (mx > 0.f && mx < kXTiny)) != 0u;
-      recent = (recent << 1) | (bad ? 1u : 0u);
-      if (!t.halo && (run_bad || (recent & kReadMask)) && lane == 0) {
+      // an fp16 overflow, or every value of some lane tiny but not zero (fp16 subnormals, or
+      // values that rounded to zero); the bits of a non-negative float order like the float
+      const uint32_t mb = __float_as_uint(mx);
+      const bool lane_bad = mb > kF16MaxBits || mb - 1u < kXTinyBits - 1u;
+      recent = (recent << 1) | (__any_sync(0xffffffffu, lane_bad) ? 1u : 0u);
+      if ((recent & kReadMask) && !t.halo && lane == 0) {
         // list the output tile for the recomputation warp
         const uint32_t n = atomicAdd(bad_count, 1u);
         if (n < kNBad) bad_w[n] = (static_cast<long long>(t.g / gmul) * p.B + t.b) * p.nT + t.i;
@@ -859,7 +865,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bars[kBarGate]);
         if (!warp_wait(&bars[kBarGate], gphase++ & 1, abort, lim)) break;
         int eh[kNG];
-        run_bad = false;
+        bool run_bad = false;  // the run's scales were clamped: all its tiles go to fp32
 #pragma unroll
         for (int gg = 0; gg < kNG; ++gg) eh[gg] = tap_scale_exp(maxw[8 * par + gg], run_bad);
         tap_store_scaled<kNG>(hz, taps, p.halo, gtid, eh);
@@ -874,16 +880,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                           hz + gg * (258 + p.halo) + 2, p.halo, warp & 3, lane);
         tc_fence_before_sync();
         mbar_arrive(&bars[kBarAFull + pa]);
-        // x's scale from the largest |k v| of the run's first tile, once every warp has merged
-        // its own
-        const int ks = kc % kNKV;
+        // x's scale from the largest |k v| of the run's first tile: that tile is converted
+        // unscaled first (no scale is the usual case), every warp merges its maximum, and the
+        // tile is converted again, scaled, only if the run needs it
+        const int ks = kc % kNKV, xs = xc % kNX;
         if (!warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort, lim)) break;
+        if (!warp_wait(&bars[kBarXEmpty + xs], ((xc / kNX) & 1) ^ 1, abort, lim)) break;
         const uint32_t kbase = smem_u32(kv_st + ks * 2 * kTileBytes);
-        const uint32_t xm = kv_absmax(kbase, kbase + kTileBytes, gw, lane);
+        const uint32_t xbase = smem_u32(x_st + xs * kTileBytes);
+        const float m0 = gate_x_tile<false>(kbase, kbase + kTileBytes, xbase, gw, lane, 1.f);
+        const uint32_t xm = __reduce_max_sync(0xffffffffu, __float_as_uint(m0));
         if (lane == 0 && xm) atomicMax(&maxw[8 * par + 4], xm);
         mbar_arrive(&bars[kBarGate]);
         if (!warp_wait(&bars[kBarGate], gphase++ & 1, abort, lim)) break;
         const int ex = x_scale_exp(maxw[8 * par + 4], eh[0], run_bad);
+        if (ex != 0) gate_x_tile<true>(kbase, kbase + kTileBytes, xbase, gw, lane, exp2i(ex));
+        first_mx = m0 * exp2i(ex);  // exact: the lane's maximum after the scale
         sx = exp2i(ex);
         uint32_t fexp = 0;
 #pragma unroll
@@ -899,19 +911,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bars[kBarSegFull + par]);
           }
         }
-        recent = 0;
+        recent = run_bad ? 0x80000000u : 0u;
         ok = true;
       } while (false);
       if (!ok) break;
-      // ------------------------------------ the run's items, with or without x's scale
+      // ------------------------------------ the run's items, with or without x's scale (the
+      // first one's X is built; it finishes like the others)
+      bool first = true;
       if (sx == 1.f) {
         do {
-          if (!(ok = gate_item(std::false_type()))) break;
+          if (!(ok = gate_item(std::false_type(), first))) break;
+          first = false;
           have = it.next(t);
         } while (have && t.seg == seg);
       } else {
         do {
-          if (!(ok = gate_item(std::true_type()))) break;
+          if (!(ok = gate_item(std::true_type(), first))) break;
+          first = false;
           have = it.next(t);
         } while (have && t.seg == seg);
       }
@@ -1030,22 +1046,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kWarpFix) {
     // ---------------------------------------------------------------- recomputation
-    // Sleeps until the epilogue is done (the whole kernel, so with a long limit), then
-    // recomputes in fp32 the tiles the gate listed: 4 rows of each per lane.
-    const uint64_t t0 = global_timer_ns();
+    // Once the gate has listed every tile (it finishes well before the epilogue) there is
+    // usually nothing to do and the warp leaves.  Otherwise it sleeps until the epilogue is done
+    // (possibly most of the kernel, so with a long limit) and recomputes the listed tiles in
+    // fp32: 4 rows of each per lane.
     bool go = false;
-    for (;;) {
-      if (mbar_try_wait(smem_u32(&bars[kBarEpiDone]), 0)) {
-        go = true;
-        break;
+    if (warp_wait(&bars[kBarGateDone], 0, abort, lim) &&
+        *reinterpret_cast<volatile uint32_t *>(bad_count) > 0) {
+      const uint64_t t0 = global_timer_ns();
+      for (;;) {
+        if (mbar_try_wait(smem_u32(&bars[kBarEpiDone]), 0)) {
+          go = true;
+          break;
+        }
+        if (*abort) break;
+        if (global_timer_ns() - t0 > kFixWaitNs) {
+          *abort = 1;
+          atomicOr(&g_device_status, kTimeoutBit);
+          break;
+        }
+        __nanosleep(1000);
       }
-      if (*abort) break;
-      if (global_timer_ns() - t0 > kFixWaitNs) {
-        *abort = 1;
-        atomicOr(&g_device_status, kTimeoutBit);
-        break;
-      }
-      __nanosleep(4000);
     }
     const uint32_t nbad = go ? *reinterpret_cast<volatile uint32_t *>(bad_count) : 0u;
     if (nbad > 0) {
