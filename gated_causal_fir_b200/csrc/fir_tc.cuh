@@ -1050,24 +1050,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     // usually nothing to do and the warp leaves.  Otherwise it sleeps until the epilogue is done
     // (possibly most of the kernel, so with a long limit) and recomputes the listed tiles in
     // fp32: 4 rows of each per lane.
-    bool go = false;
-    if (warp_wait(&bars[kBarGateDone], 0, abort, lim) &&
-        *reinterpret_cast<volatile uint32_t *>(bad_count) > 0) {
+    // Both waits sleep between polls: this warp shares its scheduler with a gate warp and an
+    // epilogue warp, and spinning would take issue slots from them.
+    auto sleep_wait = [&](int bar) -> bool {
       const uint64_t t0 = global_timer_ns();
       for (;;) {
-        if (mbar_try_wait(smem_u32(&bars[kBarEpiDone]), 0)) {
-          go = true;
-          break;
-        }
-        if (*abort) break;
+        if (mbar_try_wait(smem_u32(&bars[bar]), 0)) return true;
+        if (*abort) return false;
         if (global_timer_ns() - t0 > kFixWaitNs) {
           *abort = 1;
           atomicOr(&g_device_status, kTimeoutBit);
-          break;
+          return false;
         }
         __nanosleep(1000);
       }
-    }
+    };
+    const bool go = sleep_wait(kBarGateDone) &&
+                    *reinterpret_cast<volatile uint32_t *>(bad_count) > 0 &&
+                    sleep_wait(kBarEpiDone);
     const uint32_t nbad = go ? *reinterpret_cast<volatile uint32_t *>(bad_count) : 0u;
     if (nbad > 0) {
       if (nbad <= static_cast<uint32_t>(kNBad)) {
