@@ -12,11 +12,14 @@ stream, and reduced as the max over ranks.  Under torchrun each rank runs an ind
 replica on its own batch (weak scaling, no collective on the data path).
 
 Rank 0 prints one JSON line.  Besides the throughput it reports the roofline of the kernel
-(algorithmic bytes / mean launch time vs the measured HBM copy bandwidth), SM clocks sampled
+(algorithmic bytes / mean launch time vs the measured HBM copy bandwidth, with the median and
+minimum of a separate pass that times each launch on its own), SM clocks sampled
 through NVML during the timed region, an end-to-end figure through
 ``hyena_conv_fwd_from_host`` (pinned host buffers, copies inside the timed region) and the
 fp64 oracle timed on the host cores as a CPU baseline.  Beside the forward it reports the
-backward (``backward``) and two longer-filter cases (``long_filters``: the Hyena-LI-shaped
+backward (``backward``), the forward on the other configurations of the workload table
+(``configs``: SE, MR batched, MR with 2^20 tokens, each with its roofline) and two
+longer-filter cases (``long_filters``: the Hyena-LI-shaped
 workload through the FFT entry point, and l_h = 513 on the tensor-core path) and, as context,
 the pages' naive baseline (``comparator``: PyTorch's depthwise F.conv1d with the gating
 products, on the same inputs).
@@ -47,6 +50,8 @@ def parse():
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--workload", default="mr")
+    p.add_argument("--algo", default="auto", choices=["auto", "tensor", "window", "direct"],
+                   help="forward algorithm of the timed launches (auto = the library's choice)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -59,6 +64,10 @@ def parse():
                    help="timed steps of the torch F.conv1d comparator; 0 skips")
     p.add_argument("--long-steps", type=int, default=20,
                    help="timed steps of the long-filter measurements (FFT, l_h = 513); 0 skips")
+    p.add_argument("--stat-launches", type=int, default=300,
+                   help="launches timed one by one for the median and minimum (>= 100)")
+    p.add_argument("--config-steps", type=int, default=20,
+                   help="timed steps of the other configurations (SE, MR batched, MR 1M); 0 skips")
     return p.parse_args()
 
 
@@ -244,12 +253,91 @@ def run_reference(args, wl, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(wl),
+        "data": "synthetic", "config": workload_config(wl, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
     del torch
+
+
+def launch_stats(launch, n, stream):
+    """Per-launch durations of n back-to-back launches (one CUDA event between consecutive
+    launches on the launching stream): mean, median and minimum in microseconds."""
+    import torch
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(n):
+        launch(i)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    us = [1e3 * ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
+    return {"launches": n, "mean_us": statistics.fmean(us), "median_us": statistics.median(us),
+            "min_us": min(us)}
+
+
+def time_configs(args, stream, dev, D, g, _native, peak, peak_kind):
+    """The forward on the other configurations of the workload table (SE, MR batched, MR with
+    2^20 tokens), timed like the headline: CUDA events over K back-to-back launches on the
+    launching stream (max over ranks), plus per-launch median and minimum.  Inputs: three
+    rotating sets where they fit in a few GiB, one set beyond (then every step's inputs exceed
+    the 126 MB L2 on their own).  Algorithmic bytes per launch: q, k, v read and y written, plus
+    the filters."""
+    import torch
+    from gated_causal_fir_b200.workloads import WORKLOADS, make_inputs
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    out = {}
+    for name in ("se", "mr_batched", "mr_1m"):
+        wl = WORKLOADS[name]
+        nsets = 3 if wl.algorithmic_bytes() * 3 < (8 << 30) else 1
+        sets = [make_inputs(wl, device=dev, seed=wl.seed + 101 * s, l_slice=1 << 16)
+                for s in range(nsets)]
+        ys = [torch.empty_like(x[0]) for x in sets]
+        # the inputs are made on torch's current stream and read on `stream` (non-blocking):
+        # they must be complete, and their temporaries retired, before the first launch
+        torch.cuda.synchronize()
+        code = g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16
+        algo = g.hyena_select_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, code)
+        cfn = _native.lib().hyena_conv_fwd_f32 if wl.dtype == "f32" else _native.lib().hyena_conv_fwd
+        cargs = [(x[0].data_ptr(), x[1].data_ptr(), x[2].data_ptr(), x[3].data_ptr(),
+                  y.data_ptr(), wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, sh)
+                 for x, y in zip(sets, ys)]
+
+        def launch(i):
+            rc = cfn(*cargs[i % nsets])
+            if rc != 0:
+                raise _native.HyenaError(name, rc)
+
+        for i in range(max(3, args.warmup)):
+            launch(i)
+        torch.cuda.synchronize()
+        K = args.config_steps
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        D.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(K):
+            launch(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = D.max_over_ranks(e0.elapsed_time(e1), device=dev) / K
+        stats = launch_stats(launch, max(100, K) if wl.tokens <= (1 << 16) else K, stream)
+        nbytes = wl.algorithmic_bytes()
+        achieved = nbytes / (ms / 1e3) / 1e9
+        kernel = {g.HYENA_ALGO_TENSOR: "fir_tc_kernel", g.HYENA_ALGO_WINDOW: "fir_window_kernel",
+                  g.HYENA_ALGO_DIRECT: "fir_tiled_kernel"}[algo]
+        out[name] = {"workload": wl.describe(), "ms_per_step": ms, "steps": K,
+                     "value": D.env_world()[2] * wl.tokens / (ms / 1e3), "unit": UNIT,
+                     "gpu_launches": K, "kernel": kernel, "launch_stats": stats,
+                     "l2": "%d rotating input sets" % nsets,
+                     "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
+                                  "unit": "GB/s", "frac": achieved / peak,
+                                  "algorithmic_bytes_per_launch": nbytes,
+                                  "peak_source": peak_kind}}
+        del sets, ys, cargs
+        torch.cuda.empty_cache()
+    return out
 
 
 def time_long_filters(args, stream, dev, D, g, _native, peak, peak_kind):
@@ -272,9 +360,11 @@ def time_long_filters(args, stream, dev, D, g, _native, peak, peak_kind):
                                               "mr", seed=6), False)):
         sets = [make_inputs(wl, device=dev, seed=wl.seed + 101 * s) for s in range(2)]
         ys = [torch.empty_like(x[0]) for x in sets]
+        torch.cuda.synchronize()  # inputs complete before `stream` reads them
         if fft:
             need = g.hyena_conv_fwd_fft_workspace_bytes(wl.B, wl.L, wl.D, wl.d_g, wl.l_h)
             ws = torch.empty(need, dtype=torch.uint8, device=dev)
+            torch.cuda.synchronize()
             cfn = _native.lib().hyena_conv_fwd_fft
             cargs = [(x[0].data_ptr(), x[1].data_ptr(), x[2].data_ptr(), x[3].data_ptr(),
                       y.data_ptr(), wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, 0, ws.data_ptr(),
@@ -332,6 +422,7 @@ def time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind):
         dy = make_grad(wl, device=dev, seed=wl.seed + 977 * n)
         dq, dk, dv, dh = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q),
                           torch.empty_like(h))
+        torch.cuda.synchronize()  # dy complete before `stream` reads it
         g.hyena_conv_bwd(q, k, v, h, dy, wl.d_g, wl.l_b, workspace=ws,
                          grads=(dq, dk, dv, dh), stream=stream)  # binding checks, once
         bufs.append((q, k, v, h, dy, dq, dk, dv, dh))
@@ -379,11 +470,13 @@ def time_backward(args, wl, sets, stream, dev, D, g, _native, peak, peak_kind):
                          "note": "whole backward (all its kernels) per step"}}
 
 
-def workload_config(wl):
+def workload_config(wl, world):
+    """The workload a line measures (the same keys on both arms of the bench)."""
     return {"workload": wl.describe(), "B": wl.B, "L": wl.L, "D": wl.D, "d_g": wl.d_g,
             "l_h": wl.l_h, "l_b": wl.l_b, "io_dtype": wl.dtype, "filters": wl.filt,
             "l2": "3 rotating input sets (%.0f MiB) > 126 MB L2"
-                  % (3 * wl.algorithmic_bytes() / 2 ** 20)}
+                  % (3 * wl.algorithmic_bytes() / 2 ** 20),
+            "parallelism": "replicas x%d" % world}
 
 
 def main():
@@ -412,8 +505,13 @@ def main():
         q, k, v, h = make_inputs(wl, device=dev, seed=D.rank_seed(wl.seed + 101 * s, rank),
                                  l_slice=1 << 16)
         sets.append((q, k, v, h, torch.empty_like(q)))
-    algo = g.hyena_select_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b,
-                               g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16)
+    # The inputs are made on torch's current stream and read on `stream` (a non-blocking
+    # stream): they must be complete, and their temporaries retired, before the first launch.
+    torch.cuda.synchronize()
+    dcode = g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16
+    algo = g.hyena_select_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, dcode)
+    forced = {"auto": None, "tensor": g.HYENA_ALGO_TENSOR, "window": g.HYENA_ALGO_WINDOW,
+              "direct": g.HYENA_ALGO_DIRECT}[args.algo]
     fwd = g.hyena_conv_fwd_f32 if wl.dtype == "f32" else g.hyena_conv_fwd
     stream = torch.cuda.Stream(device=dev)
 
@@ -426,6 +524,12 @@ def main():
     sh = ctypes.c_void_p(stream.cuda_stream)
     cargs = [(q.data_ptr(), k.data_ptr(), v.data_ptr(), h.data_ptr(), y.data_ptr(), wl.B, wl.L,
               wl.D, wl.d_g, wl.l_h, wl.l_b, sh) for q, k, v, h, y in sets]
+    if forced is not None:  # the same launches through hyena_conv_fwd_ex with the algorithm
+        for x in sets:
+            g.hyena_conv_fwd_ex(*x[:4], wl.d_g, wl.l_b, algo=forced, y=x[4], stream=stream)
+        cfn = _native.lib().hyena_conv_fwd_ex
+        cargs = [c[:11] + (dcode, forced, sh) for c in cargs]
+        algo = forced
 
     def launch(i):
         rc = cfn(*cargs[i % 3])
@@ -458,6 +562,10 @@ def main():
     # The timed region launches this kernel and nothing else, back to back on one stream: its
     # mean launch duration is the region's event time over K.
     mean_launch_ms = max_ms / K
+
+    # Per-launch median and minimum (outside the timed region, the same launches one by one).
+    stats = launch_stats(launch, max(100, args.stat_launches, K), stream)
+    assert g.hyena_device_status(clear=True) == 0, "device status raised during the launches"
 
     # End to end through the host-buffer entry point, pinned buffers, copies timed.
     e2e = None
@@ -496,6 +604,11 @@ def main():
         fwd(q, k, v, h, wl.d_g, wl.l_b, y=y, stream=stream)
         comparator = time_conv1d_comparator(args, wl, sets, stream, y)
 
+    configs = None
+    if args.config_steps > 0 and wl.name == "mr":
+        peak, peak_kind = measured_peak_hbm()
+        configs = time_configs(args, stream, dev, D, g, _native, peak, peak_kind)
+
     long_filters = None
     if args.long_steps > 0 and wl.name == "mr":
         peak, peak_kind = measured_peak_hbm()
@@ -526,19 +639,21 @@ def main():
             "value": world * wl.tokens * K / (max_ms / 1e3), "unit": UNIT,
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": max_ms / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": wl.dtype, "data": "synthetic", "config": dict(
-                workload_config(wl), parallelism="replicas x%d" % world,
-                mma="f16 x f16 -> f32 (tensor path)" if algo == g.HYENA_ALGO_TENSOR
-                else "fp32 FFMA"),
+            "dtype": wl.dtype, "data": "synthetic", "config": workload_config(wl, world),
+            "mma": "f16 x f16 -> f32 (tensor path)" if algo == g.HYENA_ALGO_TENSOR
+            else "fp32 FFMA",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": "%s (MEASURED_PEAKS hbm_gbs)" % peak_kind
                          if peak_kind == "measured" else "fallback 6.65 TB/s",
                          "algorithmic_bytes_per_launch": bytes_per_launch,
-                         "mean_launch_us": 1e3 * mean_launch_ms, "kernel": kernel},
+                         "mean_launch_us": 1e3 * mean_launch_ms, "kernel": kernel,
+                         "median_launch_us": stats["median_us"], "min_launch_us": stats["min_us"],
+                         "launch_stats": stats},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K,
             "clocks": clocks.summary(t_wall0, t_wall1),
-            "backward": bwd, "long_filters": long_filters, "comparator": comparator,
+            "backward": bwd, "configs": configs, "long_filters": long_filters,
+            "comparator": comparator,
             "kernel_algo": g.ALGO_NAMES[algo], "device_status": status, "parity": parity,
             "wall_s_timed_region": t_wall1 - t_wall0,
         }
