@@ -13,9 +13,9 @@ Importing the package does not load the library; the first call does.
 import ctypes
 
 from . import _native
-from ._native import (HYENA_ALGO_AUTO, HYENA_ALGO_DIRECT, HYENA_ALGO_TENSOR, HYENA_ALGO_WINDOW,
-                      HYENA_DEVICE_F16_RANGE, HYENA_DEVICE_TIMEOUT, HYENA_DTYPE_BF16,
-                      HYENA_DTYPE_F32, ALGO_NAMES, HyenaError)
+from ._native import (HYENA_ALGO_AUTO, HYENA_ALGO_DIRECT, HYENA_ALGO_FFT, HYENA_ALGO_TENSOR,
+                      HYENA_ALGO_WINDOW, HYENA_DEVICE_F16_RANGE, HYENA_DEVICE_TIMEOUT,
+                      HYENA_DTYPE_BF16, HYENA_DTYPE_F32, ALGO_NAMES, HyenaError)
 
 __all__ = [
     "hyena_conv_fwd", "hyena_conv_fwd_f32", "hyena_conv_fwd_ex", "hyena_select_algo",
@@ -23,7 +23,8 @@ __all__ = [
     "hyena_conv_bwd_workspace_bytes",
     "hyena_device_status", "hyena_status_string", "hyena_abi_version",
     "HyenaError", "HYENA_ALGO_AUTO", "HYENA_ALGO_TENSOR", "HYENA_ALGO_WINDOW",
-    "HYENA_ALGO_DIRECT", "HYENA_DTYPE_BF16", "HYENA_DTYPE_F32", "HYENA_DEVICE_TIMEOUT",
+    "HYENA_ALGO_DIRECT", "HYENA_ALGO_FFT", "HYENA_DTYPE_BF16", "HYENA_DTYPE_F32",
+    "HYENA_DEVICE_TIMEOUT",
     "HYENA_DEVICE_F16_RANGE", "ALGO_NAMES", "hyena_conv_fwd_from_host",
     "hyena_toeplitz_stages", "hyena_build_toeplitz_blocks", "hyena_conv_fwd_hist",
     "hyena_conv_fwd_fft", "hyena_conv_fwd_fft_workspace_bytes",

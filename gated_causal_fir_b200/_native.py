@@ -25,8 +25,9 @@ HYENA_ALGO_AUTO = 0
 HYENA_ALGO_TENSOR = 1
 HYENA_ALGO_WINDOW = 2
 HYENA_ALGO_DIRECT = 3
+HYENA_ALGO_FFT = 4
 ALGO_NAMES = {HYENA_ALGO_AUTO: "auto", HYENA_ALGO_TENSOR: "tensor", HYENA_ALGO_WINDOW: "window",
-              HYENA_ALGO_DIRECT: "direct"}
+              HYENA_ALGO_DIRECT: "direct", HYENA_ALGO_FFT: "fft"}
 
 HYENA_DEVICE_TIMEOUT = 1
 HYENA_DEVICE_F16_RANGE = 2

@@ -16,6 +16,7 @@
 #include "fir_bwd.cuh"
 #include "fir_cuda_core.cuh"
 #include "fir_fft.cuh"
+#include "fir_fftblk.cuh"
 #include "fir_tc.cuh"
 #include "fir_tc_bwd.cuh"
 
@@ -40,6 +41,7 @@ constexpr int kDhSmemMax =
     ((2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (64 + 1) + hyena::bwd::kDhRedFloats) *
     static_cast<int>(sizeof(float));
 constexpr int kMaxWindowTaps = 16;
+constexpr int kBlkThreads = 512;  // block FFT: one CTA of 512 threads per SM
 #ifndef HYENA_WINDOW_ROWS
 #define HYENA_WINDOW_ROWS 128
 #endif
@@ -86,6 +88,23 @@ int current_device(DeviceState *&ds) {
       e = cudaFuncSetAttribute(reinterpret_cast<const void *>(hyena::tcb::fir_tc_bwd_kernel),
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                hyena::tcb::kSmemBytes);
+    // block FFT instantiations (see kBlkConfigs)
+    const struct {
+      const void *fn;
+      int smem;
+    } blk[] = {
+#define HYENA_BLK_ATTR(T, LGN, PP, SQ)                                                          \
+  {reinterpret_cast<const void *>(hyena::fftblk::fir_fftblk_kernel<T, LGN, PP, kBlkThreads, SQ>), \
+   hyena::fftblk::Smem<T, LGN, PP, SQ>::kBytes}
+        HYENA_BLK_ATTR(__nv_bfloat16, 10, 8, true), HYENA_BLK_ATTR(__nv_bfloat16, 11, 4, true),
+        HYENA_BLK_ATTR(__nv_bfloat16, 12, 2, true), HYENA_BLK_ATTR(__nv_bfloat16, 13, 1, false),
+        HYENA_BLK_ATTR(float, 10, 4, true), HYENA_BLK_ATTR(float, 11, 2, true),
+        HYENA_BLK_ATTR(float, 12, 1, true)
+#undef HYENA_BLK_ATTR
+    };
+    for (const auto &k : blk)
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
     const void *tiled[] = {
         reinterpret_cast<const void *>(hyena::cc::fir_tiled_kernel<float, false>),
         reinterpret_cast<const void *>(hyena::cc::fir_tiled_kernel<float, true>),
@@ -209,21 +228,91 @@ bool window_supported(const Problem &P) {
   return P.l_h <= kMaxWindowTaps && P.d_g % vec == 0 && all_aligned16(P);
 }
 
+// Block FFT (overlap-save, fir_fftblk_kernel): transform length N = 2^lgn with P channel pairs
+// per CTA (P N = 8192 complex values in shared memory for bf16, 4096 for fp32, whose staged
+// rows are twice as wide), M = N - l_h + 1 outputs per block; one CTA per SM.
+struct BlkConfig {
+  int lgn, P;
+};
+constexpr BlkConfig kBlkBf16[] = {{10, 8}, {11, 4}, {12, 2}, {13, 1}};
+constexpr BlkConfig kBlkF32[] = {{10, 4}, {11, 2}, {12, 1}};
+
+struct BlkPlan {
+  BlkConfig cfg;
+  int M, nTB;
+  bool ok;
+};
+
+// The transform length with the least work, N log N per block times the blocks per sequence,
+// among those whose channel block (2P channels) lies inside one group, whose row vectors are
+// aligned and whose blocks keep at least N / 8 rows (or one block covers the sequence);
+// ok = false when none applies.
+BlkPlan blk_plan(const Problem &P) {
+  BlkPlan best{kBlkBf16[0], 0, 0, false};
+  double best_cost = 0;
+  const bool f32 = P.dtype == HYENA_DTYPE_F32;
+  const int ncfg = f32 ? 3 : 4;
+  for (int ci = 0; ci < ncfg; ++ci) {
+    const BlkConfig &c = f32 ? kBlkF32[ci] : kBlkBf16[ci];
+    const int64_t N = int64_t{1} << c.lgn;
+    if (N < P.l_h || P.d_g % (2 * c.P) != 0 || P.D % (2 * c.P) != 0) continue;
+    const uintptr_t vec = std::min<uintptr_t>(16, static_cast<uintptr_t>(2 * c.P * P.elem()));
+    if (!aligned(P.q, vec) || !aligned(P.k, vec) || !aligned(P.v, vec) || !aligned(P.y, vec) ||
+        (P.Lh > 0 && (!aligned(P.kh, vec) || !aligned(P.vh, vec))))
+      continue;
+    const int64_t M = N - P.l_h + 1, nTB = (P.L + M - 1) / M;
+    // blocks that keep less than an eighth of their rows cost more than the direct sum
+    if (M < N / 8 && nTB > 1) continue;
+    if (P.D / (2 * c.P) * nTB > std::numeric_limits<int32_t>::max()) continue;
+    const double cost = static_cast<double>(nTB) * static_cast<double>(N) * c.lgn;
+    if (!best.ok || cost < best_cost) {
+      best = BlkPlan{c, static_cast<int>(M), static_cast<int>(nTB), true};
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
+bool fftblk_supported(const Problem &P) { return blk_plan(P).ok; }
+
+// AUTO's choice between the block FFT and the direct sum: flops per output channel, ~5 N log2 N
+// per length-N transform (forward and inverse, two channels per transform) against 2 l_h, the
+// FFT's weighted by how much faster per flop its kernel runs.
+#ifndef HYENA_FFT_FLOP_WEIGHT
+#define HYENA_FFT_FLOP_WEIGHT 0.5
+#endif
+bool fftblk_beats_direct(const Problem &P) {
+  const BlkPlan bp = blk_plan(P);
+  if (!bp.ok) return false;
+  const double fft = HYENA_FFT_FLOP_WEIGHT * 5.0 * bp.nTB * static_cast<double>(1 << bp.cfg.lgn) *
+                     bp.cfg.lgn / static_cast<double>(P.L);
+  return fft < 2.0 * P.l_h;
+}
+
 // MMAs one 128-row tile issues on the tensor path (groups per tile x k-steps).  Each costs
 // ~55 cycles of issue at any N <= 64; past ~24 per tile the issuing thread, not HBM, sets the
 // pace, and for short filters the CUDA-core window kernel is faster (measured on the SE
 // workload: 36 MMAs per tile, 80 us on tensor cores vs 50 us in the window kernel).
 constexpr int kMaxTileMmas = 24;
 
+#ifndef HYENA_FFT_MIN_TAPS
+#define HYENA_FFT_MIN_TAPS 17
+#endif
+#ifndef HYENA_FFT_OVER_TENSOR_TAPS
+#define HYENA_FFT_OVER_TENSOR_TAPS 100000
+#endif
+
 int select_algo(const Problem &P) {
   const bool tensor = tensor_supported(P), window = window_supported(P);
+  const bool fft = P.l_h >= HYENA_FFT_MIN_TAPS && fftblk_beats_direct(P);
   if (tensor && window) {
     const TcPlan t = tc_plan(P);
     return t.ng * ((hyena::tc::kTM + t.halo) / 16) <= kMaxTileMmas ? HYENA_ALGO_TENSOR
                                                                    : HYENA_ALGO_WINDOW;
   }
-  if (tensor) return HYENA_ALGO_TENSOR;
+  if (tensor) return fft && P.l_h >= HYENA_FFT_OVER_TENSOR_TAPS ? HYENA_ALGO_FFT : HYENA_ALGO_TENSOR;
   if (window) return HYENA_ALGO_WINDOW;
+  if (fft) return HYENA_ALGO_FFT;
   return HYENA_ALGO_DIRECT;
 }
 
@@ -435,6 +524,58 @@ int launch_tiled(const Problem &P, const void *dy, void *out0, void *out1, cudaS
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
+template <typename T, int LGN, int PP, bool SQ>
+int launch_fftblk_cfg(const Problem &P, const BlkPlan &bp, int sm_count, cudaStream_t s) {
+  hyena::fftblk::BlkParams p;
+  p.q = P.q;
+  p.k = P.k;
+  p.v = P.v;
+  p.kh = P.Lh > 0 ? P.kh : P.k;
+  p.vh = P.Lh > 0 ? P.vh : P.v;
+  p.h = P.h;
+  p.y = P.y;
+  p.L = P.L;
+  p.D = P.D;
+  p.Lh = P.Lh;
+  p.CB = static_cast<int>(P.D / (2 * PP));
+  p.nTB = bp.nTB;
+  p.M = bp.M;
+  p.d_g = P.d_g;
+  p.l_h = P.l_h;
+  // siblings: enough consecutive channel blocks for 64 bytes of a row (one DRAM access)
+  p.Q = std::max(1, 64 / static_cast<int>(2 * PP * P.elem()));
+  while (p.CB % p.Q != 0) p.Q /= 2;
+  p.items = P.B * (p.CB / p.Q) * static_cast<long long>(p.nTB);
+  const long long groups = std::max<long long>(1, static_cast<long long>(sm_count) / p.Q);
+  const long long grid = std::min<long long>(p.items, groups) * p.Q;
+  hyena::fftblk::fir_fftblk_kernel<T, LGN, PP, kBlkThreads, SQ>
+      <<<static_cast<unsigned>(grid), kBlkThreads, hyena::fftblk::Smem<T, LGN, PP, SQ>::kBytes, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+int launch_fftblk(const Problem &P, cudaStream_t s) {
+  const BlkPlan bp = blk_plan(P);
+  if (!bp.ok) return HYENA_ERR_UNSUPPORTED;
+  DeviceState *ds = nullptr;
+  if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
+  const int sms = ds->sm_count;
+  if (P.dtype == HYENA_DTYPE_F32) {
+    switch (bp.cfg.lgn) {
+      case 10: return launch_fftblk_cfg<float, 10, 4, true>(P, bp, sms, s);
+      case 11: return launch_fftblk_cfg<float, 11, 2, true>(P, bp, sms, s);
+      case 12: return launch_fftblk_cfg<float, 12, 1, true>(P, bp, sms, s);
+      default: return HYENA_ERR_UNSUPPORTED;
+    }
+  }
+  switch (bp.cfg.lgn) {
+    case 10: return launch_fftblk_cfg<__nv_bfloat16, 10, 8, true>(P, bp, sms, s);
+    case 11: return launch_fftblk_cfg<__nv_bfloat16, 11, 4, true>(P, bp, sms, s);
+    case 12: return launch_fftblk_cfg<__nv_bfloat16, 12, 2, true>(P, bp, sms, s);
+    case 13: return launch_fftblk_cfg<__nv_bfloat16, 13, 1, false>(P, bp, sms, s);
+    default: return HYENA_ERR_UNSUPPORTED;
+  }
+}
+
 int launch_direct(const Problem &P, cudaStream_t s) {
   if (P.dtype == HYENA_DTYPE_F32) return launch_tiled<float, false>(P, nullptr, P.y, nullptr, s);
   return launch_tiled<__nv_bfloat16, false>(P, nullptr, P.y, nullptr, s);
@@ -454,6 +595,9 @@ int run(const Problem &P, int algo, cudaStream_t s) {
     case HYENA_ALGO_WINDOW:
       if (!window_supported(P)) return HYENA_ERR_UNSUPPORTED;
       break;
+    case HYENA_ALGO_FFT:
+      if (!fftblk_supported(P)) return HYENA_ERR_UNSUPPORTED;
+      break;
     case HYENA_ALGO_DIRECT:
       break;
     default:
@@ -461,6 +605,7 @@ int run(const Problem &P, int algo, cudaStream_t s) {
   }
   if (algo == HYENA_ALGO_TENSOR) return launch_tensor(P, s);
   if (algo == HYENA_ALGO_WINDOW) return launch_window(P, s);
+  if (algo == HYENA_ALGO_FFT) return launch_fftblk(P, s);
   return launch_direct(P, s);
 }
 
@@ -907,6 +1052,7 @@ int select_bwd(const Problem &P, const void *dy, const void *dq, const void *dk,
     case HYENA_ALGO_TENSOR: return tc ? HYENA_ALGO_TENSOR : -HYENA_ERR_UNSUPPORTED;
     case HYENA_ALGO_WINDOW: return win ? HYENA_ALGO_WINDOW : -HYENA_ERR_UNSUPPORTED;
     case HYENA_ALGO_DIRECT: return HYENA_ALGO_DIRECT;
+    case HYENA_ALGO_FFT: return -HYENA_ERR_UNSUPPORTED;  // a forward-only algorithm
     default: return -HYENA_ERR_INVALID_ARG;
   }
 }

@@ -66,8 +66,15 @@ enum hyena_algo {
     HYENA_ALGO_WINDOW = 2,       /* CUDA-core register sliding window, forward and backward
                                     (l_h <= 16; d_g a multiple of 8 channels for bf16, 4 for
                                     fp32; 16-byte aligned tensors) */
-    HYENA_ALGO_DIRECT = 3        /* CUDA-core direct sum, tiled through shared memory; any
+    HYENA_ALGO_DIRECT = 3,       /* CUDA-core direct sum, tiled through shared memory; any
                                     supported shape */
+    HYENA_ALGO_FFT = 4           /* forward only: single-pass block FFT (overlap-save) on the
+                                    CUDA cores in fp32, no workspace; l_h <= 8192 for bf16,
+                                    <= 4096 for fp32; d_g a multiple of 2P channels for the
+                                    transform length N chosen (bf16: P = 8, 4, 2, 1 channel
+                                    pairs at N = 1024, 2048, 4096, 8192; fp32: P = 4, 2, 1 at
+                                    N = 1024, 2048, 4096); tensors aligned to the 2P-channel
+                                    row piece (at most 16 bytes) */
 };
 
 /* Bits of the per-device status word (hyena_device_status). */
@@ -87,8 +94,10 @@ enum hyena_device_status_bits {
  * accepted: the block form with S = 1 + ceil((l_h - 1) / l_b) sub-block diagonals is exact for
  * every filter length (the two-stage form of Sec. 3 is the case S = 2, l_h <= l_b + 1), so the
  * result does not depend on l_b.  The kernels pick their own internal block size.  Filters
- * longer than the tensor path's limit (HYENA_ALGO_TENSOR above) run on the CUDA-core direct
- * sum; hyena_conv_fwd_fft is the faster entry point for them.  All tensors 2-byte aligned.
+ * of 17 taps or more that the tensor path does not take (longer than its limit, fp32, or
+ * d_g outside {16, 32, 64}) run on the single-pass block FFT (HYENA_ALGO_FFT) where it
+ * applies, else on the CUDA-core direct sum; hyena_conv_fwd_fft (with a workspace) takes
+ * filters of any length.  All tensors 2-byte aligned.
  * Precision: on the tensor-core path the MMA operands are fp16 (x = k v formed exactly in
  * fp32; h), each scaled by a power of two first (per group for h, per sequence run for x),
  * with fp32 accumulation; tiles whose scaled operands still leave fp16's range are recomputed

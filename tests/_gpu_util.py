@@ -85,3 +85,26 @@ def tc_cta_seam_rows(B, L, D, d_g, sm_count, tile_rows=128):
         if i > 0:
             rows.append((seq // B, seq % B, i * tile_rows))  # (group, b, row)
     return rows
+
+
+# (log2 N, channel pairs per CTA) of the block FFT kernel's transform lengths, by I/O type
+FFTBLK_CONFIGS = {"bf16": ((10, 8), (11, 4), (12, 2), (13, 1)),
+                  "f32": ((10, 4), (11, 2), (12, 1))}
+
+
+def fftblk_plan(L, D, d_g, l_h, dtype="bf16"):
+    """The block FFT's choice for a shape (tensors 16-byte aligned): (N, P, M) with the least
+    N log N per block times blocks per sequence, or None where no transform length applies."""
+    best = None
+    for lgn, P in FFTBLK_CONFIGS[dtype]:
+        N = 1 << lgn
+        if N < l_h or d_g % (2 * P) or D % (2 * P):
+            continue
+        M = N - l_h + 1
+        ntb = -(-L // M)
+        if M < N // 8 and ntb > 1:
+            continue
+        cost = ntb * N * lgn
+        if best is None or cost < best[0]:
+            best = (cost, N, P, M)
+    return None if best is None else best[1:]

@@ -58,7 +58,7 @@ def test_select_algo_for_the_workloads(lib):
     from gated_causal_fir_b200.workloads import WORKLOADS
     want = {"tiny": g.HYENA_ALGO_WINDOW, "se": g.HYENA_ALGO_WINDOW, "mr": g.HYENA_ALGO_TENSOR,
             "mr_batched": g.HYENA_ALGO_TENSOR, "mr_1m": g.HYENA_ALGO_TENSOR,
-            "li": g.HYENA_ALGO_DIRECT}  # long filters: the FFT entry point (workspace) is separate
+            "li": g.HYENA_ALGO_DIRECT}  # l_h = L = 8192: blocks of one row; FFT entry point
     for name, wl in WORKLOADS.items():
         dt = g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16
         assert g.hyena_select_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, dt) == want[name]
@@ -66,11 +66,16 @@ def test_select_algo_for_the_workloads(lib):
 
 def test_select_algo_fallbacks(lib):
     bf, f32 = g.HYENA_DTYPE_BF16, g.HYENA_DTYPE_F32
-    assert g.hyena_select_algo(1, 100, 256, 64, 514, 65, bf) == g.HYENA_ALGO_DIRECT  # l_h > 513
+    assert g.hyena_select_algo(1, 100, 256, 64, 514, 65, bf) == g.HYENA_ALGO_FFT     # l_h > 513
     assert g.hyena_select_algo(1, 100, 256, 64, 130, 65, bf) == g.HYENA_ALGO_TENSOR  # 2 tiles back
     assert g.hyena_select_algo(1, 100, 256, 64, 129, 65, bf) == g.HYENA_ALGO_TENSOR
     assert g.hyena_select_algo(1, 100, 128, 32, 40, 32, bf) == g.HYENA_ALGO_TENSOR
     assert g.hyena_select_algo(1, 100, 96, 32, 40, 32, bf) == g.HYENA_ALGO_DIRECT   # D % 64 != 0
+    assert g.hyena_select_algo(1, 4096, 96, 32, 40, 32, bf) == g.HYENA_ALGO_FFT     # long enough
+    assert g.hyena_select_algo(1, 100, 96, 32, 16, 32, f32) == g.HYENA_ALGO_WINDOW
+    assert g.hyena_select_algo(1, 100, 90, 30, 40, 32, bf) == g.HYENA_ALGO_DIRECT   # 8192-point
+    assert g.hyena_select_algo(1, 8192, 90, 30, 40, 32, bf) == g.HYENA_ALGO_FFT     # (P = 1) FFT
+    assert g.hyena_select_algo(1, 100, 93, 31, 40, 32, bf) == g.HYENA_ALGO_DIRECT   # odd groups
     assert g.hyena_select_algo(1, 100, 96, 32, 16, 32, bf) == g.HYENA_ALGO_WINDOW
     assert g.hyena_select_algo(1, 100, 128, 16, 65, 64, bf) == g.HYENA_ALGO_TENSOR  # 4 bands fit
     assert g.hyena_select_algo(1, 100, 128, 16, 7, 16, bf) == g.HYENA_ALGO_WINDOW   # 36 MMAs/tile
@@ -79,7 +84,9 @@ def test_select_algo_fallbacks(lib):
     assert g.hyena_select_algo(1, 100, 128, 8, 7, 16, bf) == g.HYENA_ALGO_WINDOW    # d_g = 8
     assert g.hyena_select_algo(1, 100, 96, 4, 3, 2, bf) == g.HYENA_ALGO_DIRECT      # 4 ch < 16 B
     assert g.hyena_select_algo(1, 100, 96, 4, 3, 2, f32) == g.HYENA_ALGO_WINDOW
-    assert g.hyena_select_algo(1, 64, 128, 64, 128, 64, f32) == g.HYENA_ALGO_DIRECT
+    assert g.hyena_select_algo(1, 64, 128, 64, 128, 64, f32) == g.HYENA_ALGO_DIRECT  # L = 64
+    assert g.hyena_select_algo(1, 2048, 128, 64, 128, 64, f32) == g.HYENA_ALGO_FFT
+    assert g.hyena_select_algo(1, 64, 128, 64, 16, 64, f32) == g.HYENA_ALGO_WINDOW
     n = 64 * 128 * 2
     odd = (16 + 2, 16 + n + 64, 16 + 2 * (n + 64), 16 + 3 * (n + 64), 16 + 4 * (n + 64))
     assert g.hyena_select_algo(1, 64, 128, 64, 128, 64, bf, ptrs=odd) == g.HYENA_ALGO_DIRECT
@@ -157,12 +164,15 @@ def test_long_filters_select_an_algorithm():
     bf = g.HYENA_DTYPE_BF16
     assert g.hyena_select_algo(1, 8192, 4096, 64, 130, 64, bf) == g.HYENA_ALGO_TENSOR
     assert g.hyena_select_algo(1, 8192, 4096, 64, 513, 64, bf) == g.HYENA_ALGO_TENSOR
-    assert g.hyena_select_algo(1, 8192, 4096, 64, 514, 64, bf) == g.HYENA_ALGO_DIRECT
+    assert g.hyena_select_algo(1, 8192, 4096, 64, 514, 64, bf) == g.HYENA_ALGO_FFT
     assert g.hyena_select_algo(1, 8192, 4096, 32, 257, 64, bf) == g.HYENA_ALGO_TENSOR
-    assert g.hyena_select_algo(1, 8192, 4096, 32, 258, 64, bf) == g.HYENA_ALGO_DIRECT
-    assert g.hyena_select_algo(1, 8192, 4096, 16, 66, 16, bf) == g.HYENA_ALGO_DIRECT
+    assert g.hyena_select_algo(1, 8192, 4096, 32, 258, 64, bf) == g.HYENA_ALGO_FFT
+    assert g.hyena_select_algo(1, 8192, 4096, 16, 66, 16, bf) == g.HYENA_ALGO_FFT
     assert g.hyena_select_algo(1, 8192, 4096, 64, 300, 64, g.HYENA_DTYPE_F32) == \
-        g.HYENA_ALGO_DIRECT
+        g.HYENA_ALGO_FFT
+    assert g.hyena_select_algo(1, 8192, 4096, 64, 6000, 64, bf) == g.HYENA_ALGO_FFT
+    # 8192-point blocks would keep fewer than 1024 rows: the direct sum
+    assert g.hyena_select_algo(1, 8192, 4096, 64, 7200, 64, bf) == g.HYENA_ALGO_DIRECT
 
 
 def test_history_validation(lib):

@@ -15,7 +15,8 @@ import oracle
 
 pytestmark = pytest.mark.gpu
 
-ALGOS = {"tensor": g.HYENA_ALGO_TENSOR, "window": g.HYENA_ALGO_WINDOW, "direct": g.HYENA_ALGO_DIRECT}
+ALGOS = {"tensor": g.HYENA_ALGO_TENSOR, "window": g.HYENA_ALGO_WINDOW, "direct": g.HYENA_ALGO_DIRECT,
+         "fft": g.HYENA_ALGO_FFT}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -96,6 +97,8 @@ def _tensor_fits(D, d_g, l_h):
 def _supported(algo, B, L, D, d_g, l_h, l_b, dtype):
     if algo == "direct":
         return True
+    if algo == "fft":
+        return U.fftblk_plan(L, D, d_g, l_h, dtype) is not None
     if algo == "tensor":
         return dtype == "bf16" and _tensor_fits(D, d_g, l_h)
     return l_h <= 16 and d_g % (4 if dtype == "f32" else 8) == 0
