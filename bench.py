@@ -347,7 +347,9 @@ def time_long_filters(args, stream, dev, D, g, _native, peak, peak_kind):
     * ``li_fft``: the Hyena-LI-shaped workload (B=1, L=8192, D=4096, d_g=64, l_h=8192) through
       hyena_conv_fwd_fft (four-step FFT, caller workspace);
     * ``mr_lh513``: the MR shape with l_h = 513, the longest filter of the tensor-core path
-      (hyena_conv_fwd, AUTO).
+      (hyena_conv_fwd, AUTO);
+    * ``mr_lh514``: one tap longer, past the tensor band: AUTO runs the single-pass block FFT
+      (no workspace).
 
     Algorithmic bytes per call: q, k, v read and y written (4 B L D bf16 elements); the FFT's
     spectra in the workspace are overhead, not counted."""
@@ -357,7 +359,9 @@ def time_long_filters(args, stream, dev, D, g, _native, peak, peak_kind):
     out = {}
     for name, wl, fft in (("li_fft", WORKLOADS["li"], True),
                           ("mr_lh513", custom("mr_lh513", 1, 8192, 4096, 64, 513, 64, "bf16",
-                                              "mr", seed=6), False)):
+                                              "mr", seed=6), False),
+                          ("mr_lh514", custom("mr_lh514", 1, 8192, 4096, 64, 514, 64, "bf16",
+                                              "mr", seed=7), False)):
         sets = [make_inputs(wl, device=dev, seed=wl.seed + 101 * s) for s in range(2)]
         ys = [torch.empty_like(x[0]) for x in sets]
         torch.cuda.synchronize()  # inputs complete before `stream` reads them
@@ -376,7 +380,9 @@ def time_long_filters(args, stream, dev, D, g, _native, peak, peak_kind):
             cargs = [(x[0].data_ptr(), x[1].data_ptr(), x[2].data_ptr(), x[3].data_ptr(),
                       y.data_ptr(), wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, sh)
                      for x, y in zip(sets, ys)]
-            kernels = ["fir_tc_kernel"]
+            algo = g.hyena_select_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b)
+            kernels = [{g.HYENA_ALGO_TENSOR: "fir_tc_kernel", g.HYENA_ALGO_FFT: "fir_fftblk_kernel",
+                        g.HYENA_ALGO_DIRECT: "fir_tiled_kernel"}[algo]]
         for i in range(max(3, args.warmup)):
             if cfn(*cargs[i % 2]) != 0:
                 raise _native.HyenaError(name, cfn(*cargs[i % 2]))

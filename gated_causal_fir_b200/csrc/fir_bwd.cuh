@@ -50,10 +50,20 @@ __global__ void __launch_bounds__(kDhTaps)
     fir_bwd_dh_partial_kernel(const T *__restrict__ q, const T *__restrict__ k,
                               const T *__restrict__ v, const T *__restrict__ dy,
                               float *__restrict__ partial, long long L, long long D, int l_h,
-                              int cp) {
+                              int cp, int nchunk, int npieces, int B,
+                              const unsigned *__restrict__ run_if, unsigned run_token) {
+  if (run_if) {  // as fir_tiled_kernel's run_if
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (*run_if != run_token) return;
+  }
   extern __shared__ float sm[];
-  const int chunk = blockIdx.x, piece = blockIdx.y, b = blockIdx.z;
-  const int nchunk = gridDim.x, npieces = gridDim.y;
+  // one (chunk, piece, sequence) block after another, grid-stride
+  const long long nblk = static_cast<long long>(nchunk) * npieces * B;
+  for (long long blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+  const int chunk = static_cast<int>(blk % nchunk);
+  const int piece = static_cast<int>((blk / nchunk) % npieces);
+  const int b = static_cast<int>(blk / (static_cast<long long>(nchunk) * npieces));
+  __syncthreads();  // the previous block's rows and sums have been read
   const long long t0 = static_cast<long long>(chunk) * kDhRows;
   const long long c0 = static_cast<long long>(piece) * cp;
   const long long base = static_cast<long long>(b) * L * D;
@@ -118,6 +128,7 @@ __global__ void __launch_bounds__(kDhTaps)
       for (int g = 0; g < kDhGroups; ++g) s += red[g * kDhTaps + threadIdx.x];
       out[j] = s;
     }
+  }
   }
 }
 
@@ -246,7 +257,12 @@ __global__ void __launch_bounds__(kBwdWindowBlock)
 constexpr int kReduceBlock = 256;
 __global__ void __launch_bounds__(kReduceBlock)
     fir_bwd_dh_reduce_kernel(const float *__restrict__ partial, float *__restrict__ dh, int B,
-                             int nchunk, int npieces, int pieces_per_group, int G, int l_h) {
+                             int nchunk, int npieces, int pieces_per_group, int G, int l_h,
+                             const unsigned *__restrict__ run_if, unsigned run_token) {
+  if (run_if) {  // as fir_tiled_kernel's run_if
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (*run_if != run_token) return;
+  }
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (kReduceBlock / 32);
   const long long n = static_cast<long long>(G) * l_h;

@@ -208,8 +208,19 @@ __global__ void __launch_bounds__(kTileThreads)
                      const T *__restrict__ k, const T *__restrict__ v,
                      const float *__restrict__ h, T *__restrict__ o0, T *__restrict__ o1,
                      long long B, long long L, long long D, int d_g, int l_h,
-                     const T *__restrict__ kh, const T *__restrict__ vh, long long Lh) {
-  // forward: a0 = q, a1 unused, o0 = y;  anti: a0 = q, a1 = dy, o0 = dk, o1 = dv
+                     const T *__restrict__ kh, const T *__restrict__ vh, long long Lh,
+                     const unsigned *__restrict__ run_if, unsigned run_token) {
+  // forward: a0 = q, a1 unused, o0 = y;  anti: a0 = q, a1 = dy, o0 = dk, o1 = dv.
+  // run_if (anti only; may be null): a device word; unless it holds run_token the kernel does
+  // nothing (the fp32 recomputation behind the tensor-core backward, needed only where that
+  // kernel raised its flag).  Such a launch may start early (programmatic dependent launch): it
+  // waits for the previous kernels of the stream before it reads anything.
+  if constexpr (kAnti) {
+    if (run_if) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      if (*run_if != run_token) return;
+    }
+  }
   extern __shared__ float xs[];  // [kTileWin][kTileC]
   const int cl = threadIdx.x % kTileC, rg = threadIdx.x / kTileC;
   const long long n_ct = (D + kTileC - 1) / kTileC, n_rt = (L + kTileR - 1) / kTileR;

@@ -36,6 +36,14 @@
 //    its k, v rows from the stage into registers, releases it, and stores dk, dv rows directly;
 //    it also sums the dh anti-diagonals.  Every wait is bounded; a timeout raises
 //    HYENA_DEVICE_TIMEOUT and all roles drain and leave.
+//  * Operand range.  x, dz and h are rounded to fp16 unscaled.  Where a value of any of them
+//    lies above 65504 (it would round to inf), or a group's taps all lie below 2^-10 (deep in
+//    fp16's subnormals), the gate writes the call's token into the range flag in the host's
+//    workspace and raises HYENA_DEVICE_F16_RANGE; the host queues the fp32 CUDA-core backward
+//    behind this kernel, gated on that token, and it rewrites dk, dv and dh.  (Scaling x and dz
+//    by powers of two chosen per CTA, as the forward does per sequence run, measured 233 us
+//    instead of 192 us at the MR shape: this kernel's time follows its gate and epilogue
+//    warps' critical path, and every added step on it showed in the total.)
 #pragma once
 #include "fir_tc.cuh"
 
@@ -95,7 +103,12 @@ constexpr int kBarRedDone = kBarAEmpty + 1;
 constexpr int kBarDone = kBarRedDone + 1;
 constexpr int kNumBars = kBarDone + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+// kOffMisc: TMEM address, abort flag, then each gate warp's largest |h| of the segment (float
+// bits; two sets by segment parity)
+constexpr int kMiscTapMax = 8;
+constexpr int kSmemBytes = kOffMisc + 48 + 1024;  // + slack for 1024-byte alignment
+// A group whose largest |tap| is below 2^-10 (float bits): its taps sit in fp16's subnormals.
+constexpr uint32_t kTapTinyBits = 0x3A800000u;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget of one CTA exceeded");
 
 constexpr int kThreads = 352;
@@ -115,6 +128,8 @@ struct Params {
   int max_segs;       // partial slots per CTA
   long long D;        // channels (row length of every [B, L, D] tensor)
   __nv_bfloat16 *dk, *dv;  // outputs, written by rows
+  unsigned *range_flag;    // set to range_token where an operand leaves fp16's range
+  unsigned range_token;    // this call's token (the host's fallback kernels run on a match)
 };
 
 enum ItemKind { kNextHalo = 0, kMain = 1 };
@@ -336,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint16_t *hz = reinterpret_cast<uint16_t *>(smem + kOffHz);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  uint32_t *tapmax = reinterpret_cast<uint32_t *>(smem + kOffMisc + kMiscTapMax);  // [2][4]
   volatile int *abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -387,13 +403,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   // inputs are complete when this grid starts, and nothing here reads what the forward writes
   // (dq), so the work overlaps the forward's last tiles without a grid-dependency wait.
   griddep_launch_dependents();
-  // The gate threads issue the loads of the first segment's filter taps before the barrier.
+  // The gate threads issue the loads of the first segment's filter taps before the barrier
+  // (and each gate warp leaves the group's largest |h| among its taps in tapmax[0][warp]).
   bool over = false;
   float taps[kTapPer];
+  auto tap_share_max = [&](uint32_t *slot) {
+    uint32_t hm = 0;
+#pragma unroll
+    for (int k2 = 0; k2 < kTapPer; ++k2) hm = max(hm, __float_as_uint(fabsf(taps[k2])));
+    hm = __reduce_max_sync(0xffffffffu, hm);
+    if (lane == 0) *slot = hm;
+  };
   if (warp >= kWarpGate0 && warp < kWarpGate0 + 4 && w_begin < w_end) {
     const int g0 = static_cast<int>((w_begin / p.nT) / p.B);
     tc::tap_load(taps, p.h + static_cast<size_t>(g0) * p.l_h, p.l_h, p.halo, 1,
                  threadIdx.x - kWarpGate0 * 32);
+    tap_share_max(&tapmax[warp - kWarpGate0]);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -517,13 +542,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gw = warp - kWarpGate0, gtid = threadIdx.x - kWarpGate0 * 32;
     while (it.next(t)) {
       if (t.seg_first) {
+        const uint32_t *tm = tapmax + 4 * (t.seg & 1);
         if (t.seg > 0) {
           if (!tc::warp_wait(&bars[kBarAEmpty], (t.seg - 1) & 1, abort)) break;
           tc::tap_load(taps, p.h + static_cast<size_t>(t.g) * p.l_h, p.l_h, p.halo, 1, gtid);
-          // every gate thread has finished reading the previous taps ...
+          tap_share_max(&tapmax[4 * (t.seg & 1) + gw]);
+          // every gate thread has finished reading the previous taps (and left its warp's
+          // largest tap) ...
           mbar_arrive(&bars[kBarGate]);
           if (!tc::warp_wait(&bars[kBarGate], gphase++ & 1, abort)) break;
         }
+        // (segment 0's maxima were left before the CTA barrier; a slot set is rewritten two
+        // segments later, after a barrier that every reader of it has passed)
+        const uint32_t hmax = max(max(tm[0], tm[1]), max(tm[2], tm[3]));
+        over |= hmax != 0 && hmax < kTapTinyBits;
         tc::tap_store(hz, taps, p.halo, 1, gtid, over);
         // ... and has written its share of the new ones
         mbar_arrive(&bars[kBarGate]);
@@ -558,7 +590,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++qc;
       ++dc;
     }
-    if (over) atomicOr(&g_device_status, kF16RangeBit);
+    if (over) {  // (per thread: a lane's own products; writers all store the same token)
+      atomicOr(&g_device_status, kF16RangeBit);
+      *p.range_flag = p.range_token;
+    }
   } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
     // ------------------------------------------------------------ epilogue
     // Thread = one tile row.  It copies its k, v rows from the input stage into registers and
@@ -701,6 +736,7 @@ __global__ void __launch_bounds__(256)
                              const int *__restrict__ seg_count, int max_segs,
                              float *__restrict__ dh, int G, int l_h, long long per, long long rem,
                              long long span) {
+  griddep_wait();  // launched with programmatic stream serialisation after fir_tc_bwd_kernel
   const long long n = static_cast<long long>(G) * l_h;
   for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {

@@ -508,20 +508,44 @@ int launch_window(const Problem &P, cudaStream_t s) {
 
 // The tiled direct sum (fir_tiled_kernel): forward (y) or, with kAnti, the backward's
 // transposed product (dk, dv from q, dy).  Persistent CTAs over the tiles.
+// A kernel launch, with programmatic stream serialisation where `pdl` (the kernel then waits
+// for the previous kernels of the stream itself, with griddepcontrol.wait).
+template <typename... Exp, typename... Act>
+cudaError_t launch_ex(bool pdl, void (*kernel)(Exp...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t s, Act &&...args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl && HYENA_PDL;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Act>(args)...);
+}
+
+// run_if (anti only): the kernel's gate word, run_token the value that lets it run; a gated
+// launch takes one block per SM and starts early (programmatic dependent launch), so that it
+// costs little when the word does not match.
 template <typename T, bool kAnti>
-int launch_tiled(const Problem &P, const void *dy, void *out0, void *out1, cudaStream_t s) {
+int launch_tiled(const Problem &P, const void *dy, void *out0, void *out1, cudaStream_t s,
+                 const unsigned *run_if = nullptr, unsigned run_token = 0) {
   DeviceState *ds = nullptr;
   if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
   namespace cc = hyena::cc;
   const long long tiles = P.B * ((P.L + cc::kTileR - 1) / cc::kTileR) *
                           ((P.D + cc::kTileC - 1) / cc::kTileC);
-  const long long grid = std::min<long long>(tiles, static_cast<long long>(ds->sm_count) * 4);
-  cc::fir_tiled_kernel<T, kAnti><<<static_cast<unsigned>(grid), cc::kTileThreads,
-                                   cc::kTileSmemBytes, s>>>(
-      static_cast<const T *>(P.q), static_cast<const T *>(dy), static_cast<const T *>(P.k),
-      static_cast<const T *>(P.v), P.h, static_cast<T *>(out0), static_cast<T *>(out1), P.B,
-      P.L, P.D, P.d_g, P.l_h, static_cast<const T *>(P.kh), static_cast<const T *>(P.vh), P.Lh);
-  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+  const long long grid =
+      std::min<long long>(tiles, static_cast<long long>(ds->sm_count) * (run_if ? 1 : 4));
+  const cudaError_t e = launch_ex(
+      run_if != nullptr, cc::fir_tiled_kernel<T, kAnti>, dim3(static_cast<unsigned>(grid)),
+      dim3(cc::kTileThreads), cc::kTileSmemBytes, s, static_cast<const T *>(P.q),
+      static_cast<const T *>(dy), static_cast<const T *>(P.k), static_cast<const T *>(P.v), P.h,
+      static_cast<T *>(out0), static_cast<T *>(out1), P.B, P.L, P.D, P.d_g, P.l_h,
+      static_cast<const T *>(P.kh), static_cast<const T *>(P.vh), P.Lh, run_if, run_token);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
 template <typename T, int LGN, int PP, bool SQ>
@@ -659,11 +683,18 @@ int64_t window_bwd_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h, int6
 }
 
 // The workspace a backward call needs at least (every algorithm runs in it) ...
-int64_t bwd_required_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
+// The partials of every algorithm fit below this offset; the tensor-core path keeps its
+// operand-range flag at it (the fp32 fallback behind that path reuses the partials' room).
+int64_t bwd_flag_offset(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
   const int64_t cc = round256(bwd_plan(B, L, D, d_g, l_h).partial_floats * 4);
   const int64_t tc = tc_bwd_bytes_bound(B, L, D, d_g, l_h);
   const int64_t win = window_bwd_bytes(B, L, D, d_g, l_h, std::max<int64_t>(L, 1));
   return std::max(cc, std::max(tc, win));
+}
+
+int64_t bwd_required_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
+  if (B == 0 || L == 0) return 0;  // nothing runs but the zeroing of dh
+  return bwd_flag_offset(B, L, D, d_g, l_h) + 256;
 }
 
 // ... and the size hyena_conv_bwd_workspace_bytes reports: enough for the window kernel's
@@ -673,33 +704,49 @@ int64_t bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g, int l_h) {
                   window_bwd_bytes(B, L, D, d_g, l_h, kWindowMinRows));
 }
 
+// The CUDA-core kernels' index limits: one 32-bit grid of (chunk, piece, sequence) blocks, and
+// the reduction's terms per group.
+bool cuda_core_bwd_launchable(const Problem &P) {
+  const BwdPlan b = bwd_plan(P.B, P.L, P.D, P.d_g, P.l_h);
+  const int64_t i32 = std::numeric_limits<int32_t>::max();
+  return b.nchunk <= i32 && P.B <= i32 && P.B * b.nchunk * static_cast<int64_t>(b.npieces) <= i32 &&
+         P.B * b.nchunk * (P.d_g / b.cp) <= i32;
+}
+
+// run_if, run_token: as fir_tiled_kernel's (null: always run).
 template <typename T>
 int launch_bwd_cuda_core(const Problem &P, const void *dy, void *dk, void *dv, float *dh,
-                         float *partial, cudaStream_t s) {
+                         float *partial, cudaStream_t s, const unsigned *run_if = nullptr,
+                         unsigned run_token = 0) {
   DeviceState *ds = nullptr;
   if (current_device(ds) != HYENA_OK) return HYENA_ERR_CUDA;
   const long long cap = static_cast<long long>(ds->sm_count) * 16;
-  const int rt = launch_tiled<T, true>(P, dy, dk, dv, s);  // dk, dv
+  const int rt = launch_tiled<T, true>(P, dy, dk, dv, s, run_if, run_token);  // dk, dv
   if (rt != HYENA_OK) return rt;
+  if (!cuda_core_bwd_launchable(P)) return HYENA_ERR_UNSUPPORTED;
   const BwdPlan b = bwd_plan(P.B, P.L, P.D, P.d_g, P.l_h);
-  if (b.nchunk > 2147483647 || P.B > 65535 || b.npieces > 65535 ||
-      P.B * b.nchunk * (P.d_g / b.cp) > std::numeric_limits<int32_t>::max())
-    return HYENA_ERR_UNSUPPORTED;
-  const dim3 grid(static_cast<unsigned>(b.nchunk), static_cast<unsigned>(b.npieces),
-                  static_cast<unsigned>(P.B));
+  // gated: one block per SM walks every (chunk, piece, sequence); else one block each
+  const long long nblk = P.B * b.nchunk * static_cast<long long>(b.npieces);
+  const long long grid = run_if ? std::min<long long>(nblk, ds->sm_count) : nblk;
   const int smem = ((2 * hyena::bwd::kDhRows + hyena::bwd::kDhTaps - 1) * (b.cp + 1) +
                     hyena::bwd::kDhRedFloats) * 4;
-  hyena::bwd::fir_bwd_dh_partial_kernel<T><<<grid, hyena::bwd::kDhTaps, smem, s>>>(
-      static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v),
-      static_cast<const T *>(dy), partial, P.L, P.D, P.l_h, b.cp);
-  if (cudaGetLastError() != cudaSuccess) return HYENA_ERR_CUDA;
+  if (launch_ex(run_if != nullptr, hyena::bwd::fir_bwd_dh_partial_kernel<T>,
+                dim3(static_cast<unsigned>(grid)), dim3(hyena::bwd::kDhTaps), smem, s,
+                static_cast<const T *>(P.q), static_cast<const T *>(P.k),
+                static_cast<const T *>(P.v), static_cast<const T *>(dy), partial, P.L, P.D,
+                P.l_h, b.cp, b.nchunk, b.npieces, static_cast<int>(P.B), run_if,
+                run_token) != cudaSuccess ||
+      cudaGetLastError() != cudaSuccess)
+    return HYENA_ERR_CUDA;
   const long long gn = P.G() * P.l_h;  // one warp per output
   long long rblocks = (gn + hyena::bwd::kReduceBlock / 32 - 1) / (hyena::bwd::kReduceBlock / 32);
-  if (rblocks > cap) rblocks = cap;
-  hyena::bwd::fir_bwd_dh_reduce_kernel<<<static_cast<unsigned>(rblocks),
-                                         hyena::bwd::kReduceBlock, 0, s>>>(
-      partial, dh, static_cast<int>(P.B), b.nchunk, b.npieces, P.d_g / b.cp,
-      static_cast<int>(P.G()), P.l_h);
+  if (rblocks > (run_if ? ds->sm_count : cap)) rblocks = run_if ? ds->sm_count : cap;
+  if (launch_ex(run_if != nullptr, hyena::bwd::fir_bwd_dh_reduce_kernel,
+                dim3(static_cast<unsigned>(rblocks)), dim3(hyena::bwd::kReduceBlock), 0, s,
+                static_cast<const float *>(partial), dh, static_cast<int>(P.B), b.nchunk,
+                b.npieces, P.d_g / b.cp, static_cast<int>(P.G()), P.l_h, run_if,
+                run_token) != cudaSuccess)
+    return HYENA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
@@ -741,7 +788,7 @@ int launch_window_bwd_lh(const Problem &P, WindowParams wp, const void *dy, void
   hyena::bwd::fir_bwd_dh_reduce_kernel<<<static_cast<unsigned>(rblocks),
                                          hyena::bwd::kReduceBlock, 0, s>>>(
       partial, dh, static_cast<int>(P.B), static_cast<int>(wp.n_tb), static_cast<int>(wp.cv),
-      static_cast<int>(P.d_g / (wp.D / wp.cv)), static_cast<int>(P.G()), P.l_h);
+      static_cast<int>(P.d_g / (wp.D / wp.cv)), static_cast<int>(P.G()), P.l_h, nullptr, 0u);
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
@@ -808,8 +855,10 @@ int run_bwd_cuda_core(const Problem &P, const void *dy, void *dq, void *dk, void
 
 bool tc_bwd_supported(const Problem &P, const void *dy, const void *dq, const void *dk,
                       const void *dv) {
+  // the CUDA-core kernels stand behind it for operands outside fp16's range
   return P.dtype == HYENA_DTYPE_BF16 && P.d_g == hyena::tc::kNC && P.D % hyena::tc::kNC == 0 &&
-         P.l_h <= hyena::tcb::kMaxHalo + 1 && P.L <= (int64_t{1} << 30) &&
+         cuda_core_bwd_launchable(P) && P.l_h <= hyena::tcb::kMaxHalo + 1 &&
+         P.L <= (int64_t{1} << 30) &&
          P.B <= (int64_t{1} << 30) && aligned(P.q, 16) && aligned(P.k, 16) &&
          aligned(P.v, 16) && aligned(dy, 16) && aligned(dq, 16) && aligned(dk, 16) &&
          aligned(dv, 16);
@@ -862,6 +911,17 @@ int launch_tensor_bwd(const Problem &P, const void *dy, void *dq, void *dk, void
   p.D = P.D;
   p.dk = static_cast<__nv_bfloat16 *>(dk);
   p.dv = static_cast<__nv_bfloat16 *>(dv);
+  const int64_t flag_off = bwd_flag_offset(P.B, P.L, P.D, P.d_g, P.l_h);
+  if (flag_off + 4 > static_cast<int64_t>(workspace_bytes)) return HYENA_ERR_INVALID_ARG;
+  // The flag word is never reset: the kernel writes this call's token into it, and the fallback
+  // kernels run only where they find that token (a stale word from an earlier call, or
+  // whatever the workspace held, cannot match; if it ever did, the fp32 kernels would only
+  // redo the same gradients).
+  static std::atomic<unsigned> tokens{0};
+  unsigned token = tokens.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (token == 0) token = tokens.fetch_add(1, std::memory_order_relaxed) + 1;
+  p.range_flag = reinterpret_cast<unsigned *>(ws + flag_off);
+  p.range_token = token;
   Problem F = P;  // dq through the forward kernels
   F.q = dy;
   F.y = dq;
@@ -885,10 +945,17 @@ int launch_tensor_bwd(const Problem &P, const void *dy, void *dq, void *dk, void
   const long long gn = static_cast<long long>(p.G) * P.l_h;
   long long rblocks = (gn + 255) / 256;
   if (rblocks > ds->sm_count) rblocks = ds->sm_count;
-  tb::fir_bwd_tc_reduce_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
-      p.partial, p.seg_group, p.seg_count, p.max_segs, dh, p.G, P.l_h, per, p.W % grid,
-      static_cast<long long>(P.B) * p.nT);
-  return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+  if (launch_ex(true, tb::fir_bwd_tc_reduce_kernel, dim3(static_cast<unsigned>(rblocks)),
+                dim3(256), 0, s, static_cast<const float *>(p.partial),
+                static_cast<const int *>(p.seg_group), static_cast<const int *>(p.seg_count),
+                p.max_segs, dh, p.G, P.l_h, per, static_cast<long long>(p.W % grid),
+                static_cast<long long>(P.B) * p.nT) != cudaSuccess ||
+      cudaGetLastError() != cudaSuccess)
+    return HYENA_ERR_CUDA;
+  // Where an fp16 operand left its range (the kernel raised the flag), the fp32 CUDA-core
+  // kernels redo dk, dv and dh; otherwise each of them returns at once.
+  return launch_bwd_cuda_core<__nv_bfloat16>(P, dy, dk, dv, dh, reinterpret_cast<float *>(ws), s,
+                                             p.range_flag, token);
 }
 
 // FFT path: N = N1 N2 >= L + l_h - 1 (power of two, >= 256), N1 >= N2, both in [16, 256].

@@ -85,7 +85,10 @@ enum hyena_device_status_bits {
                                        power-of-two scaling (a scaled |k*v| above 65504, or a
                                        warp's rows all far below the sequence run's first
                                        tile), and the tiles reading it were recomputed in fp32
-                                       on the CUDA cores; outputs are valid */
+                                       on the CUDA cores; in the tensor-core backward an fp16
+                                       operand exceeded 65504 (or a group's taps all lay below
+                                       2^-10) and dk, dv, dh were recomputed in fp32; outputs
+                                       are valid */
 };
 
 /*
@@ -224,7 +227,8 @@ int hyena_select_algo(const void *q, const void *k, const void *v, const float *
  * shape.  The workspace holds fp32 partial filter gradients: on the CUDA-core path one per
  * sequence, 64-step chunk, channel piece and tap; on the register-window path (l_h <= 16) one
  * per thread (a 16-byte channel vector over a run of at least 32 time steps) and tap; on the
- * tensor path one per (CTA, sequence run) and tap, with the run's group and a run count per CTA.
+ * tensor path one per (CTA, sequence run) and tap, with the run's group and a run count per CTA,
+ * and after all partials one 256-byte slot for the tensor path's operand-range flag.
  * Touches no device.  A smaller workspace still runs where it holds what the chosen algorithm
  * needs at least (the window path then takes longer runs); the size returned here runs every
  * algorithm at full speed.
@@ -246,7 +250,11 @@ int64_t hyena_conv_bwd_workspace_bytes(int64_t B, int64_t L, int64_t D, int d_g,
  * comes from the forward kernels (dy in the place of q); where the tensor path applies (bf16,
  * d_g == 64, D % 64 == 0, l_h <= 129, all seven tensors 16-byte aligned) one tcgen05 kernel
  * reads q, k, v, dy once and writes dk, dv once, with fp16 operands (x = k v, dz = q dy, h
- * rounded to fp16) and fp32 accumulation; else, for l_h <= 16 with d_g a multiple of 8 (bf16)
+ * rounded to fp16) and fp32 accumulation -- where one of them holds a value above 65504, or a
+ * group's taps all lie below 2^-10, the kernel raises HYENA_DEVICE_F16_RANGE and fp32
+ * CUDA-core kernels queued behind it recompute dk, dv and dh (values of x or dz within fp16's
+ * subnormal range, below about 6e-5, take the fp16 path with reduced relative precision);
+ * else, for l_h <= 16 with d_g a multiple of 8 (bf16)
  * or 4 (fp32) and q, k, v, dy, dk, dv 16-byte aligned, one CUDA-core register-window kernel
  * (HYENA_ALGO_WINDOW) does the same in fp32; otherwise CUDA-core kernels in fp32 (one for dk,
  * dv, one for the dh partials).  dh is summed in a fixed order on every path: results are

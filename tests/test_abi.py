@@ -272,10 +272,11 @@ def test_python_binding_rejects_cpu_tensors():
 
 def test_bwd_workspace_bytes(lib):
     # D = 4096, d_g = 64 (pieces of 64 channels), l_h = 128, 8192 tokens: 128 chunks x 64 x 128
-    assert lib.hyena_conv_bwd_workspace_bytes(1, 8192, 4096, 64, 128) == 128 * 64 * 128 * 4
+    # partials, then 256 bytes for the tensor path's operand-range flag
+    assert lib.hyena_conv_bwd_workspace_bytes(1, 8192, 4096, 64, 128) == 128 * 64 * 128 * 4 + 256
     assert lib.hyena_conv_bwd_workspace_bytes(1, 8192, 4096, 63, 128) == -1
     assert lib.hyena_conv_bwd_workspace_bytes(0, 8192, 4096, 64, 128) == 0
-    assert lib.hyena_conv_bwd_workspace_bytes(1, 1, 6, 6, 5) == 256  # rounded up
+    assert lib.hyena_conv_bwd_workspace_bytes(1, 1, 6, 6, 5) == 512  # rounded up, + the flag
     # SE (l_h = 7, d_g = 16): the window kernel's partials at its shortest runs, one per
     # 32-row block and 4-channel vector (the fp32 width): 256 x 1024 x 7 floats
     assert lib.hyena_conv_bwd_workspace_bytes(1, 8192, 4096, 16, 7) == 256 * 1024 * 7 * 4
