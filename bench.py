@@ -50,7 +50,7 @@ def parse():
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--workload", default="mr")
-    p.add_argument("--algo", default="auto", choices=["auto", "tensor", "window", "direct"],
+    p.add_argument("--algo", default="auto", choices=["auto", "tensor", "window", "direct", "fft"],
                    help="forward algorithm of the timed launches (auto = the library's choice)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=10)
@@ -326,7 +326,7 @@ def time_configs(args, stream, dev, D, g, _native, peak, peak_kind):
         nbytes = wl.algorithmic_bytes()
         achieved = nbytes / (ms / 1e3) / 1e9
         kernel = {g.HYENA_ALGO_TENSOR: "fir_tc_kernel", g.HYENA_ALGO_WINDOW: "fir_window_kernel",
-                  g.HYENA_ALGO_DIRECT: "fir_tiled_kernel"}[algo]
+                  g.HYENA_ALGO_DIRECT: "fir_tiled_kernel", g.HYENA_ALGO_FFT: "fir_fftblk_kernel"}[algo]
         out[name] = {"workload": wl.describe(), "ms_per_step": ms, "steps": K,
                      "value": D.env_world()[2] * wl.tokens / (ms / 1e3), "unit": UNIT,
                      "gpu_launches": K, "kernel": kernel, "launch_stats": stats,
@@ -517,7 +517,7 @@ def main():
     dcode = g.HYENA_DTYPE_F32 if wl.dtype == "f32" else g.HYENA_DTYPE_BF16
     algo = g.hyena_select_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b, dcode)
     forced = {"auto": None, "tensor": g.HYENA_ALGO_TENSOR, "window": g.HYENA_ALGO_WINDOW,
-              "direct": g.HYENA_ALGO_DIRECT}[args.algo]
+              "direct": g.HYENA_ALGO_DIRECT, "fft": g.HYENA_ALGO_FFT}[args.algo]
     fwd = g.hyena_conv_fwd_f32 if wl.dtype == "f32" else g.hyena_conv_fwd
     stream = torch.cuda.Stream(device=dev)
 
@@ -637,7 +637,7 @@ def main():
         bytes_per_launch = wl.algorithmic_bytes()
         achieved = bytes_per_launch / (mean_launch_ms / 1e3) / 1e9
         kernel = {g.HYENA_ALGO_TENSOR: "fir_tc_kernel", g.HYENA_ALGO_WINDOW: "fir_window_kernel",
-                  g.HYENA_ALGO_DIRECT: "fir_tiled_kernel"}[algo]
+                  g.HYENA_ALGO_DIRECT: "fir_tiled_kernel", g.HYENA_ALGO_FFT: "fir_fftblk_kernel"}[algo]
         traffic = committed_traffic(kernel, wl.name)
         line = {
             "metric": METRIC if wl.name == "mr" else
