@@ -304,7 +304,8 @@ int hyena_select_bwd_algo(const void *q, const void *k, const void *v, const flo
  * allocates nothing.  Arguments, results and errors are those of hyena_conv_bwd, plus:
  *   - HYENA_ERR_UNSUPPORTED, with nothing queued, when the least workspace the shape needs
  *     exceeds HYENA_BWD_STATIC_SCRATCH_BYTES (e.g. the D = 4096, d_g = 64, l_h = 128 shape
- *     above B * L = 16384 tokens); use hyena_conv_bwd with a workspace there.
+ *     from B * L = 16384 tokens on: 8 MiB of partials and the range flag); use
+ *     hyena_conv_bwd with a workspace there.
  *   - The first call on each device looks up the array's address (cudaGetSymbolAddress) with
  *     that device current and keeps it (a failed lookup returns HYENA_ERR_CUDA and is tried
  *     again on the next call); make that first call before any stream capture.
