@@ -102,6 +102,10 @@ __global__ void __launch_bounds__(kWindowBlock, HYENA_WINDOW_MIN_BLOCKS)
   constexpr int VN = Vec<T>::N;
   // Longer windows hold more registers: they unroll no further than 4 rows.
   constexpr int U = LH <= 8 ? kWindowUnroll : (kWindowUnroll < 4 ? kWindowUnroll : 4);
+  // Launched with programmatic stream serialisation: the next kernel of the stream may be
+  // scheduled at once, and this one reads nothing before the previous kernel has completed.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (gid >= p.B * p.n_tb * p.cv) return;
   const long long cvi = gid % p.cv;

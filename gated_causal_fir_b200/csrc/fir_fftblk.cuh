@@ -336,6 +336,11 @@ __global__ void __launch_bounds__(NT, 1) fir_fftblk_kernel(const BlkParams p) {
   uint8_t *qst = smem_raw + SM::kOffQ;                        // staged q rows
   const int tid = threadIdx.x;
   for (int r = tid; r < N / 4; r += NT) tw[r] = fft::twiddle(r, N);
+  // Launched with programmatic stream serialisation: the next kernel of the stream may be
+  // scheduled at once, and this one reads no global memory before the previous kernel has
+  // completed (the twiddle table above overlaps its tail).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const uint8_t *q = static_cast<const uint8_t *>(p.q), *k = static_cast<const uint8_t *>(p.k),
                 *v = static_cast<const uint8_t *>(p.v), *kh = static_cast<const uint8_t *>(p.kh),

@@ -442,6 +442,24 @@ int resident_blocks(K kernel, int block, std::atomic<int> (&cache)[kMaxDevices],
   return HYENA_OK;
 }
 
+// A kernel launch, with programmatic stream serialisation where `pdl` (the kernel then waits
+// for the previous kernels of the stream itself, with griddepcontrol.wait).
+template <typename... Exp, typename... Act>
+cudaError_t launch_ex(bool pdl, void (*kernel)(Exp...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t s, Act &&...args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl && HYENA_PDL;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Act>(args)...);
+}
+
 // Run length of the window kernels: with `units` thread columns per time block and `wave`
 // resident threads, the rows that make the whole problem one full wave.
 long long window_rows(long long units, long long L, long long wave) {
@@ -470,9 +488,11 @@ int launch_window_lh(const Problem &P, WindowParams wp, int sm_count, cudaStream
   const long long threads = units * wp.n_tb;
   const long long blocks = (threads + hyena::cc::kWindowBlock - 1) / hyena::cc::kWindowBlock;
   if (blocks > std::numeric_limits<int32_t>::max()) return HYENA_ERR_UNSUPPORTED;
-  kernel<<<static_cast<unsigned>(blocks), hyena::cc::kWindowBlock, 0, s>>>(
-      static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v), P.h,
-      static_cast<T *>(P.y), wp);
+  if (launch_ex(true, kernel, dim3(static_cast<unsigned>(blocks)), dim3(hyena::cc::kWindowBlock), 0,
+                s, static_cast<const T *>(P.q), static_cast<const T *>(P.k),
+                static_cast<const T *>(P.v), static_cast<const float *>(P.h),
+                static_cast<T *>(P.y), wp) != cudaSuccess)
+    return HYENA_ERR_CUDA;
   return HYENA_OK;
 }
 
@@ -508,24 +528,6 @@ int launch_window(const Problem &P, cudaStream_t s) {
 
 // The tiled direct sum (fir_tiled_kernel): forward (y) or, with kAnti, the backward's
 // transposed product (dk, dv from q, dy).  Persistent CTAs over the tiles.
-// A kernel launch, with programmatic stream serialisation where `pdl` (the kernel then waits
-// for the previous kernels of the stream itself, with griddepcontrol.wait).
-template <typename... Exp, typename... Act>
-cudaError_t launch_ex(bool pdl, void (*kernel)(Exp...), dim3 grid, dim3 block, size_t smem,
-                      cudaStream_t s, Act &&...args) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = pdl && HYENA_PDL;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Act>(args)...);
-}
-
 // run_if (anti only): the kernel's gate word, run_token the value that lets it run; a gated
 // launch takes one block per SM and starts early (programmatic dependent launch), so that it
 // costs little when the word does not match.
@@ -572,8 +574,10 @@ int launch_fftblk_cfg(const Problem &P, const BlkPlan &bp, int sm_count, cudaStr
   p.items = P.B * (p.CB / p.Q) * static_cast<long long>(p.nTB);
   const long long groups = std::max<long long>(1, static_cast<long long>(sm_count) / p.Q);
   const long long grid = std::min<long long>(p.items, groups) * p.Q;
-  hyena::fftblk::fir_fftblk_kernel<T, LGN, PP, kBlkThreads, SQ>
-      <<<static_cast<unsigned>(grid), kBlkThreads, hyena::fftblk::Smem<T, LGN, PP, SQ>::kBytes, s>>>(p);
+  if (launch_ex(true, hyena::fftblk::fir_fftblk_kernel<T, LGN, PP, kBlkThreads, SQ>,
+                dim3(static_cast<unsigned>(grid)), dim3(kBlkThreads),
+                hyena::fftblk::Smem<T, LGN, PP, SQ>::kBytes, s, p) != cudaSuccess)
+    return HYENA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
