@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kBwdWindowBlock)
                           const T *__restrict__ v, const float *__restrict__ h,
                           const T *__restrict__ dy, T *__restrict__ dk, T *__restrict__ dv,
                           float *__restrict__ partial, const cc::WindowParams p) {
+  cc::pdl_enter();  // launched with programmatic stream serialisation
   using V = cc::Vec<T>;
   constexpr int VN = V::N;
   constexpr int U = LH <= 8 ? 4 : 2;  // rows of loads issued before their arithmetic

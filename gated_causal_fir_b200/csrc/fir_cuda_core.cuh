@@ -66,6 +66,14 @@ struct Vec<float> {
   }
 };
 
+// Programmatic dependent launch, for kernels launched with programmatic stream serialisation:
+// let the next kernel of the stream be scheduled at once, then wait until the previous one has
+// completed and its writes are visible.  Call before the first global-memory access.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ void from_f32(float v, __nv_bfloat16 *p) { *p = __float2bfloat16_rn(v); }
@@ -102,10 +110,7 @@ __global__ void __launch_bounds__(kWindowBlock, HYENA_WINDOW_MIN_BLOCKS)
   constexpr int VN = Vec<T>::N;
   // Longer windows hold more registers: they unroll no further than 4 rows.
   constexpr int U = LH <= 8 ? kWindowUnroll : (kWindowUnroll < 4 ? kWindowUnroll : 4);
-  // Launched with programmatic stream serialisation: the next kernel of the stream may be
-  // scheduled at once, and this one reads nothing before the previous kernel has completed.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_enter();  // launched with programmatic stream serialisation
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (gid >= p.B * p.n_tb * p.cv) return;
   const long long cvi = gid % p.cv;

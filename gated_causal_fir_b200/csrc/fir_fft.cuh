@@ -283,6 +283,7 @@ __global__ void __launch_bounds__(kThreads)
   const int N = N1 * p.N2;
   const int idx = threadIdx.x / kP, sig = threadIdx.x % kP;
   fill_twiddles(tw, N1, tw2, n2, N);
+  cc::pdl_enter();  // launched with programmatic stream serialisation (the tables overlap)
   // stage the rows t = N2 n1 + n2 of the CTA's 16 signals: ex[n1 * 16 + signal]
   if constexpr (kSpectrum) {
     for (int e = threadIdx.x; e < N1 * kP; e += blockDim.x) {
@@ -351,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, N2 <= 128 ? 8 : (kSpectrum ? 1 : 4))
   const int idx = threadIdx.x / kP, sig = threadIdx.x % kP;
   const bool live = s0 + sig < p.PT;
   fill_twiddles(tw, N2);
+  cc::pdl_enter();  // launched with programmatic stream serialisation (the table overlaps)
   // A[b][k1][n2][s0 + sig] at row[n2 PT]
   float2 *row = A + (b * p.N1 + k1) * N2 * p.PT + s0 + sig;
   float2 va[R1], vb[BLay<N2>::M];
@@ -393,6 +395,7 @@ __global__ void __launch_bounds__(kThreads)
   const int N = N1 * p.N2;
   const int idx = threadIdx.x / kP, sig = threadIdx.x % kP;
   fill_twiddles(tw, N1, tw2, n2, N);
+  cc::pdl_enter();  // launched with programmatic stream serialisation (the tables overlap)
   __syncthreads();
   float2 va[R1], vb[BLay<N1>::M];
   {

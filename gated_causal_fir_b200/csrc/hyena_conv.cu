@@ -781,10 +781,13 @@ int launch_window_bwd_lh(const Problem &P, WindowParams wp, const void *dy, void
       wp.cv > std::numeric_limits<int32_t>::max() ||
       wp.B * wp.n_tb * (P.d_g / (wp.D / wp.cv)) > std::numeric_limits<int32_t>::max())
     return HYENA_ERR_UNSUPPORTED;
-  kernel<<<static_cast<unsigned>(blocks), hyena::bwd::kBwdWindowBlock, 0, s>>>(
-      static_cast<const T *>(P.q), static_cast<const T *>(P.k), static_cast<const T *>(P.v), P.h,
-      static_cast<const T *>(dy), static_cast<T *>(dk), static_cast<T *>(dv), partial, wp);
-  if (cudaGetLastError() != cudaSuccess) return HYENA_ERR_CUDA;
+  if (launch_ex(true, kernel, dim3(static_cast<unsigned>(blocks)),
+                dim3(hyena::bwd::kBwdWindowBlock), 0, s, static_cast<const T *>(P.q),
+                static_cast<const T *>(P.k), static_cast<const T *>(P.v),
+                static_cast<const float *>(P.h), static_cast<const T *>(dy),
+                static_cast<T *>(dk), static_cast<T *>(dv), partial, wp) != cudaSuccess ||
+      cudaGetLastError() != cudaSuccess)
+    return HYENA_ERR_CUDA;
   const long long gn = P.G() * P.l_h;  // one warp per output
   long long rblocks = (gn + hyena::bwd::kReduceBlock / 32 - 1) / (hyena::bwd::kReduceBlock / 32);
   const long long cap = static_cast<long long>(sm_count) * 16;
@@ -1012,28 +1015,31 @@ int fft_supported(const Problem &P, FftPlan &f) {
 template <typename T, int N1>
 void launch_fft_p1(const Problem &P, const hyena::fft::FftParams &p, dim3 grid, float2 *A,
                    cudaStream_t s) {
-  hyena::fft::fft_pass1_kernel<T, false, N1><<<grid, hyena::fft::kThreads, 0, s>>>(
-      static_cast<const T *>(P.k), static_cast<const T *>(P.v), nullptr, A, p);
+  launch_ex(true, hyena::fft::fft_pass1_kernel<T, false, N1>, grid, dim3(hyena::fft::kThreads), 0,
+            s, static_cast<const T *>(P.k), static_cast<const T *>(P.v),
+            static_cast<const float *>(nullptr), A, p);
 }
 
 template <int N1>
 void launch_fft_spec1(const Problem &P, const hyena::fft::FftParams &p, dim3 grid, float2 *A,
                       cudaStream_t s) {
-  hyena::fft::fft_pass1_kernel<float, true, N1><<<grid, hyena::fft::kThreads, 0, s>>>(
-      nullptr, nullptr, P.h, A, p);
+  launch_ex(true, hyena::fft::fft_pass1_kernel<float, true, N1>, grid,
+            dim3(hyena::fft::kThreads), 0, s, static_cast<const float *>(nullptr),
+            static_cast<const float *>(nullptr), P.h, A, p);
 }
 
 template <typename T, int N1>
 void launch_fft_p3(const Problem &P, const hyena::fft::FftParams &p, dim3 grid, const float2 *A,
                    cudaStream_t s) {
-  hyena::fft::fft_pass3_kernel<T, N1><<<grid, hyena::fft::kThreads, 0, s>>>(
-      A, static_cast<const T *>(P.q), static_cast<T *>(P.y), p);
+  launch_ex(true, hyena::fft::fft_pass3_kernel<T, N1>, grid, dim3(hyena::fft::kThreads), 0, s, A,
+            static_cast<const T *>(P.q), static_cast<T *>(P.y), p);
 }
 
 template <bool kSpectrum, int N2>
 void launch_fft_p2(const hyena::fft::FftParams &p, dim3 grid, float2 *A, float2 *H,
                    cudaStream_t s) {
-  hyena::fft::fft_pass2_kernel<kSpectrum, N2><<<grid, hyena::fft::kThreads, 0, s>>>(A, H, p);
+  launch_ex(true, hyena::fft::fft_pass2_kernel<kSpectrum, N2>, grid, dim3(hyena::fft::kThreads), 0,
+            s, A, H, p);
 }
 
 // Calls F<n>() for the transform length n in {16, ..., 256}.
