@@ -1,0 +1,97 @@
+"""Back-to-back calls on one stream, each reading the previous call's output (needs a B200).
+
+Every forward and backward kernel is launched with programmatic stream serialisation: it may
+start while the previous kernel of the stream still runs, and it must not touch global memory
+before that kernel has completed.  These chains make each call read what the one before wrote
+(y of call i is k of call i + 1, cycling through the algorithms), queued with no
+synchronisation in between, and compare with the same chain run with a device synchronisation
+after every call: the kernels are deterministic, so the two must agree bit for bit.  A read
+that raced ahead of the previous kernel's writes would see stale or partial data and differ.
+Every output is also checked against the oracle on the same inputs."""
+import pytest
+import torch
+
+import gated_causal_fir_b200 as g
+from gated_causal_fir_b200.workloads import custom, make_grad, make_inputs
+from tests import _gpu_util as U
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    from gated_causal_fir_b200 import build
+    build.build()
+    g.hyena_device_status(clear=True)
+    yield
+    assert g.hyena_device_status(clear=True) == 0, "a kernel raised its device status word"
+
+
+T, W, F, Dd = g.HYENA_ALGO_TENSOR, g.HYENA_ALGO_WINDOW, g.HYENA_ALGO_FFT, g.HYENA_ALGO_DIRECT
+CHAINS = [
+    # name, B, L, D, d_g, l_h, algorithms in call order
+    ("se_shape", 2, 3000, 256, 16, 7, (W, T, F, W, Dd, T, W)),
+    ("mr_shape", 1, 5000, 512, 64, 128, (T, F, T, Dd, T, F, T)),
+    ("long_filter", 1, 4000, 256, 64, 514, (F, Dd, F, F)),
+]
+
+
+def _chain(q, k, v, h, d_g, algos, sync):
+    ys = []
+    for a in algos:
+        y = g.hyena_conv_fwd_ex(q, k, v, h, d_g, 64, algo=a)
+        if sync:
+            torch.cuda.synchronize()
+        ys.append(y)
+        k = y
+    torch.cuda.synchronize()
+    return ys
+
+
+@pytest.mark.parametrize("chain", CHAINS, ids=[c[0] for c in CHAINS])
+def test_forward_chain_without_sync(chain):
+    name, B, L, D, d_g, l_h, algos = chain
+    wl = custom(name, B, L, D, d_g, l_h, 64, "bf16", "mr" if l_h > 16 else "se", seed=L + l_h)
+    q, k, v, h = make_inputs(wl, device="cuda")
+    fast = _chain(q, k, v, h, d_g, algos, sync=False)
+    slow = _chain(q, k, v, h, d_g, algos, sync=True)
+    for i, (a, b) in enumerate(zip(fast, slow)):
+        assert torch.equal(a, b), "call %d (%s) differs without synchronisation" % (
+            i, g.ALGO_NAMES[algos[i]])
+    # each call against the oracle on the same inputs: the first elementwise under the bf16
+    # bound; the later ones, whose k is a previous output with heavier tails than N(0, 1) (the
+    # bound's absolute term assumes unit-scale inputs), normwise within 2^-8
+    kk = k
+    for i, a in enumerate(algos):
+        ref = oracle.gated_fir(q, kk, v, h, d_g)
+        if i == 0:
+            U.assert_parity(fast[i], ref, q.dtype)
+        else:
+            assert torch.isfinite(fast[i]).all()
+            r = U.f32_normwise(fast[i], ref)
+            assert r <= 2.0 ** -8, "call %d: normwise error %.2e" % (i, r)
+        kk = fast[i]
+
+
+def test_backward_after_forward_without_sync():
+    """A forward whose output is the backward's dy, then a forward reading the backward's dk,
+    all queued at once: equal to the synchronised run."""
+    wl = custom("bwd_chain", 1, 4096, 512, 64, 128, 64, "bf16", "mr", seed=9)
+    q, k, v, h = make_inputs(wl, device="cuda")
+
+    def run(sync):
+        y = g.hyena_conv_fwd_ex(q, k, v, h, 64, 64, algo=T)
+        if sync:
+            torch.cuda.synchronize()
+        dq, dk, dv, dh = g.hyena_conv_bwd_ex(q, k, v, h, y, 64, 64, algo=T)
+        if sync:
+            torch.cuda.synchronize()
+        y2 = g.hyena_conv_fwd_ex(q, dk, v, h, 64, 64, algo=T)
+        torch.cuda.synchronize()
+        return [y, dq, dk, dv, dh, y2]
+
+    for a, b in zip(run(False), run(True)):
+        assert torch.equal(a, b)
