@@ -346,10 +346,10 @@ def time_long_filters(args, stream, dev, D, g, _native, peak, peak_kind):
 
     * ``li_fft``: the Hyena-LI-shaped workload (B=1, L=8192, D=4096, d_g=64, l_h=8192) through
       hyena_conv_fwd_fft (four-step FFT, caller workspace);
-    * ``mr_lh513``: the MR shape with l_h = 513, the longest filter of the tensor-core path
-      (hyena_conv_fwd, AUTO);
-    * ``mr_lh514``: one tap longer, past the tensor band: AUTO runs the single-pass block FFT
-      (no workspace).
+    * ``mr_lh513``, ``mr_lh514``: the MR shape with l_h = 513 (four history tiles on the
+      tensor-core path) and 514 (five, with one band set and two k/v stages) (AUTO);
+    * ``mr_lh641``, ``mr_lh642``: the longest filter of the tensor-core path, and one tap
+      longer, past the tensor band: AUTO runs the single-pass block FFT (no workspace).
 
     Algorithmic bytes per call: q, k, v read and y written (4 B L D bf16 elements); the FFT's
     spectra in the workspace are overhead, not counted."""
@@ -361,7 +361,11 @@ def time_long_filters(args, stream, dev, D, g, _native, peak, peak_kind):
                           ("mr_lh513", custom("mr_lh513", 1, 8192, 4096, 64, 513, 64, "bf16",
                                               "mr", seed=6), False),
                           ("mr_lh514", custom("mr_lh514", 1, 8192, 4096, 64, 514, 64, "bf16",
-                                              "mr", seed=7), False)):
+                                              "mr", seed=7), False),
+                          ("mr_lh641", custom("mr_lh641", 1, 8192, 4096, 64, 641, 64, "bf16",
+                                              "mr", seed=8), False),
+                          ("mr_lh642", custom("mr_lh642", 1, 8192, 4096, 64, 642, 64, "bf16",
+                                              "mr", seed=9), False)):
         sets = [make_inputs(wl, device=dev, seed=wl.seed + 101 * s) for s in range(2)]
         ys = [torch.empty_like(x[0]) for x in sets]
         torch.cuda.synchronize()  # inputs complete before `stream` reads them

@@ -10,8 +10,9 @@
 // One tile = 128 output rows x 64 channels (64 / d_g groups).  The block size of the
 // decomposition is 128 rows, the largest M of one tcgen05.mma.  A tile reads its own 128 input
 // rows and halo = roundup16(l_h - 1) rows before them, which lie in the kNH = ceil(halo / 128)
-// earlier tiles (one for l_h <= 129, where this is the two-stage form of Sec. 3; up to four for
-// l_h <= 513, the general block form of Sec. 2).  As one GEMM per tile and group:
+// earlier tiles (one for l_h <= 129, where this is the two-stage form of Sec. 3; up to five for
+// l_h <= 641, the general block form of Sec. 2; five hold one band set in tensor memory and two
+// k/v stages).  As one GEMM per tile and group:
 //   D[128 x d_g] = A[128 x K] * X[K x d_g],  K = 128 + halo,
 // A is the Toeplitz band over input rows [t0 - halo, t0 + 128), X = k*v over those rows.
 //
@@ -47,12 +48,12 @@ namespace tc {
 
 constexpr int kTM = 128;             // output rows per tile (MMA M)
 constexpr int kNC = 64;              // channels per tile: 64 / d_g groups of d_g (MMA N = d_g)
-constexpr int kMaxHist = 4;          // history tiles a tile may read: l_h - 1 <= 4 * 128
+constexpr int kMaxHist = 5;          // history tiles a tile may read: l_h - 1 <= 5 * 128
 constexpr int kMaxHalo = kMaxHist * kTM;
 #ifndef HYENA_TC_KV_STAGES
 #define HYENA_TC_KV_STAGES 3
 #endif
-constexpr int kNKV = HYENA_TC_KV_STAGES;  // k/v stages
+constexpr int kNKV = HYENA_TC_KV_STAGES;  // k/v stages (two where five history tiles are held)
 // Unrolling of the gate's and the epilogue's per-tile loops (8 iterations each).  The kernel's
 // warp roles run different code side by side, so hot-loop code size competes for the
 // instruction cache.
@@ -87,6 +88,7 @@ constexpr int kGroupThreads = 128;
 // history, the current tile and the next one being gated).
 template <int kNH>
 struct Layout {
+  static constexpr int kNKV = kNH >= 5 ? 2 : tc::kNKV;  // k/v stages
   static constexpr int kNQ = kNH >= 4 ? 2 : 3;   // q (and in-place y) stages
   static constexpr int kNX = kNH + 2;            // fp16 X slots
   static constexpr int kOffKV = 0;
@@ -94,7 +96,8 @@ struct Layout {
   static constexpr int kOffX = kOffQ + kNQ * kTileBytes;
   // fp16 filter taps of the tile's groups, zero-padded: 258 + halo per group (see stage_taps);
   // kPer of them per gate thread
-  static constexpr int kHzBytes = kNH == 1 ? 2688 : (kNH == 2 ? 2064 : (kNH == 3 ? 1296 : 1552));
+  static constexpr int kHzBytes =
+      kNH == 1 ? 2688 : (kNH == 2 ? 2064 : (kNH == 3 ? 1296 : (kNH == 4 ? 1552 : 1808)));
   static constexpr int kPer = (kHzBytes / 2 + kGroupThreads - 1) / kGroupThreads;
   static constexpr int kOffHz = kOffX + kNX * kTileBytes;
   // Output tiles whose fp16 operands left the range, listed by the gate warps for the
@@ -542,7 +545,7 @@ __device__ __forceinline__ void build_band_tmem(uint32_t band_col, int band_cols
 }
 
 // kNG = 64 / d_g groups per tile (1, 2 or 4); MMA N = d_g.  kNH = ceil(halo / 128) earlier
-// tiles feed each tile's product (1 for l_h <= 129, up to 4 for l_h <= 513).  kHooks builds
+// tiles feed each tile's product (1 for l_h <= 129, up to 5 for l_h <= 641).  kHooks builds
 // the test instantiation: the waits between roles use p.wait_ns, and p.fault == 1 withholds
 // the first accumulator arrive; the product instantiations carry neither.
 template <int kNG, int kNH, bool kHooks = false>
@@ -589,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long w_end = w_begin + per + (bx < rem ? 1 : 0);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNKV; ++i) {
+    for (int i = 0; i < Ly::kNKV; ++i) {
       mbar_init(&bars[kBarKVFull + i], 1);
       mbar_init(&bars[kBarKVEmpty + i], kGroupThreads);
     }
@@ -655,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t kv_count = 0;
   bool kv_done = false;
   if (threadIdx.x == 0) {
-    while (kv_count < kNKV) {
+    while (kv_count < Ly::kNKV) {
       if (!kv_it.next(kv_t)) {
         kv_done = true;
         break;
@@ -685,15 +688,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kc = kv_count;
       while (!kv_done && kv_it.next(kv_t)) {
         const Item &t = kv_t;
-        const int ks = kc % kNKV;
-        if (!thread_wait(&bars[kBarKVEmpty + ks], ((kc / kNKV) & 1) ^ 1, abort, lim)) break;
+        const int ks = kc % Ly::kNKV;
+        if (!thread_wait(&bars[kBarKVEmpty + ks], ((kc / Ly::kNKV) & 1) ^ 1, abort, lim)) break;
         mbar_arrive_expect_tx(&bars[kBarKVFull + ks], 2 * kTileBytes);
         load_kv(ks, t);
         ++kc;
       }
       // Every load this thread issued must land before the CTA may exit.
-      for (uint32_t n = kc > kNKV ? kc - kNKV : 0; n < kc; ++n)
-        drain_wait(&bars[kBarKVFull + n % kNKV], (n / kNKV) & 1);
+      for (uint32_t n = kc > Ly::kNKV ? kc - Ly::kNKV : 0; n < kc; ++n)
+        drain_wait(&bars[kBarKVFull + n % Ly::kNKV], (n / Ly::kNKV) & 1);
     }
   } else if (warp == kWarpTmaQ) {
     // ---------------------------------------------------------------- TMA producer: q
@@ -822,10 +825,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float first_mx = 0.f;  // this lane's largest scaled |x| of the run's first tile
     auto gate_item = [&](auto scaled, bool built) -> bool {
       constexpr bool kScaled = decltype(scaled)::value;
-      const int ks = kc % kNKV, xs = xc % kNX;
+      const int ks = kc % Ly::kNKV, xs = xc % kNX;
       float mx = first_mx;  // the run's first tile was converted at the run's start
       if (!built) {
-        if (!warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort, lim)) return false;
+        if (!warp_wait(&bars[kBarKVFull + ks], (kc / Ly::kNKV) & 1, abort, lim)) return false;
         if (!warp_wait(&bars[kBarXEmpty + xs], ((xc / kNX) & 1) ^ 1, abort, lim)) return false;
         const uint32_t kbase = smem_u32(kv_st + ks * 2 * kTileBytes);
         mx = gate_x_tile<kScaled>(kbase, kbase + kTileBytes, smem_u32(x_st + xs * kTileBytes),
@@ -883,8 +886,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // x's scale from the largest |k v| of the run's first tile: that tile is converted
         // unscaled first (no scale is the usual case), every warp merges its maximum, and the
         // tile is converted again, scaled, only if the run needs it
-        const int ks = kc % kNKV, xs = xc % kNX;
-        if (!warp_wait(&bars[kBarKVFull + ks], (kc / kNKV) & 1, abort, lim)) break;
+        const int ks = kc % Ly::kNKV, xs = xc % kNX;
+        if (!warp_wait(&bars[kBarKVFull + ks], (kc / Ly::kNKV) & 1, abort, lim)) break;
         if (!warp_wait(&bars[kBarXEmpty + xs], ((xc / kNX) & 1) ^ 1, abort, lim)) break;
         const uint32_t kbase = smem_u32(kv_st + ks * 2 * kTileBytes);
         const uint32_t xbase = smem_u32(x_st + xs * kTileBytes);

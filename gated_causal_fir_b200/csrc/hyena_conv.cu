@@ -71,6 +71,7 @@ int current_device(DeviceState *&ds) {
         {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 2>), hyena::tc::Layout<2>::kSmemBytes},
         {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 3>), hyena::tc::Layout<3>::kSmemBytes},
         {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 4>), hyena::tc::Layout<4>::kSmemBytes},
+        {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<1, 5>), hyena::tc::Layout<5>::kSmemBytes},
         {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<2, 1>), hyena::tc::Layout<1>::kSmemBytes},
         {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<2, 2>), hyena::tc::Layout<2>::kSmemBytes},
         {reinterpret_cast<const void *>(hyena::tc::fir_tc_kernel<4, 1>), hyena::tc::Layout<1>::kSmemBytes},
@@ -408,6 +409,7 @@ int launch_tensor(const Problem &P, cudaStream_t s, const TcTestHooks &hooks = T
     case 10: HYENA_TC_LAUNCH(1, 2); break;
     case 11: HYENA_TC_LAUNCH(1, 3); break;
     case 12: HYENA_TC_LAUNCH(1, 4); break;
+    case 13: HYENA_TC_LAUNCH(1, 5); break;
     case 17: HYENA_TC_LAUNCH(2, 1); break;
     case 18: HYENA_TC_LAUNCH(2, 2); break;
     case 33: HYENA_TC_LAUNCH(4, 1); break;

@@ -60,7 +60,7 @@ enum hyena_dtype {
 enum hyena_algo {
     HYENA_ALGO_AUTO = 0,         /* pick the fastest algorithm that supports the problem */
     HYENA_ALGO_TENSOR = 1,       /* tcgen05 tensor-core block-Toeplitz GEMM (bf16 only;
-                                    D % 64 == 0, d_g in {16, 32, 64}; l_h <= 513 for
+                                    D % 64 == 0, d_g in {16, 32, 64}; l_h <= 641 for
                                     d_g == 64, <= 257 for d_g == 32, <= 65 for d_g == 16;
                                     16-byte aligned tensors) */
     HYENA_ALGO_WINDOW = 2,       /* CUDA-core register sliding window, forward and backward

@@ -66,7 +66,8 @@ def test_select_algo_for_the_workloads(lib):
 
 def test_select_algo_fallbacks(lib):
     bf, f32 = g.HYENA_DTYPE_BF16, g.HYENA_DTYPE_F32
-    assert g.hyena_select_algo(1, 100, 256, 64, 514, 65, bf) == g.HYENA_ALGO_FFT     # l_h > 513
+    assert g.hyena_select_algo(1, 100, 256, 64, 642, 65, bf) == g.HYENA_ALGO_FFT     # l_h > 641
+    assert g.hyena_select_algo(1, 100, 256, 64, 641, 65, bf) == g.HYENA_ALGO_TENSOR  # 5 tiles back
     assert g.hyena_select_algo(1, 100, 256, 64, 130, 65, bf) == g.HYENA_ALGO_TENSOR  # 2 tiles back
     assert g.hyena_select_algo(1, 100, 256, 64, 129, 65, bf) == g.HYENA_ALGO_TENSOR
     assert g.hyena_select_algo(1, 100, 128, 32, 40, 32, bf) == g.HYENA_ALGO_TENSOR
@@ -109,7 +110,7 @@ def _call(lib, q=0x10000, k=0x20000, v=0x30000, h=0x40000, y=0x50000, dtype=0, a
     (dict(algo=1, dtype=1), 2), (dict(algo=1, d_g=8, l_h=8, l_b=8), 2),
     (dict(algo=2, l_h=17, l_b=16), 2),
     (dict(algo=1, q=0x10002), 2),
-    (dict(algo=1, l_h=514, l_b=16), 2),                  # past the tensor path's 513 taps
+    (dict(algo=1, l_h=642, l_b=16), 2),                  # past the tensor path's 641 taps
     (dict(algo=1, d_g=32, l_h=258, l_b=16), 2),          # d_g 32: bands fit up to 257 taps
 ])
 def test_host_validation(lib, kw, code):
@@ -164,7 +165,9 @@ def test_long_filters_select_an_algorithm():
     bf = g.HYENA_DTYPE_BF16
     assert g.hyena_select_algo(1, 8192, 4096, 64, 130, 64, bf) == g.HYENA_ALGO_TENSOR
     assert g.hyena_select_algo(1, 8192, 4096, 64, 513, 64, bf) == g.HYENA_ALGO_TENSOR
-    assert g.hyena_select_algo(1, 8192, 4096, 64, 514, 64, bf) == g.HYENA_ALGO_FFT
+    assert g.hyena_select_algo(1, 8192, 4096, 64, 514, 64, bf) == g.HYENA_ALGO_TENSOR
+    assert g.hyena_select_algo(1, 8192, 4096, 64, 641, 64, bf) == g.HYENA_ALGO_TENSOR
+    assert g.hyena_select_algo(1, 8192, 4096, 64, 642, 64, bf) == g.HYENA_ALGO_FFT
     assert g.hyena_select_algo(1, 8192, 4096, 32, 257, 64, bf) == g.HYENA_ALGO_TENSOR
     assert g.hyena_select_algo(1, 8192, 4096, 32, 258, 64, bf) == g.HYENA_ALGO_FFT
     assert g.hyena_select_algo(1, 8192, 4096, 16, 66, 16, bf) == g.HYENA_ALGO_FFT

@@ -35,7 +35,7 @@ CHAINS = [
     # name, B, L, D, d_g, l_h, algorithms in call order
     ("se_shape", 2, 3000, 256, 16, 7, (W, T, F, W, Dd, T, W)),
     ("mr_shape", 1, 5000, 512, 64, 128, (T, F, T, Dd, T, F, T)),
-    ("long_filter", 1, 4000, 256, 64, 514, (F, Dd, F, F)),
+    ("long_filter", 1, 4000, 256, 64, 600, (F, T, Dd, F, T)),
 ]
 
 

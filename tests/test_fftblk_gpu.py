@@ -33,7 +33,7 @@ SHAPES = [
     # name, B, L, D, d_g, l_h, dtype; the transform length the plan picks in the comment
     ("n1024_lh17", 2, 3000, 128, 64, 17, "bf16"),        # 1024, 3 blocks, 8 pairs per CTA
     ("n1024_lh300", 1, 2500, 256, 16, 300, "bf16"),      # 1024
-    ("n2048_lh514", 1, 3000, 256, 64, 514, "bf16"),      # the first filter past the band
+    ("n2048_lh514", 1, 3000, 256, 64, 514, "bf16"),      # forced: the tensor path takes it too
     ("n2048_lh1000_ragged", 3, 1777, 64, 8, 1000, "bf16"),   # 2048 (4 pairs: d_g = 8)
     ("n4096_lh1500", 1, 5000, 32, 4, 1500, "bf16"),      # 4096 (2 pairs: d_g = 4)
     ("n4096_lh2049", 2, 4000, 64, 32, 2049, "bf16"),
@@ -100,16 +100,17 @@ def test_fftblk_history():
 
 
 def test_fftblk_deterministic_and_auto():
-    """The MR shape with l_h = 514 (past the tensor band): AUTO picks the block FFT, runs it
+    """The MR shape with l_h = 700 (past the tensor band): AUTO picks the block FFT, runs it
     bit for bit like the forced call, and repeats bit for bit; sampled rows against the
     oracle."""
-    wl = custom("mr514", 1, 8192, 4096, 64, 514, 64, "bf16", "mr", seed=19)
+    wl = custom("mr700", 1, 8192, 4096, 64, 700, 64, "bf16", "mr", seed=19)
     assert g.hyena_select_algo(wl.B, wl.L, wl.D, wl.d_g, wl.l_h, wl.l_b) == g.HYENA_ALGO_FFT
     q, k, v, h = make_inputs(wl, device="cuda")
     a = _run(q, k, v, h, 64, g.HYENA_ALGO_AUTO)
     b = _run(q, k, v, h, 64)
     assert torch.equal(a, b)
     assert torch.equal(a, _run(q, k, v, h, 64))
-    rows = [(0, t) for t in (0, 1, 512, 513, 1534, 1535, 1536, 3070, 3071, 4000, 8191)]
+    # 4096-point blocks of 3397 rows
+    rows = [(0, t) for t in (0, 1, 698, 699, 3396, 3397, 3398, 6793, 6794, 8191)]
     ref = oracle.gated_fir_rows(q, k, v, h, 64, rows)
     U.assert_parity(torch.stack([a[bb, t] for bb, t in rows]), ref, q.dtype)

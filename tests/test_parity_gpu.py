@@ -73,6 +73,8 @@ SHAPES = [
     ("lh513_ragged", 2, 1700, 128, 64, 513, 32, "bf16"),
     ("lh300_multiseg", 3, 1100, 512, 64, 300, 64, "bf16"),
     ("lh513_short_runs", 1, 19200, 128, 64, 513, 64, "bf16"),
+    ("lh514_ragged", 2, 1700, 128, 64, 514, 64, "bf16"),     # five history tiles
+    ("lh641_runs", 1, 19200, 128, 64, 641, 64, "bf16"),
     ("lh400_L77", 1, 77, 128, 64, 400, 64, "bf16"),
     ("dg32_lh257", 1, 900, 128, 32, 257, 64, "bf16"),
     ("dg32_lh200_multiseg", 2, 3000, 256, 32, 200, 16, "bf16"),
@@ -88,7 +90,7 @@ def _tensor_fits(D, d_g, l_h):
     """The tensor kernel's plan: 64-channel tiles of 64 / d_g groups, one Toeplitz band of
     (128 + halo) / 2 TMEM columns per group, next to 128 accumulator columns (512 in all);
     at most 4 earlier 128-row tiles of history (halo <= 512)."""
-    if d_g not in (16, 32, 64) or D % 64 or l_h > 513:
+    if d_g not in (16, 32, 64) or D % 64 or l_h > 641:
         return False
     halo = (l_h - 1 + 15) // 16 * 16
     return (64 // d_g) * (128 + halo) // 2 <= 384
@@ -205,6 +207,8 @@ def test_toeplitz_blocks_builder(l_h, l_b, S):
     ("int_lh385", 1, 2100, 128, 64, 385),
     ("int_lh513", 3, 900, 128, 64, 513),
     ("int_lh513_runs", 1, 19200, 128, 64, 513),
+    ("int_lh641", 2, 1500, 128, 64, 641),            # five history tiles, two k/v stages
+    ("int_lh600_runs", 1, 19200, 128, 64, 600),
     ("int_dg32_lh250", 2, 1000, 128, 32, 250),
 ], ids=lambda s: s[0])
 def test_long_filter_integer_exact(shape):

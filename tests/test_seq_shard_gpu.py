@@ -47,6 +47,7 @@ CASES = [
     ("mr_short_hist", 2, 520, 40, 128, 64, 128, "bf16"),     # zero before the 40 rows
     ("lh300_hist", 1, 900, 299, 128, 64, 300, "bf16"),       # 3 history tiles
     ("lh513_hist", 2, 300, 700, 128, 64, 513, "bf16"),       # 4 history tiles, L < l_h
+    ("lh600_hist", 1, 900, 650, 128, 64, 600, "bf16"),       # 5 history tiles
     ("se_hist", 2, 777, 6, 512, 16, 7, "bf16"),
     ("se_hist_1row", 1, 300, 1, 128, 16, 7, "bf16"),
     ("dg32_hist", 1, 640, 60, 128, 32, 40, "bf16"),
@@ -62,7 +63,7 @@ def _supported(algo, D, d_g, l_h, dtype, L):
     if algo == "fft":
         return U.fftblk_plan(L, D, d_g, l_h, dtype) is not None
     if algo == "tensor":
-        if dtype != "bf16" or d_g not in (16, 32, 64) or D % 64 or l_h > 513:
+        if dtype != "bf16" or d_g not in (16, 32, 64) or D % 64 or l_h > 641:
             return False
         halo = (l_h - 1 + 15) // 16 * 16
         return (64 // d_g) * (128 + halo) // 2 <= 384
@@ -112,7 +113,8 @@ def test_shards_compose_to_the_whole_sequence(algo, bounds):
     U.assert_parity(y, oracle.gated_fir(q, k, v, h, d_g), q.dtype)
 
 
-@pytest.mark.parametrize("l_h,Lh", [(128, 127), (200, 150), (513, 512), (385, 1000)])
+@pytest.mark.parametrize("l_h,Lh", [(128, 127), (200, 150), (513, 512), (385, 1000),
+                                     (641, 700)])
 def test_history_integer_exact(l_h, Lh):
     """Integer inputs: every fp16 operand and fp32 partial sum of the tensor path is exact, so
     the result equals the oracle's rounded once to bf16 -- any history row taken from the wrong
