@@ -643,6 +643,13 @@ def main():
         kernel = {g.HYENA_ALGO_TENSOR: "fir_tc_kernel", g.HYENA_ALGO_WINDOW: "fir_window_kernel",
                   g.HYENA_ALGO_DIRECT: "fir_tiled_kernel", g.HYENA_ALGO_FFT: "fir_fftblk_kernel"}[algo]
         traffic = committed_traffic(kernel, wl.name)
+        # the step in SM clock cycles (time x median sampled SM clock): comparable across boxes
+        # whose clocks differ
+        clock_summary = clocks.summary(t_wall0, t_wall1)
+        try:
+            clock_summary["sm_cycles_per_step"] = (max_ms / K) * 1e3 * clock_summary["sm_mhz"]
+        except (KeyError, TypeError):
+            pass
         line = {
             "metric": METRIC if wl.name == "mr" else
             "gated causal FIR fwd tokens/s (%s); HBM GB/s vs peak" % wl.describe(),
@@ -661,7 +668,7 @@ def main():
                          "median_launch_us": stats["median_us"], "min_launch_us": stats["min_us"],
                          "launch_stats": stats},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K,
-            "clocks": clocks.summary(t_wall0, t_wall1),
+            "clocks": clock_summary,
             "backward": bwd, "configs": configs, "long_filters": long_filters,
             "comparator": comparator,
             "kernel_algo": g.ALGO_NAMES[algo], "device_status": status, "parity": parity,
