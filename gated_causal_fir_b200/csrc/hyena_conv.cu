@@ -238,16 +238,22 @@ struct BlkConfig {
 constexpr BlkConfig kBlkBf16[] = {{10, 8}, {11, 4}, {12, 2}, {13, 1}};
 constexpr BlkConfig kBlkF32[] = {{10, 4}, {11, 2}, {12, 1}};
 
+// Time per point of each transform length relative to N = 1024 and 2048 (see blk_plan).
+double blk_weight(int lgn) { return lgn <= 11 ? 1.0 : (lgn == 12 ? 2.2 : 2.6); }
+
 struct BlkPlan {
   BlkConfig cfg;
   int M, nTB;
   bool ok;
 };
 
-// The transform length with the least work, N log N per block times the blocks per sequence,
-// among those whose channel block (2P channels) lies inside one group, whose row vectors are
-// aligned and whose blocks keep at least N / 8 rows (or one block covers the sequence);
-// ok = false when none applies.
+// The transform length with the least estimated time: N log N per block times the blocks per
+// sequence, weighted by how fast each length's kernel runs per point (measured on the MR shape:
+// ~80 ns per 8192 complex points at N = 1024 and 2048, ~2.2x that at N = 4096 and ~2.6x at
+// 8192, whose narrower row pieces of 2 and 1 channel pairs per CTA make the staging copies
+// small), among the lengths whose channel block (2P channels) lies inside one group, whose row
+// vectors are aligned and whose blocks keep at least N / 8 rows (or one block covers the
+// sequence); ok = false when none applies.
 BlkPlan blk_plan(const Problem &P) {
   BlkPlan best{kBlkBf16[0], 0, 0, false};
   double best_cost = 0;
@@ -265,7 +271,7 @@ BlkPlan blk_plan(const Problem &P) {
     // blocks that keep less than an eighth of their rows cost more than the direct sum
     if (M < N / 8 && nTB > 1) continue;
     if (P.D / (2 * c.P) * nTB > std::numeric_limits<int32_t>::max()) continue;
-    const double cost = static_cast<double>(nTB) * static_cast<double>(N) * c.lgn;
+    const double cost = static_cast<double>(nTB) * static_cast<double>(N) * c.lgn * blk_weight(c.lgn);
     if (!best.ok || cost < best_cost) {
       best = BlkPlan{c, static_cast<int>(M), static_cast<int>(nTB), true};
       best_cost = cost;
@@ -285,8 +291,8 @@ bool fftblk_supported(const Problem &P) { return blk_plan(P).ok; }
 bool fftblk_beats_direct(const Problem &P) {
   const BlkPlan bp = blk_plan(P);
   if (!bp.ok) return false;
-  const double fft = HYENA_FFT_FLOP_WEIGHT * 5.0 * bp.nTB * static_cast<double>(1 << bp.cfg.lgn) *
-                     bp.cfg.lgn / static_cast<double>(P.L);
+  const double fft = HYENA_FFT_FLOP_WEIGHT * blk_weight(bp.cfg.lgn) * 5.0 * bp.nTB *
+                     static_cast<double>(1 << bp.cfg.lgn) * bp.cfg.lgn / static_cast<double>(P.L);
   return fft < 2.0 * P.l_h;
 }
 

@@ -94,7 +94,8 @@ FFTBLK_CONFIGS = {"bf16": ((10, 8), (11, 4), (12, 2), (13, 1)),
 
 def fftblk_plan(L, D, d_g, l_h, dtype="bf16"):
     """The block FFT's choice for a shape (tensors 16-byte aligned): (N, P, M) with the least
-    N log N per block times blocks per sequence, or None where no transform length applies."""
+    N log N per block times blocks per sequence, weighted per transform length as the library
+    weights it (1 up to N = 2048, 2.2 at 4096, 2.6 at 8192), or None where no length applies."""
     best = None
     for lgn, P in FFTBLK_CONFIGS[dtype]:
         N = 1 << lgn
@@ -104,7 +105,7 @@ def fftblk_plan(L, D, d_g, l_h, dtype="bf16"):
         ntb = -(-L // M)
         if M < N // 8 and ntb > 1:
             continue
-        cost = ntb * N * lgn
+        cost = ntb * N * lgn * (1.0 if lgn <= 11 else (2.2 if lgn == 12 else 2.6))
         if best is None or cost < best[0]:
             best = (cost, N, P, M)
     return None if best is None else best[1:]

@@ -75,7 +75,10 @@ def test_select_algo_fallbacks(lib):
     assert g.hyena_select_algo(1, 4096, 96, 32, 40, 32, bf) == g.HYENA_ALGO_FFT     # long enough
     assert g.hyena_select_algo(1, 100, 96, 32, 16, 32, f32) == g.HYENA_ALGO_WINDOW
     assert g.hyena_select_algo(1, 100, 90, 30, 40, 32, bf) == g.HYENA_ALGO_DIRECT   # 8192-point
-    assert g.hyena_select_algo(1, 8192, 90, 30, 40, 32, bf) == g.HYENA_ALGO_FFT     # (P = 1) FFT
+    # d_g = 30: only the 8192-point length applies (one channel pair per CTA, its slowest
+    # configuration): at 40 taps the direct sum wins, at 400 the block FFT
+    assert g.hyena_select_algo(1, 8192, 90, 30, 40, 32, bf) == g.HYENA_ALGO_DIRECT
+    assert g.hyena_select_algo(1, 8192, 90, 30, 400, 32, bf) == g.HYENA_ALGO_FFT
     assert g.hyena_select_algo(1, 100, 93, 31, 40, 32, bf) == g.HYENA_ALGO_DIRECT   # odd groups
     assert g.hyena_select_algo(1, 100, 96, 32, 16, 32, bf) == g.HYENA_ALGO_WINDOW
     assert g.hyena_select_algo(1, 100, 128, 16, 65, 64, bf) == g.HYENA_ALGO_TENSOR  # 4 bands fit
