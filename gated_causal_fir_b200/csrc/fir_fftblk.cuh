@@ -24,12 +24,13 @@
 // software-pipelined through shared memory with cp.async: the next item's k and v rows are
 // copied while the current item is transformed, and the current item's q rows while its
 // forward transform runs.  The first stage reads k and v from there and forms x = k v on the
-// way in; the last inverse stage multiplies by q and writes y to global memory directly.  Q sibling CTAs (consecutive block indices)
-// walk the same range in step, on Q consecutive channel blocks: together they read whole
-// 64-byte pieces of each row at the same time, where one CTA alone would use 4P bytes (bf16)
-// of every 64 that DRAM delivers.  Shared memory rows of 16 complex values are
-// padded to 18, so that every stage's 64-bit accesses and the middle stage's 128-bit row
-// accesses are free of bank conflicts.  All arithmetic is fp32; q, k, v, y are bf16 or fp32.
+// way in; the last inverse stage multiplies by q and writes y to global memory directly.
+// Q sibling CTAs (consecutive block indices) walk the same range in step, on Q consecutive
+// channel blocks: together they read whole 64-byte pieces of each row at the same time, where
+// one CTA alone would use 4P bytes (bf16) of every 64 that DRAM delivers.  Shared-memory rows
+// of 16 complex values are padded to 18, so that every stage's 64-bit accesses and the middle
+// stage's 128-bit row accesses are free of bank conflicts.  All arithmetic is fp32; q, k, v, y
+// are bf16 or fp32.  The kernel launches with programmatic stream serialisation.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
