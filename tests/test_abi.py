@@ -115,6 +115,7 @@ def _call(lib, q=0x10000, k=0x20000, v=0x30000, h=0x40000, y=0x50000, dtype=0, a
     (dict(algo=1, q=0x10002), 2),
     (dict(algo=1, l_h=642, l_b=16), 2),                  # past the tensor path's 641 taps
     (dict(algo=1, d_g=32, l_h=258, l_b=16), 2),          # d_g 32: bands fit up to 257 taps
+    (dict(algo=4, D=96, d_g=3, l_h=40), 2),              # block FFT: channel pairs need even d_g
 ])
 def test_host_validation(lib, kw, code):
     assert _call(lib, **kw) == code
@@ -311,3 +312,23 @@ def test_select_bwd_algo(lib):
     assert g.hyena_select_bwd_algo(1, 300, 4096, 64, 130, 65) == Dd   # l_h > 129
     assert g.hyena_select_bwd_algo(1, 300, 96, 32, 16, 16) == W
     assert g.hyena_select_bwd_algo(1, 300, 4096, 64, 300, 16) == Dd   # l_h > 2 l_b: block form
+
+
+def test_fft_block_refuses_short_blocks_on_host(lib):
+    """A filter whose 8192-point blocks would keep fewer than 1024 of their rows (and no shorter
+    transform holds it): the forced block FFT returns HYENA_ERR_UNSUPPORTED before any device
+    work.  Distinct stand-in addresses, 16 MiB apart."""
+    B, L, D, d_g, l_h = 1, 20000, 128, 64, 8000
+    p = [0x1000000 * (i + 1) for i in range(5)]
+    rc = lib.hyena_conv_fwd_ex(*p, B, L, D, d_g, l_h, 64, 0, g.HYENA_ALGO_FFT, None)
+    assert rc == _native.HYENA_ERR_UNSUPPORTED
+
+
+def test_backward_refuses_the_forward_only_fft(lib):
+    """HYENA_ALGO_FFT is a forward algorithm: the backward refuses it on the host."""
+    B, L, D, d_g, l_h = 1, 256, 128, 64, 16
+    p = [0x1000000 * (i + 1) for i in range(9)]
+    need = lib.hyena_conv_bwd_workspace_bytes(B, L, D, d_g, l_h)
+    ws = 0x1000000 * 12
+    rc = lib.hyena_conv_bwd_ex(*p, B, L, D, d_g, l_h, 16, 0, g.HYENA_ALGO_FFT, ws, need, None)
+    assert rc == _native.HYENA_ERR_UNSUPPORTED
