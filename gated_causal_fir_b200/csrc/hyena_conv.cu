@@ -305,9 +305,6 @@ constexpr int kMaxTileMmas = 24;
 #ifndef HYENA_FFT_MIN_TAPS
 #define HYENA_FFT_MIN_TAPS 17
 #endif
-#ifndef HYENA_FFT_OVER_TENSOR_TAPS
-#define HYENA_FFT_OVER_TENSOR_TAPS 100000
-#endif
 
 int select_algo(const Problem &P) {
   const bool tensor = tensor_supported(P), window = window_supported(P);
@@ -317,13 +314,14 @@ int select_algo(const Problem &P) {
     return t.ng * ((hyena::tc::kTM + t.halo) / 16) <= kMaxTileMmas ? HYENA_ALGO_TENSOR
                                                                    : HYENA_ALGO_WINDOW;
   }
-  if (tensor) return fft && P.l_h >= HYENA_FFT_OVER_TENSOR_TAPS ? HYENA_ALGO_FFT : HYENA_ALGO_TENSOR;
+  if (tensor) return HYENA_ALGO_TENSOR;  // up to 641 taps it beats the block FFT (50-108 us
+                                         // against 170-250 us at the MR shape)
   if (window) return HYENA_ALGO_WINDOW;
   if (fft) return HYENA_ALGO_FFT;
   return HYENA_ALGO_DIRECT;
 }
 
-// Test hooks of the tensor-core forward (hyena_testing_fwd_wait_fault): a shorter limit for the
+// Test hooks of the tensor-core forward (hyena_testing_fwd_fault): a shorter limit for the
 // waits between roles, and an arrive the MMA issuer withholds.  Zero = the product behaviour.
 struct TcTestHooks {
   unsigned long long wait_ns = 0;
